@@ -1,0 +1,412 @@
+#!/usr/bin/env python3
+"""Benchmark: NVFP4 sparse MLA decode on B200.
+
+One step = one decode launch of the hot path (list compaction, row gather,
+on-chip NVFP4 unpack, QK^T, online softmax, PV, split combine) over the
+35-token x 64-head workload: 35 query tokens from 35 requests, each request
+with a 140,000-row context in a shared paged NVFP4 cache (4.9M rows), 2048
+indexer-selected rows per token.  The staged FP8 comparison path and the
+append kernel are timed in the same run and reported beside the headline.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+Prints one JSON line (rank 0).  ``--impl reference`` times the CPU oracle
+(the reference arm for this build) on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "NVFP4 sparse MLA decode µs/launch & TFLOP/s, % of roofline (1×B200)"
+FLOP_PER_ROW_HEAD = 2 * 576 + 2 * 512          # QK^T + PV per (token, head, valid row)
+ROW_BYTES = 352
+N_SETS = 8                                      # rotating index/query sets
+L2_BYTES = 126 * 2 ** 20
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--no-extras", action="store_true", help="skip staged/append/e2e/cpu legs")
+    return ap.parse_args()
+
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML on a thread."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+               0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+    def __init__(self, torch_device: int, period: float = 0.01):
+        self.samples = []
+        self.period = period
+        self.ok = False
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = None
+            p = torch.cuda.get_device_properties(torch_device)
+            bus = getattr(p, "pci_bus_id", None)
+            if bus is not None:  # match the CUDA device to its NVML handle by PCI location
+                bus_id = "%08X:%02X:%02X.0" % (getattr(p, "pci_domain_id", 0), bus, getattr(p, "pci_device_id", 0))
+                try:
+                    self.h = pynvml.nvmlDeviceGetHandleByPciBusId(bus_id.encode())
+                except Exception:  # noqa: BLE001
+                    self.h = None
+            if self.h is None:
+                vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+                ids = [v for v in vis.split(",") if v.strip()]
+                idx = int(ids[torch_device]) if ids and ids[torch_device].strip().isdigit() else torch_device
+                self.h = pynvml.nvmlDeviceGetHandleByIndex(idx)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # noqa: BLE001
+            self.err = str(e)
+            self.max_mhz = None
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                mhz = self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM)
+                rs = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                self.samples.append((time.perf_counter(), mhz, rs))
+            except Exception:  # noqa: BLE001
+                pass
+            time.sleep(self.period)
+
+    def start(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+
+    def stop(self):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self, t0: float, t1: float):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0, "note": "nvml unavailable"}
+        inside = [s for s in self.samples if t0 <= s[0] <= t1]
+        note = "sampled during the timed region"
+        if not inside:  # region shorter than one period: take the samples nearest to it
+            inside = sorted(self.samples, key=lambda s: min(abs(s[0] - t0), abs(s[0] - t1)))[:3]
+            note = "timed region shorter than the sampling period; nearest samples"
+        mhz = [s[1] for s in inside]
+        bits = 0
+        for s in inside:
+            bits |= s[2]
+        reasons = sorted(v for k, v in self.REASONS.items() if bits & k and v != "gpu_idle")
+        return {"sm_mhz": statistics.median(mhz) if mhz else None, "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(inside), "note": note}
+
+
+def kernel_traffic(kernel_file: str):
+    """DRAM bytes per launch from a committed ncu summary, valid only while
+    the kernel source is unchanged since the capture."""
+    path = os.path.join(ROOT, "profiles", "decode_traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f)
+    sha = hashlib.sha256(open(kernel_file, "rb").read()).hexdigest()
+    if d.get("decode_cu_sha256") != sha:
+        return None
+    return d.get("dram_bytes_per_launch")
+
+
+def workload_stats(indices_sets, T, H):
+    """Valid rows per launch and algorithmic bytes / FLOP of one launch."""
+    import torch
+    valid = [int(((ix >= 0)).sum().item()) for ix in indices_sets]
+    rows = statistics.mean(valid)
+    flop = FLOP_PER_ROW_HEAD * H * rows
+    bytes_ = ROW_BYTES * rows + T * indices_sets[0].shape[1] * 4 + T * H * (576 * 2 + 512 * 2 + 4)
+    return rows, flop, bytes_
+
+
+def reference_arm(args, rank, world):
+    """CPU oracle on host cores, rank 0 only, bounded sample of the workload."""
+    if rank != 0:
+        return
+    import numpy as np
+    import torch
+    import oracle
+    from nvfp4_sparse_mla_decode_b200 import synth
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    w = synth.decode35(dev)
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    from harness import oracle_inputs
+    cores = oracle.max_threads()
+    # one token first, to size the sample to ~10-20 s per step
+    qn, qr, rows, remap, _ = oracle_inputs(w, [0])
+    t0 = time.perf_counter()
+    oracle.sparse_mla(qn, qr, rows, remap, w.sm_scale)
+    one = time.perf_counter() - t0
+    ntok = max(1, min(w.T, int(12.0 / max(one, 1e-3))))
+    tokens = list(range(ntok))
+    qn, qr, rows, remap, _ = oracle_inputs(w, tokens)
+    for _ in range(min(args.warmup, 1)):
+        oracle.sparse_mla(qn[:1], qr[:1], rows, remap[:1], w.sm_scale)
+    times = []
+    for _ in range(args.steps if args.steps <= 3 else 3):
+        t0 = time.perf_counter()
+        oracle.sparse_mla(qn, qr, rows, remap, w.sm_scale)
+        times.append(time.perf_counter() - t0)
+    sec = statistics.median(times)
+    flop = FLOP_PER_ROW_HEAD * w.H * int((remap >= 0).sum())
+    tflops = flop / sec / 1e12
+    sample = "%d of %d tokens of decode35x64 (H=64, 2048 valid rows each), FP64 oracle incl. row dequantization" % (
+        ntok, w.T)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": tflops, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": len(times), "warmup": min(args.warmup, 1), "ms_per_step": sec * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": "decode35x64", "T": w.T, "H": w.H, "topk": 2048, "ctx_rows": 140000,
+                   "sample_tokens": ntok},
+        "cpu_baseline": {"value": tflops, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": tflops, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    rank, world, local = dist_env()
+    if args.impl == "reference":
+        return reference_arm(args, rank, world)
+
+    import torch
+    import torch.distributed as tdist
+    import nvfp4_sparse_mla_decode_b200 as nv
+    from nvfp4_sparse_mla_decode_b200 import synth
+
+    assert torch.cuda.is_available(), "bench.py needs a CUDA GPU"
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    nv.lib()  # fails loudly if the library is missing
+
+    # ------------------------------------------------------------ workload
+    w = synth.decode35("cuda", seed=1 + 1000 * rank)
+    from nvfp4_sparse_mla_decode_b200.cache import build_cache
+    t_build = time.perf_counter()
+    cache = build_cache(w)
+    torch.cuda.synchronize()
+    t_build = time.perf_counter() - t_build
+    sets = [(w.indices, w.q_nope, w.q_rope)] + [synth.redraw(w, 100 + k + 1000 * rank) for k in range(N_SETS - 1)]
+    rows, flop, alg_bytes = workload_stats([s[0] for s in sets], w.T, w.H)
+    T, H, topk = w.T, w.H, 2048
+    out = torch.empty(T, H, 512, dtype=torch.float16, device="cuda")
+    lse = torch.empty(T, H, dtype=torch.float32, device="cuda")
+    ws = torch.empty(max(1, nv.workspace_size(T, H, topk)), dtype=torch.uint8, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    stream = torch.cuda.current_stream()
+    launches_per_step = 1 + (1 if nv.num_splits(T, H, topk) > 1 else 0)
+
+    def step(k):
+        ix, qn, qr = sets[k % N_SETS]
+        nv.decode(qn, qr, cache, ix, w.sm_scale, out=out, lse=lse, workspace=ws, dev_status=status)
+
+    for k in range(args.warmup):
+        step(k)
+    torch.cuda.synchronize()
+
+    sampler = ClockSampler(torch.cuda.current_device())
+    sampler.start()
+    time.sleep(0.05)
+    if world > 1:
+        tdist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    h0 = time.perf_counter()
+    e0.record(stream)
+    for k in range(args.steps):
+        step(k)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    h1 = time.perf_counter()
+    if world > 1:
+        tdist.barrier()
+    sampler.stop()
+    ms = e0.elapsed_time(e1)
+    if world > 1:
+        tmax = torch.tensor([ms], device="cuda")
+        tdist.all_reduce(tmax, op=tdist.ReduceOp.MAX)
+        ms = float(tmax.item())
+    assert int(status.item()) == 0, "device status %d" % int(status.item())
+    sec_per = ms * 1e-3 / args.steps
+    tflops = flop / sec_per / 1e12 * world
+    us = sec_per * 1e6
+    peaks, peak_kind = measured_peaks()
+    peak_tf = float(peaks["bf16_tflops"])    # FP16 and BF16 share the nominal dense rate
+    peak_bw = float(peaks["hbm_gbs"])
+    t_roof = max(flop / (peak_tf * 1e12), alg_bytes / (peak_bw * 1e9))
+    clocks = sampler.summary(h0, h1)
+
+    line = {
+        "metric": METRIC, "value": tflops, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f16", "data": "synthetic",
+        "config": {"workload": "decode35x64", "T": T, "H": H, "topk": topk, "ctx_rows": 140000,
+                   "cache_rows": w.num_slots, "valid_rows_per_launch": rows, "splits": nv.num_splits(T, H, topk),
+                   "l2": "inputs larger than L2: %d rotating index/query sets, %.0f MB gathered per cycle > %d MB L2"
+                         % (N_SETS, N_SETS * rows * ROW_BYTES / 1e6, L2_BYTES >> 20),
+                   "parallelism": "replicas" if world > 1 else "single"},
+        "us_per_launch": us,
+        "gathered_gbs": rows * ROW_BYTES / sec_per / 1e9,
+        "alg_bytes_per_launch": alg_bytes, "alg_flop_per_launch": flop,
+        "roofline": {"bound": "tensor", "achieved": flop / sec_per / 1e12, "peak": peak_tf, "unit": "TFLOP/s",
+                     "frac": (flop / sec_per / 1e12) / peak_tf,
+                     "traffic": kernel_traffic(os.path.join(ROOT, "nvfp4_sparse_mla_decode_b200", "csrc", "decode.cu")),
+                     "peak_source": "%s bf16_tflops (burst) from MEASURED_PEAKS.json" % peak_kind
+                                    if peak_kind == "measured" else "fallback 1590 TFLOP/s",
+                     "roofline_us": t_roof * 1e6, "frac_of_roofline_time": t_roof / sec_per,
+                     "mem_bound_us": alg_bytes / (peak_bw * 1e9) * 1e6, "hbm_peak_gbs": peak_bw},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks,
+        "cache_build_s": t_build,
+    }
+
+    if not args.no_extras:
+        # ----------------------------------------------------- staged path
+        staging = torch.empty(nv.staging_size(T, topk), dtype=torch.uint8, device="cuda")
+        nst = max(20, min(2000, args.steps // 10))
+
+        def sstep(k):
+            ix, qn, qr = sets[k % N_SETS]
+            nv.staged_decode(qn, qr, cache, ix, w.sm_scale, out=out, lse=lse, staging=staging, workspace=ws,
+                             dev_status=status)
+
+        for k in range(5):
+            sstep(k)
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for k in range(nst):
+            sstep(k)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        sus = e0.elapsed_time(e1) * 1e3 / nst
+        line["staged_fp8"] = {"us_per_launch": sus, "tflops": flop / (sus * 1e-6) / 1e12,
+                              "native_speedup": sus / us, "launches": 2 + (launches_per_step - 1),
+                              "staging_bytes": staging.numel()}
+        del staging
+        # ------------------------------------------------------------ e2e
+        h_sets = []
+        for ix, qn, qr in sets:
+            h_sets.append((ix.cpu().pin_memory(), qn.cpu().pin_memory(), qr.cpu().pin_memory()))
+        d_ix = torch.empty_like(sets[0][0])
+        d_qn = torch.empty_like(sets[0][1])
+        d_qr = torch.empty_like(sets[0][2])
+        h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        h_lse = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+        ne = max(20, min(2000, args.steps // 10))
+
+        def estep(k):
+            ix, qn, qr = h_sets[k % N_SETS]
+            d_ix.copy_(ix, non_blocking=True)
+            d_qn.copy_(qn, non_blocking=True)
+            d_qr.copy_(qr, non_blocking=True)
+            nv.decode(d_qn, d_qr, cache, d_ix, w.sm_scale, out=out, lse=lse, workspace=ws, dev_status=status)
+            h_out.copy_(out, non_blocking=True)
+            h_lse.copy_(lse, non_blocking=True)
+
+        for k in range(5):
+            estep(k)
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for k in range(ne):
+            estep(k)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        eus = e0.elapsed_time(e1) * 1e3 / ne
+        h2d = d_ix.numel() * 4 + d_qn.numel() * 2 + d_qr.numel() * 2
+        d2h = out.numel() * 2 + lse.numel() * 4
+        line["e2e"] = {"value": flop / (eus * 1e-6) / 1e12 * world, "unit": "TFLOP/s",
+                       "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "us_per_step": eus}
+        # ----------------------------------------------------------- append
+        wa = synth.append_prefill("cuda")
+        acache = torch.zeros(wa.num_slots, nv.ROW_BYTES, dtype=torch.uint8, device="cuda")
+        flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device="cuda")
+        for _ in range(3):
+            nv.kv_append(wa.new_lat, wa.new_rope, wa.new_slots, acache)
+        ta = []
+        for _ in range(20):
+            flush.fill_(1)
+            e0.record(stream)
+            nv.kv_append(wa.new_lat, wa.new_rope, wa.new_slots, acache)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            ta.append(e0.elapsed_time(e1) * 1e3)
+        aus = statistics.median(ta)
+        abytes = wa.T * (1152 + 352 + 4)
+        line["append"] = {"rows": wa.T, "us_per_launch": aus, "gbs": abytes / (aus * 1e-6) / 1e9,
+                          "frac_of_hbm": abytes / (aus * 1e-6) / 1e9 / peak_bw, "l2": "flushed before each launch"}
+        del acache, flush
+        # ---------------------------------------------------- cpu baseline
+        if rank == 0:
+            try:
+                import oracle
+                sys.path.insert(0, os.path.join(ROOT, "tests"))
+                from harness import oracle_inputs
+                qn, qr, rrows, remap, _ = oracle_inputs(w, [0])
+                t0 = time.perf_counter()
+                oracle.sparse_mla(qn, qr, rrows, remap, w.sm_scale)
+                one = time.perf_counter() - t0
+                ntok = max(1, min(T, int(10.0 / max(one, 1e-3))))
+                qn, qr, rrows, remap, _ = oracle_inputs(w, list(range(ntok)))
+                t0 = time.perf_counter()
+                oracle.sparse_mla(qn, qr, rrows, remap, w.sm_scale)
+                sec = time.perf_counter() - t0
+                cflop = FLOP_PER_ROW_HEAD * H * int((remap >= 0).sum())
+                line["cpu_baseline"] = {
+                    "value": cflop / sec / 1e12, "unit": "TFLOP/s", "cores": oracle.max_threads(), "kind": "oracle",
+                    "sample": "%d of %d tokens of decode35x64 (H=64, 2048 rows each), FP64 oracle incl. row "
+                              "dequantization, %.1f s" % (ntok, T, sec)}
+            except Exception as e:  # noqa: BLE001
+                line["cpu_baseline"] = {"value": None, "unit": "TFLOP/s", "cores": None, "kind": "oracle",
+                                        "sample": "oracle unavailable: %s" % e}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        tdist.barrier()
+        tdist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

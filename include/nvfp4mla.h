@@ -1,0 +1,171 @@
+/*
+ * nvfp4mla.h -- C ABI of libnvfp4mla: sparse multi-head-latent-attention
+ * (MLA) decode over a KV cache stored as NVFP4, for NVIDIA B200 (sm_100a).
+ *
+ * What the library computes follows page "Prime Intellect Launches Prime
+ * Inference, Serving 600B Tokens Daily", section "Four-bit caches make room":
+ * the MLA latent cache is compressed with NVFP4 (4-bit values, one FP8 scale
+ * per group of 16), shrinking each row from 576 to 352 bytes; a native
+ * sparse-attention kernel loads only the rows picked by the sparse indexer,
+ * unpacks them on chip and runs attention with FP16 operands and FP32
+ * accumulation; the index list has 2,048 positions and its empty entries
+ * are zero-filled; a staged implementation that first unpacks NVFP4 into FP8
+ * buffers in GPU memory is the comparison path.
+ *
+ * Row layout (352 bytes, the pages fix only the size and the grouping):
+ *   [0,256)   latent dims 0..511 as E2M1 nibbles; byte b = dim 2b (low
+ *             nibble) | dim 2b+1 (high nibble)
+ *   [256,288) 32 E4M3 scales; scale g covers latent dims 16g..16g+15
+ *   [288,352) 64 RoPE dims as E4M3, byte k = RoPE dim k
+ * Latent dim d dequantizes to e2m1(nibble) * e4m3(scale[d/16]); RoPE dim k
+ * to e4m3(byte k).  Both values are exact in FP16.
+ *
+ * Conventions for every call:
+ *   - all data pointers are DEVICE pointers; the caller owns every buffer;
+ *     the library allocates no device memory and keeps no global state;
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream); work is enqueued asynchronously on it;
+ *   - arguments the host can check are checked before anything is enqueued;
+ *     on error the call returns a non-OK status and launches nothing;
+ *   - problems only the device can see (an index or slot out of range, a
+ *     bounded wait that ran out) are OR-ed as status bits into *dev_status
+ *     when dev_status is not NULL; read it after synchronizing the stream;
+ *   - calls on different streams are independent; concurrent calls that
+ *     write the same output or workspace race.
+ */
+#ifndef NVFP4MLA_H
+#define NVFP4MLA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define NVFP4MLA_ROW_BYTES 352        /* 256 nibble bytes + 32 scales + 64 RoPE */
+#define NVFP4MLA_STAGED_ROW_BYTES 576 /* staged FP8 row: 512 latent + 64 RoPE */
+#define NVFP4MLA_LATENT 512
+#define NVFP4MLA_ROPE 64
+#define NVFP4MLA_GROUP 16
+#define NVFP4MLA_MAX_TOPK 2048        /* positions of one index list */
+#define NVFP4MLA_MAX_HEADS 128
+
+typedef enum {
+    NVFP4MLA_OK = 0,
+    NVFP4MLA_ERR_INVALID_ARG = 1, /* null/misaligned pointer, bad size */
+    NVFP4MLA_ERR_UNSUPPORTED = 2, /* shape outside what the kernels cover */
+    NVFP4MLA_ERR_WORKSPACE = 3,   /* workspace/staging buffer too small */
+    NVFP4MLA_ERR_CUDA = 4,        /* a CUDA runtime call failed */
+    NVFP4MLA_ERR_TIMEOUT = 5,     /* device: a bounded wait ran out */
+    NVFP4MLA_ERR_BAD_INDEX = 6    /* device: index/slot outside [0,num_slots) */
+} nvfp4mla_status;
+
+/* Device status bits OR-ed into *dev_status (int32). */
+#define NVFP4MLA_DEV_TIMEOUT 1   /* a bounded wait ran out; results invalid */
+#define NVFP4MLA_DEV_BAD_INDEX 2 /* an index/slot outside [-1, num_slots) */
+#define NVFP4MLA_DEV_LAYOUT 4    /* shared memory base not 1 KB aligned */
+
+/*
+ * nvfp4_kv_append -- quantize n BF16 cache rows into NVFP4 rows at scattered
+ * slots (page "Prime Intellect Launches Prime Inference, Serving 600B Tokens
+ * Daily", section "Four-bit caches make room": 4-bit values with an FP8
+ * scale shared by every 16 of them, 352-byte rows).
+ *
+ *   latent_bf16   [n, latent_stride] BF16, first 512 elements of a row used;
+ *                 16-byte aligned, latent_stride % 8 == 0
+ *   rope_bf16     [n, rope_stride] BF16, first 64 used; 16-byte aligned,
+ *                 rope_stride % 8 == 0
+ *   slot_mapping  [n] int32: row i goes to cache slot slot_mapping[i];
+ *                 a negative slot skips the row; a slot >= num_slots skips
+ *                 it and sets NVFP4MLA_DEV_BAD_INDEX
+ *   cache         [num_slots, 352] bytes, 16-byte aligned
+ * Per group of 16 latent values: a = max|x|, scale = E4M3 round-to-nearest-
+ * even, saturating, of a/6 (FP32 division); each value becomes the E2M1
+ * round-to-nearest-even, saturating, of x/scale (FP32 division), or +0 when
+ * the scale is 0.  RoPE values are E4M3-rounded the same way, unscaled.
+ * n == 0 is a no-op.  Returns INVALID_ARG for null pointers (when n > 0),
+ * misalignment or negative sizes.
+ */
+nvfp4mla_status nvfp4_kv_append(const void *latent_bf16, int64_t latent_stride, const void *rope_bf16,
+                                int64_t rope_stride, const int32_t *slot_mapping, int32_t n, uint8_t *cache,
+                                int64_t num_slots, int32_t *dev_status, void *stream);
+
+/*
+ * nvfp4_sparse_mla_num_splits -- how many CTAs the decode splits each
+ * token's index list across (chosen from T and H to fill the 148 SMs; the
+ * pages size SM clusters from the token batch size, same section).  Pure
+ * host function; returns 0 for unsupported shapes.
+ */
+int32_t nvfp4_sparse_mla_num_splits(int32_t T, int32_t H, int32_t topk);
+
+/*
+ * nvfp4_sparse_mla_workspace_size -- bytes of device workspace
+ * nvfp4_sparse_mla_decode needs for (T, H, topk): FP32 partial outputs and
+ * softmax statistics of the splits.  0 means no workspace is needed.
+ */
+size_t nvfp4_sparse_mla_workspace_size(int32_t T, int32_t H, int32_t topk);
+
+/*
+ * nvfp4_sparse_mla_decode -- sparse MLA decode over the NVFP4 cache (same
+ * page and section: load only the indexer-selected rows, unpack on chip,
+ * FP16 operands, FP32 accumulation, zero-filled empty entries).
+ *
+ *   q_nope_f16  [T, H, 512] FP16, contiguous, 16-byte aligned
+ *   q_rope_f16  [T, H, 64]  FP16, contiguous, 16-byte aligned
+ *   cache       [num_slots, 352] NVFP4 rows, 16-byte aligned
+ *   indices     [T, topk] int32 slot ids, 16-byte aligned; an entry outside
+ *               [0, num_slots) is empty: it takes no part in the softmax
+ *               (entries < -1 or >= num_slots also set DEV_BAD_INDEX)
+ *   sm_scale    softmax scale applied to q.k
+ *   out_f16     [T, H, 512] FP16:  sum_j p_j V_j with p = softmax over the
+ *               valid entries of sm_scale * (q_nope.k_lat + q_rope.k_rope),
+ *               V_j = the 512 latent values of row j; all-empty -> 0
+ *   lse         [T, H] FP32 natural-log sum-exp of the scaled scores;
+ *               all-empty -> -inf
+ *   workspace   device buffer of at least nvfp4_sparse_mla_workspace_size
+ *               bytes (may be NULL when that size is 0), 256-byte aligned
+ * Supported: 1 <= topk <= 2048; H in {16, 32, 64, 128}; T >= 0 (T == 0
+ * is a no-op); num_slots >= 1.  Results are undefined for NaN/Inf queries.
+ */
+nvfp4mla_status nvfp4_sparse_mla_decode(const void *q_nope_f16, const void *q_rope_f16, const uint8_t *cache,
+                                        int64_t num_slots, const int32_t *indices, int32_t topk, int32_t T,
+                                        int32_t H, float sm_scale, void *out_f16, float *lse, void *workspace,
+                                        size_t workspace_bytes, int32_t *dev_status, void *stream);
+
+/*
+ * nvfp4_staged_fp8_staging_size -- bytes of the FP8 staging buffer the
+ * staged path writes: T * topk * 576.
+ */
+size_t nvfp4_staged_fp8_staging_size(int32_t T, int32_t topk);
+
+/*
+ * nvfp4_staged_fp8_mla_decode -- the staged comparison path (same page and
+ * section: the earlier implementation expanded NVFP4 into FP8 buffers in GPU
+ * memory before attention, which costs one more trip through HBM).  Kernel 1 gathers each
+ * valid row, dequantizes it and re-encodes every value as E4M3 (round to
+ * nearest even, saturating) into staging[t, j, 0:576] (512 latent then 64
+ * RoPE); kernel 2 runs the same attention over the staging buffer.  Empty
+ * entries leave their staging rows untouched and stay excluded.
+ * Arguments as nvfp4_sparse_mla_decode, plus
+ *   staging   [T, topk, 576] bytes, 16-byte aligned, at least
+ *             nvfp4_staged_fp8_staging_size bytes
+ * The result equals attention over the E4M3-rounded dequantized values.
+ */
+nvfp4mla_status nvfp4_staged_fp8_mla_decode(const void *q_nope_f16, const void *q_rope_f16, const uint8_t *cache,
+                                            int64_t num_slots, const int32_t *indices, int32_t topk, int32_t T,
+                                            int32_t H, float sm_scale, void *out_f16, float *lse,
+                                            uint8_t *staging, size_t staging_bytes, void *workspace,
+                                            size_t workspace_bytes, int32_t *dev_status, void *stream);
+
+/* Human-readable name of a status code (static storage). */
+const char *nvfp4mla_status_string(nvfp4mla_status status);
+
+/* Library ABI version: major*10000 + minor*100 + patch. */
+int32_t nvfp4mla_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NVFP4MLA_H */

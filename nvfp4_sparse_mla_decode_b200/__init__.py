@@ -1,0 +1,190 @@
+"""Python binding of libnvfp4mla (NVFP4 sparse MLA decode on B200, sm_100a).
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels of ``libnvfp4mla.so`` behind the C ABI of ``include/nvfp4mla.h``.
+PyTorch supplies device memory and the current stream.  There is no CPU or
+PyTorch fallback: if the shared library is missing or the device is not a
+CUDA GPU, calls raise.
+
+Build the library with ``python -m nvfp4_sparse_mla_decode_b200.build``.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Optional
+
+import torch
+
+__all__ = [
+    "ROW_BYTES", "STAGED_ROW_BYTES", "LATENT", "ROPE", "MAX_TOPK", "NVFP4MLAError",
+    "lib", "lib_path", "kv_append", "decode", "staged_decode", "num_splits",
+    "workspace_size", "staging_size", "status_string", "version",
+    "DEV_TIMEOUT", "DEV_BAD_INDEX", "DEV_LAYOUT",
+]
+
+ROW_BYTES = 352
+STAGED_ROW_BYTES = 576
+LATENT = 512
+ROPE = 64
+MAX_TOPK = 2048
+DEV_TIMEOUT = 1
+DEV_BAD_INDEX = 2
+DEV_LAYOUT = 4
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+lib_path = os.path.join(_HERE, "libnvfp4mla.so")
+_lib = None
+
+_vp, _i32, _i64, _f32, _sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
+
+
+class NVFP4MLAError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__("%s: %s (status %d)" % (what, status_string(status), status))
+        self.status = status
+
+
+def lib() -> ctypes.CDLL:
+    """Load libnvfp4mla.so from the package directory (raises if absent)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(lib_path):
+            raise RuntimeError("libnvfp4mla.so is not built; run `python -m nvfp4_sparse_mla_decode_b200.build`")
+        L = ctypes.CDLL(lib_path)
+        L.nvfp4_kv_append.restype = _i32
+        L.nvfp4_kv_append.argtypes = [_vp, _i64, _vp, _i64, _vp, _i32, _vp, _i64, _vp, _vp]
+        L.nvfp4_sparse_mla_num_splits.restype = _i32
+        L.nvfp4_sparse_mla_num_splits.argtypes = [_i32, _i32, _i32]
+        L.nvfp4_sparse_mla_workspace_size.restype = _sz
+        L.nvfp4_sparse_mla_workspace_size.argtypes = [_i32, _i32, _i32]
+        L.nvfp4_sparse_mla_decode.restype = _i32
+        L.nvfp4_sparse_mla_decode.argtypes = [_vp, _vp, _vp, _i64, _vp, _i32, _i32, _i32, _f32, _vp, _vp, _vp,
+                                              _sz, _vp, _vp]
+        L.nvfp4_staged_fp8_staging_size.restype = _sz
+        L.nvfp4_staged_fp8_staging_size.argtypes = [_i32, _i32]
+        L.nvfp4_staged_fp8_mla_decode.restype = _i32
+        L.nvfp4_staged_fp8_mla_decode.argtypes = [_vp, _vp, _vp, _i64, _vp, _i32, _i32, _i32, _f32, _vp, _vp,
+                                                  _vp, _sz, _vp, _sz, _vp, _vp]
+        L.nvfp4mla_status_string.restype = ctypes.c_char_p
+        L.nvfp4mla_status_string.argtypes = [_i32]
+        L.nvfp4mla_version.restype = _i32
+        L.nvfp4mla_version.argtypes = []
+        _lib = L
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().nvfp4mla_status_string(int(status)).decode()
+
+
+def version() -> int:
+    return int(lib().nvfp4mla_version())
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(device: torch.device) -> int:
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def _need_cuda(*ts: torch.Tensor) -> torch.device:
+    dev = ts[0].device
+    for t in ts:
+        if t.device.type != "cuda" or t.device != dev:
+            raise ValueError("all tensors must live on the same CUDA device")
+    return dev
+
+
+def _check(status: int, what: str) -> None:
+    if status != 0:
+        raise NVFP4MLAError(status, what)
+
+
+def num_splits(T: int, H: int, topk: int = MAX_TOPK) -> int:
+    return int(lib().nvfp4_sparse_mla_num_splits(T, H, topk))
+
+
+def workspace_size(T: int, H: int, topk: int = MAX_TOPK) -> int:
+    return int(lib().nvfp4_sparse_mla_workspace_size(T, H, topk))
+
+
+def staging_size(T: int, topk: int = MAX_TOPK) -> int:
+    return int(lib().nvfp4_staged_fp8_staging_size(T, topk))
+
+
+def kv_append(latent: torch.Tensor, rope: torch.Tensor, slot_mapping: torch.Tensor, cache: torch.Tensor,
+              dev_status: Optional[torch.Tensor] = None) -> None:
+    """Quantize BF16 rows latent [n, >=512] / rope [n, >=64] (row strides in
+    elements, unit inner stride) into ``cache`` uint8 [num_slots, 352] at
+    ``slot_mapping`` int32 [n]."""
+    dev = _need_cuda(latent, rope, slot_mapping, cache)
+    assert latent.dtype == torch.bfloat16 and rope.dtype == torch.bfloat16
+    assert slot_mapping.dtype == torch.int32 and cache.dtype == torch.uint8 and cache.is_contiguous()
+    assert latent.stride(-1) == 1 and rope.stride(-1) == 1 and slot_mapping.is_contiguous()
+    n = slot_mapping.numel()
+    assert latent.shape[0] == n and rope.shape[0] == n
+    st = lib().nvfp4_kv_append(_ptr(latent), latent.stride(0) if n else LATENT, _ptr(rope),
+                               rope.stride(0) if n else ROPE, _ptr(slot_mapping), n, _ptr(cache),
+                               cache.shape[0], _ptr(dev_status), _stream(dev))
+    _check(st, "nvfp4_kv_append")
+
+
+def _decode_args(q_nope, q_rope, cache, indices, out, lse):
+    dev = _need_cuda(q_nope, q_rope, cache, indices)
+    T, H = q_nope.shape[0], q_nope.shape[1]
+    assert q_nope.dtype == torch.float16 and q_rope.dtype == torch.float16
+    assert q_nope.shape == (T, H, LATENT) and q_rope.shape == (T, H, ROPE)
+    assert q_nope.is_contiguous() and q_rope.is_contiguous()
+    assert indices.dtype == torch.int32 and indices.dim() == 2 and indices.shape[0] == T and indices.is_contiguous()
+    assert cache.dtype == torch.uint8 and cache.is_contiguous()
+    if out is None:
+        out = torch.empty(T, H, LATENT, dtype=torch.float16, device=dev)
+    if lse is None:
+        lse = torch.empty(T, H, dtype=torch.float32, device=dev)
+    return dev, T, H, indices.shape[1], out, lse
+
+
+def decode(q_nope: torch.Tensor, q_rope: torch.Tensor, cache: torch.Tensor, indices: torch.Tensor,
+           sm_scale: float, out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+           workspace: Optional[torch.Tensor] = None, dev_status: Optional[torch.Tensor] = None,
+           num_slots: Optional[int] = None):
+    """Sparse MLA decode over the NVFP4 cache; returns (out [T,H,512] f16, lse [T,H] f32)."""
+    dev, T, H, topk, out, lse = _decode_args(q_nope, q_rope, cache, indices, out, lse)
+    ws_need = workspace_size(T, H, topk)
+    if workspace is None and ws_need:
+        workspace = torch.empty(ws_need, dtype=torch.uint8, device=dev)
+    st = lib().nvfp4_sparse_mla_decode(_ptr(q_nope), _ptr(q_rope), _ptr(cache),
+                                       num_slots if num_slots is not None else cache.shape[0], _ptr(indices),
+                                       topk, T, H, float(sm_scale), _ptr(out), _ptr(lse), _ptr(workspace),
+                                       workspace.numel() * workspace.element_size() if workspace is not None else 0,
+                                       _ptr(dev_status), _stream(dev))
+    _check(st, "nvfp4_sparse_mla_decode")
+    return out, lse
+
+
+def staged_decode(q_nope: torch.Tensor, q_rope: torch.Tensor, cache: torch.Tensor, indices: torch.Tensor,
+                  sm_scale: float, out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                  staging: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                  dev_status: Optional[torch.Tensor] = None):
+    """The staged FP8 comparison path; returns (out, lse)."""
+    dev, T, H, topk, out, lse = _decode_args(q_nope, q_rope, cache, indices, out, lse)
+    if staging is None:
+        staging = torch.empty(max(1, staging_size(T, topk)), dtype=torch.uint8, device=dev)
+    ws_need = workspace_size(T, H, topk)
+    if workspace is None and ws_need:
+        workspace = torch.empty(ws_need, dtype=torch.uint8, device=dev)
+    st = lib().nvfp4_staged_fp8_mla_decode(_ptr(q_nope), _ptr(q_rope), _ptr(cache), cache.shape[0], _ptr(indices),
+                                           topk, T, H, float(sm_scale), _ptr(out), _ptr(lse), _ptr(staging),
+                                           staging.numel(), _ptr(workspace),
+                                           workspace.numel() if workspace is not None else 0,
+                                           _ptr(dev_status), _stream(dev))
+    _check(st, "nvfp4_staged_fp8_mla_decode")
+    return out, lse
+
+
+def default_sm_scale() -> float:
+    return 1.0 / math.sqrt(LATENT + ROPE)

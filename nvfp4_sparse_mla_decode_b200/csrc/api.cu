@@ -1,0 +1,117 @@
+// api.cu -- the C ABI of libnvfp4mla (declared in include/nvfp4mla.h):
+// argument checks, work planning, launches.  Nothing here allocates memory.
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "../../include/nvfp4mla.h"
+#include "kernels.h"
+
+using namespace nvfp4mla;
+
+namespace {
+
+bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+nvfp4mla_status from_cuda(cudaError_t e) { return e == cudaSuccess ? NVFP4MLA_OK : NVFP4MLA_ERR_CUDA; }
+
+// Checks shared by the native and staged decode entry points.
+nvfp4mla_status check_decode(const void *q_nope, const void *q_rope, const uint8_t *cache, int64_t num_slots,
+                             const int32_t *indices, int32_t topk, int32_t T, int32_t H, float sm_scale,
+                             const void *out, const float *lse, DecodePlan *plan) {
+    if (T < 0 || topk < 1 || topk > NVFP4MLA_MAX_TOPK || num_slots < 1 || num_slots > INT32_MAX)
+        return NVFP4MLA_ERR_INVALID_ARG;
+    if (!(sm_scale == sm_scale) || sm_scale > 3.0e38f || sm_scale < -3.0e38f) return NVFP4MLA_ERR_INVALID_ARG;
+    if (!make_decode_plan(T, H, topk, plan)) return NVFP4MLA_ERR_UNSUPPORTED;
+    if (T == 0) return NVFP4MLA_OK;
+    if (!q_nope || !q_rope || !cache || !indices || !out || !lse) return NVFP4MLA_ERR_INVALID_ARG;
+    if (!aligned(q_nope, 16) || !aligned(q_rope, 16) || !aligned(cache, 16) || !aligned(indices, 16) ||
+        !aligned(out, 16) || !aligned(lse, 4))
+        return NVFP4MLA_ERR_INVALID_ARG;
+    return NVFP4MLA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+nvfp4mla_status nvfp4_kv_append(const void *latent_bf16, int64_t latent_stride, const void *rope_bf16,
+                                int64_t rope_stride, const int32_t *slot_mapping, int32_t n, uint8_t *cache,
+                                int64_t num_slots, int32_t *dev_status, void *stream) {
+    if (n < 0 || num_slots < 0 || latent_stride < NVFP4MLA_LATENT || rope_stride < NVFP4MLA_ROPE)
+        return NVFP4MLA_ERR_INVALID_ARG;
+    if (n == 0) return NVFP4MLA_OK;
+    if (!latent_bf16 || !rope_bf16 || !slot_mapping || !cache) return NVFP4MLA_ERR_INVALID_ARG;
+    if (latent_stride % 8 || rope_stride % 8 || !aligned(latent_bf16, 16) || !aligned(rope_bf16, 16) ||
+        !aligned(cache, 16) || !aligned(slot_mapping, 4))
+        return NVFP4MLA_ERR_INVALID_ARG;
+    return from_cuda(launch_kv_append(latent_bf16, latent_stride, rope_bf16, rope_stride, slot_mapping, n, cache,
+                                      num_slots, dev_status, static_cast<cudaStream_t>(stream)));
+}
+
+int32_t nvfp4_sparse_mla_num_splits(int32_t T, int32_t H, int32_t topk) {
+    DecodePlan p;
+    return make_decode_plan(T, H, topk, &p) ? p.splits : 0;
+}
+
+size_t nvfp4_sparse_mla_workspace_size(int32_t T, int32_t H, int32_t topk) {
+    DecodePlan p;
+    return make_decode_plan(T, H, topk, &p) ? p.workspace_bytes : 0;
+}
+
+nvfp4mla_status nvfp4_sparse_mla_decode(const void *q_nope_f16, const void *q_rope_f16, const uint8_t *cache,
+                                        int64_t num_slots, const int32_t *indices, int32_t topk, int32_t T,
+                                        int32_t H, float sm_scale, void *out_f16, float *lse, void *workspace,
+                                        size_t workspace_bytes, int32_t *dev_status, void *stream) {
+    DecodePlan plan;
+    nvfp4mla_status st =
+        check_decode(q_nope_f16, q_rope_f16, cache, num_slots, indices, topk, T, H, sm_scale, out_f16, lse, &plan);
+    if (st != NVFP4MLA_OK || T == 0) return st;
+    if (plan.workspace_bytes > 0 && (!workspace || workspace_bytes < plan.workspace_bytes)) return NVFP4MLA_ERR_WORKSPACE;
+    if (workspace && !aligned(workspace, 256)) return NVFP4MLA_ERR_INVALID_ARG;
+    return from_cuda(launch_sparse_mla_decode(false, q_nope_f16, q_rope_f16, cache, num_slots, indices, topk, T, H,
+                                              sm_scale, out_f16, lse, workspace, plan, dev_status,
+                                              static_cast<cudaStream_t>(stream)));
+}
+
+size_t nvfp4_staged_fp8_staging_size(int32_t T, int32_t topk) {
+    if (T < 0 || topk < 0) return 0;
+    return (size_t)T * (size_t)topk * NVFP4MLA_STAGED_ROW_BYTES;
+}
+
+nvfp4mla_status nvfp4_staged_fp8_mla_decode(const void *q_nope_f16, const void *q_rope_f16, const uint8_t *cache,
+                                            int64_t num_slots, const int32_t *indices, int32_t topk, int32_t T,
+                                            int32_t H, float sm_scale, void *out_f16, float *lse,
+                                            uint8_t *staging, size_t staging_bytes, void *workspace,
+                                            size_t workspace_bytes, int32_t *dev_status, void *stream) {
+    DecodePlan plan;
+    nvfp4mla_status st =
+        check_decode(q_nope_f16, q_rope_f16, cache, num_slots, indices, topk, T, H, sm_scale, out_f16, lse, &plan);
+    if (st != NVFP4MLA_OK || T == 0) return st;
+    if (!staging || staging_bytes < nvfp4_staged_fp8_staging_size(T, topk)) return NVFP4MLA_ERR_WORKSPACE;
+    if (!aligned(staging, 16)) return NVFP4MLA_ERR_INVALID_ARG;
+    if (plan.workspace_bytes > 0 && (!workspace || workspace_bytes < plan.workspace_bytes)) return NVFP4MLA_ERR_WORKSPACE;
+    if (workspace && !aligned(workspace, 256)) return NVFP4MLA_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = launch_stage_fp8(cache, num_slots, indices, topk, T, staging, s);
+    if (e != cudaSuccess) return NVFP4MLA_ERR_CUDA;
+    return from_cuda(launch_sparse_mla_decode(true, q_nope_f16, q_rope_f16, staging, num_slots, indices, topk, T, H,
+                                              sm_scale, out_f16, lse, workspace, plan, dev_status, s));
+}
+
+const char *nvfp4mla_status_string(nvfp4mla_status status) {
+    switch (status) {
+        case NVFP4MLA_OK: return "ok";
+        case NVFP4MLA_ERR_INVALID_ARG: return "invalid argument";
+        case NVFP4MLA_ERR_UNSUPPORTED: return "unsupported shape";
+        case NVFP4MLA_ERR_WORKSPACE: return "workspace or staging buffer too small";
+        case NVFP4MLA_ERR_CUDA: return "CUDA runtime error";
+        case NVFP4MLA_ERR_TIMEOUT: return "device wait timed out";
+        case NVFP4MLA_ERR_BAD_INDEX: return "index or slot out of range";
+    }
+    return "unknown status";
+}
+
+int32_t nvfp4mla_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,35 @@
+// kernels.h -- internal launchers of libnvfp4mla (host side, no checks:
+// the C ABI in api.cu validates arguments before calling these).
+#pragma once
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace nvfp4mla {
+
+cudaError_t launch_kv_append(const void *latent, int64_t latent_stride, const void *rope, int64_t rope_stride,
+                             const int32_t *slot_mapping, int32_t n, uint8_t *cache, int64_t num_slots,
+                             int32_t *dev_status, cudaStream_t stream);
+
+// Work decomposition of one decode launch.
+struct DecodePlan {
+    int heads_per_cta;  // HG: heads handled by one CTA (N of the MMAs)
+    int head_groups;    // G = H / HG
+    int splits;         // S: CTAs sharing one token's list
+    size_t workspace_bytes;
+};
+bool make_decode_plan(int32_t T, int32_t H, int32_t topk, DecodePlan *plan);
+
+// Sparse MLA decode over NVFP4 rows (staged == false: `src` is the cache of
+// num_slots 352-byte rows, list entries are slots) or over the staging
+// buffer (staged == true: `src` is [T, topk, 576] E4M3 rows addressed by list
+// position; entries outside [0, num_slots) are still the empty ones).
+cudaError_t launch_sparse_mla_decode(bool staged, const void *q_nope, const void *q_rope, const uint8_t *src,
+                                     int64_t num_slots, const int32_t *indices, int32_t topk, int32_t T,
+                                     int32_t H, float sm_scale, void *out, float *lse, void *workspace,
+                                     const DecodePlan &plan, int32_t *dev_status, cudaStream_t stream);
+
+cudaError_t launch_stage_fp8(const uint8_t *cache, int64_t num_slots, const int32_t *indices, int32_t topk,
+                             int32_t T, uint8_t *staging, cudaStream_t stream);
+
+}  // namespace nvfp4mla

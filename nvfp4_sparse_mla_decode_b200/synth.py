@@ -183,6 +183,8 @@ class Workload:
     new_lat: Optional[torch.Tensor] = None
     new_rope: Optional[torch.Tensor] = None
     new_slots: Optional[torch.Tensor] = None
+    ctx_lens: Optional[list] = None
+    tables: Optional[list] = None
 
     def source_rows(self, slots: torch.Tensor):
         """BF16 source of the given slots as the cache holds them after any
@@ -237,7 +239,22 @@ def per_request(device, ctx_lens: Sequence[int], H: int, seed: int, name: str,
             else:
                 idx[t] = idx[t][torch.randperm(TOPK, generator=g, device=device)]
     qn, qr = queries(T, H, seed, device)
-    return Workload(name, T, H, num_slots, idx, qn, qr, SlotRows(seed, num_slots, device))
+    return Workload(name, T, H, num_slots, idx, qn, qr, SlotRows(seed, num_slots, device),
+                    ctx_lens=list(ctx_lens), tables=tables)
+
+
+def redraw(w: Workload, seed: int) -> tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+    """A fresh (indices, q_nope, q_rope) for the same requests, contexts and
+    cache as ``w`` (one request per token, full 2048-entry lists)."""
+    assert w.ctx_lens is not None and w.tables is not None
+    device = w.indices.device
+    lim = torch.tensor(list(w.ctx_lens), dtype=torch.int64)
+    pos = draw_positions(lim, w.indices.shape[1], seed, device)
+    idx = torch.empty_like(w.indices)
+    for t in range(w.T):
+        idx[t] = positions_to_slots(pos[t], w.tables[t])
+    qn, qr = queries(w.T, w.H, seed, device)
+    return idx, qn, qr
 
 
 def decode35(device, seed=1, ctx=140_000, T=35, H=64) -> Workload:

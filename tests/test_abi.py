@@ -1,0 +1,97 @@
+"""Host-side checks of the C ABI (no GPU needed): the library builds and
+loads, exports every function include/nvfp4mla.h declares, plans work, and
+rejects bad arguments before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import nvfp4_sparse_mla_decode_b200 as nv
+from nvfp4_sparse_mla_decode_b200 import build as nvbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    nvbuild.build()
+    return nv.lib()
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "nvfp4mla.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(nvfp4\w*)\s*\(", src)))
+
+
+def test_exports_every_declared_symbol(L):
+    names = declared_functions()
+    assert "nvfp4_sparse_mla_decode" in names and "nvfp4_kv_append" in names
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_status_strings(L):
+    for s in range(7):
+        assert nv.status_string(s)
+    assert nv.status_string(0) == "ok"
+    assert nv.version() >= 100
+
+
+def test_plan_splits_fill_the_gpu(L):
+    assert nv.num_splits(35, 64) == 4          # 140 CTAs on 148 SMs
+    assert nv.num_splits(1, 16) == 16
+    assert nv.num_splits(1, 128) == 16         # 2 head groups x 16
+    assert nv.num_splits(64, 128) == 1
+    assert nv.num_splits(4000, 64) == 1
+    assert nv.num_splits(1, 64, 100) == 1      # a 100-entry list is one tile
+    assert nv.num_splits(1, 48) == 0           # unsupported head count
+    assert nv.workspace_size(35, 64) == 35 * 4 * 64 * 514 * 4
+    assert nv.workspace_size(4000, 64) == 0
+    assert nv.staging_size(35) == 35 * 2048 * 576
+
+
+def _decode(L, **kw):
+    a = dict(q=1 << 20, qr=1 << 20, cache=1 << 20, ns=100, idx=1 << 20, topk=2048, T=1, H=64, sc=0.1,
+             out=1 << 20, lse=1 << 20, ws=1 << 20, wsb=1 << 30, st=None, stream=None)
+    a.update(kw)
+    return L.nvfp4_sparse_mla_decode(a["q"], a["qr"], a["cache"], a["ns"], a["idx"], a["topk"], a["T"], a["H"],
+                                     a["sc"], a["out"], a["lse"], a["ws"], a["wsb"], a["st"], a["stream"])
+
+
+def test_decode_argument_errors(L):
+    INVALID, UNSUP, WS = 1, 2, 3
+    assert _decode(L, T=0) == 0                      # nothing to do, nothing launched
+    assert _decode(L, q=None) == INVALID
+    assert _decode(L, q=(1 << 20) + 8) == INVALID    # misaligned
+    assert _decode(L, topk=0) == INVALID
+    assert _decode(L, topk=4096) == INVALID
+    assert _decode(L, ns=0) == INVALID
+    assert _decode(L, H=48) == UNSUP
+    assert _decode(L, H=256) == UNSUP
+    assert _decode(L, T=35, ws=None, wsb=0) == WS
+    assert _decode(L, T=35, wsb=1000) == WS
+    assert _decode(L, sc=float("nan")) == INVALID
+
+
+def test_append_argument_errors(L):
+    f = L.nvfp4_kv_append
+    assert f(None, 512, None, 64, None, 0, None, 10, None, None) == 0
+    assert f(None, 512, 1 << 20, 64, 1 << 20, 4, 1 << 20, 10, None, None) == 1
+    assert f(1 << 20, 500, 1 << 20, 64, 1 << 20, 4, 1 << 20, 10, None, None) == 1
+    assert f(1 << 20, 512, 1 << 20, 60, 1 << 20, 4, 1 << 20, 10, None, None) == 1
+
+
+def test_staged_argument_errors(L):
+    f = L.nvfp4_staged_fp8_mla_decode
+    base = [1 << 20, 1 << 20, 1 << 20, 100, 1 << 20, 2048, 1, 64, 0.1, 1 << 20, 1 << 20]
+    assert f(*base, None, 0, None, 0, None, None) == 3            # no staging buffer
+    assert f(*base, 1 << 20, 1000, None, 0, None, None) == 3      # staging too small
+    assert f(*base, (1 << 20) + 4, 1 << 30, None, 0, None, None) == 1
+
+
+def test_library_is_sm100a_only():
+    log = os.path.join(ROOT, "nvfp4_sparse_mla_decode_b200", "build.log")
+    if os.path.exists(log):
+        assert "arch=compute_100a,code=sm_100a" in open(log).read()

@@ -1,0 +1,125 @@
+"""Sparse MLA decode on the GPU vs the FP64 CPU oracle.
+
+Tolerance (from the target stated for this path): per (token, head)
+max|out - ref| <= 2e-3 * max|ref| + 1e-4 and |lse - ref| <= 1e-3; all-empty
+lists give out = 0 and lse = -inf on both sides.  The oracle sees only the
+BF16 source rows (it quantizes them itself) and the index lists."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import nvfp4_sparse_mla_decode_b200 as nv
+from nvfp4_sparse_mla_decode_b200 import synth
+from harness import build_cache, check_close, oracle_decode
+
+pytestmark = pytest.mark.gpu
+
+
+def run(w, cache, staged=False, tokens=None):
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    fn = nv.staged_decode if staged else nv.decode
+    out, lse = fn(w.q_nope, w.q_rope, cache, w.indices, w.sm_scale, dev_status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0, "device status %d" % int(status.item())
+    tokens = list(range(w.T)) if tokens is None else list(tokens)
+    ref_o, ref_l = oracle_decode(w, tokens, staged=staged)
+    return check_close(out[tokens], lse[tokens], ref_o, ref_l)
+
+
+def test_tiny_1500_valid_of_2048():
+    w = synth.tiny("cuda")
+    run(w, build_cache(w))
+
+
+@pytest.mark.parametrize("H", [16, 32, 64, 128])
+def test_ragged_tiles_all_head_counts(H):
+    # lists of 1, 100, 128, 129, 700, 2048 valid entries, -1 elsewhere
+    T = 6
+    w = synth.per_request("cuda", [9000] * T, H, seed=11, name="ragged")
+    counts = [1, 100, 128, 129, 700, 2048]
+    for t, n in enumerate(counts):
+        w.indices[t, n:] = -1
+    run(w, build_cache(w))
+
+
+def test_decode35x64_full():
+    w = synth.decode35("cuda")
+    assert nv.num_splits(w.T, w.H) == 4
+    run(w, build_cache(w))
+
+
+def test_staged_path_matches_staged_oracle():
+    w = synth.decode35("cuda", T=6, ctx=20000)
+    run(w, build_cache(w), staged=True)
+
+
+def test_staged_tiny():
+    w = synth.tiny("cuda")
+    run(w, build_cache(w), staged=True)
+
+
+@pytest.mark.parametrize("T", [1, 8, 32, 64, 128, 256])
+def test_sweep_h128(T):
+    w = synth.sweep("cuda", T)
+    cache = build_cache(w)
+    tokens = sorted(set([0, T - 1, T // 2]))
+    run(w, cache, tokens=tokens)
+    del cache
+    torch.cuda.empty_cache()
+
+
+def test_padded_lists_256x64():
+    w = synth.padded("cuda")
+    cache = build_cache(w)
+    tokens = list(range(0, 256, 11)) + [127, 128, 255]
+    run(w, cache, tokens=sorted(set(tokens)))
+
+
+def test_append_then_prefill_4000x64():
+    w = synth.append_prefill("cuda")
+    cache = build_cache(w)
+    tokens = [0, 1, 2, 999, 2000, 3998, 3999]
+    run(w, cache, tokens=tokens)
+
+
+def test_all_empty_and_out_of_range_entries():
+    w = synth.per_request("cuda", [5000] * 4, 64, seed=21, name="empty")
+    w.indices[0, :] = -1
+    w.indices[1, 5:] = -1
+    w.indices[2, ::2] = w.num_slots + 7       # out of range: empty, flagged
+    w.indices[3, ::3] = -(2 ** 31)
+    cache = build_cache(w)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out, lse = nv.decode(w.q_nope, w.q_rope, cache, w.indices, w.sm_scale, dev_status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) & nv.DEV_BAD_INDEX
+    assert torch.all(out[0] == 0) and torch.all(torch.isneginf(lse[0]))
+    ref_o, ref_l = oracle_decode(w, range(4))
+    check_close(out, lse, ref_o, ref_l)
+
+
+@pytest.mark.parametrize("topk", [1, 64, 100, 777, 2047])
+def test_short_lists(topk):
+    w = synth.per_request("cuda", [4000] * 3, 64, seed=31, name="short")
+    w.indices = w.indices[:, :topk].contiguous()
+    run(w, build_cache(w))
+
+
+def test_duplicates_and_permutation():
+    w = synth.per_request("cuda", [3000] * 2, 64, seed=41, name="dup")
+    w.indices[0, 1000:] = w.indices[0, :1048].clone()   # duplicates count per position
+    perm = torch.randperm(2048, device="cuda")
+    w.indices[1] = w.indices[1][perm]
+    run(w, build_cache(w))
+
+
+def test_zero_tokens_is_noop():
+    cache = torch.zeros(16, nv.ROW_BYTES, dtype=torch.uint8, device="cuda")
+    qn = torch.empty(0, 64, 512, dtype=torch.float16, device="cuda")
+    qr = torch.empty(0, 64, 64, dtype=torch.float16, device="cuda")
+    idx = torch.empty(0, 2048, dtype=torch.int32, device="cuda")
+    out, lse = nv.decode(qn, qr, cache, idx, 0.1)
+    assert out.numel() == 0 and lse.numel() == 0
