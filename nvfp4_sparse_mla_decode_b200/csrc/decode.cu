@@ -44,11 +44,15 @@
 #include <cmath>
 
 #include "common.cuh"
+#include "decode_common.cuh"
 #include "kernels.h"
 #include "ptx.cuh"
 
 namespace nvfp4mla {
 using namespace ptx;
+#ifdef NVFP4MLA_TRACE
+void set_trace_buffer(unsigned long long *p) { set_trace_local(p); }
+#endif
 
 namespace dec {
 constexpr int kTileRows = 128;
@@ -66,6 +70,7 @@ constexpr int kNumBars = 16;
 constexpr int kOffMisc = kOffBar + kNumBars * 8;
 constexpr int kSmemBytes = kOffMisc + 64;
 static_assert(kSmemBytes <= 232448, "shared memory budget");
+static_assert(kMaxHG * kLatent * 4 <= kTileBytes, "FP32 output staging must fit in the tile region");
 constexpr int kThreads = 512;
 
 constexpr int BAR_CHUNK_FULL = 0;  // [9] unpack -> MMA, count 8 warps
@@ -80,79 +85,14 @@ constexpr uint32_t kColS = 256;    // S^T: HG columns
 constexpr float kRescaleThreshold = 8.0f;
 }  // namespace dec
 
-struct DecodeArgs {
-    const __half *q_nope;
-    const __half *q_rope;
-    const uint8_t *src;
-    int64_t num_slots;
-    const int32_t *indices;
-    int topk, T, H, G, S;
-    float scale_log2;
-    __half *out;
-    float *lse;
-    float *ws_o;
-    float *ws_ml;
-    int32_t *dev_status;
-};
-
-__device__ __forceinline__ float ex2(float x) {
-    float y;
-    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-    return y;
-}
-__device__ __forceinline__ float lg2(float x) {
-    float y;
-    asm("lg2.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
-    return y;
-}
-// Named barrier 1 over the 128 softmax threads, optionally OR-reducing a flag.
-__device__ __forceinline__ void sm_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
-__device__ __forceinline__ bool sm_bar_or(bool p) {
-    uint32_t r;
-    asm volatile(
-        "{\n\t.reg .pred pi, po;\n\tsetp.ne.u32 pi, %1, 0;\n\tbar.red.or.pred po, 1, 128, pi;\n\tselp.u32 %0, 1, 0, po;\n\t}"
-        : "=r"(r)
-        : "r"((uint32_t)p)
-        : "memory");
-    return r != 0;
-}
-__device__ __forceinline__ uint32_t ldg32(const uint8_t *p) {
-    return __ldg(reinterpret_cast<const unsigned int *>(p));
-}
-__device__ __forceinline__ uint2 ldg64(const uint8_t *p) { return __ldg(reinterpret_cast<const uint2 *>(p)); }
-
-// In-warp transpose reduction: on entry each lane holds W column values; on
-// exit lane l holds op-reduced columns [l*W/32, (l+1)*W/32) in v[0..W/32)
-// (W == 16: column l/2 in v[0], duplicated in lane pairs).
-template <int W, bool kMax>
-__device__ __forceinline__ void warp_transpose_reduce(float (&v)[W], int lane) {
-#pragma unroll
-    for (int o = 16, w = W; o >= 1 && w >= 2; o >>= 1, w >>= 1) {
-        const bool upper = (lane & o) != 0;
-#pragma unroll
-        for (int j = 0; j < w / 2; ++j) {
-            const float keep = upper ? v[j + w / 2] : v[j];
-            const float send = upper ? v[j] : v[j + w / 2];
-            const float got = __shfl_xor_sync(0xffffffffu, send, o);
-            v[j] = kMax ? fmaxf(keep, got) : keep + got;
-        }
-    }
-    if (W == 16) {
-        const float got = __shfl_xor_sync(0xffffffffu, v[0], 1);
-        v[0] = kMax ? fmaxf(v[0], got) : v[0] + got;
-    }
-}
-template <int W>
-__device__ __forceinline__ int transposed_col(int lane, int j) {
-    return W >= 32 ? lane * (W / 32) + j : lane >> 1;
-}
-constexpr int cols_per_lane(int W) { return W >= 32 ? W / 32 : 1; }
-
 template <int HG, bool kStaged>
 __global__ void __launch_bounds__(dec::kThreads, 1) sparse_mla_decode_kernel(const DecodeArgs a) {
     using namespace dec;
     extern __shared__ __align__(1024) uint8_t smem[];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+#ifdef NVFP4MLA_TRACE
+    const unsigned long long t_start = clock64();
+#endif
     const int split = blockIdx.x % a.S;
     const int rest = blockIdx.x / a.S;
     const int g = rest % a.G;
@@ -171,15 +111,16 @@ __global__ void __launch_bounds__(dec::kThreads, 1) sparse_mla_decode_kernel(con
     uint32_t *cnt_s = reinterpret_cast<uint32_t *>(smem + kOffRed);  // reused before the softmax starts
 
     // ---------------------------------------------------------------- setup
-    if (tid == 0) {
-        for (int c = 0; c < kChunks; ++c) mbar_init(&bars[BAR_CHUNK_FULL + c], 8);
-        for (int c = 0; c < 4; ++c) mbar_init(&bars[BAR_CHUNK_FREE + c], 1);
-        mbar_init(&bars[BAR_S_FULL], 1);
-        mbar_init(&bars[BAR_P_FULL], 4);
-        mbar_init(&bars[BAR_DRAIN], 1);
+    if (warp == 1) {  // one barrier per lane
+        uint32_t count = 0;
+        if (lane < BAR_CHUNK_FREE) count = 8;           // chunk written by the 8 unpack warps
+        else if (lane < BAR_P_FULL) count = 1;          // MMA commits
+        else if (lane == BAR_P_FULL) count = 4;         // 4 softmax warps
+        else if (lane == BAR_DRAIN) count = 1;
+        if (count) mbar_init(&bars[lane], count);
         fence_mbar_init();
     }
-    if (warp == 0) {
+    if (warp == 3) {  // a warp with no setup work: the allocation can take a while
         tmem_alloc(&misc[0], kTmemCols);
         tmem_relinquish();
     }
@@ -187,16 +128,17 @@ __global__ void __launch_bounds__(dec::kThreads, 1) sparse_mla_decode_kernel(con
 
     // Q of (t, heads g*HG ..) -> shared memory, K-major, 128-byte swizzle:
     // chunk c holds dims 64c..64c+63 of every head (chunk 8 = RoPE).
+    // Issued as 16-byte async copies so every load of the CTA is in flight
+    // at once; they complete before the setup barrier below.
     if (warp >= 8) {
         const int ut = tid - 256;
         const int64_t head0 = (int64_t)t * a.H + (int64_t)g * HG;
         for (int u = ut; u < HG * 72; u += 256) {
             const int h = u / 72, v = u % 72;
-            const uint4 val = v < 64 ? __ldg(reinterpret_cast<const uint4 *>(a.q_nope + (head0 + h) * kLatent) + v)
-                                     : __ldg(reinterpret_cast<const uint4 *>(a.q_rope + (head0 + h) * kRope) + (v - 64));
-            *reinterpret_cast<uint4 *>(smem + kOffQ + (v >> 3) * (HG * 128) + sw128_offset(h, v & 7)) = val;
+            const void *src = v < 64 ? static_cast<const void *>(a.q_nope + (head0 + h) * kLatent + 8 * v)
+                                     : static_cast<const void *>(a.q_rope + (head0 + h) * kRope + 8 * (v - 64));
+            cp_async16(smem + kOffQ + (v >> 3) * (HG * 128) + sw128_offset(h, v & 7), src);
         }
-        fence_proxy_async_smem();
     }
 
     // Compact the token's list: keep valid entries in list order; this CTA
@@ -218,17 +160,27 @@ __global__ void __launch_bounds__(dec::kThreads, 1) sparse_mla_decode_kernel(con
     if (__any_sync(0xffffffffu, bad) && lane == 0 && split == 0 && g == 0 && a.dev_status)
         atomicOr(a.dev_status, NVFP4MLA_DEV_BAD_INDEX);
     __syncthreads();
-    int n_valid = 0;
+    // exclusive prefix of the 64 per-(round, warp) counts: warp 0 scans them
+    // (2 per lane), everyone reads its 4 offsets and the total back
+    uint32_t *pre_s = cnt_s + 64;
+    if (warp == 0) {
+        const uint32_t c0 = cnt_s[2 * lane], c1 = cnt_s[2 * lane + 1];
+        uint32_t incl = c0 + c1;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+        }
+        const uint32_t excl = incl - c0 - c1;
+        pre_s[2 * lane] = excl;
+        pre_s[2 * lane + 1] = excl + c0;
+        if (lane == 31) pre_s[64] = incl;
+    }
+    __syncthreads();
     int before[4];
 #pragma unroll
-    for (int k = 0; k < 4; ++k) before[k] = 0;
-    for (int q = 0; q < 64; ++q) {
-        const int c = (int)cnt_s[q];
-#pragma unroll
-        for (int k = 0; k < 4; ++k)
-            if (q < k * 16 + warp) before[k] += c;
-        n_valid += c;
-    }
+    for (int k = 0; k < 4; ++k) before[k] = (int)pre_s[k * 16 + warp];
+    const int n_valid = (int)pre_s[64];
     const int per = (n_valid + a.S - 1) / a.S;
     const int lo = split * per;
     const int hi = min(n_valid, lo + per);
@@ -241,14 +193,24 @@ __global__ void __launch_bounds__(dec::kThreads, 1) sparse_mla_decode_kernel(con
             if (pos >= lo && pos < hi) idx_s[pos - lo] = kStaged ? (tid + 512 * k) : vals[k];
         }
     }
+    if (warp >= 8) {
+        cp_async_wait_all();
+        fence_proxy_async_smem();
+    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = misc[0];
+    if (tid == 0) TRACE(0);
 
-    if (warp == 0) {
+    // Register budget (launched with 128 x 512): the MMA/idle warpgroup gives
+    // registers to the softmax and unpack warps, 128 x 48 + 128 x 144 +
+    // 256 x 160 = 65536.  Each role changes its budget inside its own branch
+    // so the compiler sizes each role's code separately.
+    if (warp < 4) {
+        regs_dec<48>();
         // ------------------------------------------------------------- MMA
-        if (lane == 0) {
+        if (warp == 0 && lane == 0) {
             const uint32_t idesc_qk = idesc_f16_f32(128, HG, false, false);
             const uint32_t idesc_pv = idesc_f16_f32(128, HG, true, true);
             const uint64_t dK0 = smem_desc(smem_u32(smem), 16, 1024);
@@ -256,129 +218,152 @@ __global__ void __launch_bounds__(dec::kThreads, 1) sparse_mla_decode_kernel(con
             const uint64_t dV0 = smem_desc(smem_u32(smem), kChunkBytes, 1024);
             const uint64_t dP0 = smem_desc(smem_u32(smem + 8 * kChunkBytes), kChunkBytes, 1024);
             bool ok = true;
+            // Descriptors advance by adding (byte offset >> 4) to the start
+            // address field; the chunk and block loops stay rolled so the
+            // compiler keeps a handful of descriptors live, not one per MMA.
             for (int i = 0; i < ntiles && ok; ++i) {
                 const uint32_t par = i & 1;
-#pragma unroll
+                uint64_t dk = dK0, dq = dQ0;
+#pragma unroll 1
                 for (int c = 0; c < kChunks; ++c) {
                     if (!mbar_wait(&bars[BAR_CHUNK_FULL + c], par)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-#pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        mma_ss(tmem + kColS, dK0 + (uint64_t)((c * kChunkBytes + kk * 32) >> 4),
-                               dQ0 + (uint64_t)((c * HG * 128 + kk * 32) >> 4), idesc_qk, (c | kk) != 0);
+                    mma_ss(tmem + kColS, dk, dq, idesc_qk, c != 0);
+                    mma_ss(tmem + kColS, dk + 2, dq + 2, idesc_qk, 1u);
+                    mma_ss(tmem + kColS, dk + 4, dq + 4, idesc_qk, 1u);
+                    mma_ss(tmem + kColS, dk + 6, dq + 6, idesc_qk, 1u);
+                    dk += (uint64_t)(kChunkBytes >> 4);
+                    dq += (uint64_t)((HG * 128) >> 4);
                 }
                 if (!ok) break;
                 mma_commit(&bars[BAR_S_FULL]);
+                if (i < 8) TRACE(1 + 6 * i);
                 if (!mbar_wait(&bars[BAR_P_FULL], par)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-#pragma unroll
+                if (i < 8) TRACE(2 + 6 * i);
+                uint64_t dv = dV0;
+#pragma unroll 1
                 for (int dc = 0; dc < 4; ++dc) {
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk)
-                        mma_ss(tmem + kColO + dc * HG, dV0 + (uint64_t)((2 * dc * kChunkBytes + kk * 2048) >> 4),
-                               dP0 + (uint64_t)((kk * 2048) >> 4), idesc_pv, (i > 0 || kk > 0) ? 1u : 0u);
+                        mma_ss(tmem + kColO + dc * HG, dv + (uint64_t)(kk * 128), dP0 + (uint64_t)(kk * 128),
+                               idesc_pv, (i > 0 || kk > 0) ? 1u : 0u);
                     mma_commit(&bars[BAR_CHUNK_FREE + dc]);
+                    dv += (uint64_t)((2 * kChunkBytes) >> 4);
                 }
+                if (i < 8) TRACE(3 + 6 * i);
             }
             if (!ok && a.dev_status) atomicOr(a.dev_status, NVFP4MLA_DEV_TIMEOUT);
             mma_commit(&bars[BAR_DRAIN]);  // nothing may still write TMEM at teardown
             mbar_wait(&bars[BAR_DRAIN], 0);
+            TRACE(60);
         }
         __syncwarp();
-    } else if (warp >= 4 && warp < 8) {
+    } else if (warp < 8) {
         // --------------------------------------------------------- softmax
-        constexpr int CPL = cols_per_lane(HG);
-        const int st = tid - 128;         // tile row == TMEM lane
+        regs_inc<144>();
+        // Heads are processed in halves of HW = min(HG, 32): the reference
+        // max, rescale and row sums of a head never depend on other heads.
+        constexpr int HW = HG < 32 ? HG : 32;
+        constexpr int NH = HG / HW;
+        const int st = tid - 128;  // tile row == TMEM lane
         const int wq = st >> 5;
         const uint32_t lane_base = (uint32_t)(32 * wq) << 16;
-        uint8_t *p_tile = smem + 8 * kChunkBytes;
-        float lp[CPL];
+        uint8_t *p_tile = smem + 8 * kChunkBytes;  // P^T overwrites the RoPE chunk
+        float lp[NH];  // warp-partial row sums, column h0 + transposed_col<HW>(lane)
 #pragma unroll
-        for (int j = 0; j < CPL; ++j) lp[j] = 0.0f;
+        for (int j = 0; j < NH; ++j) lp[j] = 0.0f;
         bool ok = true;
         for (int i = 0; i < ntiles; ++i) {
+            // S_FULL(i) also covers PV(i-1): the MMA thread issued it earlier,
+            // so O^T is quiescent and may be rescaled here.
             if (!mbar_wait(&bars[BAR_S_FULL], i & 1)) {
                 ok = false;
                 break;
             }
             tc_fence_after();
+            if (st == 0 && i < 8) TRACE(4 + 6 * i);
+            uint32_t rs[HG];
+            tmem_ld_cols<HG>(tmem + lane_base + kColS, rs);
+            tmem_ld_wait();
             const int nrows = min(kTileRows, n_mine - kTileRows * i);
             const bool valid = st < nrows;
-            float sv[HG];
 #pragma unroll
-            for (int cb = 0; cb < HG; cb += 16) {
-                uint32_t r[16];
-                tmem_ld16(tmem + lane_base + kColS + cb, r);
-                tmem_ld_wait();
+            for (int hh = 0; hh < NH; ++hh) {
+                const int h0 = hh * HW;
+                float sv[HW];
 #pragma unroll
-                for (int j = 0; j < 16; ++j) sv[cb + j] = __uint_as_float(r[j]) * a.scale_log2;
-            }
-            bool need = false;
-            if (valid) {
+                for (int h = 0; h < HW; ++h) sv[h] = __uint_as_float(rs[h0 + h]) * a.scale_log2;
+                bool need = false;
+                if (valid) {
 #pragma unroll
-                for (int h = 0; h < HG; ++h) need |= sv[h] > m_s[h] + kRescaleThreshold;
-            }
-            if (sm_bar_or(need)) {
-                float mx[HG];
-#pragma unroll
-                for (int h = 0; h < HG; ++h) mx[h] = valid ? sv[h] : -INFINITY;
-                warp_transpose_reduce<HG, true>(mx, lane);
-#pragma unroll
-                for (int j = 0; j < CPL; ++j) red_s[wq * 64 + transposed_col<HG>(lane, j)] = mx[j];
-                sm_bar();
-                if (st < HG) {
-                    const float old = m_s[st];
-                    float nm = old;
-#pragma unroll
-                    for (int w = 0; w < 4; ++w) nm = fmaxf(nm, red_s[w * 64 + st]);
-                    aux_s[st] = (old == -INFINITY) ? 0.0f : ex2(old - nm);
-                    m_s[st] = nm;
+                    for (int h = 0; h < HW; ++h) need |= sv[h] > m_s[h0 + h] + kRescaleThreshold;
                 }
-                sm_bar();
+                if (sm_bar_or(need)) {
+                    {
+                        float mx[HW];
 #pragma unroll
-                for (int j = 0; j < CPL; ++j) lp[j] *= aux_s[transposed_col<HG>(lane, j)];
-                if (i > 0) {
+                        for (int h = 0; h < HW; ++h) mx[h] = valid ? sv[h] : -INFINITY;
+                        warp_transpose_reduce<HW, true>(mx, lane);
+                        red_s[wq * 64 + h0 + transposed_col<HW>(lane, 0)] = mx[0];
+                    }
+                    sm_bar();
+                    if (st < HW) {
+                        const int h = h0 + st;
+                        const float old = m_s[h];
+                        float nm = old;
 #pragma unroll
-                    for (int dc = 0; dc < 4; ++dc) {
-#pragma unroll
-                        for (int cb = 0; cb < HG; cb += 16) {
-                            uint32_t r[16];
-                            const uint32_t addr = tmem + lane_base + kColO + dc * HG + cb;
-                            tmem_ld16(addr, r);
+                        for (int w = 0; w < 4; ++w) nm = fmaxf(nm, red_s[w * 64 + h]);
+                        aux_s[h] = (old == -INFINITY) ? 0.0f : ex2(old - nm);
+                        m_s[h] = nm;
+                    }
+                    sm_bar();
+                    lp[hh] *= aux_s[h0 + transposed_col<HW>(lane, 0)];
+                    if (i > 0) {
+#pragma unroll 1
+                        for (int dc = 0; dc < 4; ++dc) {
+                            uint32_t r[HW];
+                            const uint32_t addr = tmem + lane_base + kColO + dc * HG + h0;
+                            tmem_ld_cols<HW>(addr, r);
                             tmem_ld_wait();
 #pragma unroll
-                            for (int j = 0; j < 16; ++j) r[j] = __float_as_uint(__uint_as_float(r[j]) * aux_s[cb + j]);
-                            tmem_st16(addr, r);
+                            for (int h = 0; h < HW; ++h) r[h] = __float_as_uint(__uint_as_float(r[h]) * aux_s[h0 + h]);
+#pragma unroll
+                            for (int cb = 0; cb < HW; cb += 16) {
+                                uint32_t q[16];
+#pragma unroll
+                                for (int j = 0; j < 16; ++j) q[j] = r[cb + j];
+                                tmem_st16(addr + cb, q);
+                            }
                         }
+                        tmem_st_wait();
                     }
-                    tmem_st_wait();
                 }
-            }
-            // P = 2^(s - m) for valid rows, 0 for the zero-filled ones
 #pragma unroll
-            for (int h = 0; h < HG; ++h) sv[h] = valid ? ex2(sv[h] - m_s[h]) : 0.0f;
+                for (int h = 0; h < HW; ++h) sv[h] = valid ? ex2(sv[h] - m_s[h0 + h]) : 0.0f;
 #pragma unroll
-            for (int j = 0; j < HG / 8; ++j) {
-                uint4 pk;
-                pk.x = pack_half2(sv[8 * j + 0], sv[8 * j + 1]);
-                pk.y = pack_half2(sv[8 * j + 2], sv[8 * j + 3]);
-                pk.z = pack_half2(sv[8 * j + 4], sv[8 * j + 5]);
-                pk.w = pack_half2(sv[8 * j + 6], sv[8 * j + 7]);
-                *reinterpret_cast<uint4 *>(p_tile + sw128_offset(st, j)) = pk;
+                for (int j = 0; j < HW / 8; ++j) {
+                    uint4 pk;
+                    pk.x = pack_half2(sv[8 * j + 0], sv[8 * j + 1]);
+                    pk.y = pack_half2(sv[8 * j + 2], sv[8 * j + 3]);
+                    pk.z = pack_half2(sv[8 * j + 4], sv[8 * j + 5]);
+                    pk.w = pack_half2(sv[8 * j + 6], sv[8 * j + 7]);
+                    *reinterpret_cast<uint4 *>(p_tile + sw128_offset(st, h0 / 8 + j)) = pk;
+                }
+                warp_transpose_reduce<HW, false>(sv, lane);
+                lp[hh] += sv[0];
             }
             fence_proxy_async_smem();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars[BAR_P_FULL]);
-            warp_transpose_reduce<HG, false>(sv, lane);
-#pragma unroll
-            for (int j = 0; j < CPL; ++j) lp[j] += sv[j];
+            if (st == 0 && i < 8) TRACE(5 + 6 * i);
         }
         if (!ok && a.dev_status) atomicOr(a.dev_status, NVFP4MLA_DEV_TIMEOUT);
         // ---------------------------------------------------------- epilogue
@@ -390,10 +375,9 @@ __global__ void __launch_bounds__(dec::kThreads, 1) sparse_mla_decode_kernel(con
             tc_fence_after();
         }
         const bool have = ok && ntiles > 0;
-        if (HG < 32 && (lane & 1)) {
-        } else {
+        if (!(HW < 32 && (lane & 1))) {
 #pragma unroll
-            for (int j = 0; j < CPL; ++j) red_s[wq * 64 + transposed_col<HG>(lane, j)] = lp[j];
+            for (int hh = 0; hh < NH; ++hh) red_s[wq * 64 + hh * HW + transposed_col<HW>(lane, 0)] = lp[hh];
         }
         sm_bar();
         if (st < HG) {
@@ -410,34 +394,64 @@ __global__ void __launch_bounds__(dec::kThreads, 1) sparse_mla_decode_kernel(con
             }
         }
         sm_bar();
-#pragma unroll 1
-        for (int dc = 0; dc < 4; ++dc) {
-            const int dv = 128 * dc + st;
+        // O^T (TMEM, lanes = dv) -> normalized rows staged in the (now free)
+        // tile region, then bulk copies to global memory.
+        //  one split:   out[t, g*HG + h, :] (FP16), one copy of HG x 1 KB;
+        //  split parts: ws_o[t, split, dc, g*HG + h, 0:128] (FP32, dv block
+        //               major), one 32 KB copy per 128-dv block, issued as soon
+        //               as the block is staged.
+        float inv_l[HG];
 #pragma unroll
-            for (int cb = 0; cb < HG; cb += 16) {
-                uint32_t r[16];
+        for (int h = 0; h < HG; ++h) inv_l[h] = aux_s[h];
+        uint8_t *stage = smem;
+        if (a.S == 1) {
+#pragma unroll 1
+            for (int dc = 0; dc < 4; ++dc) {
+                const int dv = 128 * dc + st;
+                uint32_t r[HG];
                 if (have) {
-                    tmem_ld16(tmem + lane_base + kColO + dc * HG + cb, r);
+                    tmem_ld_cols<HG>(tmem + lane_base + kColO + dc * HG, r);
                     tmem_ld_wait();
                 } else {
 #pragma unroll
-                    for (int j = 0; j < 16; ++j) r[j] = 0u;
+                    for (int h = 0; h < HG; ++h) r[h] = 0u;
                 }
 #pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    const int h = cb + j;
-                    const float o = __uint_as_float(r[j]) * aux_s[h];
-                    if (a.S == 1) {
-                        a.out[((int64_t)t * a.H + (int64_t)g * HG + h) * kLatent + dv] = __float2half_rn(o);
-                    } else {
-                        const int64_t prow = ((int64_t)t * a.S + split) * a.H + (int64_t)g * HG + h;
-                        a.ws_o[prow * kLatent + dv] = o;
-                    }
-                }
+                for (int h = 0; h < HG; ++h)
+                    reinterpret_cast<__half *>(stage)[h * kLatent + dv] = __float2half_rn(__uint_as_float(r[h]) * inv_l[h]);
             }
+            fence_proxy_async_smem();
+            sm_bar();
+            if (st == 0) {
+                bulk_s2g(a.out + ((int64_t)t * a.H + (int64_t)g * HG) * kLatent, stage, HG * kLatent * 2);
+                bulk_commit_wait_read();
+            }
+        } else {
+#pragma unroll 1
+            for (int dc = 0; dc < 4; ++dc) {
+                float *blk = reinterpret_cast<float *>(stage + dc * (HG * 128 * 4));
+                uint32_t r[HG];
+                if (have) {
+                    tmem_ld_cols<HG>(tmem + lane_base + kColO + dc * HG, r);
+                    tmem_ld_wait();
+                } else {
+#pragma unroll
+                    for (int h = 0; h < HG; ++h) r[h] = 0u;
+                }
+#pragma unroll
+                for (int h = 0; h < HG; ++h) blk[h * 128 + st] = __uint_as_float(r[h]) * inv_l[h];
+                fence_proxy_async_smem();
+                sm_bar();
+                if (st == 0)
+                    bulk_s2g(a.ws_o + ((((int64_t)t * a.S + split) * 4 + dc) * a.H + (int64_t)g * HG) * 128, blk,
+                             HG * 128 * 4);
+            }
+            if (st == 0) bulk_commit_wait_read();
         }
-    } else if (warp >= 8) {
+        if (st == 0) TRACE(61);
+    } else {
         // ---------------------------------------------------- gather + unpack
+        regs_inc<160>();
         const int ut = tid - 256;
         const int sub = ut & 7;   // 8-dim slice of every 64-dim chunk
         const int rg = ut >> 3;   // rows rg, rg+32, rg+64, rg+96 of each tile
@@ -508,50 +522,61 @@ __global__ void __launch_bounds__(dec::kThreads, 1) sparse_mla_decode_kernel(con
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&bars[BAR_CHUNK_FULL + c]);
             }
+            if (ut == 0 && i < 8) TRACE(6 + 6 * i);
             if (ok && i + 1 < ntiles) load_tile(i + 1);
         }
+        if (ut == 0) TRACE(62);
         if (!ok && a.dev_status) atomicOr(a.dev_status, NVFP4MLA_DEV_TIMEOUT);
     }
 
     // ---------------------------------------------------------------- teardown
     tc_fence_before();
     __syncthreads();
-    if (warp == 0) {
+    if (warp == 3) {
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
     }
 }
 
 // Merge split partials: out = sum_s w_s o_s / sum_s w_s with
-// w_s = l_s 2^(m_s - max m), lse = (max m + log2 sum w) ln 2.
+// w_s = l_s 2^(m_s - max m), lse = (max m + log2 sum w) ln 2.  One block per
+// (token, head); every load is issued before any of them is used.
+template <int S>
 __global__ void __launch_bounds__(128) combine_splits_kernel(const float *__restrict__ ws_o,
-                                                             const float *__restrict__ ws_ml, int H, int S,
+                                                             const float *__restrict__ ws_ml, int H,
                                                              __half *__restrict__ out, float *__restrict__ lse) {
     const int th = blockIdx.x;  // t*H + h
     const int t = th / H, h = th % H;
-    float mmax = -INFINITY;
+    float m[S], l[S];
+    float4 o[S];
+#pragma unroll
     for (int s = 0; s < S; ++s) {
         const int64_t prow = ((int64_t)t * S + s) * H + h;
-        if (ws_ml[2 * prow + 1] > 0.0f) mmax = fmaxf(mmax, ws_ml[2 * prow]);
+        const float2 ml = *reinterpret_cast<const float2 *>(ws_ml + 2 * prow);
+        m[s] = ml.x;
+        l[s] = ml.y;
+        // partial rows are stored per 128-dv block: [t][s][dc][h][128]
+        const int dc = threadIdx.x >> 5, d = 4 * (threadIdx.x & 31);
+        o[s] = *reinterpret_cast<const float4 *>(ws_o + ((((int64_t)t * S + s) * 4 + dc) * H + h) * 128 + d);
     }
-    float L = 0.0f;
-    float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    float mmax = -INFINITY;
+#pragma unroll
+    for (int s = 0; s < S; ++s)
+        if (l[s] > 0.0f) mmax = fmaxf(mmax, m[s]);
+    float L = 0.0f, acc0 = 0.0f, acc1 = 0.0f, acc2 = 0.0f, acc3 = 0.0f;
+#pragma unroll
     for (int s = 0; s < S; ++s) {
-        const int64_t prow = ((int64_t)t * S + s) * H + h;
-        const float l = ws_ml[2 * prow + 1];
-        if (!(l > 0.0f)) continue;
-        const float w = l * ex2(ws_ml[2 * prow] - mmax);
+        const float w = l[s] > 0.0f ? l[s] * ex2(m[s] - mmax) : 0.0f;
         L += w;
-        const float4 o = *reinterpret_cast<const float4 *>(ws_o + prow * kLatent + 4 * threadIdx.x);
-        acc[0] += w * o.x;
-        acc[1] += w * o.y;
-        acc[2] += w * o.z;
-        acc[3] += w * o.w;
+        acc0 += w * o[s].x;
+        acc1 += w * o[s].y;
+        acc2 += w * o[s].z;
+        acc3 += w * o[s].w;
     }
     const float inv = L > 0.0f ? 1.0f / L : 0.0f;
     __half2 *dst = reinterpret_cast<__half2 *>(out + (int64_t)th * kLatent + 4 * threadIdx.x);
-    dst[0] = __floats2half2_rn(acc[0] * inv, acc[1] * inv);
-    dst[1] = __floats2half2_rn(acc[2] * inv, acc[3] * inv);
+    dst[0] = __floats2half2_rn(acc0 * inv, acc1 * inv);
+    dst[1] = __floats2half2_rn(acc2 * inv, acc3 * inv);
     if (threadIdx.x == 0) lse[th] = L > 0.0f ? (mmax + lg2(L)) * 0.69314718055994531f : -INFINITY;
 }
 
@@ -627,8 +652,14 @@ cudaError_t launch_sparse_mla_decode(bool staged, const void *q_nope, const void
         default: return cudaErrorInvalidValue;
     }
     if (e != cudaSuccess || plan.splits == 1) return e;
-    combine_splits_kernel<<<(unsigned)((int64_t)T * H), 128, 0, stream>>>(a.ws_o, a.ws_ml, H, plan.splits, a.out,
-                                                                          a.lse);
+    const unsigned cblocks = (unsigned)((int64_t)T * H);
+    switch (plan.splits) {
+        case 2: combine_splits_kernel<2><<<cblocks, 128, 0, stream>>>(a.ws_o, a.ws_ml, H, a.out, a.lse); break;
+        case 4: combine_splits_kernel<4><<<cblocks, 128, 0, stream>>>(a.ws_o, a.ws_ml, H, a.out, a.lse); break;
+        case 8: combine_splits_kernel<8><<<cblocks, 128, 0, stream>>>(a.ws_o, a.ws_ml, H, a.out, a.lse); break;
+        case 16: combine_splits_kernel<16><<<cblocks, 128, 0, stream>>>(a.ws_o, a.ws_ml, H, a.out, a.lse); break;
+        default: return cudaErrorInvalidValue;
+    }
     return cudaGetLastError();
 }
 

@@ -1,0 +1,106 @@
+// decode_common.cuh -- pieces shared by the decode kernels: launch
+// arguments, base-2 exp/log instructions, softmax-warp barriers, the in-warp
+// transpose reduction and debug-only tracing.
+#pragma once
+#include <cuda_runtime.h>
+
+#include <cmath>
+
+#include "common.cuh"
+#include "ptx.cuh"
+
+namespace nvfp4mla {
+
+struct DecodeArgs {
+    const __half *q_nope;
+    const __half *q_rope;
+    const uint8_t *src;
+    int64_t num_slots;
+    const int32_t *indices;
+    int topk, T, H, G, S;
+    float scale_log2;
+    __half *out;
+    float *lse;
+    float *ws_o;
+    float *ws_ml;
+    int32_t *dev_status;
+};
+
+#ifdef NVFP4MLA_TRACE
+// Debug builds only: per-CTA phase timestamps (clock64 deltas) for the
+// first 16 CTAs, 64 slots each.
+static __device__ unsigned long long *g_trace;
+#define TRACE(slot)                                                                  \
+    do {                                                                             \
+        if (g_trace && blockIdx.x < 16) g_trace[blockIdx.x * 64 + (slot)] = clock64() - t_start; \
+    } while (0)
+static inline void set_trace_local(unsigned long long *p) { cudaMemcpyToSymbol(g_trace, &p, sizeof(p)); }
+#else
+#define TRACE(slot) \
+    do {            \
+    } while (0)
+#endif
+
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+__device__ __forceinline__ float lg2(float x) {
+    float y;
+    asm("lg2.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+// Named barrier 1 over the 128 softmax threads, optionally OR-reducing a flag.
+__device__ __forceinline__ void sm_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+__device__ __forceinline__ bool sm_bar_or(bool p) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred pi, po;\n\tsetp.ne.u32 pi, %1, 0;\n\tbar.red.or.pred po, 1, 128, pi;\n\tselp.u32 %0, 1, 0, po;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)p)
+        : "memory");
+    return r != 0;
+}
+__device__ __forceinline__ uint32_t ldg32(const uint8_t *p) {
+    return __ldg(reinterpret_cast<const unsigned int *>(p));
+}
+__device__ __forceinline__ uint2 ldg64(const uint8_t *p) { return __ldg(reinterpret_cast<const uint2 *>(p)); }
+
+// In-warp transpose reduction: on entry each lane holds W column values; on
+// exit lane l holds op-reduced columns [l*W/32, (l+1)*W/32) in v[0..W/32)
+// (W == 16: column l/2 in v[0], duplicated in lane pairs).
+template <int W, bool kMax>
+__device__ __forceinline__ void warp_transpose_reduce(float (&v)[W], int lane) {
+#pragma unroll
+    for (int o = 16, w = W; o >= 1 && w >= 2; o >>= 1, w >>= 1) {
+        const bool upper = (lane & o) != 0;
+#pragma unroll
+        for (int j = 0; j < w / 2; ++j) {
+            const float keep = upper ? v[j + w / 2] : v[j];
+            const float send = upper ? v[j] : v[j + w / 2];
+            const float got = __shfl_xor_sync(0xffffffffu, send, o);
+            v[j] = kMax ? fmaxf(keep, got) : keep + got;
+        }
+    }
+    if (W == 16) {
+        const float got = __shfl_xor_sync(0xffffffffu, v[0], 1);
+        v[0] = kMax ? fmaxf(v[0], got) : v[0] + got;
+    }
+}
+template <int W>
+__device__ __forceinline__ int transposed_col(int lane, int j) {
+    return W >= 32 ? lane * (W / 32) + j : lane >> 1;
+}
+__host__ __device__ constexpr int cols_per_lane(int W) { return W >= 32 ? W / 32 : 1; }
+
+
+// N consecutive TMEM columns (32 lanes x 32 bit) in one instruction.
+template <int N>
+__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&r)[N]) {
+    if constexpr (N == 64) ptx::tmem_ld64(taddr, r);
+    else if constexpr (N == 32) ptx::tmem_ld32(taddr, r);
+    else ptx::tmem_ld16(taddr, r);
+}
+
+}  // namespace nvfp4mla
