@@ -93,23 +93,29 @@ nvfp4mla_status nvfp4_kv_append(const void *latent_bf16, int64_t latent_stride, 
 
 /*
  * nvfp4_sparse_mla_num_splits -- how many CTAs the decode splits each
- * token's index list across (chosen from T and H to fill the 148 SMs; the
- * pages size SM clusters from the token batch size, same section).  Pure
- * host function; returns 0 for unsupported shapes.
+ * token's index list across: the largest power of two S <= 16 (and <= the
+ * number of 128-row tiles of topk) with T * (H / min(H, 64)) * S no larger
+ * than the SM count of the current device (148 when no device can be
+ * queried).  The pages size their SM clusters from the token batch in the
+ * same spirit (same section).  Host-only; returns 0 for unsupported shapes.
  */
 int32_t nvfp4_sparse_mla_num_splits(int32_t T, int32_t H, int32_t topk);
 
 /*
  * nvfp4_sparse_mla_workspace_size -- bytes of device workspace
- * nvfp4_sparse_mla_decode needs for (T, H, topk): FP32 partial outputs and
- * softmax statistics of the splits.  0 means no workspace is needed.
+ * nvfp4_sparse_mla_decode needs for (T, H, topk) on the current device:
+ * 0 when the lists are not split (S == 1), else 4096 bytes of split
+ * counters followed by the softmax statistics and FP32 partial outputs of
+ * the S splits.  Layout: [0, 4096) uint32 counter pairs, then [T][S][H][2]
+ * FP32 (max, row sum), then [T][S][H][512] FP32.
  */
 size_t nvfp4_sparse_mla_workspace_size(int32_t T, int32_t H, int32_t topk);
 
 /*
  * nvfp4_sparse_mla_decode -- sparse MLA decode over the NVFP4 cache (same
- * page and section: load only the indexer-selected rows, unpack on chip,
- * FP16 operands, FP32 accumulation, zero-filled empty entries).
+ * page and section: only the rows the indexer selected are read, they are
+ * unpacked on chip to FP16 MMA operands with FP32 accumulation, and list
+ * entries that name no row contribute nothing).
  *
  *   q_nope_f16  [T, H, 512] FP16, contiguous, 16-byte aligned
  *   q_rope_f16  [T, H, 64]  FP16, contiguous, 16-byte aligned
@@ -124,7 +130,15 @@ size_t nvfp4_sparse_mla_workspace_size(int32_t T, int32_t H, int32_t topk);
  *   lse         [T, H] FP32 natural-log sum-exp of the scaled scores;
  *               all-empty -> -inf
  *   workspace   device buffer of at least nvfp4_sparse_mla_workspace_size
- *               bytes (may be NULL when that size is 0), 256-byte aligned
+ *               bytes (may be NULL when that size is 0), 256-byte aligned,
+ *               owned by the caller.  Its first 4096 bytes (the split
+ *               counters) must be zero before the first call that uses it
+ *               (e.g. allocate it zero-filled); every call that completes
+ *               leaves them zero again, for any shape.  After a call that
+ *               raised NVFP4MLA_DEV_TIMEOUT they must be cleared again.
+ *               When S > 1 the launch is cooperative: it fails with
+ *               NVFP4MLA_ERR_CUDA if the device cannot hold all
+ *               T * (H / min(H, 64)) * S CTAs at once.
  * Supported: 1 <= topk <= 2048; H in {16, 32, 64, 128}; T >= 0 (T == 0
  * is a no-op); num_slots >= 1.  Results are undefined for NaN/Inf queries.
  */

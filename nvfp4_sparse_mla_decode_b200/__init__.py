@@ -152,11 +152,14 @@ def decode(q_nope: torch.Tensor, q_rope: torch.Tensor, cache: torch.Tensor, indi
            sm_scale: float, out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
            workspace: Optional[torch.Tensor] = None, dev_status: Optional[torch.Tensor] = None,
            num_slots: Optional[int] = None):
-    """Sparse MLA decode over the NVFP4 cache; returns (out [T,H,512] f16, lse [T,H] f32)."""
+    """Sparse MLA decode over the NVFP4 cache; returns (out [T,H,512] f16, lse [T,H] f32).
+
+    A caller-supplied `workspace` must start zero-filled (its first 4096
+    bytes hold split counters that every completed call leaves at zero)."""
     dev, T, H, topk, out, lse = _decode_args(q_nope, q_rope, cache, indices, out, lse)
     ws_need = workspace_size(T, H, topk)
     if workspace is None and ws_need:
-        workspace = torch.empty(ws_need, dtype=torch.uint8, device=dev)
+        workspace = torch.zeros(ws_need, dtype=torch.uint8, device=dev)
     st = lib().nvfp4_sparse_mla_decode(_ptr(q_nope), _ptr(q_rope), _ptr(cache),
                                        num_slots if num_slots is not None else cache.shape[0], _ptr(indices),
                                        topk, T, H, float(sm_scale), _ptr(out), _ptr(lse), _ptr(workspace),
@@ -176,7 +179,7 @@ def staged_decode(q_nope: torch.Tensor, q_rope: torch.Tensor, cache: torch.Tenso
         staging = torch.empty(max(1, staging_size(T, topk)), dtype=torch.uint8, device=dev)
     ws_need = workspace_size(T, H, topk)
     if workspace is None and ws_need:
-        workspace = torch.empty(ws_need, dtype=torch.uint8, device=dev)
+        workspace = torch.zeros(ws_need, dtype=torch.uint8, device=dev)
     st = lib().nvfp4_staged_fp8_mla_decode(_ptr(q_nope), _ptr(q_rope), _ptr(cache), cache.shape[0], _ptr(indices),
                                            topk, T, H, float(sm_scale), _ptr(out), _ptr(lse), _ptr(staging),
                                            staging.numel(), _ptr(workspace),

@@ -22,7 +22,7 @@ nvfp4mla_status check_decode(const void *q_nope, const void *q_rope, const uint8
     if (T < 0 || topk < 1 || topk > NVFP4MLA_MAX_TOPK || num_slots < 1 || num_slots > INT32_MAX)
         return NVFP4MLA_ERR_INVALID_ARG;
     if (!(sm_scale == sm_scale) || sm_scale > 3.0e38f || sm_scale < -3.0e38f) return NVFP4MLA_ERR_INVALID_ARG;
-    if (!make_decode_plan(T, H, topk, plan)) return NVFP4MLA_ERR_UNSUPPORTED;
+    if (!make_decode_plan(T, H, topk, current_device_sm_count(), plan)) return NVFP4MLA_ERR_UNSUPPORTED;
     if (T == 0) return NVFP4MLA_OK;
     if (!q_nope || !q_rope || !cache || !indices || !out || !lse) return NVFP4MLA_ERR_INVALID_ARG;
     if (!aligned(q_nope, 16) || !aligned(q_rope, 16) || !aligned(cache, 16) || !aligned(indices, 16) ||
@@ -51,12 +51,12 @@ nvfp4mla_status nvfp4_kv_append(const void *latent_bf16, int64_t latent_stride, 
 
 int32_t nvfp4_sparse_mla_num_splits(int32_t T, int32_t H, int32_t topk) {
     DecodePlan p;
-    return make_decode_plan(T, H, topk, &p) ? p.splits : 0;
+    return make_decode_plan(T, H, topk, current_device_sm_count(), &p) ? p.splits : 0;
 }
 
 size_t nvfp4_sparse_mla_workspace_size(int32_t T, int32_t H, int32_t topk) {
     DecodePlan p;
-    return make_decode_plan(T, H, topk, &p) ? p.workspace_bytes : 0;
+    return make_decode_plan(T, H, topk, current_device_sm_count(), &p) ? p.workspace_bytes : 0;
 }
 
 nvfp4mla_status nvfp4_sparse_mla_decode(const void *q_nope_f16, const void *q_rope_f16, const uint8_t *cache,

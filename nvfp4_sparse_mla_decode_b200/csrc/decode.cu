@@ -71,7 +71,29 @@ constexpr int kOffMisc = kOffBar + kNumBars * 8;
 constexpr int kSmemBytes = kOffMisc + 64;
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 static_assert(kMaxHG * kLatent * 4 <= kTileBytes, "FP32 output staging must fit in the tile region");
-constexpr int kThreads = 512;
+constexpr int kThreads = 640;
+// warps 0-3: MMA issue (warp 0) + TMEM allocation (warp 3); warps 4-11: two
+// softmax warpgroups (half of the heads each); warps 12-19: gather + unpack.
+constexpr int kSoftmaxWarp0 = 4;
+constexpr int kUnpackWarp0 = 12;
+// Per-thread register budgets per role (setmaxnreg).  At launch every thread
+// holds kRegsLaunch registers (65536 / 640 rounded down to a multiple of 8);
+// a role may only decrease below it with .dec and increase above it with .inc,
+// and the new total must fit in what the block was launched with.  The split
+// depends on the instantiation: 64 heads per CTA keep 32 per-head values per
+// softmax thread, and the staged source keeps 18 raw words per row in the
+// unpack warps instead of 11 (chosen so ptxas reports no spills, or the
+// fewest).
+constexpr int kRegsLaunch = 96;
+template <int HG, bool kStaged>
+struct RegSplit {
+    static constexpr int mma = 40;                                         // warpgroup 0 (.dec)
+    static constexpr int softmax = HG == 64 ? (kStaged ? 136 : 144) : 128;  // warpgroups 1-2 (.inc)
+    static constexpr int unpack = HG == 64 ? (kStaged ? 80 : 72) : 88;      // warpgroups 3-4 (.dec)
+    static_assert(mma < kRegsLaunch && unpack < kRegsLaunch && softmax > kRegsLaunch, "setmaxnreg direction");
+    static_assert(mma % 8 == 0 && softmax % 8 == 0 && unpack % 8 == 0, "setmaxnreg granularity");
+    static_assert(128 * mma + 256 * softmax + 256 * unpack <= 640 * kRegsLaunch, "register budget");
+};
 
 constexpr int BAR_CHUNK_FULL = 0;  // [9] unpack -> MMA, count 8 warps
 constexpr int BAR_CHUNK_FREE = 9;  // [4] output MMAs of a 128-dv block done
@@ -83,7 +105,111 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColO = 0;      // O^T: 4 blocks of HG columns
 constexpr uint32_t kColS = 256;    // S^T: HG columns
 constexpr float kRescaleThreshold = 8.0f;
+constexpr int kMaxSplits = 16;
+static_assert((kMaxSplits + 1) * kMaxHG * 4 <= kTileBytes, "merge weights must fit in the tile region");
 }  // namespace dec
+
+// Merge of the S split partials of one (token, head group), run by the 256
+// softmax threads of each of the S CTAs of the group once their own partial
+// is written: each CTA announces its partial on the group's arrival
+// counter, waits (bounded) until all S have, then combines the dv slice
+// [split*512/S, (split+1)*512/S) of every head:
+//   out = sum_s w_s O_s / sum_s w_s l_s,  w_s = 2^(m_s - max m)
+// over the splits with rows (l_s > 0); split 0 also writes
+// lse = (max m + log2 of the denominator) ln 2.  The launch is cooperative,
+// so all S CTAs are resident together and the wait ends.  The last CTA to
+// leave resets both counters, which lets the next call start from zero.
+// Loads of up to 16 partial vectors are issued before any is used.
+template <int HG, int S>
+__device__ __forceinline__ void merge_splits(const DecodeArgs &a, int t, int g, int split, uint8_t *smem, int mt) {
+    using namespace dec;
+    constexpr int kMergeThreads = 256;
+    constexpr int D = kLatent / S;        // dv per CTA
+    constexpr int NQ = D / 4;             // float4 per head
+    constexpr int ITEMS = HG * NQ;
+    constexpr int B = S >= 16 ? 1 : 16 / S;  // items per batch: B * S loads in flight
+    uint32_t *arrive = a.counters + 2 * ((int64_t)t * a.G + g);
+    uint32_t *depart = arrive + 1;
+    uint32_t *flag = reinterpret_cast<uint32_t *>(smem + kOffMisc) + 1;
+    float *w_s = reinterpret_cast<float *>(smem);  // [S][HG] weights (free tile region)
+    float *inv_den = w_s + kMaxSplits * HG;         // [HG]
+    named_bar(3, kMergeThreads);                    // every partial store of this CTA is fenced
+    if (mt == 0) {
+        red_release_gpu_add(arrive, 1u);
+        const bool ok = spin_until_geq(arrive, (uint32_t)S);
+        if (!ok && a.dev_status) atomicOr(a.dev_status, NVFP4MLA_DEV_TIMEOUT);
+        *flag = ok ? 1u : 0u;
+    }
+    named_bar(3, kMergeThreads);
+    if (!*flag) return;  // counters stay raised: the caller must clear them after a timeout
+    if (mt < HG) {
+        const float *ml = a.ws_ml + 2 * ((int64_t)t * S * a.H + (int64_t)g * HG + mt);
+        float2 v[S];
+#pragma unroll
+        for (int s = 0; s < S; ++s) v[s] = __ldcg(reinterpret_cast<const float2 *>(ml + 2 * (int64_t)s * a.H));
+        float mmax = -INFINITY;
+#pragma unroll
+        for (int s = 0; s < S; ++s)
+            if (v[s].y > 0.0f) mmax = fmaxf(mmax, v[s].x);
+        float den = 0.0f;
+#pragma unroll
+        for (int s = 0; s < S; ++s) {
+            const float w = v[s].y > 0.0f ? ex2(v[s].x - mmax) : 0.0f;
+            w_s[s * HG + mt] = w;
+            den += w * v[s].y;
+        }
+        inv_den[mt] = den > 0.0f ? 1.0f / den : 0.0f;
+        if (split == 0)
+            a.lse[(int64_t)t * a.H + (int64_t)g * HG + mt] =
+                den > 0.0f ? (mmax + lg2(den)) * 0.69314718055994531f : -INFINITY;
+    }
+    named_bar(3, kMergeThreads);
+    const int dv0 = split * D;
+    const int64_t part = (int64_t)a.H * kLatent;  // next split of the same (t, head)
+    const float *src = a.ws_o + ((int64_t)t * S * a.H + (int64_t)g * HG) * kLatent + dv0;
+    __half *dst = a.out + ((int64_t)t * a.H + (int64_t)g * HG) * kLatent + dv0;
+    for (int base = mt; base < ITEMS; base += kMergeThreads * B) {
+        float4 o[B][S];
+#pragma unroll
+        for (int b = 0; b < B; ++b) {
+            const int item = base + b * kMergeThreads;
+            const int h = item / NQ, q = item - h * NQ;
+#pragma unroll
+            for (int s = 0; s < S; ++s)
+                o[b][s] = item < ITEMS
+                              ? __ldcg(reinterpret_cast<const float4 *>(src + (int64_t)h * kLatent + 4 * q + s * part))
+                              : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+        }
+#pragma unroll
+        for (int b = 0; b < B; ++b) {
+            const int item = base + b * kMergeThreads;
+            if (item < ITEMS) {
+                const int h = item / NQ, q = item - h * NQ;
+                float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+#pragma unroll
+                for (int s = 0; s < S; ++s) {  // an empty split's partial is zero and its weight 0
+                    const float w = w_s[s * HG + h];
+                    acc.x += w * o[b][s].x;
+                    acc.y += w * o[b][s].y;
+                    acc.z += w * o[b][s].z;
+                    acc.w += w * o[b][s].w;
+                }
+                const float r = inv_den[h];
+                __half2 *d2 = reinterpret_cast<__half2 *>(dst + (int64_t)h * kLatent + 4 * q);
+                d2[0] = __floats2half2_rn(acc.x * r, acc.y * r);
+                d2[1] = __floats2half2_rn(acc.z * r, acc.w * r);
+            }
+        }
+    }
+    named_bar(3, kMergeThreads);
+    if (mt == 0) {
+        const uint32_t old = atomicAdd(depart, 1u);
+        if (old == (uint32_t)S - 1u) {  // every CTA of the group is past its wait
+            atomicExch(arrive, 0u);
+            atomicExch(depart, 0u);
+        }
+    }
+}
 
 template <int HG, bool kStaged>
 __global__ void __launch_bounds__(dec::kThreads, 1) sparse_mla_decode_kernel(const DecodeArgs a) {
@@ -115,7 +241,7 @@ __global__ void __launch_bounds__(dec::kThreads, 1) sparse_mla_decode_kernel(con
         uint32_t count = 0;
         if (lane < BAR_CHUNK_FREE) count = 8;           // chunk written by the 8 unpack warps
         else if (lane < BAR_P_FULL) count = 1;          // MMA commits
-        else if (lane == BAR_P_FULL) count = 4;         // 4 softmax warps
+        else if (lane == BAR_P_FULL) count = 8;         // 8 softmax warps
         else if (lane == BAR_DRAIN) count = 1;
         if (count) mbar_init(&bars[lane], count);
         fence_mbar_init();
@@ -123,23 +249,9 @@ __global__ void __launch_bounds__(dec::kThreads, 1) sparse_mla_decode_kernel(con
     if (warp == 3) {  // a warp with no setup work: the allocation can take a while
         tmem_alloc(&misc[0], kTmemCols);
         tmem_relinquish();
+        if (lane == 0) TRACE(260);
     }
     if (tid < HG) m_s[tid] = -INFINITY;
-
-    // Q of (t, heads g*HG ..) -> shared memory, K-major, 128-byte swizzle:
-    // chunk c holds dims 64c..64c+63 of every head (chunk 8 = RoPE).
-    // Issued as 16-byte async copies so every load of the CTA is in flight
-    // at once; they complete before the setup barrier below.
-    if (warp >= 8) {
-        const int ut = tid - 256;
-        const int64_t head0 = (int64_t)t * a.H + (int64_t)g * HG;
-        for (int u = ut; u < HG * 72; u += 256) {
-            const int h = u / 72, v = u % 72;
-            const void *src = v < 64 ? static_cast<const void *>(a.q_nope + (head0 + h) * kLatent + 8 * v)
-                                     : static_cast<const void *>(a.q_rope + (head0 + h) * kRope + 8 * (v - 64));
-            cp_async16(smem + kOffQ + (v >> 3) * (HG * 128) + sw128_offset(h, v & 7), src);
-        }
-    }
 
     // Compact the token's list: keep valid entries in list order; this CTA
     // keeps entries [lo, hi) of the compacted order.
@@ -149,21 +261,40 @@ __global__ void __launch_bounds__(dec::kThreads, 1) sparse_mla_decode_kernel(con
     bool bad = false;
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
-        const int p = tid + 512 * k;
-        const int32_t v = p < a.topk ? __ldg(lst + p) : -1;
+        const int p = tid + 512 * k;  // warps 16.. have no list entries (p >= 2048)
+        const int32_t v = (p < a.topk && tid < 512) ? __ldg(lst + p) : -1;
         const bool ok = v >= 0 && (int64_t)v < a.num_slots;
         bad |= (p < a.topk) && (v < -1 || (int64_t)v >= a.num_slots);
         vals[k] = v;
         bal[k] = __ballot_sync(0xffffffffu, ok);
-        if (lane == 0) cnt_s[k * 16 + warp] = __popc(bal[k]);
+        if (lane == 0 && warp < 16) cnt_s[k * 16 + warp] = __popc(bal[k]);
     }
     if (__any_sync(0xffffffffu, bad) && lane == 0 && split == 0 && g == 0 && a.dev_status)
         atomicOr(a.dev_status, NVFP4MLA_DEV_BAD_INDEX);
+    if (tid == 0) TRACE(261);
     __syncthreads();
-    // exclusive prefix of the 64 per-(round, warp) counts: warp 0 scans them
-    // (2 per lane), everyone reads its 4 offsets and the total back
-    uint32_t *pre_s = cnt_s + 64;
-    if (warp == 0) {
+    if (tid == 0) TRACE(262);
+    // Q of (t, heads g*HG ..) -> shared memory, K-major, 128-byte swizzle:
+    // chunk c holds dims 64c..64c+63 of every head (chunk 8 = RoPE).  Issued
+    // as 16-byte async copies after the list loads (so they do not queue
+    // ahead of them); each unpack thread waits for its own copies before its
+    // first chunk arrival, which orders them before the first score MMAs.
+    if (warp >= kUnpackWarp0) {
+        const int ut = tid - 32 * kUnpackWarp0;
+        const int64_t head0 = (int64_t)t * a.H + (int64_t)g * HG;
+        for (int u = ut; u < HG * 72; u += 256) {
+            const int h = u / 72, v = u % 72;
+            const void *src = v < 64 ? static_cast<const void *>(a.q_nope + (head0 + h) * kLatent + 8 * v)
+                                     : static_cast<const void *>(a.q_rope + (head0 + h) * kRope + 8 * (v - 64));
+            cp_async16(smem + kOffQ + (v >> 3) * (HG * 128) + sw128_offset(h, v & 7), src);
+        }
+    }
+    // Exclusive prefix of the 64 per-(round, warp) counts.  Every warp scans
+    // them itself (two per lane) and reads its own offsets from the lane that
+    // holds them, so no second block barrier is needed.
+    int before[4];
+    int n_valid;
+    {
         const uint32_t c0 = cnt_s[2 * lane], c1 = cnt_s[2 * lane + 1];
         uint32_t incl = c0 + c1;
 #pragma unroll
@@ -172,15 +303,15 @@ __global__ void __launch_bounds__(dec::kThreads, 1) sparse_mla_decode_kernel(con
             if (lane >= o) incl += y;
         }
         const uint32_t excl = incl - c0 - c1;
-        pre_s[2 * lane] = excl;
-        pre_s[2 * lane + 1] = excl + c0;
-        if (lane == 31) pre_s[64] = incl;
-    }
-    __syncthreads();
-    int before[4];
+        n_valid = (int)__shfl_sync(0xffffffffu, incl, 31);
 #pragma unroll
-    for (int k = 0; k < 4; ++k) before[k] = (int)pre_s[k * 16 + warp];
-    const int n_valid = (int)pre_s[64];
+        for (int k = 0; k < 4; ++k) {
+            const int j = k * 16 + (warp & 15);  // count index of (round k, this warp)
+            const uint32_t mine = (j & 1) ? excl + c0 : excl;
+            const uint32_t b = __shfl_sync(0xffffffffu, mine, j >> 1);
+            before[k] = warp < 16 ? (int)b : 0;
+        }
+    }
     const int per = (n_valid + a.S - 1) / a.S;
     const int lo = split * per;
     const int hi = min(n_valid, lo + per);
@@ -188,14 +319,10 @@ __global__ void __launch_bounds__(dec::kThreads, 1) sparse_mla_decode_kernel(con
     const int ntiles = (n_mine + kTileRows - 1) / kTileRows;
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
-        if ((bal[k] >> lane) & 1u) {
+        if (warp < 16 && ((bal[k] >> lane) & 1u)) {
             const int pos = before[k] + __popc(bal[k] & ((1u << lane) - 1u));
             if (pos >= lo && pos < hi) idx_s[pos - lo] = kStaged ? (tid + 512 * k) : vals[k];
         }
-    }
-    if (warp >= 8) {
-        cp_async_wait_all();
-        fence_proxy_async_smem();
     }
     tc_fence_before();
     __syncthreads();
@@ -203,12 +330,12 @@ __global__ void __launch_bounds__(dec::kThreads, 1) sparse_mla_decode_kernel(con
     const uint32_t tmem = misc[0];
     if (tid == 0) TRACE(0);
 
-    // Register budget (launched with 128 x 512): the MMA/idle warpgroup gives
-    // registers to the softmax and unpack warps, 128 x 48 + 128 x 144 +
-    // 256 x 160 = 65536.  Each role changes its budget inside its own branch
-    // so the compiler sizes each role's code separately.
+    // Register budget (launched with 96 x 640 = 61440): the MMA/idle
+    // warpgroup and the unpack warps give registers to the softmax warps
+    // (see RegSplit).  Each role changes its budget inside its own branch so
+    // the compiler sizes each role's code separately.
     if (warp < 4) {
-        regs_dec<48>();
+        regs_dec<RegSplit<HG, kStaged>::mma>();
         // ------------------------------------------------------------- MMA
         if (warp == 0 && lane == 0) {
             const uint32_t idesc_qk = idesc_f16_f32(128, HG, false, false);
@@ -230,6 +357,7 @@ __global__ void __launch_bounds__(dec::kThreads, 1) sparse_mla_decode_kernel(con
                         ok = false;
                         break;
                     }
+                    if (i == 1) TRACE(64 + c);
                     tc_fence_after();
                     mma_ss(tmem + kColS, dk, dq, idesc_qk, c != 0);
                     mma_ss(tmem + kColS, dk + 2, dq + 2, idesc_qk, 1u);
@@ -255,6 +383,7 @@ __global__ void __launch_bounds__(dec::kThreads, 1) sparse_mla_decode_kernel(con
                         mma_ss(tmem + kColO + dc * HG, dv + (uint64_t)(kk * 128), dP0 + (uint64_t)(kk * 128),
                                idesc_pv, (i > 0 || kk > 0) ? 1u : 0u);
                     mma_commit(&bars[BAR_CHUNK_FREE + dc]);
+                    if (i == 0) TRACE(112 + dc);
                     dv += (uint64_t)((2 * kChunkBytes) >> 4);
                 }
                 if (i < 8) TRACE(3 + 6 * i);
@@ -265,20 +394,27 @@ __global__ void __launch_bounds__(dec::kThreads, 1) sparse_mla_decode_kernel(con
             TRACE(60);
         }
         __syncwarp();
-    } else if (warp < 8) {
+    } else if (warp < kUnpackWarp0) {
         // --------------------------------------------------------- softmax
-        regs_inc<144>();
-        // Heads are processed in halves of HW = min(HG, 32): the reference
-        // max, rescale and row sums of a head never depend on other heads.
-        constexpr int HW = HG < 32 ? HG : 32;
-        constexpr int NH = HG / HW;
-        const int st = tid - 128;  // tile row == TMEM lane
+        regs_inc<RegSplit<HG, kStaged>::softmax>();
+        // Two warpgroups; warpgroup sw owns heads [h0, h0 + HWG).  A head's
+        // reference max, rescale and row sum never depend on other heads, so
+        // the groups only meet at the P^T barrier and the epilogue.  With
+        // HG = 16 the second group has no heads and only keeps the barrier
+        // count.
+        constexpr int NSW = HG >= 32 ? 2 : 1;
+        constexpr int HWG = HG / NSW;
+        const int sw = (warp - kSoftmaxWarp0) >> 2;
+        const int st = tid - 32 * kSoftmaxWarp0 - 128 * sw;  // tile row == TMEM lane
         const int wq = st >> 5;
+        const uint32_t bar_id = 1 + sw;
         const uint32_t lane_base = (uint32_t)(32 * wq) << 16;
         uint8_t *p_tile = smem + 8 * kChunkBytes;  // P^T overwrites the RoPE chunk
-        float lp[NH];  // warp-partial row sums, column h0 + transposed_col<HW>(lane)
+        const int h0 = sw * HWG;
+        const bool active = sw < NSW;
+        float lp[HWG];  // this thread's (row slot's) running sum per head
 #pragma unroll
-        for (int j = 0; j < NH; ++j) lp[j] = 0.0f;
+        for (int j = 0; j < HWG; ++j) lp[j] = 0.0f;
         bool ok = true;
         for (int i = 0; i < ntiles; ++i) {
             // S_FULL(i) also covers PV(i-1): the MMA thread issued it earlier,
@@ -288,33 +424,34 @@ __global__ void __launch_bounds__(dec::kThreads, 1) sparse_mla_decode_kernel(con
                 break;
             }
             tc_fence_after();
-            if (st == 0 && i < 8) TRACE(4 + 6 * i);
-            uint32_t rs[HG];
-            tmem_ld_cols<HG>(tmem + lane_base + kColS, rs);
-            tmem_ld_wait();
-            const int nrows = min(kTileRows, n_mine - kTileRows * i);
-            const bool valid = st < nrows;
+            if (st == 0 && sw == 0 && i < 8) TRACE(4 + 6 * i);
+            if (active) {
+                float sv[HWG];
+                {
+                    uint32_t rs[HWG];
+                    tmem_ld_cols<HWG>(tmem + lane_base + kColS + h0, rs);
+                    tmem_ld_wait();
 #pragma unroll
-            for (int hh = 0; hh < NH; ++hh) {
-                const int h0 = hh * HW;
-                float sv[HW];
-#pragma unroll
-                for (int h = 0; h < HW; ++h) sv[h] = __uint_as_float(rs[h0 + h]) * a.scale_log2;
+                    for (int h = 0; h < HWG; ++h) sv[h] = __uint_as_float(rs[h]) * a.scale_log2;
+                }
+                const int nrows = min(kTileRows, n_mine - kTileRows * i);
+                const bool valid = st < nrows;
                 bool need = false;
                 if (valid) {
 #pragma unroll
-                    for (int h = 0; h < HW; ++h) need |= sv[h] > m_s[h0 + h] + kRescaleThreshold;
+                    for (int h = 0; h < HWG; ++h) need |= sv[h] > m_s[h0 + h] + kRescaleThreshold;
                 }
-                if (sm_bar_or(need)) {
-                    {
-                        float mx[HW];
+                if (named_bar_or(bar_id, 128, need)) {
 #pragma unroll
-                        for (int h = 0; h < HW; ++h) mx[h] = valid ? sv[h] : -INFINITY;
-                        warp_transpose_reduce<HW, true>(mx, lane);
-                        red_s[wq * 64 + h0 + transposed_col<HW>(lane, 0)] = mx[0];
+                    for (int c0 = 0; c0 < HWG; c0 += 16) {  // column max, 16 heads at a time
+                        float mx[16];
+#pragma unroll
+                        for (int h = 0; h < 16; ++h) mx[h] = valid ? sv[c0 + h] : -INFINITY;
+                        warp_transpose_reduce<16, true>(mx, lane);
+                        if (!(lane & 1)) red_s[wq * 64 + h0 + c0 + transposed_col<16>(lane, 0)] = mx[0];
                     }
-                    sm_bar();
-                    if (st < HW) {
+                    named_bar(bar_id, 128);
+                    if (st < HWG) {
                         const int h = h0 + st;
                         const float old = m_s[h];
                         float nm = old;
@@ -323,32 +460,34 @@ __global__ void __launch_bounds__(dec::kThreads, 1) sparse_mla_decode_kernel(con
                         aux_s[h] = (old == -INFINITY) ? 0.0f : ex2(old - nm);
                         m_s[h] = nm;
                     }
-                    sm_bar();
-                    lp[hh] *= aux_s[h0 + transposed_col<HW>(lane, 0)];
+                    named_bar(bar_id, 128);
+#pragma unroll
+                    for (int h = 0; h < HWG; ++h) lp[h] *= aux_s[h0 + h];
                     if (i > 0) {
 #pragma unroll 1
                         for (int dc = 0; dc < 4; ++dc) {
-                            uint32_t r[HW];
-                            const uint32_t addr = tmem + lane_base + kColO + dc * HG + h0;
-                            tmem_ld_cols<HW>(addr, r);
-                            tmem_ld_wait();
 #pragma unroll
-                            for (int h = 0; h < HW; ++h) r[h] = __float_as_uint(__uint_as_float(r[h]) * aux_s[h0 + h]);
+                            for (int cb = 0; cb < HWG; cb += 16) {  // 16 columns per round trip
+                                uint32_t r[16];
+                                const uint32_t addr = tmem + lane_base + kColO + dc * HG + h0 + cb;
+                                tmem_ld16(addr, r);
+                                tmem_ld_wait();
 #pragma unroll
-                            for (int cb = 0; cb < HW; cb += 16) {
-                                uint32_t q[16];
-#pragma unroll
-                                for (int j = 0; j < 16; ++j) q[j] = r[cb + j];
-                                tmem_st16(addr + cb, q);
+                                for (int h = 0; h < 16; ++h)
+                                    r[h] = __float_as_uint(__uint_as_float(r[h]) * aux_s[h0 + cb + h]);
+                                tmem_st16(addr, r);
                             }
                         }
                         tmem_st_wait();
                     }
                 }
 #pragma unroll
-                for (int h = 0; h < HW; ++h) sv[h] = valid ? ex2(sv[h] - m_s[h0 + h]) : 0.0f;
+                for (int h = 0; h < HWG; ++h) {
+                    sv[h] = valid ? ex2(sv[h] - m_s[h0 + h]) : 0.0f;
+                    lp[h] += sv[h];
+                }
 #pragma unroll
-                for (int j = 0; j < HW / 8; ++j) {
+                for (int j = 0; j < HWG / 8; ++j) {
                     uint4 pk;
                     pk.x = pack_half2(sv[8 * j + 0], sv[8 * j + 1]);
                     pk.y = pack_half2(sv[8 * j + 2], sv[8 * j + 3]);
@@ -356,14 +495,12 @@ __global__ void __launch_bounds__(dec::kThreads, 1) sparse_mla_decode_kernel(con
                     pk.w = pack_half2(sv[8 * j + 6], sv[8 * j + 7]);
                     *reinterpret_cast<uint4 *>(p_tile + sw128_offset(st, h0 / 8 + j)) = pk;
                 }
-                warp_transpose_reduce<HW, false>(sv, lane);
-                lp[hh] += sv[0];
+                fence_proxy_async_smem();
+                tc_fence_before();
             }
-            fence_proxy_async_smem();
-            tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars[BAR_P_FULL]);
-            if (st == 0 && i < 8) TRACE(5 + 6 * i);
+            if (st == 0 && sw == 0 && i < 8) TRACE(5 + 6 * i);
         }
         if (!ok && a.dev_status) atomicOr(a.dev_status, NVFP4MLA_DEV_TIMEOUT);
         // ---------------------------------------------------------- epilogue
@@ -374,91 +511,115 @@ __global__ void __launch_bounds__(dec::kThreads, 1) sparse_mla_decode_kernel(con
             }
             tc_fence_after();
         }
+        if (st == 0 && sw == 0) TRACE(270);
         const bool have = ok && ntiles > 0;
-        if (!(HW < 32 && (lane & 1))) {
+        if (active) {
+            // row sums: reduce each head's 128 per-row partials (16 heads at a time)
 #pragma unroll
-            for (int hh = 0; hh < NH; ++hh) red_s[wq * 64 + hh * HW + transposed_col<HW>(lane, 0)] = lp[hh];
-        }
-        sm_bar();
-        if (st < HG) {
-            const float l = have ? red_s[st] + red_s[64 + st] + red_s[128 + st] + red_s[192 + st] : 0.0f;
-            const float m = m_s[st];
-            aux_s[st] = l > 0.0f ? 1.0f / l : 0.0f;
-            const int64_t hrow = (int64_t)t * a.H + (int64_t)g * HG + st;
-            if (a.S == 1) {
-                a.lse[hrow] = l > 0.0f ? (m + lg2(l)) * 0.69314718055994531f : -INFINITY;
-            } else {
-                const int64_t prow = ((int64_t)t * a.S + split) * a.H + (int64_t)g * HG + st;
-                a.ws_ml[2 * prow] = l > 0.0f ? m : -INFINITY;
-                a.ws_ml[2 * prow + 1] = l;
+            for (int c0 = 0; c0 < HWG; c0 += 16) {
+                float v[16];
+#pragma unroll
+                for (int h = 0; h < 16; ++h) v[h] = lp[c0 + h];
+                warp_transpose_reduce<16, false>(v, lane);
+                if (!(lane & 1)) red_s[wq * 64 + h0 + c0 + transposed_col<16>(lane, 0)] = v[0];
             }
-        }
-        sm_bar();
-        // O^T (TMEM, lanes = dv) -> normalized rows staged in the (now free)
-        // tile region, then bulk copies to global memory.
-        //  one split:   out[t, g*HG + h, :] (FP16), one copy of HG x 1 KB;
-        //  split parts: ws_o[t, split, dc, g*HG + h, 0:128] (FP32, dv block
-        //               major), one 32 KB copy per 128-dv block, issued as soon
-        //               as the block is staged.
-        float inv_l[HG];
-#pragma unroll
-        for (int h = 0; h < HG; ++h) inv_l[h] = aux_s[h];
-        uint8_t *stage = smem;
-        if (a.S == 1) {
-#pragma unroll 1
-            for (int dc = 0; dc < 4; ++dc) {
-                const int dv = 128 * dc + st;
-                uint32_t r[HG];
-                if (have) {
-                    tmem_ld_cols<HG>(tmem + lane_base + kColO + dc * HG, r);
-                    tmem_ld_wait();
+            named_bar(bar_id, 128);
+            if (st < HWG) {
+                const int h = h0 + st;
+                const float l = have ? red_s[h] + red_s[64 + h] + red_s[128 + h] + red_s[192 + h] : 0.0f;
+                const float m = m_s[h];
+                aux_s[h] = l > 0.0f ? 1.0f / l : 0.0f;
+                const int64_t hrow = (int64_t)t * a.H + (int64_t)g * HG + h;
+                if (a.S == 1) {
+                    a.lse[hrow] = l > 0.0f ? (m + lg2(l)) * 0.69314718055994531f : -INFINITY;
                 } else {
-#pragma unroll
-                    for (int h = 0; h < HG; ++h) r[h] = 0u;
+                    const int64_t prow = ((int64_t)t * a.S + split) * a.H + (int64_t)g * HG + h;
+                    a.ws_ml[2 * prow] = l > 0.0f ? m : -INFINITY;
+                    a.ws_ml[2 * prow + 1] = l;
                 }
-#pragma unroll
-                for (int h = 0; h < HG; ++h)
-                    reinterpret_cast<__half *>(stage)[h * kLatent + dv] = __float2half_rn(__uint_as_float(r[h]) * inv_l[h]);
             }
-            fence_proxy_async_smem();
-            sm_bar();
-            if (st == 0) {
+            named_bar(bar_id, 128);
+        }
+        if (st == 0 && sw == 0) TRACE(271);
+        const bool leader = (warp == kSoftmaxWarp0 && lane == 0);
+        if (a.S == 1) {
+            // O^T (TMEM, lanes = dv) -> normalised FP16 rows staged in the
+            // (now free) tile region, then one bulk copy of HG x 1 KB to
+            // out[t, g*HG .., :].
+            float inv_l[HWG];
+#pragma unroll
+            for (int h = 0; h < HWG; ++h) inv_l[h] = active ? aux_s[h0 + h] : 0.0f;
+            uint8_t *stage = smem;
+            if (active) {
+#pragma unroll 1
+                for (int dc = 0; dc < 4; ++dc) {
+                    const int dv = 128 * dc + st;
+                    uint32_t r[HWG];
+                    if (have) {
+                        tmem_ld_cols<HWG>(tmem + lane_base + kColO + dc * HG + h0, r);
+                        tmem_ld_wait();
+                    } else {
+#pragma unroll
+                        for (int h = 0; h < HWG; ++h) r[h] = 0u;
+                    }
+#pragma unroll
+                    for (int h = 0; h < HWG; ++h)
+                        reinterpret_cast<__half *>(stage)[(h0 + h) * kLatent + dv] =
+                            __float2half_rn(__uint_as_float(r[h]) * inv_l[h]);
+                }
+                fence_proxy_async_smem();
+            }
+            named_bar(3, 256);
+            if (leader) {
                 bulk_s2g(a.out + ((int64_t)t * a.H + (int64_t)g * HG) * kLatent, stage, HG * kLatent * 2);
                 bulk_commit_wait_read();
             }
-        } else {
+        } else if (active) {
+            // Unnormalised partial O (this split's rows, scaled to its own
+            // reference max) straight from registers: for each head a warp
+            // writes 32 consecutive dv, one 128-byte segment.  The fence makes
+            // these and the statistics above visible before the arrival that
+            // the teardown signals.
+            float *dst = a.ws_o + (((int64_t)t * a.S + split) * a.H + (int64_t)g * HG + h0) * kLatent + st;
 #pragma unroll 1
             for (int dc = 0; dc < 4; ++dc) {
-                float *blk = reinterpret_cast<float *>(stage + dc * (HG * 128 * 4));
-                uint32_t r[HG];
+                uint32_t r[HWG];
                 if (have) {
-                    tmem_ld_cols<HG>(tmem + lane_base + kColO + dc * HG, r);
+                    tmem_ld_cols<HWG>(tmem + lane_base + kColO + dc * HG + h0, r);
                     tmem_ld_wait();
                 } else {
 #pragma unroll
-                    for (int h = 0; h < HG; ++h) r[h] = 0u;
+                    for (int h = 0; h < HWG; ++h) r[h] = 0u;
                 }
 #pragma unroll
-                for (int h = 0; h < HG; ++h) blk[h * 128 + st] = __uint_as_float(r[h]) * inv_l[h];
-                fence_proxy_async_smem();
-                sm_bar();
-                if (st == 0)
-                    bulk_s2g(a.ws_o + ((((int64_t)t * a.S + split) * 4 + dc) * a.H + (int64_t)g * HG) * 128, blk,
-                             HG * 128 * 4);
+                for (int h = 0; h < HWG; ++h) __stcg(dst + (int64_t)h * kLatent + 128 * dc, __uint_as_float(r[h]));
             }
-            if (st == 0) bulk_commit_wait_read();
+            __threadfence();
         }
-        if (st == 0) TRACE(61);
+        if (a.S > 1) {
+            const int mt = tid - 32 * kSoftmaxWarp0;
+            switch (a.S) {
+                case 2: merge_splits<HG, 2>(a, t, g, split, smem, mt); break;
+                case 4: merge_splits<HG, 4>(a, t, g, split, smem, mt); break;
+                case 8: merge_splits<HG, 8>(a, t, g, split, smem, mt); break;
+                default: merge_splits<HG, 16>(a, t, g, split, smem, mt); break;
+            }
+        }
+        if (leader) TRACE(61);
     } else {
         // ---------------------------------------------------- gather + unpack
-        regs_inc<160>();
-        const int ut = tid - 256;
+        regs_dec<RegSplit<HG, kStaged>::unpack>();
+        const int ut = tid - 32 * kUnpackWarp0;
         const int sub = ut & 7;   // 8-dim slice of every 64-dim chunk
         const int rg = ut >> 3;   // rows rg, rg+32, rg+64, rg+96 of each tile
         const uint8_t *row_ptr[4];
         bool rvalid[4];
         constexpr int kWords = kStaged ? 18 : 11;  // raw 32-bit words per row held per tile
         uint32_t raw[4][kWords];
+        // Loads of a tile's rows, issued in the order the chunks consume
+        // them (scales first, then chunk by chunk, RoPE last) so chunk 0
+        // does not wait for the whole tile.  Rows past the end are not read
+        // and stay zero.
         auto load_tile = [&](int i) {
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
@@ -469,58 +630,85 @@ __global__ void __launch_bounds__(dec::kThreads, 1) sparse_mla_decode_kernel(con
                     row_ptr[k] = a.src + ((int64_t)t * a.topk + v) * kStagedRowBytes;
                 else
                     row_ptr[k] = a.src + (int64_t)v * kRowBytes;
-                if (rvalid[k]) {
-                    if (kStaged) {
+            }
+            if (kStaged) {
 #pragma unroll
-                        for (int c = 0; c < kChunks; ++c) {
-                            const uint2 w2 = ldg64(row_ptr[k] + 64 * c + 8 * sub);
-                            raw[k][2 * c] = w2.x;
-                            raw[k][2 * c + 1] = w2.y;
-                        }
-                    } else {
+                for (int c = 0; c < kChunks; ++c) {
 #pragma unroll
-                        for (int c = 0; c < 8; ++c) raw[k][c] = ldg32(row_ptr[k] + 32 * c + 4 * sub);
-                        raw[k][8] = ldg32(row_ptr[k] + kScaleOff + 4 * sub);
-                        const uint2 rp = ldg64(row_ptr[k] + kRopeOff + 8 * sub);
-                        raw[k][9] = rp.x;
-                        raw[k][10] = rp.y;
+                    for (int k = 0; k < 4; ++k) {
+                        const uint2 w2 = rvalid[k] ? ldg64(row_ptr[k] + 64 * c + 8 * sub) : make_uint2(0u, 0u);
+                        raw[k][2 * c] = w2.x;
+                        raw[k][2 * c + 1] = w2.y;
                     }
-                } else {
+                }
+            } else {
 #pragma unroll
-                    for (int w = 0; w < kWords; ++w) raw[k][w] = 0u;
+                for (int k = 0; k < 4; ++k) raw[k][8] = rvalid[k] ? ldg32(row_ptr[k] + kScaleOff + 4 * sub) : 0u;
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) raw[k][c] = rvalid[k] ? ldg32(row_ptr[k] + 32 * c + 4 * sub) : 0u;
+                }
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const uint2 rp = rvalid[k] ? ldg64(row_ptr[k] + kRopeOff + 8 * sub) : make_uint2(0u, 0u);
+                    raw[k][9] = rp.x;
+                    raw[k][10] = rp.y;
                 }
             }
         };
         bool ok = true;
         if (ntiles > 0) load_tile(0);
-        for (int i = 0; i < ntiles && ok; ++i) {
+        if (ut == 0) TRACE(277);
+        cp_async_wait_all();  // this thread's Q copies
+        fence_proxy_async_smem();
+        if (ut == 0) TRACE(264);
+        // Decode chunk c of this thread's 4 rows into the swizzled tile.
+        auto unpack_chunk = [&](int c) {
 #pragma unroll
-            for (int c = 0; c < kChunks; ++c) {
-                if (i > 0 && !mbar_wait(&bars[BAR_CHUNK_FREE + (c < 8 ? (c >> 1) : 3)], (i - 1) & 1)) {
+            for (int k = 0; k < 4; ++k) {
+                uint32_t o[4];
+                if (kStaged) {
+                    e4m3x8_to_f16x8(raw[k][2 * c], raw[k][2 * c + 1], o);
+                } else if (c < 8) {
+                    const uint32_t sw = __shfl_sync(0xffffffffu, raw[k][8], (lane & ~7) | c);
+                    const uint32_t sb = (sw >> (8 * (sub >> 1))) & 0xFFu;
+                    const uint32_t s2 = e4m3x2_to_f16x2(sb | (sb << 8));
+                    e2m1x8_to_f16x8(raw[k][c], o);
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) o[j] = hmul2_u32(o[j], s2);
+                } else {
+                    e4m3x8_to_f16x8(raw[k][9], raw[k][10], o);
+                }
+                *reinterpret_cast<uint4 *>(smem + c * kChunkBytes + sw128_offset(rg + 32 * k, sub)) =
+                    make_uint4(o[0], o[1], o[2], o[3]);
+            }
+        };
+        for (int i = 0; i < ntiles && ok; ++i) {
+            // Chunks 2p and 2p+1 are released together by output block p, so
+            // they are written as a pair behind one wait and one fence; the
+            // RoPE chunk (8, where P^T lives) was released by block 3.
+#pragma unroll
+            for (int p = 0; p < 5; ++p) {
+                if (p < 4 && i > 0 && !mbar_wait(&bars[BAR_CHUNK_FREE + p], (i - 1) & 1)) {
                     ok = false;
                     break;
                 }
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    uint32_t o[4];
-                    if (kStaged) {
-                        e4m3x8_to_f16x8(raw[k][2 * c], raw[k][2 * c + 1], o);
-                    } else if (c < 8) {
-                        const uint32_t sw = __shfl_sync(0xffffffffu, raw[k][8], (lane & ~7) | c);
-                        const uint32_t sb = (sw >> (8 * (sub >> 1))) & 0xFFu;
-                        const uint32_t s2 = e4m3x2_to_f16x2(sb | (sb << 8));
-                        e2m1x8_to_f16x8(raw[k][c], o);
-#pragma unroll
-                        for (int j = 0; j < 4; ++j) o[j] = hmul2_u32(o[j], s2);
-                    } else {
-                        e4m3x8_to_f16x8(raw[k][9], raw[k][10], o);
-                    }
-                    *reinterpret_cast<uint4 *>(smem + c * kChunkBytes + sw128_offset(rg + 32 * k, sub)) =
-                        make_uint4(o[0], o[1], o[2], o[3]);
+                if (ut == 0 && i == 1) TRACE(80 + p);
+                if (p < 4) {
+                    unpack_chunk(2 * p);
+                    unpack_chunk(2 * p + 1);
+                } else {
+                    unpack_chunk(8);
                 }
                 fence_proxy_async_smem();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&bars[BAR_CHUNK_FULL + c]);
+                if (lane == 0) {
+                    mbar_arrive(&bars[BAR_CHUNK_FULL + (p < 4 ? 2 * p : 8)]);
+                    if (p < 4) mbar_arrive(&bars[BAR_CHUNK_FULL + 2 * p + 1]);
+                }
+                if (ut == 0 && i == 1) TRACE(96 + p);
+                if (lane == 0 && i == 1) TRACE(128 + 16 * (ut >> 5) + p);
             }
             if (ut == 0 && i < 8) TRACE(6 + 6 * i);
             if (ok && i + 1 < ntiles) load_tile(i + 1);
@@ -538,49 +726,25 @@ __global__ void __launch_bounds__(dec::kThreads, 1) sparse_mla_decode_kernel(con
     }
 }
 
-// Merge split partials: out = sum_s w_s o_s / sum_s w_s with
-// w_s = l_s 2^(m_s - max m), lse = (max m + log2 sum w) ln 2.  One block per
-// (token, head); every load is issued before any of them is used.
-template <int S>
-__global__ void __launch_bounds__(128) combine_splits_kernel(const float *__restrict__ ws_o,
-                                                             const float *__restrict__ ws_ml, int H,
-                                                             __half *__restrict__ out, float *__restrict__ lse) {
-    const int th = blockIdx.x;  // t*H + h
-    const int t = th / H, h = th % H;
-    float m[S], l[S];
-    float4 o[S];
-#pragma unroll
-    for (int s = 0; s < S; ++s) {
-        const int64_t prow = ((int64_t)t * S + s) * H + h;
-        const float2 ml = *reinterpret_cast<const float2 *>(ws_ml + 2 * prow);
-        m[s] = ml.x;
-        l[s] = ml.y;
-        // partial rows are stored per 128-dv block: [t][s][dc][h][128]
-        const int dc = threadIdx.x >> 5, d = 4 * (threadIdx.x & 31);
-        o[s] = *reinterpret_cast<const float4 *>(ws_o + ((((int64_t)t * S + s) * 4 + dc) * H + h) * 128 + d);
+int current_device_sm_count() {
+    static int cached[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+        (void)cudaGetLastError();  // no device: leave no error behind for later launches
+        return 148;
     }
-    float mmax = -INFINITY;
-#pragma unroll
-    for (int s = 0; s < S; ++s)
-        if (l[s] > 0.0f) mmax = fmaxf(mmax, m[s]);
-    float L = 0.0f, acc0 = 0.0f, acc1 = 0.0f, acc2 = 0.0f, acc3 = 0.0f;
-#pragma unroll
-    for (int s = 0; s < S; ++s) {
-        const float w = l[s] > 0.0f ? l[s] * ex2(m[s] - mmax) : 0.0f;
-        L += w;
-        acc0 += w * o[s].x;
-        acc1 += w * o[s].y;
-        acc2 += w * o[s].z;
-        acc3 += w * o[s].w;
+    if (!cached[dev]) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1) {
+            (void)cudaGetLastError();
+            return 148;
+        }
+        cached[dev] = n;
     }
-    const float inv = L > 0.0f ? 1.0f / L : 0.0f;
-    __half2 *dst = reinterpret_cast<__half2 *>(out + (int64_t)th * kLatent + 4 * threadIdx.x);
-    dst[0] = __floats2half2_rn(acc0 * inv, acc1 * inv);
-    dst[1] = __floats2half2_rn(acc2 * inv, acc3 * inv);
-    if (threadIdx.x == 0) lse[th] = L > 0.0f ? (mmax + lg2(L)) * 0.69314718055994531f : -INFINITY;
+    return cached[dev];
 }
 
-bool make_decode_plan(int32_t T, int32_t H, int32_t topk, DecodePlan *plan) {
+bool make_decode_plan(int32_t T, int32_t H, int32_t topk, int sm_count, DecodePlan *plan) {
     DecodePlan p{};
     if (H == 16 || H == 32 || H == 64) {
         p.heads_per_cta = H;
@@ -591,13 +755,16 @@ bool make_decode_plan(int32_t T, int32_t H, int32_t topk, DecodePlan *plan) {
     } else {
         return false;
     }
-    if (topk < 1 || topk > kMaxTopk || T < 0) return false;
+    if (topk < 1 || topk > kMaxTopk || T < 0 || sm_count < 1) return false;
+    // Split a token's list over S CTAs only while the whole grid still fits
+    // in one wave of one CTA per SM (the merge needs every CTA resident).
     const int64_t units = (int64_t)T * p.head_groups;
-    const int max_s = std::min(16, (topk + dec::kTileRows - 1) / dec::kTileRows);
+    const int max_s = std::min(dec::kMaxSplits, (topk + dec::kTileRows - 1) / dec::kTileRows);
     int S = 1;
-    while (S * 2 <= max_s && units * S * 2 <= 148) S *= 2;
+    while (S * 2 <= max_s && units * S * 2 <= sm_count) S *= 2;
+    if (S > 1 && units > (int64_t)(kSplitCounterBytes / 8)) S = 1;
     p.splits = S;
-    p.workspace_bytes = S > 1 ? (size_t)T * S * H * (kLatent + 2) * sizeof(float) : 0;
+    p.workspace_bytes = S > 1 ? kSplitCounterBytes + (size_t)T * S * H * (kLatent + 2) * sizeof(float) : 0;
     *plan = p;
     return true;
 }
@@ -610,12 +777,30 @@ static cudaError_t launch_hg(const DecodeArgs &a, int64_t nblocks, cudaStream_t 
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= 64 || !attr_set[dev]) {
+        // The per-role register split (setmaxnreg) assumes the block starts
+        // with kRegsLaunch registers per thread; with fewer, a role's
+        // increase could never be granted, so refuse to launch.
+        cudaFuncAttributes fa;
+        e = cudaFuncGetAttributes(&fa, kern);
+        if (e != cudaSuccess) return e;
+        if (fa.numRegs != dec::kRegsLaunch || fa.maxThreadsPerBlock < dec::kThreads) return cudaErrorInvalidConfiguration;
         e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, dec::kSmemBytes);
         if (e != cudaSuccess) return e;
         if (dev >= 0 && dev < 64) attr_set[dev] = true;
     }
-    kern<<<(unsigned)nblocks, dec::kThreads, dec::kSmemBytes, stream>>>(a);
-    return cudaGetLastError();
+    // Split launches are cooperative: the runtime refuses the launch unless
+    // every CTA can be resident at once, which the merge's wait relies on.
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)nblocks);
+    cfg.blockDim = dim3(dec::kThreads);
+    cfg.dynamicSmemBytes = dec::kSmemBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = a.S > 1 ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kern, a);
 }
 
 cudaError_t launch_sparse_mla_decode(bool staged, const void *q_nope, const void *q_rope, const uint8_t *src,
@@ -637,8 +822,11 @@ cudaError_t launch_sparse_mla_decode(bool staged, const void *q_nope, const void
     a.scale_log2 = (float)((double)sm_scale * 1.4426950408889634);
     a.out = static_cast<__half *>(out);
     a.lse = lse;
-    a.ws_o = static_cast<float *>(workspace);
-    a.ws_ml = a.ws_o ? a.ws_o + (size_t)T * plan.splits * H * kLatent : nullptr;
+    // workspace: [split counters, kSplitCounterBytes][ws_ml][ws_o]
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    a.counters = plan.splits > 1 ? reinterpret_cast<uint32_t *>(ws) : nullptr;
+    a.ws_ml = plan.splits > 1 ? reinterpret_cast<float *>(ws + kSplitCounterBytes) : nullptr;
+    a.ws_o = plan.splits > 1 ? a.ws_ml + (size_t)T * plan.splits * H * 2 : nullptr;
     a.dev_status = dev_status;
     const int64_t nblocks = (int64_t)T * plan.head_groups * plan.splits;
     cudaError_t e;
@@ -651,16 +839,7 @@ cudaError_t launch_sparse_mla_decode(bool staged, const void *q_nope, const void
         case 129: e = launch_hg<64, true>(a, nblocks, stream); break;
         default: return cudaErrorInvalidValue;
     }
-    if (e != cudaSuccess || plan.splits == 1) return e;
-    const unsigned cblocks = (unsigned)((int64_t)T * H);
-    switch (plan.splits) {
-        case 2: combine_splits_kernel<2><<<cblocks, 128, 0, stream>>>(a.ws_o, a.ws_ml, H, a.out, a.lse); break;
-        case 4: combine_splits_kernel<4><<<cblocks, 128, 0, stream>>>(a.ws_o, a.ws_ml, H, a.out, a.lse); break;
-        case 8: combine_splits_kernel<8><<<cblocks, 128, 0, stream>>>(a.ws_o, a.ws_ml, H, a.out, a.lse); break;
-        case 16: combine_splits_kernel<16><<<cblocks, 128, 0, stream>>>(a.ws_o, a.ws_ml, H, a.out, a.lse); break;
-        default: return cudaErrorInvalidValue;
-    }
-    return cudaGetLastError();
+    return e;
 }
 
 }  // namespace nvfp4mla

@@ -21,18 +21,19 @@ struct DecodeArgs {
     float scale_log2;
     __half *out;
     float *lse;
-    float *ws_o;
-    float *ws_ml;
+    float *ws_o;        // split partials: [T][S][H][512] FP32, unnormalised
+    float *ws_ml;       // split statistics: [T][S][H] x (max in log2 units, row sum)
+    uint32_t *counters; // per (token, head group): arrivals, departures
     int32_t *dev_status;
 };
 
 #ifdef NVFP4MLA_TRACE
 // Debug builds only: per-CTA phase timestamps (clock64 deltas) for the
-// first 16 CTAs, 64 slots each.
+// first 16 CTAs, 512 slots each.
 static __device__ unsigned long long *g_trace;
 #define TRACE(slot)                                                                  \
     do {                                                                             \
-        if (g_trace && blockIdx.x < 16) g_trace[blockIdx.x * 64 + (slot)] = clock64() - t_start; \
+        if (g_trace && blockIdx.x < 16) g_trace[blockIdx.x * 512 + (slot)] = clock64() - t_start; \
     } while (0)
 static inline void set_trace_local(unsigned long long *p) { cudaMemcpyToSymbol(g_trace, &p, sizeof(p)); }
 #else
@@ -52,13 +53,16 @@ __device__ __forceinline__ float lg2(float x) {
     return y;
 }
 // Named barrier 1 over the 128 softmax threads, optionally OR-reducing a flag.
-__device__ __forceinline__ void sm_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
-__device__ __forceinline__ bool sm_bar_or(bool p) {
+// Named barrier `id` over `n` threads, optionally OR-reducing a flag.
+__device__ __forceinline__ void named_bar(uint32_t id, uint32_t n) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+__device__ __forceinline__ bool named_bar_or(uint32_t id, uint32_t n, bool p) {
     uint32_t r;
     asm volatile(
-        "{\n\t.reg .pred pi, po;\n\tsetp.ne.u32 pi, %1, 0;\n\tbar.red.or.pred po, 1, 128, pi;\n\tselp.u32 %0, 1, 0, po;\n\t}"
+        "{\n\t.reg .pred pi, po;\n\tsetp.ne.u32 pi, %3, 0;\n\tbar.red.or.pred po, %1, %2, pi;\n\tselp.u32 %0, 1, 0, po;\n\t}"
         : "=r"(r)
-        : "r"((uint32_t)p)
+        : "r"(id), "r"(n), "r"((uint32_t)p)
         : "memory");
     return r != 0;
 }

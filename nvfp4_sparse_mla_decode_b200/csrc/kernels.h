@@ -18,7 +18,16 @@ struct DecodePlan {
     int splits;         // S: CTAs sharing one token's list
     size_t workspace_bytes;
 };
-bool make_decode_plan(int32_t T, int32_t H, int32_t topk, DecodePlan *plan);
+// Split launches keep one (arrivals, departures) pair of uint32 counters per
+// (token, head group) at the start of the workspace; splitting needs
+// T * G * S <= SMs, so a fixed 4 KB region (512 pairs) always suffices and
+// sits at the same place for every shape.
+constexpr size_t kSplitCounterBytes = 4096;
+// sm_count: SMs of the device the launch will run on (one CTA per SM).
+bool make_decode_plan(int32_t T, int32_t H, int32_t topk, int sm_count, DecodePlan *plan);
+// SM count of the current device, or 148 when no device can be queried
+// (pure host use, e.g. sizing a workspace on a machine without a GPU).
+int current_device_sm_count();
 
 // Sparse MLA decode over NVFP4 rows (staged == false: `src` is the cache of
 // num_slots 352-byte rows, list entries are slots) or over the staging

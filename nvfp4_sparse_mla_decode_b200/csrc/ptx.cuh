@@ -56,6 +56,30 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity,
     }
 }
 
+// ------------------------------------------------- grid-scope counters
+// Release-add / acquire-load on a global counter (GPU scope), used to hand
+// split partials from one CTA to the others of its group.
+__device__ __forceinline__ void red_release_gpu_add(uint32_t *p, uint32_t v) {
+    asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t *p) {
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+// Wait until *p >= target, for at most max_cycles SM clocks; false on
+// timeout.  Only meaningful when every CTA that adds to *p is resident at
+// the same time (cooperative launch).
+__device__ __forceinline__ bool spin_until_geq(const uint32_t *p, uint32_t target,
+                                               unsigned long long max_cycles = kWaitCycles) {
+    const unsigned long long t0 = clock64();
+    while (ld_acquire_gpu(p) < target) {
+        if (clock64() - t0 > max_cycles) return false;
+        __nanosleep(64);
+    }
+    return true;
+}
+
 // --------------------------------------------------------------- bulk copies
 // Untiled bulk copy global -> this CTA's shared memory, completing `bytes`
 // transaction bytes on `bar`.  Both addresses 16-byte aligned, bytes % 16 == 0.

@@ -227,8 +227,9 @@ void oracle_stage_row(const uint8_t *row, uint8_t *out576)
 /* Sparse MLA decode in FP64 over dequantized rows.
  *
  * For token t and head h, over list positions j with 0 <= idx[t,j] < num_slots
- * (any other entry is empty and contributes nothing -- the reading of
- * "zero-filled empty entries"; a duplicate index counts once per position):
+ * (any other entry is empty and contributes nothing -- this is how the
+ * pages' treatment of list slots the indexer leaves unfilled is read here;
+ * a duplicate index counts once per position):
  *   s_j   = sm_scale * ( sum_{d<512} q_nope[t,h,d] k_j[d]
  *                      + sum_{d<64}  q_rope[t,h,d] k_j[512+d] )
  *   m     = max_j s_j ;  l = sum_j exp(s_j - m)

@@ -47,7 +47,7 @@ def test_plan_splits_fill_the_gpu(L):
     assert nv.num_splits(4000, 64) == 1
     assert nv.num_splits(1, 64, 100) == 1      # a 100-entry list is one tile
     assert nv.num_splits(1, 48) == 0           # unsupported head count
-    assert nv.workspace_size(35, 64) == 35 * 4 * 64 * 514 * 4
+    assert nv.workspace_size(35, 64) == 4096 + 35 * 4 * 64 * 514 * 4
     assert nv.workspace_size(4000, 64) == 0
     assert nv.staging_size(35) == 35 * 2048 * 576
 

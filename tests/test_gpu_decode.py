@@ -123,3 +123,31 @@ def test_zero_tokens_is_noop():
     idx = torch.empty(0, 2048, dtype=torch.int32, device="cuda")
     out, lse = nv.decode(qn, qr, cache, idx, 0.1)
     assert out.numel() == 0 and lse.numel() == 0
+
+
+def test_split_workspace_reused_across_shapes_and_calls():
+    # One zero-filled workspace serves split launches of different shapes
+    # (S = 4, 8 and 16 here); every call must leave the 4096-byte counter
+    # region at zero and repeat its results bit for bit.
+    shapes = [(synth.per_request("cuda", [6000] * 35, 64, seed=51, name="ws35"), [0, 17, 34]),
+              (synth.per_request("cuda", [6000] * 6, 128, seed=52, name="ws6"), [0, 5]),
+              (synth.tiny("cuda", seed=53), [0])]
+    need = max(nv.workspace_size(w.T, w.H) for w, _ in shapes)
+    assert [nv.num_splits(w.T, w.H) for w, _ in shapes] == [4, 8, 16]
+    ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
+    for w, tokens in shapes:
+        cache = build_cache(w)
+        status = torch.zeros(1, dtype=torch.int32, device="cuda")
+        first = None
+        for _ in range(2):
+            out, lse = nv.decode(w.q_nope, w.q_rope, cache, w.indices, w.sm_scale, workspace=ws, dev_status=status)
+            torch.cuda.synchronize()
+            assert int(status.item()) == 0
+            assert int(ws[:4096].count_nonzero().item()) == 0, "split counters not reset"
+            if first is None:
+                first = (out.clone(), lse.clone())
+            else:
+                assert torch.equal(out, first[0]) and torch.equal(lse, first[1])
+        ref_o, ref_l = oracle_decode(w, tokens)
+        check_close(out[tokens], lse[tokens], ref_o, ref_l)
+        del cache
