@@ -66,7 +66,7 @@ constexpr int kOffM = kOffIdx + kMaxTopk * 4;        // reference max per head (
 constexpr int kOffAux = kOffM + kMaxHG * 4;          // rescale factors / 1/l per head
 constexpr int kOffRed = kOffAux + kMaxHG * 4;        // 4 warps x 64 floats
 constexpr int kOffBar = kOffRed + 4 * kMaxHG * 4;
-constexpr int kNumBars = 16;
+constexpr int kNumBars = 17;
 constexpr int kOffMisc = kOffBar + kNumBars * 8;
 constexpr int kSmemBytes = kOffMisc + 64;
 static_assert(kSmemBytes <= 232448, "shared memory budget");
@@ -100,45 +100,60 @@ constexpr int BAR_CHUNK_FREE = 9;  // [4] output MMAs of a 128-dv block done
 constexpr int BAR_S_FULL = 13;     // score MMAs of a tile done
 constexpr int BAR_P_FULL = 14;     // P^T written (4 softmax warps)
 constexpr int BAR_DRAIN = 15;      // every MMA issued so far done
+constexpr int BAR_Q_FULL = 16;     // Q copies landed (4 warps of the MMA warpgroup)
 
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColO = 0;      // O^T: 4 blocks of HG columns
 constexpr uint32_t kColS = 256;    // S^T: HG columns
 constexpr float kRescaleThreshold = 8.0f;
 constexpr int kMaxSplits = 16;
-static_assert((kMaxSplits + 1) * kMaxHG * 4 <= kTileBytes, "merge weights must fit in the tile region");
+// Merge scratch in the (by then free) tile region: split weights at 0, and
+// at kOffPart the CTA's own partial dv slice (S <= 4) at its place in an
+// [S][HG][512/S] FP32 array (HG x 2 KB).
+constexpr int kOffPart = 16384;
+static_assert((kMaxSplits + 1) * kMaxHG * 4 <= kOffPart, "merge weights must fit below the slices");
+static_assert(kOffPart + kMaxHG * kLatent * 4 <= kTileBytes, "partial slices must fit in the tile region");
 }  // namespace dec
 
 // Merge of the S split partials of one (token, head group), run by the 256
-// softmax threads of each of the S CTAs of the group once their own partial
-// is written: each CTA announces its partial on the group's arrival
-// counter, waits (bounded) until all S have, then combines the dv slice
-// [split*512/S, (split+1)*512/S) of every head:
+// softmax threads of each of the S CTAs of the group once their partial is
+// written: one thread announces this CTA's partial on the group's arrival
+// counter (release; the softmax-group barrier before it orders every
+// thread's partial stores ahead of it), waits (bounded) until all S have,
+// and then the group combines the dv slice [split*512/S, (split+1)*512/S)
+// of every head:
 //   out = sum_s w_s O_s / sum_s w_s l_s,  w_s = 2^(m_s - max m)
 // over the splits with rows (l_s > 0); split 0 also writes
-// lse = (max m + log2 of the denominator) ln 2.  The launch is cooperative,
-// so all S CTAs are resident together and the wait ends.  The last CTA to
-// leave resets both counters, which lets the next call start from zero.
-// Loads of up to 16 partial vectors are issued before any is used.
+// lse = (max m + log2 of the denominator) ln 2.  With S <= 4 the CTA's own
+// slice is already in shared memory; the others are read with 16-byte
+// loads, up to 16 in flight per thread.  The launch is cooperative, so all S
+// CTAs are resident together and the wait ends.  The last CTA to leave
+// resets both counters, which lets the next call start from zero.
 template <int HG, int S>
-__device__ __forceinline__ void merge_splits(const DecodeArgs &a, int t, int g, int split, uint8_t *smem, int mt) {
+__device__ __forceinline__ void merge_splits(const DecodeArgs &a, int t, int g, int split, uint8_t *smem, int mt,
+                                             [[maybe_unused]] unsigned long long t_start) {
     using namespace dec;
     constexpr int kMergeThreads = 256;
-    constexpr int D = kLatent / S;        // dv per CTA
-    constexpr int NQ = D / 4;             // float4 per head
+    constexpr int D = kLatent / S;           // dv per CTA
+    constexpr int NQ = D / 4;                // float4 per head
     constexpr int ITEMS = HG * NQ;
-    constexpr int B = S >= 16 ? 1 : 16 / S;  // items per batch: B * S loads in flight
+    constexpr int B = S >= 16 ? 1 : 16 / S;  // items per batch: B * S vectors in flight per thread
+    constexpr bool kOwnInSmem = S <= 4;
     uint32_t *arrive = a.counters + 2 * ((int64_t)t * a.G + g);
     uint32_t *depart = arrive + 1;
     uint32_t *flag = reinterpret_cast<uint32_t *>(smem + kOffMisc) + 1;
-    float *w_s = reinterpret_cast<float *>(smem);  // [S][HG] weights (free tile region)
+    float *w_s = reinterpret_cast<float *>(smem);  // [S][HG] weights
     float *inv_den = w_s + kMaxSplits * HG;         // [HG]
-    named_bar(3, kMergeThreads);                    // every partial store of this CTA is fenced
+    const float *own = reinterpret_cast<const float *>(smem + kOffPart) + (int64_t)split * HG * D;  // [HG][D]
+    named_bar(3, kMergeThreads);  // every partial store of the group precedes the release
     if (mt == 0) {
+        TRACE(280);
+        __threadfence();
         red_release_gpu_add(arrive, 1u);
         const bool ok = spin_until_geq(arrive, (uint32_t)S);
         if (!ok && a.dev_status) atomicOr(a.dev_status, NVFP4MLA_DEV_TIMEOUT);
         *flag = ok ? 1u : 0u;
+        TRACE(281);
     }
     named_bar(3, kMergeThreads);
     if (!*flag) return;  // counters stay raised: the caller must clear them after a timeout
@@ -164,6 +179,7 @@ __device__ __forceinline__ void merge_splits(const DecodeArgs &a, int t, int g, 
                 den > 0.0f ? (mmax + lg2(den)) * 0.69314718055994531f : -INFINITY;
     }
     named_bar(3, kMergeThreads);
+    if (mt == 0) TRACE(282);
     const int dv0 = split * D;
     const int64_t part = (int64_t)a.H * kLatent;  // next split of the same (t, head)
     const float *src = a.ws_o + ((int64_t)t * S * a.H + (int64_t)g * HG) * kLatent + dv0;
@@ -175,10 +191,14 @@ __device__ __forceinline__ void merge_splits(const DecodeArgs &a, int t, int g, 
             const int item = base + b * kMergeThreads;
             const int h = item / NQ, q = item - h * NQ;
 #pragma unroll
-            for (int s = 0; s < S; ++s)
-                o[b][s] = item < ITEMS
-                              ? __ldcg(reinterpret_cast<const float4 *>(src + (int64_t)h * kLatent + 4 * q + s * part))
-                              : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+            for (int s = 0; s < S; ++s) {
+                if (item >= ITEMS)
+                    o[b][s] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+                else if (kOwnInSmem && s == split)
+                    o[b][s] = *reinterpret_cast<const float4 *>(own + h * D + 4 * q);
+                else
+                    o[b][s] = __ldcg(reinterpret_cast<const float4 *>(src + (int64_t)h * kLatent + 4 * q + s * part));
+            }
         }
 #pragma unroll
         for (int b = 0; b < B; ++b) {
@@ -203,6 +223,7 @@ __device__ __forceinline__ void merge_splits(const DecodeArgs &a, int t, int g, 
     }
     named_bar(3, kMergeThreads);
     if (mt == 0) {
+        TRACE(283);
         const uint32_t old = atomicAdd(depart, 1u);
         if (old == (uint32_t)S - 1u) {  // every CTA of the group is past its wait
             atomicExch(arrive, 0u);
@@ -218,6 +239,8 @@ __global__ void __launch_bounds__(dec::kThreads, 1) sparse_mla_decode_kernel(con
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 #ifdef NVFP4MLA_TRACE
     const unsigned long long t_start = clock64();
+#else
+    const unsigned long long t_start = 0;  // timestamps exist only in trace builds
 #endif
     const int split = blockIdx.x % a.S;
     const int rest = blockIdx.x / a.S;
@@ -243,6 +266,7 @@ __global__ void __launch_bounds__(dec::kThreads, 1) sparse_mla_decode_kernel(con
         else if (lane < BAR_P_FULL) count = 1;          // MMA commits
         else if (lane == BAR_P_FULL) count = 8;         // 8 softmax warps
         else if (lane == BAR_DRAIN) count = 1;
+        else if (lane == BAR_Q_FULL) count = 4;         // MMA warpgroup
         if (count) mbar_init(&bars[lane], count);
         fence_mbar_init();
     }
@@ -274,21 +298,6 @@ __global__ void __launch_bounds__(dec::kThreads, 1) sparse_mla_decode_kernel(con
     if (tid == 0) TRACE(261);
     __syncthreads();
     if (tid == 0) TRACE(262);
-    // Q of (t, heads g*HG ..) -> shared memory, K-major, 128-byte swizzle:
-    // chunk c holds dims 64c..64c+63 of every head (chunk 8 = RoPE).  Issued
-    // as 16-byte async copies after the list loads (so they do not queue
-    // ahead of them); each unpack thread waits for its own copies before its
-    // first chunk arrival, which orders them before the first score MMAs.
-    if (warp >= kUnpackWarp0) {
-        const int ut = tid - 32 * kUnpackWarp0;
-        const int64_t head0 = (int64_t)t * a.H + (int64_t)g * HG;
-        for (int u = ut; u < HG * 72; u += 256) {
-            const int h = u / 72, v = u % 72;
-            const void *src = v < 64 ? static_cast<const void *>(a.q_nope + (head0 + h) * kLatent + 8 * v)
-                                     : static_cast<const void *>(a.q_rope + (head0 + h) * kRope + 8 * (v - 64));
-            cp_async16(smem + kOffQ + (v >> 3) * (HG * 128) + sw128_offset(h, v & 7), src);
-        }
-    }
     // Exclusive prefix of the 64 per-(round, warp) counts.  Every warp scans
     // them itself (two per lane) and reads its own offsets from the lane that
     // holds them, so no second block barrier is needed.
@@ -336,6 +345,24 @@ __global__ void __launch_bounds__(dec::kThreads, 1) sparse_mla_decode_kernel(con
     // the compiler sizes each role's code separately.
     if (warp < 4) {
         regs_dec<RegSplit<HG, kStaged>::mma>();
+        // Q of (t, heads g*HG ..) -> shared memory, K-major, 128-byte swizzle:
+        // chunk c holds dims 64c..64c+63 of every head (chunk 8 = RoPE).  The
+        // MMA warpgroup is otherwise idle here, so its 128 threads issue the
+        // 16-byte async copies while the unpack warps start on the rows, and
+        // signal Q_FULL once their own copies have landed.
+        {
+            const int64_t head0 = (int64_t)t * a.H + (int64_t)g * HG;
+            for (int u = tid; u < HG * 72; u += 128) {
+                const int h = u / 72, v = u % 72;
+                const void *src = v < 64 ? static_cast<const void *>(a.q_nope + (head0 + h) * kLatent + 8 * v)
+                                         : static_cast<const void *>(a.q_rope + (head0 + h) * kRope + 8 * (v - 64));
+                cp_async16(smem + kOffQ + (v >> 3) * (HG * 128) + sw128_offset(h, v & 7), src);
+            }
+            cp_async_wait_all();
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars[BAR_Q_FULL]);
+        }
         // ------------------------------------------------------------- MMA
         if (warp == 0 && lane == 0) {
             const uint32_t idesc_qk = idesc_f16_f32(128, HG, false, false);
@@ -344,7 +371,7 @@ __global__ void __launch_bounds__(dec::kThreads, 1) sparse_mla_decode_kernel(con
             const uint64_t dQ0 = smem_desc(smem_u32(smem + kOffQ), 16, 1024);
             const uint64_t dV0 = smem_desc(smem_u32(smem), kChunkBytes, 1024);
             const uint64_t dP0 = smem_desc(smem_u32(smem + 8 * kChunkBytes), kChunkBytes, 1024);
-            bool ok = true;
+            bool ok = ntiles == 0 || mbar_wait(&bars[BAR_Q_FULL], 0);
             // Descriptors advance by adding (byte offset >> 4) to the start
             // address field; the chunk and block loops stay rolled so the
             // compiler keeps a handful of descriptors live, not one per MMA.
@@ -576,33 +603,52 @@ __global__ void __launch_bounds__(dec::kThreads, 1) sparse_mla_decode_kernel(con
             }
         } else if (active) {
             // Unnormalised partial O (this split's rows, scaled to its own
-            // reference max) straight from registers: for each head a warp
-            // writes 32 consecutive dv, one 128-byte segment.  The fence makes
-            // these and the statistics above visible before the arrival that
-            // the teardown signals.
+            // reference max), two 128-dv blocks per TMEM round trip.  Blocks
+            // inside this CTA's own merge slice (S <= 4) go straight to their
+            // place in shared memory; the rest go to the workspace from registers
+            // (for each head a warp writes 32 consecutive dv, one 128-byte
+            // segment).  The block barrier and release in the merge order
+            // these stores ahead of the arrival.
             float *dst = a.ws_o + (((int64_t)t * a.S + split) * a.H + (int64_t)g * HG + h0) * kLatent + st;
+            const int own_n = a.S <= 4 ? 4 / a.S : 0;  // 128-dv blocks in the own slice
+            const int own_dc0 = split * own_n;
+            const int own_d = kLatent / a.S;
+            // own slice: its place [split][h][own_d] among the merge's slices
+            float *own = reinterpret_cast<float *>(smem + kOffPart) + (int64_t)split * HG * own_d;
 #pragma unroll 1
-            for (int dc = 0; dc < 4; ++dc) {
-                uint32_t r[HWG];
+            for (int dc = 0; dc < 4; dc += 2) {
+                uint32_t r[2][HWG];
                 if (have) {
-                    tmem_ld_cols<HWG>(tmem + lane_base + kColO + dc * HG + h0, r);
+                    tmem_ld_cols<HWG>(tmem + lane_base + kColO + dc * HG + h0, r[0]);
+                    tmem_ld_cols<HWG>(tmem + lane_base + kColO + (dc + 1) * HG + h0, r[1]);
                     tmem_ld_wait();
                 } else {
 #pragma unroll
-                    for (int h = 0; h < HWG; ++h) r[h] = 0u;
+                    for (int h = 0; h < HWG; ++h) r[0][h] = r[1][h] = 0u;
                 }
 #pragma unroll
-                for (int h = 0; h < HWG; ++h) __stcg(dst + (int64_t)h * kLatent + 128 * dc, __uint_as_float(r[h]));
+                for (int j = 0; j < 2; ++j) {
+                    const int b = dc + j;
+                    if (b >= own_dc0 && b < own_dc0 + own_n) {
+                        float *o = own + (int64_t)h0 * own_d + 128 * (b - own_dc0) + st;
+#pragma unroll
+                        for (int h = 0; h < HWG; ++h) o[h * own_d] = __uint_as_float(r[j][h]);
+                    } else {
+#pragma unroll
+                        for (int h = 0; h < HWG; ++h)
+                            __stcg(dst + (int64_t)h * kLatent + 128 * b, __uint_as_float(r[j][h]));
+                    }
+                }
             }
-            __threadfence();
         }
+        if (st == 0 && sw == 0) TRACE(279);
         if (a.S > 1) {
             const int mt = tid - 32 * kSoftmaxWarp0;
             switch (a.S) {
-                case 2: merge_splits<HG, 2>(a, t, g, split, smem, mt); break;
-                case 4: merge_splits<HG, 4>(a, t, g, split, smem, mt); break;
-                case 8: merge_splits<HG, 8>(a, t, g, split, smem, mt); break;
-                default: merge_splits<HG, 16>(a, t, g, split, smem, mt); break;
+                case 2: merge_splits<HG, 2>(a, t, g, split, smem, mt, t_start); break;
+                case 4: merge_splits<HG, 4>(a, t, g, split, smem, mt, t_start); break;
+                case 8: merge_splits<HG, 8>(a, t, g, split, smem, mt, t_start); break;
+                default: merge_splits<HG, 16>(a, t, g, split, smem, mt, t_start); break;
             }
         }
         if (leader) TRACE(61);
@@ -660,9 +706,6 @@ __global__ void __launch_bounds__(dec::kThreads, 1) sparse_mla_decode_kernel(con
         bool ok = true;
         if (ntiles > 0) load_tile(0);
         if (ut == 0) TRACE(277);
-        cp_async_wait_all();  // this thread's Q copies
-        fence_proxy_async_smem();
-        if (ut == 0) TRACE(264);
         // Decode chunk c of this thread's 4 rows into the swizzled tile.
         auto unpack_chunk = [&](int c) {
 #pragma unroll
