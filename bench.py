@@ -177,6 +177,24 @@ def oracle_passes(w, seconds: float):
     return flop * passes / t_all, passes, t_all, oracle.max_threads()
 
 
+def max_over_ranks(value: float, world: int, device) -> float:
+    """The largest of every rank's value (the job is as slow as its slowest
+    replica); every rank takes the same collective step."""
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as tdist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tflops(flop_per_launch: float, ms_total: float, steps: int, world: int) -> float:
+    """Whole-job throughput: every rank ran `steps` launches of the same work,
+    timed as the slowest rank's `ms_total`."""
+    return flop_per_launch * steps * world / (ms_total * 1e-3) / 1e12
+
+
 def reference_arm(args, rank, world):
     """CPU oracle on host cores, rank 0 only, bounded sample of the workload."""
     if rank != 0:
@@ -270,14 +288,10 @@ def main():
     if world > 1:
         tdist.barrier()
     sampler.stop()
-    ms = e0.elapsed_time(e1)
-    if world > 1:
-        tmax = torch.tensor([ms], device="cuda")
-        tdist.all_reduce(tmax, op=tdist.ReduceOp.MAX)
-        ms = float(tmax.item())
+    ms = max_over_ranks(e0.elapsed_time(e1), world, "cuda")
     assert int(status.item()) == 0, "device status %d" % int(status.item())
     sec_per = ms * 1e-3 / args.steps
-    tflops = flop / sec_per / 1e12 * world
+    tflops = job_tflops(flop, ms, args.steps, world)
     us = sec_per * 1e6
     peaks, peak_kind = measured_peaks()
     peak_tf = float(peaks["bf16_tflops"])    # FP16 and BF16 share the nominal dense rate
