@@ -148,6 +148,34 @@ nvfp4mla_status nvfp4_sparse_mla_decode(const void *q_nope_f16, const void *q_ro
                                         size_t workspace_bytes, int32_t *dev_status, void *stream);
 
 /*
+ * nvfp4_sparse_mla_decode_noalloc -- nvfp4_sparse_mla_decode without a
+ * caller-supplied workspace.  The pages have no counterpart: this is a
+ * library convenience for callers that cannot hand out device memory per
+ * call -- e.g. a serving engine that gave all free HBM to its paged KV cache
+ * at start-up, or a code path that must not reach a device allocator.  The
+ * split scratch is a static device array of 20 MiB per device (enough for
+ * every plan on a device of up to 148 SMs); a plan that needs more returns
+ * NVFP4MLA_ERR_WORKSPACE.  Nothing is allocated, no allocating library
+ * routine is called.
+ *
+ *   Arguments, layouts and results: as nvfp4_sparse_mla_decode, minus the
+ *   workspace.
+ *   The first call on each device looks the scratch up
+ *   (cudaGetSymbolAddress); make that call before any stream capture.
+ *   The scratch's first 4096 bytes (split counters) start at zero when the
+ *   library loads and every completed call leaves them zero; after a call
+ *   that raised NVFP4MLA_DEV_TIMEOUT this entry point must not be used again
+ *   in the process.
+ *   All calls on one device share the scratch: calls that can overlap in time
+ *   (different streams, or different host threads) race -- use
+ *   nvfp4_sparse_mla_decode with separate workspaces for those.
+ */
+nvfp4mla_status nvfp4_sparse_mla_decode_noalloc(const void *q_nope_f16, const void *q_rope_f16,
+                                                const uint8_t *cache, int64_t num_slots, const int32_t *indices,
+                                                int32_t topk, int32_t T, int32_t H, float sm_scale, void *out_f16,
+                                                float *lse, int32_t *dev_status, void *stream);
+
+/*
  * nvfp4_staged_fp8_staging_size -- bytes of the FP8 staging buffer the
  * staged path writes: T * topk * 576.
  */

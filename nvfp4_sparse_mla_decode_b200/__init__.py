@@ -19,7 +19,7 @@ import torch
 
 __all__ = [
     "ROW_BYTES", "STAGED_ROW_BYTES", "LATENT", "ROPE", "MAX_TOPK", "NVFP4MLAError",
-    "lib", "lib_path", "kv_append", "decode", "staged_decode", "num_splits",
+    "lib", "lib_path", "kv_append", "decode", "decode_noalloc", "staged_decode", "num_splits",
     "workspace_size", "staging_size", "status_string", "version",
     "DEV_TIMEOUT", "DEV_BAD_INDEX", "DEV_LAYOUT",
 ]
@@ -62,6 +62,9 @@ def lib() -> ctypes.CDLL:
         L.nvfp4_sparse_mla_decode.restype = _i32
         L.nvfp4_sparse_mla_decode.argtypes = [_vp, _vp, _vp, _i64, _vp, _i32, _i32, _i32, _f32, _vp, _vp, _vp,
                                               _sz, _vp, _vp]
+        L.nvfp4_sparse_mla_decode_noalloc.restype = _i32
+        L.nvfp4_sparse_mla_decode_noalloc.argtypes = [_vp, _vp, _vp, _i64, _vp, _i32, _i32, _i32, _f32, _vp, _vp,
+                                                      _vp, _vp]
         L.nvfp4_staged_fp8_staging_size.restype = _sz
         L.nvfp4_staged_fp8_staging_size.argtypes = [_i32, _i32]
         L.nvfp4_staged_fp8_mla_decode.restype = _i32
@@ -166,6 +169,21 @@ def decode(q_nope: torch.Tensor, q_rope: torch.Tensor, cache: torch.Tensor, indi
                                        workspace.numel() * workspace.element_size() if workspace is not None else 0,
                                        _ptr(dev_status), _stream(dev))
     _check(st, "nvfp4_sparse_mla_decode")
+    return out, lse
+
+
+def decode_noalloc(q_nope: torch.Tensor, q_rope: torch.Tensor, cache: torch.Tensor, indices: torch.Tensor,
+                   sm_scale: float, out: torch.Tensor, lse: torch.Tensor,
+                   dev_status: Optional[torch.Tensor] = None, num_slots: Optional[int] = None):
+    """decode() without a workspace: the library's static per-device scratch
+    is used, so calls that may overlap in time must not use it.  `out` and
+    `lse` are caller-provided so nothing is allocated on this path."""
+    dev, T, H, topk, out, lse = _decode_args(q_nope, q_rope, cache, indices, out, lse)
+    st = lib().nvfp4_sparse_mla_decode_noalloc(_ptr(q_nope), _ptr(q_rope), _ptr(cache),
+                                               num_slots if num_slots is not None else cache.shape[0],
+                                               _ptr(indices), topk, T, H, float(sm_scale), _ptr(out), _ptr(lse),
+                                               _ptr(dev_status), _stream(dev))
+    _check(st, "nvfp4_sparse_mla_decode_noalloc")
     return out, lse
 
 

@@ -13,6 +13,32 @@ namespace {
 
 bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
+// Scratch of nvfp4_sparse_mla_decode_noalloc: a file-scope device array, one
+// per device, so that entry point never asks for memory.  Every split plan
+// on a device with up to 148 SMs needs at most
+// 4096 + 148 * 64 * (512 + 2) * 4 = 19,478,528 bytes; 20 MiB covers them, and
+// a larger plan is refused.  Device globals are zero when the module loads,
+// which is the state the split counters at its start must begin in.
+constexpr size_t kNoAllocWorkspaceBytes = size_t(20) << 20;
+static_assert(kSplitCounterBytes + size_t(148) * 64 * (NVFP4MLA_LATENT + 2) * 4 <= kNoAllocWorkspaceBytes,
+              "the no-allocation scratch must hold every plan on a 148-SM device");
+static __device__ __align__(256) uint8_t g_noalloc_workspace[kNoAllocWorkspaceBytes];
+
+// Device address of the scratch on `dev`, looked up once per device.
+void *noalloc_workspace(int dev) {
+    static void *addr[64] = {};
+    if (dev < 0 || dev >= 64) return nullptr;
+    if (!addr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_workspace) != cudaSuccess) {
+            (void)cudaGetLastError();
+            return nullptr;
+        }
+        addr[dev] = p;
+    }
+    return addr[dev];
+}
+
 nvfp4mla_status from_cuda(cudaError_t e) { return e == cudaSuccess ? NVFP4MLA_OK : NVFP4MLA_ERR_CUDA; }
 
 // Checks shared by the native and staged decode entry points.
@@ -71,6 +97,27 @@ nvfp4mla_status nvfp4_sparse_mla_decode(const void *q_nope_f16, const void *q_ro
     if (workspace && !aligned(workspace, 256)) return NVFP4MLA_ERR_INVALID_ARG;
     return from_cuda(launch_sparse_mla_decode(false, q_nope_f16, q_rope_f16, cache, num_slots, indices, topk, T, H,
                                               sm_scale, out_f16, lse, workspace, plan, dev_status,
+                                              static_cast<cudaStream_t>(stream)));
+}
+
+nvfp4mla_status nvfp4_sparse_mla_decode_noalloc(const void *q_nope_f16, const void *q_rope_f16,
+                                                const uint8_t *cache, int64_t num_slots, const int32_t *indices,
+                                                int32_t topk, int32_t T, int32_t H, float sm_scale, void *out_f16,
+                                                float *lse, int32_t *dev_status, void *stream) {
+    DecodePlan plan;
+    nvfp4mla_status st =
+        check_decode(q_nope_f16, q_rope_f16, cache, num_slots, indices, topk, T, H, sm_scale, out_f16, lse, &plan);
+    if (st != NVFP4MLA_OK || T == 0) return st;
+    if (plan.workspace_bytes > kNoAllocWorkspaceBytes) return NVFP4MLA_ERR_WORKSPACE;
+    void *ws = nullptr;
+    if (plan.workspace_bytes > 0) {
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess) return NVFP4MLA_ERR_CUDA;
+        ws = noalloc_workspace(dev);
+        if (!ws) return NVFP4MLA_ERR_CUDA;
+    }
+    return from_cuda(launch_sparse_mla_decode(false, q_nope_f16, q_rope_f16, cache, num_slots, indices, topk, T, H,
+                                              sm_scale, out_f16, lse, ws, plan, dev_status,
                                               static_cast<cudaStream_t>(stream)));
 }
 

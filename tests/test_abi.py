@@ -95,3 +95,26 @@ def test_library_is_sm100a_only():
     log = os.path.join(ROOT, "nvfp4_sparse_mla_decode_b200", "build.log")
     if os.path.exists(log):
         assert "arch=compute_100a,code=sm_100a" in open(log).read()
+
+
+def test_noalloc_argument_errors(L):
+    # the same host checks as the workspace entry point, all before any
+    # device call; the largest plan on 148 SMs fits the static scratch
+    INVALID, UNSUP = 1, 2
+    f = L.nvfp4_sparse_mla_decode_noalloc
+
+    def call(**kw):
+        a = dict(q=1 << 20, qr=1 << 20, cache=1 << 20, ns=100, idx=1 << 20, topk=2048, T=1, H=64, sc=0.1,
+                 out=1 << 20, lse=1 << 20, st=None, stream=None)
+        a.update(kw)
+        return f(a["q"], a["qr"], a["cache"], a["ns"], a["idx"], a["topk"], a["T"], a["H"], a["sc"], a["out"],
+                 a["lse"], a["st"], a["stream"])
+
+    assert call(T=0) == 0
+    assert call(q=None) == INVALID
+    assert call(out=(1 << 20) + 4) == INVALID
+    assert call(topk=0) == INVALID
+    assert call(H=48) == UNSUP
+    assert call(sc=float("inf")) == INVALID
+    worst = max(nv.workspace_size(T, H) for T in range(1, 149) for H in (16, 32, 64, 128))
+    assert worst <= 20 << 20
