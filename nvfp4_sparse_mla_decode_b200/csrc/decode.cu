@@ -39,6 +39,8 @@
 //
 // Splits (several CTAs per token) write normalized FP32 partials plus
 // (m, l) to the workspace and a small combine kernel merges them.
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
 #include <cmath>
@@ -100,7 +102,7 @@ constexpr int BAR_CHUNK_FREE = 9;  // [4] output MMAs of a 128-dv block done
 constexpr int BAR_S_FULL = 13;     // score MMAs of a tile done
 constexpr int BAR_P_FULL = 14;     // P^T written (4 softmax warps)
 constexpr int BAR_DRAIN = 15;      // every MMA issued so far done
-constexpr int BAR_Q_FULL = 16;     // Q copies landed (4 warps of the MMA warpgroup)
+constexpr int BAR_Q_FULL = 16;     // Q tensor copies landed (one arrive with the byte count)
 
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColO = 0;      // O^T: 4 blocks of HG columns
@@ -108,11 +110,10 @@ constexpr uint32_t kColS = 256;    // S^T: HG columns
 constexpr float kRescaleThreshold = 8.0f;
 constexpr int kMaxSplits = 16;
 // Merge scratch in the (by then free) tile region: split weights at 0, and
-// at kOffPart the CTA's own partial dv slice (S <= 4) at its place in an
-// [S][HG][512/S] FP32 array (HG x 2 KB).
-constexpr int kOffPart = 16384;
-static_assert((kMaxSplits + 1) * kMaxHG * 4 <= kOffPart, "merge weights must fit below the slices");
-static_assert(kOffPart + kMaxHG * kLatent * 4 <= kTileBytes, "partial slices must fit in the tile region");
+// at kOffOwn the CTA's own partial dv slice (S <= 4: [HG][512/S] FP32).
+constexpr int kOffOwn = 16384;
+static_assert((kMaxSplits + 1) * kMaxHG * 4 <= kOffOwn, "merge weights must fit below the own slice");
+static_assert(kOffOwn + kMaxHG * (kLatent / 2) * 4 <= kTileBytes, "own slice must fit in the tile region");
 }  // namespace dec
 
 // Merge of the S split partials of one (token, head group), run by the 256
@@ -144,7 +145,7 @@ __device__ __forceinline__ void merge_splits(const DecodeArgs &a, int t, int g, 
     uint32_t *flag = reinterpret_cast<uint32_t *>(smem + kOffMisc) + 1;
     float *w_s = reinterpret_cast<float *>(smem);  // [S][HG] weights
     float *inv_den = w_s + kMaxSplits * HG;         // [HG]
-    const float *own = reinterpret_cast<const float *>(smem + kOffPart) + (int64_t)split * HG * D;  // [HG][D]
+    const float *own = reinterpret_cast<const float *>(smem + kOffOwn);  // [HG][D]
     named_bar(3, kMergeThreads);  // every partial store of the group precedes the release
     if (mt == 0) {
         TRACE(280);
@@ -233,7 +234,9 @@ __device__ __forceinline__ void merge_splits(const DecodeArgs &a, int t, int g, 
 }
 
 template <int HG, bool kStaged>
-__global__ void __launch_bounds__(dec::kThreads, 1) sparse_mla_decode_kernel(const DecodeArgs a) {
+__global__ void __launch_bounds__(dec::kThreads, 1)
+    sparse_mla_decode_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_qn,
+                             const __grid_constant__ CUtensorMap tm_qr) {
     using namespace dec;
     extern __shared__ __align__(1024) uint8_t smem[];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -266,7 +269,7 @@ __global__ void __launch_bounds__(dec::kThreads, 1) sparse_mla_decode_kernel(con
         else if (lane < BAR_P_FULL) count = 1;          // MMA commits
         else if (lane == BAR_P_FULL) count = 8;         // 8 softmax warps
         else if (lane == BAR_DRAIN) count = 1;
-        else if (lane == BAR_Q_FULL) count = 4;         // MMA warpgroup
+        else if (lane == BAR_Q_FULL) count = 1;         // thread 0, with the Q byte count
         if (count) mbar_init(&bars[lane], count);
         fence_mbar_init();
     }
@@ -346,22 +349,16 @@ __global__ void __launch_bounds__(dec::kThreads, 1) sparse_mla_decode_kernel(con
     if (warp < 4) {
         regs_dec<RegSplit<HG, kStaged>::mma>();
         // Q of (t, heads g*HG ..) -> shared memory, K-major, 128-byte swizzle:
-        // chunk c holds dims 64c..64c+63 of every head (chunk 8 = RoPE).  The
-        // MMA warpgroup is otherwise idle here, so its 128 threads issue the
-        // 16-byte async copies while the unpack warps start on the rows, and
-        // signal Q_FULL once their own copies have landed.
-        {
-            const int64_t head0 = (int64_t)t * a.H + (int64_t)g * HG;
-            for (int u = tid; u < HG * 72; u += 128) {
-                const int h = u / 72, v = u % 72;
-                const void *src = v < 64 ? static_cast<const void *>(a.q_nope + (head0 + h) * kLatent + 8 * v)
-                                         : static_cast<const void *>(a.q_rope + (head0 + h) * kRope + 8 * (v - 64));
-                cp_async16(smem + kOffQ + (v >> 3) * (HG * 128) + sw128_offset(h, v & 7), src);
-            }
-            cp_async_wait_all();
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bars[BAR_Q_FULL]);
+        // chunk c holds dims 64c..64c+63 of every head (chunk 8 = RoPE).  Nine
+        // tensor copies (box: 64 dims x HG heads, swizzled by the copy engine
+        // into exactly the MMA operand layout), so Q takes no load/store-unit
+        // slots from the row gather.
+        if (tid == 0) {
+            const int32_t row = t * a.H + g * HG;
+            mbar_arrive_expect_tx(&bars[BAR_Q_FULL], (uint32_t)(HG * kDim * 2));
+#pragma unroll 1
+            for (int c = 0; c < 8; ++c) tma_load_2d(smem + kOffQ + c * (HG * 128), &tm_qn, 64 * c, row, &bars[BAR_Q_FULL]);
+            tma_load_2d(smem + kOffQ + 8 * (HG * 128), &tm_qr, 0, row, &bars[BAR_Q_FULL]);
         }
         // ------------------------------------------------------------- MMA
         if (warp == 0 && lane == 0) {
@@ -531,14 +528,8 @@ __global__ void __launch_bounds__(dec::kThreads, 1) sparse_mla_decode_kernel(con
         }
         if (!ok && a.dev_status) atomicOr(a.dev_status, NVFP4MLA_DEV_TIMEOUT);
         // ---------------------------------------------------------- epilogue
-        if (ok && ntiles > 0) {
-            if (!mbar_wait(&bars[BAR_CHUNK_FREE + 3], (ntiles - 1) & 1)) {
-                ok = false;
-                if (a.dev_status) atomicOr(a.dev_status, NVFP4MLA_DEV_TIMEOUT);
-            }
-            tc_fence_after();
-        }
-        if (st == 0 && sw == 0) TRACE(270);
+        // Row sums and the per-head statistics need no TMEM, so they are
+        // done while the last tile's output MMAs still run.
         const bool have = ok && ntiles > 0;
         if (active) {
             // row sums: reduce each head's 128 per-row partials (16 heads at a time)
@@ -567,12 +558,24 @@ __global__ void __launch_bounds__(dec::kThreads, 1) sparse_mla_decode_kernel(con
             }
             named_bar(bar_id, 128);
         }
+        // Output block b is final once the last tile's block-b MMAs are done.
+        auto wait_block = [&](int b) {
+            if (ok && ntiles > 0) {
+                if (!mbar_wait(&bars[BAR_CHUNK_FREE + b], (ntiles - 1) & 1)) {
+                    ok = false;
+                    if (a.dev_status) atomicOr(a.dev_status, NVFP4MLA_DEV_TIMEOUT);
+                }
+                tc_fence_after();
+            }
+        };
+        if (st == 0 && sw == 0) TRACE(270);
         if (st == 0 && sw == 0) TRACE(271);
         const bool leader = (warp == kSoftmaxWarp0 && lane == 0);
         if (a.S == 1) {
             // O^T (TMEM, lanes = dv) -> normalised FP16 rows staged in the
             // (now free) tile region, then one bulk copy of HG x 1 KB to
             // out[t, g*HG .., :].
+            wait_block(3);
             float inv_l[HWG];
 #pragma unroll
             for (int h = 0; h < HWG; ++h) inv_l[h] = active ? aux_s[h0 + h] : 0.0f;
@@ -601,26 +604,29 @@ __global__ void __launch_bounds__(dec::kThreads, 1) sparse_mla_decode_kernel(con
                 bulk_s2g(a.out + ((int64_t)t * a.H + (int64_t)g * HG) * kLatent, stage, HG * kLatent * 2);
                 bulk_commit_wait_read();
             }
-        } else if (active) {
+        } else {
             // Unnormalised partial O (this split's rows, scaled to its own
-            // reference max), two 128-dv blocks per TMEM round trip.  Blocks
-            // inside this CTA's own merge slice (S <= 4) go straight to their
-            // place in shared memory; the rest go to the workspace from registers
-            // (for each head a warp writes 32 consecutive dv, one 128-byte
-            // segment).  The block barrier and release in the merge order
-            // these stores ahead of the arrival.
+            // reference max), up to two 128-dv blocks per TMEM round trip.
+            // Blocks 0-1 that go to the workspace leave as soon as they are
+            // final, while blocks 2-3 are still being accumulated; the rest
+            // follow once everything is done.  Blocks inside this CTA's own
+            // merge slice (S <= 4) go to shared memory at kOffOwn (the tile
+            // is no longer read by then); the others go to the workspace
+            // straight from registers (for each head a warp writes 32
+            // consecutive dv, one 128-byte segment).  The softmax-group
+            // barrier and the release in the merge order these stores ahead
+            // of the arrival.
             float *dst = a.ws_o + (((int64_t)t * a.S + split) * a.H + (int64_t)g * HG + h0) * kLatent + st;
             const int own_n = a.S <= 4 ? 4 / a.S : 0;  // 128-dv blocks in the own slice
             const int own_dc0 = split * own_n;
             const int own_d = kLatent / a.S;
-            // own slice: its place [split][h][own_d] among the merge's slices
-            float *own = reinterpret_cast<float *>(smem + kOffPart) + (int64_t)split * HG * own_d;
-#pragma unroll 1
-            for (int dc = 0; dc < 4; dc += 2) {
+            float *own = reinterpret_cast<float *>(smem + kOffOwn) + (int64_t)h0 * own_d + st;
+            auto is_own = [&](int b) { return b >= own_dc0 && b < own_dc0 + own_n; };
+            auto drain = [&](int b0, int b1) {  // b1 < 0: one block
                 uint32_t r[2][HWG];
                 if (have) {
-                    tmem_ld_cols<HWG>(tmem + lane_base + kColO + dc * HG + h0, r[0]);
-                    tmem_ld_cols<HWG>(tmem + lane_base + kColO + (dc + 1) * HG + h0, r[1]);
+                    tmem_ld_cols<HWG>(tmem + lane_base + kColO + b0 * HG + h0, r[0]);
+                    if (b1 >= 0) tmem_ld_cols<HWG>(tmem + lane_base + kColO + b1 * HG + h0, r[1]);
                     tmem_ld_wait();
                 } else {
 #pragma unroll
@@ -628,16 +634,36 @@ __global__ void __launch_bounds__(dec::kThreads, 1) sparse_mla_decode_kernel(con
                 }
 #pragma unroll
                 for (int j = 0; j < 2; ++j) {
-                    const int b = dc + j;
-                    if (b >= own_dc0 && b < own_dc0 + own_n) {
-                        float *o = own + (int64_t)h0 * own_d + 128 * (b - own_dc0) + st;
+                    const int b = j == 0 ? b0 : b1;
+                    if (b < 0) continue;
+                    if (is_own(b)) {
 #pragma unroll
-                        for (int h = 0; h < HWG; ++h) o[h * own_d] = __uint_as_float(r[j][h]);
+                        for (int h = 0; h < HWG; ++h) own[h * own_d + 128 * (b - own_dc0)] = __uint_as_float(r[j][h]);
                     } else {
 #pragma unroll
                         for (int h = 0; h < HWG; ++h)
                             __stcg(dst + (int64_t)h * kLatent + 128 * b, __uint_as_float(r[j][h]));
                     }
+                }
+            };
+            wait_block(1);
+            if (active) {
+                const bool g0 = !is_own(0), g1 = !is_own(1);
+                if (g0 && g1) drain(0, 1);
+                else if (g0) drain(0, -1);
+                else if (g1) drain(1, -1);
+            }
+            wait_block(3);
+            if (active) {  // blocks 2-3 and any own block among 0-1
+                const bool o0 = is_own(0), o1 = is_own(1);
+                if (o0 && o1) {
+                    drain(0, 1);
+                    drain(2, 3);
+                } else if (o0 || o1) {
+                    drain(o0 ? 0 : 1, 2);
+                    drain(3, -1);
+                } else {
+                    drain(2, 3);
                 }
             }
         }
@@ -812,6 +838,35 @@ bool make_decode_plan(int32_t T, int32_t H, int32_t topk, int sm_count, DecodePl
     return true;
 }
 
+// Tensor maps for Q: a 2-D FP16 view [rows = T*H, cols] of q_nope (cols 512)
+// or q_rope (cols 64), box 64 cols x HG rows, 128-byte swizzle.
+static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess || !p) {
+            (void)cudaGetLastError();
+            return nullptr;
+        }
+        fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }
+    return fn;
+}
+
+static bool make_q_map(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    const cuuint64_t dims[2] = {cols, rows};
+    const cuuint64_t strides[1] = {cols * 2};
+    const cuuint32_t box[2] = {64, box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <int HG, bool kStaged>
 static cudaError_t launch_hg(const DecodeArgs &a, int64_t nblocks, cudaStream_t stream) {
     auto kern = sparse_mla_decode_kernel<HG, kStaged>;
@@ -843,7 +898,11 @@ static cudaError_t launch_hg(const DecodeArgs &a, int64_t nblocks, cudaStream_t 
     attr[0].val.cooperative = 1;
     cfg.attrs = attr;
     cfg.numAttrs = a.S > 1 ? 1 : 0;
-    return cudaLaunchKernelEx(&cfg, kern, a);
+    CUtensorMap tm_qn, tm_qr;
+    const uint64_t rows = (uint64_t)a.T * (uint64_t)a.H;
+    if (!make_q_map(&tm_qn, a.q_nope, rows, kLatent, HG) || !make_q_map(&tm_qr, a.q_rope, rows, kRope, HG))
+        return cudaErrorInvalidValue;
+    return cudaLaunchKernelEx(&cfg, kern, a, tm_qn, tm_qr);
 }
 
 cudaError_t launch_sparse_mla_decode(bool staged, const void *q_nope, const void *q_rope, const uint8_t *src,

@@ -91,6 +91,18 @@ __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t by
         : "memory");
 }
 
+// Tiled 2-D tensor copy global -> this CTA's shared memory through a tensor
+// map passed as a __grid_constant__ kernel parameter, completing its bytes
+// on `bar`.  x is the innermost coordinate in elements; x * element size must
+// be a multiple of 16 bytes.
+__device__ __forceinline__ void tma_load_2d(void *dst, const void *tmap, int32_t x, int32_t y, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+            smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(smem_u32(bar))
+        : "memory");
+}
+
 // 16-byte asynchronous copy global -> shared (no register staging); the
 // copies of a thread complete at cp_async_wait_all().
 __device__ __forceinline__ void cp_async16(void *dst, const void *src) {
