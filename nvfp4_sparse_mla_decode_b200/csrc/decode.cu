@@ -82,16 +82,16 @@ constexpr int kUnpackWarp0 = 12;
 // holds kRegsLaunch registers (65536 / 640 rounded down to a multiple of 8);
 // a role may only decrease below it with .dec and increase above it with .inc,
 // and the new total must fit in what the block was launched with.  The split
-// depends on the instantiation: 64 heads per CTA keep 32 per-head values per
-// softmax thread, and the staged source keeps 18 raw words per row in the
-// unpack warps instead of 11 (chosen so ptxas reports no spills, or the
-// fewest).
+// depends on the instantiation: with 64 heads per CTA a softmax thread keeps
+// 32 per-head values and two 32-column output blocks at once, while the
+// unpack warps hold a tile's raw words plus the next tile's row slots
+// (chosen by measurement among the splits with the fewest spills).
 constexpr int kRegsLaunch = 96;
 template <int HG, bool kStaged>
 struct RegSplit {
     static constexpr int mma = 40;                                         // warpgroup 0 (.dec)
-    static constexpr int softmax = HG == 64 ? (kStaged ? 136 : 144) : 128;  // warpgroups 1-2 (.inc)
-    static constexpr int unpack = HG == 64 ? (kStaged ? 80 : 72) : 88;      // warpgroups 3-4 (.dec)
+    static constexpr int softmax = HG == 64 ? 136 : 128;  // warpgroups 1-2 (.inc)
+    static constexpr int unpack = HG == 64 ? 80 : 88;      // warpgroups 3-4 (.dec)
     static_assert(mma < kRegsLaunch && unpack < kRegsLaunch && softmax > kRegsLaunch, "setmaxnreg direction");
     static_assert(mma % 8 == 0 && softmax % 8 == 0 && unpack % 8 == 0, "setmaxnreg granularity");
     static_assert(128 * mma + 256 * softmax + 256 * unpack <= 640 * kRegsLaunch, "register budget");
@@ -684,53 +684,68 @@ __global__ void __launch_bounds__(dec::kThreads, 1)
         const int ut = tid - 32 * kUnpackWarp0;
         const int sub = ut & 7;   // 8-dim slice of every 64-dim chunk
         const int rg = ut >> 3;   // rows rg, rg+32, rg+64, rg+96 of each tile
-        const uint8_t *row_ptr[4];
-        bool rvalid[4];
         constexpr int kWords = kStaged ? 18 : 11;  // raw 32-bit words per row held per tile
         uint32_t raw[4][kWords];
-        // Loads of a tile's rows, issued in the order the chunks consume
-        // them (scales first, then chunk by chunk, RoPE last) so chunk 0
-        // does not wait for the whole tile.  Rows past the end are not read
-        // and stay zero.
-        auto load_tile = [&](int i) {
+        int32_t slot[4];  // rows of the tile whose words are being loaded
+        bool rvalid[4];
+        // Row loads come in groups, in the order the pairs consume them:
+        // group p < 4 = chunks 2p and 2p+1, group 4 = RoPE, and for NVFP4
+        // rows group 5 = the 32 scales.  Rows past the end are not read and
+        // stay zero.
+        auto set_rows = [&](int i) {
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
                 const int e = kTileRows * i + rg + 32 * k;
                 rvalid[k] = e < n_mine;
-                const int32_t v = rvalid[k] ? idx_s[e] : 0;
-                if (kStaged)
-                    row_ptr[k] = a.src + ((int64_t)t * a.topk + v) * kStagedRowBytes;
-                else
-                    row_ptr[k] = a.src + (int64_t)v * kRowBytes;
+                slot[k] = rvalid[k] ? idx_s[e] : 0;
             }
-            if (kStaged) {
+        };
+        auto row_base = [&](int k) -> const uint8_t * {
+            return kStaged ? a.src + ((int64_t)t * a.topk + slot[k]) * kStagedRowBytes
+                           : a.src + (int64_t)slot[k] * kRowBytes;
+        };
+        auto load_group = [&](int grp) {
 #pragma unroll
-                for (int c = 0; c < kChunks; ++c) {
+            for (int k = 0; k < 4; ++k) {
+                const uint8_t *rp = row_base(k);
+                if (kStaged) {
+                    if (grp < 4) {
 #pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        const uint2 w2 = rvalid[k] ? ldg64(row_ptr[k] + 64 * c + 8 * sub) : make_uint2(0u, 0u);
-                        raw[k][2 * c] = w2.x;
-                        raw[k][2 * c + 1] = w2.y;
+                        for (int j = 0; j < 2; ++j) {
+                            const int c = 2 * grp + j;
+                            const uint2 w2 = rvalid[k] ? ldg64(rp + 64 * c + 8 * sub) : make_uint2(0u, 0u);
+                            raw[k][2 * c] = w2.x;
+                            raw[k][2 * c + 1] = w2.y;
+                        }
+                    } else if (grp == 4) {
+                        const uint2 w2 = rvalid[k] ? ldg64(rp + 64 * 8 + 8 * sub) : make_uint2(0u, 0u);
+                        raw[k][16] = w2.x;
+                        raw[k][17] = w2.y;
                     }
-                }
-            } else {
+                } else {
+                    if (grp < 4) {
 #pragma unroll
-                for (int k = 0; k < 4; ++k) raw[k][8] = rvalid[k] ? ldg32(row_ptr[k] + kScaleOff + 4 * sub) : 0u;
-#pragma unroll
-                for (int c = 0; c < 8; ++c) {
-#pragma unroll
-                    for (int k = 0; k < 4; ++k) raw[k][c] = rvalid[k] ? ldg32(row_ptr[k] + 32 * c + 4 * sub) : 0u;
-                }
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const uint2 rp = rvalid[k] ? ldg64(row_ptr[k] + kRopeOff + 8 * sub) : make_uint2(0u, 0u);
-                    raw[k][9] = rp.x;
-                    raw[k][10] = rp.y;
+                        for (int j = 0; j < 2; ++j) {
+                            const int c = 2 * grp + j;
+                            raw[k][c] = rvalid[k] ? ldg32(rp + 32 * c + 4 * sub) : 0u;
+                        }
+                    } else if (grp == 4) {
+                        const uint2 w2 = rvalid[k] ? ldg64(rp + kRopeOff + 8 * sub) : make_uint2(0u, 0u);
+                        raw[k][9] = w2.x;
+                        raw[k][10] = w2.y;
+                    } else {
+                        raw[k][8] = rvalid[k] ? ldg32(rp + kScaleOff + 4 * sub) : 0u;
+                    }
                 }
             }
         };
         bool ok = true;
-        if (ntiles > 0) load_tile(0);
+        if (ntiles > 0) {
+            set_rows(0);
+            load_group(5);
+#pragma unroll
+            for (int grp = 0; grp < 5; ++grp) load_group(grp);
+        }
         if (ut == 0) TRACE(277);
         // Decode chunk c of this thread's 4 rows into the swizzled tile.
         auto unpack_chunk = [&](int c) {
@@ -754,9 +769,13 @@ __global__ void __launch_bounds__(dec::kThreads, 1)
             }
         };
         for (int i = 0; i < ntiles && ok; ++i) {
+            const bool more = i + 1 < ntiles;
             // Chunks 2p and 2p+1 are released together by output block p, so
             // they are written as a pair behind one wait and one fence; the
-            // RoPE chunk (8, where P^T lives) was released by block 3.
+            // RoPE chunk (8, where P^T lives) was released by block 3.  As
+            // soon as a pair's words are decoded, the same registers start
+            // loading that pair of the next tile, so the gather of tile i+1
+            // is spread over the unpack of tile i.
 #pragma unroll
             for (int p = 0; p < 5; ++p) {
                 if (p < 4 && i > 0 && !mbar_wait(&bars[BAR_CHUNK_FREE + p], (i - 1) & 1)) {
@@ -778,9 +797,13 @@ __global__ void __launch_bounds__(dec::kThreads, 1)
                 }
                 if (ut == 0 && i == 1) TRACE(96 + p);
                 if (lane == 0 && i == 1) TRACE(128 + 16 * (ut >> 5) + p);
+                if (more) {
+                    if (p == 0) set_rows(i + 1);
+                    load_group(p);
+                    if (p == 3 && !kStaged) load_group(5);  // scales: last used by pair 3
+                }
             }
             if (ut == 0 && i < 8) TRACE(6 + 6 * i);
-            if (ok && i + 1 < ntiles) load_tile(i + 1);
         }
         if (ut == 0) TRACE(62);
         if (!ok && a.dev_status) atomicOr(a.dev_status, NVFP4MLA_DEV_TIMEOUT);
@@ -855,16 +878,39 @@ static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
     return fn;
 }
 
+// Encoded maps are kept in a small per-thread cache keyed by (address, rows,
+// cols, box rows), so a caller that reuses its query buffers pays for the
+// encoding once.
 static bool make_q_map(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+    struct Entry {
+        const void *base;
+        uint64_t rows, cols;
+        uint32_t box_rows;
+        CUtensorMap map;
+    };
+    constexpr int kEntries = 16;
+    thread_local Entry cache[kEntries] = {};
+    thread_local int next = 0;
+    for (int i = 0; i < kEntries; ++i) {
+        const Entry &e = cache[i];
+        if (e.base == base && e.rows == rows && e.cols == cols && e.box_rows == box_rows) {
+            *m = e.map;
+            return true;
+        }
+    }
     auto enc = tensor_map_encoder();
     if (!enc) return false;
     const cuuint64_t dims[2] = {cols, rows};
     const cuuint64_t strides[1] = {cols * 2};
     const cuuint32_t box[2] = {64, box_rows};
     const cuuint32_t estr[2] = {1, 1};
-    return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
-               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
-               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    if (enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return false;
+    cache[next] = Entry{base, rows, cols, box_rows, *m};
+    next = (next + 1) % kEntries;
+    return true;
 }
 
 template <int HG, bool kStaged>
