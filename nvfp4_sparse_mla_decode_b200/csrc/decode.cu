@@ -138,8 +138,12 @@ __device__ __forceinline__ void merge_splits(const DecodeArgs &a, int t, int g, 
     constexpr int D = kLatent / S;           // dv per CTA
     constexpr int NQ = D / 4;                // float4 per head
     constexpr int ITEMS = HG * NQ;
-    constexpr int B = S >= 16 ? 1 : 16 / S;  // items per batch: B * S vectors in flight per thread
     constexpr bool kOwnInSmem = S <= 4;
+    // items per batch: up to 24 global vectors in flight per thread (the own
+    // slice is read from shared memory when it is combined)
+    constexpr int kGlobal = kOwnInSmem ? S - 1 : S;
+    constexpr int kPerThread = (ITEMS + kMergeThreads - 1) / kMergeThreads;
+    constexpr int B = (24 / kGlobal) < 1 ? 1 : ((24 / kGlobal) > kPerThread ? kPerThread : (24 / kGlobal));
     uint32_t *arrive = a.counters + 2 * ((int64_t)t * a.G + g);
     uint32_t *depart = arrive + 1;
     uint32_t *flag = reinterpret_cast<uint32_t *>(smem + kOffMisc) + 1;
@@ -186,19 +190,17 @@ __device__ __forceinline__ void merge_splits(const DecodeArgs &a, int t, int g, 
     const float *src = a.ws_o + ((int64_t)t * S * a.H + (int64_t)g * HG) * kLatent + dv0;
     __half *dst = a.out + ((int64_t)t * a.H + (int64_t)g * HG) * kLatent + dv0;
     for (int base = mt; base < ITEMS; base += kMergeThreads * B) {
-        float4 o[B][S];
+        float4 o[B][kGlobal];  // the foreign partials (all S when the own slice is not in shared memory)
 #pragma unroll
         for (int b = 0; b < B; ++b) {
             const int item = base + b * kMergeThreads;
             const int h = item / NQ, q = item - h * NQ;
 #pragma unroll
-            for (int s = 0; s < S; ++s) {
-                if (item >= ITEMS)
-                    o[b][s] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-                else if (kOwnInSmem && s == split)
-                    o[b][s] = *reinterpret_cast<const float4 *>(own + h * D + 4 * q);
-                else
-                    o[b][s] = __ldcg(reinterpret_cast<const float4 *>(src + (int64_t)h * kLatent + 4 * q + s * part));
+            for (int j = 0; j < kGlobal; ++j) {
+                const int s = kOwnInSmem && j >= split ? j + 1 : j;
+                o[b][j] = item < ITEMS
+                              ? __ldcg(reinterpret_cast<const float4 *>(src + (int64_t)h * kLatent + 4 * q + s * part))
+                              : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
             }
         }
 #pragma unroll
@@ -207,13 +209,22 @@ __device__ __forceinline__ void merge_splits(const DecodeArgs &a, int t, int g, 
             if (item < ITEMS) {
                 const int h = item / NQ, q = item - h * NQ;
                 float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+                if (kOwnInSmem) {
+                    const float w = w_s[split * HG + h];
+                    const float4 v = *reinterpret_cast<const float4 *>(own + h * D + 4 * q);
+                    acc.x = w * v.x;
+                    acc.y = w * v.y;
+                    acc.z = w * v.z;
+                    acc.w = w * v.w;
+                }
 #pragma unroll
-                for (int s = 0; s < S; ++s) {  // an empty split's partial is zero and its weight 0
+                for (int j = 0; j < kGlobal; ++j) {  // an empty split's partial is zero and its weight 0
+                    const int s = kOwnInSmem && j >= split ? j + 1 : j;
                     const float w = w_s[s * HG + h];
-                    acc.x += w * o[b][s].x;
-                    acc.y += w * o[b][s].y;
-                    acc.z += w * o[b][s].z;
-                    acc.w += w * o[b][s].w;
+                    acc.x += w * o[b][j].x;
+                    acc.y += w * o[b][j].y;
+                    acc.z += w * o[b][j].z;
+                    acc.w += w * o[b][j].w;
                 }
                 const float r = inv_den[h];
                 __half2 *d2 = reinterpret_cast<__half2 *>(dst + (int64_t)h * kLatent + 4 * q);
