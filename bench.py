@@ -42,6 +42,8 @@ def parse():
     ap.add_argument("--warmup", type=int, default=50)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-extras", action="store_true", help="skip staged/append/e2e/cpu legs")
+    ap.add_argument("--launch", default="graph", choices=["graph", "stream"],
+                    help="time the K launches replayed from a captured CUDA graph (default) or issued one by one")
     return ap.parse_args()
 
 
@@ -271,6 +273,29 @@ def main():
         step(k)
     torch.cuda.synchronize()
 
+    # The K timed launches: a CUDA graph holding one launch per rotating set,
+    # replayed K // N_SETS times, then the K % N_SETS remaining launches --
+    # exactly K launches of the same kernel on the same stream.
+    graph = None
+    if args.launch == "graph":
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            for k in range(N_SETS):
+                step(k)
+        graph.replay()
+        torch.cuda.synchronize()
+        stream = torch.cuda.current_stream()
+
+    def timed_launches(n):
+        if graph is None:
+            for k in range(n):
+                step(k)
+            return
+        for _ in range(n // N_SETS):
+            graph.replay()
+        for k in range(n % N_SETS):
+            step(k)
+
     sampler = ClockSampler(torch.cuda.current_device())
     sampler.start()
     time.sleep(0.05)
@@ -280,8 +305,7 @@ def main():
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     h0 = time.perf_counter()
     e0.record(stream)
-    for k in range(args.steps):
-        step(k)
+    timed_launches(args.steps)
     e1.record(stream)
     torch.cuda.synchronize()
     h1 = time.perf_counter()
@@ -298,6 +322,15 @@ def main():
     peak_bw = float(peaks["hbm_gbs"])
     t_roof = max(flop / (peak_tf * 1e12), alg_bytes / (peak_bw * 1e9))
     clocks = sampler.summary(h0, h1)
+    # for reference: the same launches issued one by one from the host
+    n_stream = min(args.steps, 2000)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for k in range(n_stream):
+        step(k)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    stream_us = e0.elapsed_time(e1) * 1e3 / n_stream
 
     line = {
         "metric": METRIC, "value": tflops, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
@@ -307,8 +340,10 @@ def main():
                    "cache_rows": w.num_slots, "valid_rows_per_launch": rows, "splits": nv.num_splits(T, H, topk),
                    "l2": "inputs larger than L2: %d rotating index/query sets, %.0f MB gathered per cycle > %d MB L2"
                          % (N_SETS, N_SETS * rows * ROW_BYTES / 1e6, L2_BYTES >> 20),
-                   "parallelism": "replicas" if world > 1 else "single"},
+                   "parallelism": "replicas" if world > 1 else "single",
+                   "launch": "cuda_graph" if graph is not None else "stream"},
         "us_per_launch": us,
+        "us_per_launch_stream_issued": stream_us,
         "gathered_gbs": rows * ROW_BYTES / sec_per / 1e9,
         "alg_bytes_per_launch": alg_bytes, "alg_flop_per_launch": flop,
         "roofline": {"bound": "tensor", "achieved": flop / sec_per / 1e12, "peak": peak_tf, "unit": "TFLOP/s",
