@@ -201,6 +201,16 @@ nvfp4mla_status nvfp4_staged_fp8_mla_decode(const void *q_nope_f16, const void *
                                             size_t workspace_bytes, int32_t *dev_status, void *stream);
 
 /* Human-readable name of a status code (static storage). */
+/*
+ * nvfp4mla_selftest_wait_timeout -- checks, on the device, that the bounded
+ * waits every kernel here uses end with a status instead of hanging: one CTA
+ * waits on an mbarrier nothing arrives on and on *zero_word (which must stay
+ * 0) reaching 1, each for about a millisecond, then ORs
+ * NVFP4MLA_DEV_TIMEOUT into *dev_status and exits normally.  The context
+ * stays usable.  Both pointers are device pointers owned by the caller.
+ */
+nvfp4mla_status nvfp4mla_selftest_wait_timeout(uint32_t *zero_word, int32_t *dev_status, void *stream);
+
 const char *nvfp4mla_status_string(nvfp4mla_status status);
 
 /* Library ABI version: major*10000 + minor*100 + patch. */

@@ -70,6 +70,8 @@ def lib() -> ctypes.CDLL:
         L.nvfp4_staged_fp8_mla_decode.restype = _i32
         L.nvfp4_staged_fp8_mla_decode.argtypes = [_vp, _vp, _vp, _i64, _vp, _i32, _i32, _i32, _f32, _vp, _vp,
                                                   _vp, _sz, _vp, _sz, _vp, _vp]
+        L.nvfp4mla_selftest_wait_timeout.restype = _i32
+        L.nvfp4mla_selftest_wait_timeout.argtypes = [_vp, _vp, _vp]
         L.nvfp4mla_status_string.restype = ctypes.c_char_p
         L.nvfp4mla_status_string.argtypes = [_i32]
         L.nvfp4mla_version.restype = _i32
@@ -205,6 +207,17 @@ def staged_decode(q_nope: torch.Tensor, q_rope: torch.Tensor, cache: torch.Tenso
                                            _ptr(dev_status), _stream(dev))
     _check(st, "nvfp4_staged_fp8_mla_decode")
     return out, lse
+
+
+def selftest_wait_timeout(device="cuda") -> int:
+    """Run the bounded-wait self-test; returns the device status word it set
+    (NVFP4MLA_DEV_TIMEOUT when the waits ended as designed)."""
+    zero = torch.zeros(1, dtype=torch.int32, device=device)
+    status = torch.zeros(1, dtype=torch.int32, device=device)
+    _check(lib().nvfp4mla_selftest_wait_timeout(_ptr(zero), _ptr(status), _stream(zero.device)),
+           "nvfp4mla_selftest_wait_timeout")
+    torch.cuda.synchronize(zero.device)
+    return int(status.item())
 
 
 def default_sm_scale() -> float:

@@ -146,6 +146,12 @@ nvfp4mla_status nvfp4_staged_fp8_mla_decode(const void *q_nope_f16, const void *
                                               sm_scale, out_f16, lse, workspace, plan, dev_status, s));
 }
 
+nvfp4mla_status nvfp4mla_selftest_wait_timeout(uint32_t *zero_word, int32_t *dev_status, void *stream) {
+    if (!zero_word || !dev_status || !aligned(zero_word, 4) || !aligned(dev_status, 4))
+        return NVFP4MLA_ERR_INVALID_ARG;
+    return from_cuda(launch_wait_timeout_selftest(zero_word, dev_status, static_cast<cudaStream_t>(stream)));
+}
+
 const char *nvfp4mla_status_string(nvfp4mla_status status) {
     switch (status) {
         case NVFP4MLA_OK: return "ok";

@@ -162,35 +162,12 @@ __device__ __forceinline__ void merge_splits(const DecodeArgs &a, int t, int g, 
     }
     named_bar(3, kMergeThreads);
     if (!*flag) return;  // counters stay raised: the caller must clear them after a timeout
-    if (mt < HG) {
-        const float *ml = a.ws_ml + 2 * ((int64_t)t * S * a.H + (int64_t)g * HG + mt);
-        float2 v[S];
-#pragma unroll
-        for (int s = 0; s < S; ++s) v[s] = __ldcg(reinterpret_cast<const float2 *>(ml + 2 * (int64_t)s * a.H));
-        float mmax = -INFINITY;
-#pragma unroll
-        for (int s = 0; s < S; ++s)
-            if (v[s].y > 0.0f) mmax = fmaxf(mmax, v[s].x);
-        float den = 0.0f;
-#pragma unroll
-        for (int s = 0; s < S; ++s) {
-            const float w = v[s].y > 0.0f ? ex2(v[s].x - mmax) : 0.0f;
-            w_s[s * HG + mt] = w;
-            den += w * v[s].y;
-        }
-        inv_den[mt] = den > 0.0f ? 1.0f / den : 0.0f;
-        if (split == 0)
-            a.lse[(int64_t)t * a.H + (int64_t)g * HG + mt] =
-                den > 0.0f ? (mmax + lg2(den)) * 0.69314718055994531f : -INFINITY;
-    }
-    named_bar(3, kMergeThreads);
-    if (mt == 0) TRACE(282);
     const int dv0 = split * D;
     const int64_t part = (int64_t)a.H * kLatent;  // next split of the same (t, head)
     const float *src = a.ws_o + ((int64_t)t * S * a.H + (int64_t)g * HG) * kLatent + dv0;
     __half *dst = a.out + ((int64_t)t * a.H + (int64_t)g * HG) * kLatent + dv0;
-    for (int base = mt; base < ITEMS; base += kMergeThreads * B) {
-        float4 o[B][kGlobal];  // the foreign partials (all S when the own slice is not in shared memory)
+    float4 o[B][kGlobal];  // the foreign partials (all S when the own slice is not in shared memory)
+    auto load_batch = [&](int base) {
 #pragma unroll
         for (int b = 0; b < B; ++b) {
             const int item = base + b * kMergeThreads;
@@ -203,6 +180,8 @@ __device__ __forceinline__ void merge_splits(const DecodeArgs &a, int t, int g, 
                               : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
             }
         }
+    };
+    auto combine_batch = [&](int base) {
 #pragma unroll
         for (int b = 0; b < B; ++b) {
             const int item = base + b * kMergeThreads;
@@ -232,6 +211,37 @@ __device__ __forceinline__ void merge_splits(const DecodeArgs &a, int t, int g, 
                 d2[1] = __floats2half2_rn(acc.z * r, acc.w * r);
             }
         }
+    };
+    // The first batch of partial loads is in flight while the weights are
+    // computed from the statistics.
+    load_batch(mt);
+    if (mt < HG) {
+        const float *ml = a.ws_ml + 2 * ((int64_t)t * S * a.H + (int64_t)g * HG + mt);
+        float2 v[S];
+#pragma unroll
+        for (int s = 0; s < S; ++s) v[s] = __ldcg(reinterpret_cast<const float2 *>(ml + 2 * (int64_t)s * a.H));
+        float mmax = -INFINITY;
+#pragma unroll
+        for (int s = 0; s < S; ++s)
+            if (v[s].y > 0.0f) mmax = fmaxf(mmax, v[s].x);
+        float den = 0.0f;
+#pragma unroll
+        for (int s = 0; s < S; ++s) {
+            const float w = v[s].y > 0.0f ? ex2(v[s].x - mmax) : 0.0f;
+            w_s[s * HG + mt] = w;
+            den += w * v[s].y;
+        }
+        inv_den[mt] = den > 0.0f ? 1.0f / den : 0.0f;
+        if (split == 0)
+            a.lse[(int64_t)t * a.H + (int64_t)g * HG + mt] =
+                den > 0.0f ? (mmax + lg2(den)) * 0.69314718055994531f : -INFINITY;
+    }
+    named_bar(3, kMergeThreads);
+    if (mt == 0) TRACE(282);
+    combine_batch(mt);
+    for (int base = mt + kMergeThreads * B; base < ITEMS; base += kMergeThreads * B) {
+        load_batch(base);
+        combine_batch(base);
     }
     named_bar(3, kMergeThreads);
     if (mt == 0) {

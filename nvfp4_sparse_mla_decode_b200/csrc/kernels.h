@@ -41,4 +41,8 @@ cudaError_t launch_sparse_mla_decode(bool staged, const void *q_nope, const void
 cudaError_t launch_stage_fp8(const uint8_t *cache, int64_t num_slots, const int32_t *indices, int32_t topk,
                              int32_t T, uint8_t *staging, cudaStream_t stream);
 
+// Bounded-wait self-test: a single CTA whose two waits run out (~1 ms each);
+// `counter` must point at a zero uint32 in device memory.
+cudaError_t launch_wait_timeout_selftest(uint32_t *counter, int32_t *dev_status, cudaStream_t stream);
+
 }  // namespace nvfp4mla

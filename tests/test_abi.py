@@ -118,3 +118,10 @@ def test_noalloc_argument_errors(L):
     assert call(sc=float("inf")) == INVALID
     worst = max(nv.workspace_size(T, H) for T in range(1, 149) for H in (16, 32, 64, 128))
     assert worst <= 20 << 20
+
+
+def test_selftest_argument_errors(L):
+    f = L.nvfp4mla_selftest_wait_timeout
+    assert f(None, 1 << 20, None) == 1
+    assert f(1 << 20, None, None) == 1
+    assert f((1 << 20) + 2, 1 << 20, None) == 1
