@@ -54,6 +54,7 @@ namespace nvfp4mla {
 using namespace ptx;
 #ifdef NVFP4MLA_TRACE
 void set_trace_buffer(unsigned long long *p) { set_trace_local(p); }
+void set_trace_all_buffer(unsigned long long *p) { set_trace_all_local(p); }
 #endif
 
 namespace dec {
@@ -263,6 +264,10 @@ __global__ void __launch_bounds__(dec::kThreads, 1)
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 #ifdef NVFP4MLA_TRACE
     const unsigned long long t_start = clock64();
+    if (tid == 0 && g_trace_all) {
+        g_trace_all[3 * blockIdx.x] = global_ns();
+        g_trace_all[3 * blockIdx.x + 2] = sm_id();
+    }
 #else
     const unsigned long long t_start = 0;  // timestamps exist only in trace builds
 #endif
@@ -837,6 +842,9 @@ __global__ void __launch_bounds__(dec::kThreads, 1)
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
     }
+#ifdef NVFP4MLA_TRACE
+    if (tid == 0 && g_trace_all) g_trace_all[3 * blockIdx.x + 1] = global_ns();
+#endif
 }
 
 int current_device_sm_count() {

@@ -36,6 +36,20 @@ static __device__ unsigned long long *g_trace;
         if (g_trace && blockIdx.x < 16) g_trace[blockIdx.x * 512 + (slot)] = clock64() - t_start; \
     } while (0)
 static inline void set_trace_local(unsigned long long *p) { cudaMemcpyToSymbol(g_trace, &p, sizeof(p)); }
+// Every CTA: [start ns, end ns, SM id] from the global timer (comparable
+// across SMs, unlike clock64).
+static __device__ unsigned long long *g_trace_all;
+static inline void set_trace_all_local(unsigned long long *p) { cudaMemcpyToSymbol(g_trace_all, &p, sizeof(p)); }
+__device__ __forceinline__ unsigned long long global_ns() {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+__device__ __forceinline__ unsigned sm_id() {
+    unsigned r;
+    asm volatile("mov.u32 %0, %%smid;" : "=r"(r));
+    return r;
+}
 #else
 #define TRACE(slot) \
     do {            \
