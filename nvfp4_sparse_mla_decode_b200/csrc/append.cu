@@ -2,8 +2,8 @@
 // rows at scattered cache slots.
 //
 // Page "Prime Intellect Launches Prime Inference, Serving 600B Tokens Daily",
-// section "Four-bit caches make room": NVFP4 stores one FP8 scale per group of
-// 16 values and the cache row shrinks to 352 bytes.  Per group of 16 latent
+// section "Four-bit caches make room": NVFP4 keeps an FP8 scale for every 16
+// values and the cache row becomes 352 bytes.  Per group of 16 latent
 // values: scale = E4M3_RNE_sat(max|x| / 6), value codes = E2M1_RNE_sat(x /
 // scale) (all zero when the scale is 0); RoPE dims are E4M3_RNE_sat(x).
 //
