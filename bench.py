@@ -137,16 +137,26 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(inside), "note": note}
 
 
+def code_fingerprint(path: str) -> str:
+    """sha256 of a C/CUDA source with comments and whitespace removed, so a
+    comment edit keeps the fingerprint and any code change alters it."""
+    import re
+    src = open(path, encoding="utf-8").read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    src = re.sub(r"//[^\n]*", "", src)
+    src = re.sub(r"\s+", "", src)
+    return hashlib.sha256(src.encode()).hexdigest()
+
+
 def kernel_traffic(kernel_file: str):
     """DRAM bytes per launch from a committed ncu summary, valid only while
-    the kernel source is unchanged since the capture."""
+    the kernel code is unchanged since the capture."""
     path = os.path.join(ROOT, "profiles", "decode_traffic.json")
     if not os.path.exists(path):
         return None
     with open(path) as f:
         d = json.load(f)
-    sha = hashlib.sha256(open(kernel_file, "rb").read()).hexdigest()
-    if d.get("decode_cu_sha256") != sha:
+    if d.get("decode_cu_code_sha256") != code_fingerprint(kernel_file):
         return None
     return d.get("dram_bytes_per_launch")
 

@@ -23,22 +23,27 @@
 // row is unpacked exactly once.  P^T overwrites the RoPE chunk of the tile
 // once the score MMAs have consumed it.
 //
-// Warp roles (512 threads):
-//   warp 0      TMEM allocation; lane 0 issues every MMA
-//   warps 4-7   softmax (TMEM lanes = tile rows) and epilogue
-//   warps 8-15  gather + unpack: each thread owns 4 rows x one 8-dim slice
-//               per 64-dim chunk; a whole tile's raw bytes are requested
-//               before the tile's shared-memory chunks are released, so the
-//               gather latency hides behind the previous tile's MMAs.
-// Chunk-granular mbarriers let the unpack of tile i+1 overwrite a 64-dim
-// chunk as soon as the output MMAs of tile i no longer need it.
+// Warp roles (640 threads, five warpgroups):
+//   warps 0-3   thread 0 issues the nine Q tensor copies and every MMA;
+//               warp 1 initialises the mbarriers, warp 3 owns TMEM
+//   warps 4-11  softmax, two warpgroups with half of the heads each (TMEM
+//               lanes = tile rows), then the epilogue and the split merge
+//   warps 12-19 gather + unpack: each thread owns 4 rows x one 8-dim slice
+//               of every 64-dim chunk; chunks 2p and 2p+1 are written as a
+//               pair once output block p of the previous tile is done, and
+//               the same registers then start loading that pair of the next
+//               tile, so the gather hides behind the current tile's work.
+// Each role sets its own register budget with setmaxnreg (RegSplit).
 //
 // Online softmax in base 2 with a lazily updated reference max: a head's
 // reference moves (and O^T and the partial sums are rescaled) only when a
 // score exceeds it by more than 8, so P = 2^(s - m) <= 256 fits FP16.
 //
-// Splits (several CTAs per token) write normalized FP32 partials plus
-// (m, l) to the workspace and a small combine kernel merges them.
+// Splits: when the grid would not fill the SMs, S CTAs share a token's
+// list.  Each writes its unnormalised FP32 partial O and (max, row sum) to
+// the workspace (its own merge slice stays in shared memory), the S CTAs meet
+// on a counter (cooperative launch, bounded wait) and each merges one
+// 512/S-wide dv slice of every head; there is no second kernel.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
