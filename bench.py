@@ -42,6 +42,10 @@ def parse():
     ap.add_argument("--warmup", type=int, default=50)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-extras", action="store_true", help="skip staged/append/e2e/cpu legs")
+    ap.add_argument("--workload", default="decode35x64",
+                    choices=["decode35x64", "sweep", "padded", "prefill", "tiny", "all-others"],
+                    help="decode35x64 (default) prints the one result line; the others time the remaining "
+                         "workloads and print one line per shape")
     ap.add_argument("--launch", default="graph", choices=["graph", "stream"],
                     help="time the K launches replayed from a captured CUDA graph (default) or issued one by one")
     return ap.parse_args()
@@ -240,11 +244,74 @@ def reference_arm(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+def time_other_workload(name, w, nv, synth, args):
+    """One JSON line for a non-default workload: single launches with a cold
+    L2 (a buffer twice the L2 size is written before each), timed with CUDA
+    events on the launching stream around the decode alone; median of 20."""
+    import torch
+    from nvfp4_sparse_mla_decode_b200.cache import build_cache
+    cache = build_cache(w)
+    rows, flop, alg_bytes = workload_stats([w.indices], w.T, w.H)
+    topk = w.indices.shape[1]
+    out = torch.empty(w.T, w.H, 512, dtype=torch.float16, device="cuda")
+    lse = torch.empty(w.T, w.H, dtype=torch.float32, device="cuda")
+    ws = torch.zeros(max(1, nv.workspace_size(w.T, w.H, topk)), dtype=torch.uint8, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for _ in range(3):
+        nv.decode(w.q_nope, w.q_rope, cache, w.indices, w.sm_scale, out=out, lse=lse, workspace=ws,
+                  dev_status=status)
+    times = []
+    for _ in range(20):
+        flush.fill_(1)
+        e0.record(stream)
+        nv.decode(w.q_nope, w.q_rope, cache, w.indices, w.sm_scale, out=out, lse=lse, workspace=ws,
+                  dev_status=status)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1) * 1e3)
+    assert int(status.item()) == 0, "device status %d" % int(status.item())
+    us = statistics.median(times)
+    peaks, _ = measured_peaks()
+    t_roof = max(flop / (float(peaks["bf16_tflops"]) * 1e12), alg_bytes / (float(peaks["hbm_gbs"]) * 1e9))
+    line = {"metric": METRIC, "workload": name, "T": w.T, "H": w.H, "topk": topk,
+            "valid_rows_per_launch": rows, "splits": nv.num_splits(w.T, w.H, topk), "us_per_launch": us,
+            "tflops": flop / (us * 1e-6) / 1e12, "gathered_gbs": rows * ROW_BYTES / (us * 1e-6) / 1e9,
+            "roofline_us": t_roof * 1e6, "frac_of_roofline": t_roof / (us * 1e-6),
+            "timing": "single launch, L2 flushed before it, median of 20", "data": "synthetic"}
+    print(json.dumps(line), flush=True)
+    del cache, flush
+    torch.cuda.empty_cache()
+
+
+def other_workloads(args):
+    import torch
+    import nvfp4_sparse_mla_decode_b200 as nv
+    from nvfp4_sparse_mla_decode_b200 import synth
+    assert torch.cuda.is_available(), "bench.py needs a CUDA GPU"
+    nv.lib()
+    names = ["tiny", "sweep", "padded", "prefill"] if args.workload == "all-others" else [args.workload]
+    for name in names:
+        if name == "tiny":
+            time_other_workload("tiny1x16", synth.tiny("cuda"), nv, synth, args)
+        elif name == "sweep":
+            for T in (1, 8, 32, 64, 128, 256):
+                time_other_workload("sweep%dx128" % T, synth.sweep("cuda", T), nv, synth, args)
+        elif name == "padded":
+            time_other_workload("padded256x64", synth.padded("cuda"), nv, synth, args)
+        elif name == "prefill":
+            time_other_workload("prefill4000x64", synth.append_prefill("cuda"), nv, synth, args)
+
+
 def main():
     args = parse()
     rank, world, local = dist_env()
     if args.impl == "reference":
         return reference_arm(args, rank, world)
+    if args.workload != "decode35x64":
+        return other_workloads(args) if rank == 0 else None
 
     import torch
     import torch.distributed as tdist
