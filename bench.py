@@ -43,7 +43,7 @@ def parse():
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-extras", action="store_true", help="skip staged/append/e2e/cpu legs")
     ap.add_argument("--workload", default="decode35x64",
-                    choices=["decode35x64", "sweep", "padded", "prefill", "tiny", "all-others"],
+                    choices=["decode35x64", "sweep", "padded", "prefill", "tiny", "paged", "all-others"],
                     help="decode35x64 (default) prints the one result line; the others time the remaining "
                          "workloads and print one line per shape")
     ap.add_argument("--launch", default="graph", choices=["graph", "stream"],
@@ -286,14 +286,65 @@ def time_other_workload(name, w, nv, synth, args):
     torch.cuda.empty_cache()
 
 
+def time_paged(nv, synth, args):
+    """decode35x64 with request-local positions and block tables (the
+    translation inside the launch) against the same lists as slot ids: single
+    launches with a cold L2, median of 20 each."""
+    import torch
+    from nvfp4_sparse_mla_decode_b200.cache import build_cache
+    w = synth.decode35("cuda")
+    cache = build_cache(w)
+    table = synth.block_table(w)
+    pos = w.positions.contiguous()
+    out = torch.empty(w.T, w.H, 512, dtype=torch.float16, device="cuda")
+    lse = torch.empty(w.T, w.H, dtype=torch.float32, device="cuda")
+    ws = torch.zeros(max(1, nv.workspace_size(w.T, w.H)), dtype=torch.uint8, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    calls = {
+        "slot_ids": lambda: nv.decode(w.q_nope, w.q_rope, cache, w.indices, w.sm_scale, out=out, lse=lse,
+                                      workspace=ws, dev_status=status),
+        "positions_block_table": lambda: nv.decode_paged(w.q_nope, w.q_rope, cache, pos, table, synth.PAGE_SIZE,
+                                                         w.sm_scale, out=out, lse=lse, workspace=ws,
+                                                         dev_status=status),
+    }
+    res = {}
+    for name, fn in calls.items():
+        for _ in range(3):
+            fn()
+        times = []
+        for _ in range(20):
+            flush.fill_(1)
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            times.append(e0.elapsed_time(e1) * 1e3)
+        res[name] = statistics.median(times)
+    assert int(status.item()) == 0, "device status %d" % int(status.item())
+    print(json.dumps({"metric": METRIC, "workload": "decode35x64 paged", "T": w.T, "H": w.H,
+                      "us_per_launch_slot_ids": res["slot_ids"],
+                      "us_per_launch_positions_block_table": res["positions_block_table"],
+                      "translation_overhead_us": res["positions_block_table"] - res["slot_ids"],
+                      "page_size": synth.PAGE_SIZE, "table_stride": int(table.shape[1]),
+                      "timing": "single launch, L2 flushed before it, median of 20", "data": "synthetic"}),
+          flush=True)
+    del cache, flush
+    torch.cuda.empty_cache()
+
+
 def other_workloads(args):
     import torch
     import nvfp4_sparse_mla_decode_b200 as nv
     from nvfp4_sparse_mla_decode_b200 import synth
     assert torch.cuda.is_available(), "bench.py needs a CUDA GPU"
     nv.lib()
-    names = ["tiny", "sweep", "padded", "prefill"] if args.workload == "all-others" else [args.workload]
+    names = ["tiny", "sweep", "padded", "prefill", "paged"] if args.workload == "all-others" else [args.workload]
     for name in names:
+        if name == "paged":
+            time_paged(nv, synth, args)
         if name == "tiny":
             time_other_workload("tiny1x16", synth.tiny("cuda"), nv, synth, args)
         elif name == "sweep":

@@ -148,6 +148,33 @@ nvfp4mla_status nvfp4_sparse_mla_decode(const void *q_nope_f16, const void *q_ro
                                         size_t workspace_bytes, int32_t *dev_status, void *stream);
 
 /*
+ * nvfp4_sparse_mla_decode_paged -- nvfp4_sparse_mla_decode for lists of
+ * request-local token positions instead of slot ids: the position -> slot
+ * translation through each request's page table (the paged cache the pages'
+ * deployment uses, same page and section) happens inside the launch, while
+ * the list is compacted, so no translated list is ever written to memory.
+ *
+ *   positions    [T, topk] int32, 16-byte aligned: token positions in the
+ *                request's context; -1 = empty
+ *   block_table  [T, table_stride] int32, 4-byte aligned: page ids of token
+ *                t's request in position order (slot = page * page_size +
+ *                position % page_size); unused entries may hold -1
+ *   table_stride entries per row of block_table (>= 1)
+ *   page_size    slots per page, a power of two in [1, 2^20];
+ *                table_stride * page_size must fit in int32
+ * A position < -1 or >= table_stride * page_size, a page id < 0, or a slot
+ * >= num_slots makes that entry empty and sets NVFP4MLA_DEV_BAD_INDEX.  Every
+ * other argument, the workspace contract and the results are those of
+ * nvfp4_sparse_mla_decode.
+ */
+nvfp4mla_status nvfp4_sparse_mla_decode_paged(const void *q_nope_f16, const void *q_rope_f16, const uint8_t *cache,
+                                              int64_t num_slots, const int32_t *positions, int32_t topk,
+                                              const int32_t *block_table, int32_t table_stride, int32_t page_size,
+                                              int32_t T, int32_t H, float sm_scale, void *out_f16, float *lse,
+                                              void *workspace, size_t workspace_bytes, int32_t *dev_status,
+                                              void *stream);
+
+/*
  * nvfp4_sparse_mla_decode_noalloc -- nvfp4_sparse_mla_decode without a
  * caller-supplied workspace.  The pages have no counterpart: this is a
  * library convenience for callers that cannot hand out device memory per

@@ -19,7 +19,7 @@ import torch
 
 __all__ = [
     "ROW_BYTES", "STAGED_ROW_BYTES", "LATENT", "ROPE", "MAX_TOPK", "NVFP4MLAError",
-    "lib", "lib_path", "kv_append", "decode", "decode_noalloc", "staged_decode", "num_splits",
+    "lib", "lib_path", "kv_append", "decode", "decode_paged", "decode_noalloc", "staged_decode", "num_splits",
     "workspace_size", "staging_size", "status_string", "version",
     "DEV_TIMEOUT", "DEV_BAD_INDEX", "DEV_LAYOUT",
 ]
@@ -62,6 +62,9 @@ def lib() -> ctypes.CDLL:
         L.nvfp4_sparse_mla_decode.restype = _i32
         L.nvfp4_sparse_mla_decode.argtypes = [_vp, _vp, _vp, _i64, _vp, _i32, _i32, _i32, _f32, _vp, _vp, _vp,
                                               _sz, _vp, _vp]
+        L.nvfp4_sparse_mla_decode_paged.restype = _i32
+        L.nvfp4_sparse_mla_decode_paged.argtypes = [_vp, _vp, _vp, _i64, _vp, _i32, _vp, _i32, _i32, _i32, _i32,
+                                                    _f32, _vp, _vp, _vp, _sz, _vp, _vp]
         L.nvfp4_sparse_mla_decode_noalloc.restype = _i32
         L.nvfp4_sparse_mla_decode_noalloc.argtypes = [_vp, _vp, _vp, _i64, _vp, _i32, _i32, _i32, _f32, _vp, _vp,
                                                       _vp, _vp]
@@ -171,6 +174,28 @@ def decode(q_nope: torch.Tensor, q_rope: torch.Tensor, cache: torch.Tensor, indi
                                        workspace.numel() * workspace.element_size() if workspace is not None else 0,
                                        _ptr(dev_status), _stream(dev))
     _check(st, "nvfp4_sparse_mla_decode")
+    return out, lse
+
+
+def decode_paged(q_nope: torch.Tensor, q_rope: torch.Tensor, cache: torch.Tensor, positions: torch.Tensor,
+                 block_table: torch.Tensor, page_size: int, sm_scale: float, out: Optional[torch.Tensor] = None,
+                 lse: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                 dev_status: Optional[torch.Tensor] = None):
+    """decode() over request-local positions translated through block_table
+    ([T, stride] int32 page ids) inside the launch."""
+    dev, T, H, topk, out, lse = _decode_args(q_nope, q_rope, cache, positions, out, lse)
+    assert block_table.dtype == torch.int32 and block_table.dim() == 2 and block_table.is_contiguous()
+    assert block_table.shape[0] == T
+    ws_need = workspace_size(T, H, topk)
+    if workspace is None and ws_need:
+        workspace = torch.zeros(ws_need, dtype=torch.uint8, device=dev)
+    st = lib().nvfp4_sparse_mla_decode_paged(_ptr(q_nope), _ptr(q_rope), _ptr(cache), cache.shape[0],
+                                             _ptr(positions), topk, _ptr(block_table), block_table.shape[1],
+                                             int(page_size), T, H, float(sm_scale), _ptr(out), _ptr(lse),
+                                             _ptr(workspace),
+                                             workspace.numel() * workspace.element_size() if workspace is not None
+                                             else 0, _ptr(dev_status), _stream(dev))
+    _check(st, "nvfp4_sparse_mla_decode_paged")
     return out, lse
 
 

@@ -100,6 +100,30 @@ nvfp4mla_status nvfp4_sparse_mla_decode(const void *q_nope_f16, const void *q_ro
                                               static_cast<cudaStream_t>(stream)));
 }
 
+nvfp4mla_status nvfp4_sparse_mla_decode_paged(const void *q_nope_f16, const void *q_rope_f16, const uint8_t *cache,
+                                              int64_t num_slots, const int32_t *positions, int32_t topk,
+                                              const int32_t *block_table, int32_t table_stride, int32_t page_size,
+                                              int32_t T, int32_t H, float sm_scale, void *out_f16, float *lse,
+                                              void *workspace, size_t workspace_bytes, int32_t *dev_status,
+                                              void *stream) {
+    DecodePlan plan;
+    nvfp4mla_status st =
+        check_decode(q_nope_f16, q_rope_f16, cache, num_slots, positions, topk, T, H, sm_scale, out_f16, lse, &plan);
+    if (st != NVFP4MLA_OK) return st;
+    int shift = 0;
+    while (shift < 21 && (1 << shift) < page_size) ++shift;
+    if (page_size < 1 || page_size > (1 << 20) || (1 << shift) != page_size || table_stride < 1 ||
+        (int64_t)table_stride * page_size > INT32_MAX)
+        return NVFP4MLA_ERR_INVALID_ARG;
+    if (T == 0) return NVFP4MLA_OK;
+    if (!block_table || !aligned(block_table, 4)) return NVFP4MLA_ERR_INVALID_ARG;
+    if (plan.workspace_bytes > 0 && (!workspace || workspace_bytes < plan.workspace_bytes)) return NVFP4MLA_ERR_WORKSPACE;
+    if (workspace && !aligned(workspace, 256)) return NVFP4MLA_ERR_INVALID_ARG;
+    return from_cuda(launch_sparse_mla_decode(false, q_nope_f16, q_rope_f16, cache, num_slots, positions, topk, T, H,
+                                              sm_scale, out_f16, lse, workspace, plan, dev_status,
+                                              static_cast<cudaStream_t>(stream), block_table, table_stride, shift));
+}
+
 nvfp4mla_status nvfp4_sparse_mla_decode_noalloc(const void *q_nope_f16, const void *q_rope_f16,
                                                 const uint8_t *cache, int64_t num_slots, const int32_t *indices,
                                                 int32_t topk, int32_t T, int32_t H, float sm_scale, void *out_f16,

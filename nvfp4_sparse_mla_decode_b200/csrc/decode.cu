@@ -320,9 +320,19 @@ __global__ void __launch_bounds__(dec::kThreads, 1)
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
         const int p = tid + 512 * k;  // warps 16.. have no list entries (p >= 2048)
-        const int32_t v = (p < a.topk && tid < 512) ? __ldg(lst + p) : -1;
+        int32_t v = (p < a.topk && tid < 512) ? __ldg(lst + p) : -1;
+        bool entry_bad = false;
+        if (a.block_table && v >= 0) {  // request-local position -> slot through the block table
+            int64_t slot = -1;
+            if ((int64_t)v < a.max_pos) {
+                const int32_t blk = __ldg(a.block_table + (int64_t)t * a.table_stride + (v >> a.page_shift));
+                if (blk >= 0) slot = ((int64_t)blk << a.page_shift) + (v & ((1 << a.page_shift) - 1));
+            }
+            entry_bad = slot < 0 || slot >= a.num_slots;
+            v = entry_bad ? -1 : (int32_t)slot;
+        }
         const bool ok = v >= 0 && (int64_t)v < a.num_slots;
-        bad |= (p < a.topk) && (v < -1 || (int64_t)v >= a.num_slots);
+        bad |= (p < a.topk) && (entry_bad || v < -1 || (int64_t)v >= a.num_slots);
         vals[k] = v;
         bal[k] = __ballot_sync(0xffffffffu, ok);
         if (lane == 0 && warp < 16) cnt_s[k * 16 + warp] = __popc(bal[k]);
@@ -988,7 +998,8 @@ static cudaError_t launch_hg(const DecodeArgs &a, int64_t nblocks, cudaStream_t 
 cudaError_t launch_sparse_mla_decode(bool staged, const void *q_nope, const void *q_rope, const uint8_t *src,
                                      int64_t num_slots, const int32_t *indices, int32_t topk, int32_t T,
                                      int32_t H, float sm_scale, void *out, float *lse, void *workspace,
-                                     const DecodePlan &plan, int32_t *dev_status, cudaStream_t stream) {
+                                     const DecodePlan &plan, int32_t *dev_status, cudaStream_t stream,
+                                     const int32_t *block_table, int64_t table_stride, int page_shift) {
     if (T == 0) return cudaSuccess;
     DecodeArgs a;
     a.q_nope = static_cast<const __half *>(q_nope);
@@ -1010,6 +1021,10 @@ cudaError_t launch_sparse_mla_decode(bool staged, const void *q_nope, const void
     a.ws_ml = plan.splits > 1 ? reinterpret_cast<float *>(ws + kSplitCounterBytes) : nullptr;
     a.ws_o = plan.splits > 1 ? a.ws_ml + (size_t)T * plan.splits * H * 2 : nullptr;
     a.dev_status = dev_status;
+    a.block_table = block_table;
+    a.table_stride = table_stride;
+    a.page_shift = page_shift;
+    a.max_pos = block_table ? (table_stride << page_shift) : 0;
     const int64_t nblocks = (int64_t)T * plan.head_groups * plan.splits;
     cudaError_t e;
     switch (plan.heads_per_cta * 2 + (staged ? 1 : 0)) {

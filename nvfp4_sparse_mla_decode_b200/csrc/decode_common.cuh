@@ -25,6 +25,12 @@ struct DecodeArgs {
     float *ws_ml;       // split statistics: [T][S][H] x (max in log2 units, row sum)
     uint32_t *counters; // per (token, head group): arrivals, departures
     int32_t *dev_status;
+    // Optional block table: when set, list entries are request-local token
+    // positions and slot = table[t][pos >> page_shift] << page_shift | low bits.
+    const int32_t *block_table;
+    int64_t table_stride;  // entries per token row of the table
+    int page_shift;        // log2 of the page size
+    int64_t max_pos;       // table_stride << page_shift
 };
 
 #ifdef NVFP4MLA_TRACE

@@ -33,10 +33,15 @@ int current_device_sm_count();
 // num_slots 352-byte rows, list entries are slots) or over the staging
 // buffer (staged == true: `src` is [T, topk, 576] E4M3 rows addressed by list
 // position; entries outside [0, num_slots) are still the empty ones).
+// block_table (optional): list entries are then request-local positions,
+// translated through table[t][pos >> page_shift] (table_stride entries per
+// token) while the list is compacted.
 cudaError_t launch_sparse_mla_decode(bool staged, const void *q_nope, const void *q_rope, const uint8_t *src,
                                      int64_t num_slots, const int32_t *indices, int32_t topk, int32_t T,
                                      int32_t H, float sm_scale, void *out, float *lse, void *workspace,
-                                     const DecodePlan &plan, int32_t *dev_status, cudaStream_t stream);
+                                     const DecodePlan &plan, int32_t *dev_status, cudaStream_t stream,
+                                     const int32_t *block_table = nullptr, int64_t table_stride = 0,
+                                     int page_shift = 0);
 
 cudaError_t launch_stage_fp8(const uint8_t *cache, int64_t num_slots, const int32_t *indices, int32_t topk,
                              int32_t T, uint8_t *staging, cudaStream_t stream);

@@ -185,6 +185,7 @@ class Workload:
     new_slots: Optional[torch.Tensor] = None
     ctx_lens: Optional[list] = None
     tables: Optional[list] = None
+    positions: Optional[torch.Tensor] = None  # [T, 2048] request-local positions behind ``indices``
 
     def source_rows(self, slots: torch.Tensor):
         """BF16 source of the given slots as the cache holds them after any
@@ -240,7 +241,17 @@ def per_request(device, ctx_lens: Sequence[int], H: int, seed: int, name: str,
                 idx[t] = idx[t][torch.randperm(TOPK, generator=g, device=device)]
     qn, qr = queries(T, H, seed, device)
     return Workload(name, T, H, num_slots, idx, qn, qr, SlotRows(seed, num_slots, device),
-                    ctx_lens=list(ctx_lens), tables=tables)
+                    ctx_lens=list(ctx_lens), tables=tables, positions=None if pad_lists else pos)
+
+
+def block_table(w: Workload, width: Optional[int] = None) -> torch.Tensor:
+    """The requests' page tables as one int32 [T, width] tensor, -1 padded."""
+    assert w.tables is not None
+    width = width or max(int(tb.numel()) for tb in w.tables)
+    out = torch.full((w.T, width), -1, dtype=torch.int32, device=w.indices.device)
+    for t, tb in enumerate(w.tables):
+        out[t, :tb.numel()] = tb.to(torch.int32)
+    return out
 
 
 def redraw(w: Workload, seed: int) -> tuple[torch.Tensor, torch.Tensor, torch.Tensor]:

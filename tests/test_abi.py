@@ -125,3 +125,25 @@ def test_selftest_argument_errors(L):
     assert f(None, 1 << 20, None) == 1
     assert f(1 << 20, None, None) == 1
     assert f((1 << 20) + 2, 1 << 20, None) == 1
+
+
+def test_paged_argument_errors(L):
+    f = L.nvfp4_sparse_mla_decode_paged
+    INVALID = 1
+
+    def call(**kw):
+        a = dict(q=1 << 20, qr=1 << 20, cache=1 << 20, ns=100, pos=1 << 20, topk=2048, tb=1 << 20, stride=8,
+                 page=64, T=1, H=64, sc=0.1, out=1 << 20, lse=1 << 20, ws=1 << 20, wsb=1 << 30, st=None,
+                 stream=None)
+        a.update(kw)
+        return f(a["q"], a["qr"], a["cache"], a["ns"], a["pos"], a["topk"], a["tb"], a["stride"], a["page"],
+                 a["T"], a["H"], a["sc"], a["out"], a["lse"], a["ws"], a["wsb"], a["st"], a["stream"])
+
+    assert call(T=0) == 0
+    assert call(page=48) == INVALID
+    assert call(page=0) == INVALID
+    assert call(page=1 << 21) == INVALID
+    assert call(stride=0) == INVALID
+    assert call(tb=None) == INVALID
+    assert call(tb=(1 << 20) + 2) == INVALID
+    assert call(stride=1 << 20, page=1 << 12) == INVALID   # positions would overflow int32
