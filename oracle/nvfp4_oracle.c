@@ -193,6 +193,25 @@ void oracle_quantize_rows(const uint16_t *latent, int64_t lat_stride,
     }
 }
 
+/* The pre-NVFP4 cache row (page "Prime Intellect Launches Prime Inference,
+ * Serving 600B Tokens Daily", section "Four-bit caches make room": rows were
+ * 576 bytes before NVFP4): one E4M3 byte per dim, 512 latent dims then 64
+ * RoPE dims, each value E4M3_RNE_sat of the BF16 input with no scale.
+ * Quantizes n rows into n 576-byte rows. */
+void oracle_quantize_fp8_rows(const uint16_t *latent, int64_t lat_stride,
+                              const uint16_t *rope, int64_t rope_stride,
+                              int64_t n, uint8_t *rows)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < n; ++r) {
+        uint8_t *row = rows + r * ORACLE_STAGED_ROW;
+        for (int d = 0; d < ORACLE_LATENT; ++d)
+            row[d] = (uint8_t)oracle_e4m3_encode(bf16_to_float(latent[r * lat_stride + d]));
+        for (int k = 0; k < ORACLE_ROPE; ++k)
+            row[ORACLE_LATENT + k] = (uint8_t)oracle_e4m3_encode(bf16_to_float(rope[r * rope_stride + k]));
+    }
+}
+
 /* Dequantize one 352-byte row to 576 values: dims 0..511 are
  * e2m1(nibble) * e4m3(scale of its group), dims 512..575 are e4m3(RoPE).
  * Every such product has at most 6 significant bits and lies in
@@ -236,8 +255,10 @@ void oracle_stage_row(const uint8_t *row, uint8_t *out576)
  *   out   = sum_j exp(s_j - m) * k_j[0:512] / l      (V = the latent part)
  *   lse   = m + ln l                                  (natural log)
  * A token with no valid entry gets out = 0 and lse = -inf.
- * staged != 0 first replaces each key value by its E4M3 re-encoding (the
- * staged FP8 baseline).  q is FP16 [T,H,512] and [T,H,64]; out is FP64
+ * staged == 1 first replaces each key value by its E4M3 re-encoding (the
+ * staged FP8 baseline); staged == 2 means the cache holds 576-byte E4M3 rows
+ * (oracle_quantize_fp8_rows) and k_j is their decoded values.  q is FP16
+ * [T,H,512] and [T,H,64]; out is FP64
  * [T,H,512], lse FP64 [T,H].  Each token's valid rows are dequantized once
  * (the same values for every head); sums run over valid positions in list
  * order; OpenMP only distributes independent rows and heads.
@@ -268,9 +289,11 @@ int oracle_sparse_mla(const uint16_t *q_nope, const uint16_t *q_rope,
         }
 #pragma omp parallel for schedule(static)
         for (int jj = 0; jj < nvalid; ++jj) {
-            const uint8_t *row = cache + pos[jj] * ORACLE_ROW_BYTES;
+            const uint8_t *row = cache + pos[jj] * (staged == 2 ? ORACLE_STAGED_ROW : ORACLE_ROW_BYTES);
             double *k = K + (size_t)jj * D;
-            if (staged) {
+            if (staged == 2) {
+                for (int d = 0; d < D; ++d) k[d] = oracle_e4m3_value(row[d]);
+            } else if (staged) {
                 uint8_t st[ORACLE_STAGED_ROW];
                 oracle_stage_row(row, st);
                 for (int d = 0; d < D; ++d) k[d] = oracle_e4m3_value(st[d]);

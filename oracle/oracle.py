@@ -16,7 +16,7 @@ import numpy as np
 __all__ = [
     "build_oracle", "lib", "ROW_BYTES", "STAGED_ROW_BYTES",
     "e2m1_value", "e4m3_value", "e2m1_encode", "e4m3_encode",
-    "f16_to_double", "quantize_group", "quantize_rows", "dequant_rows",
+    "f16_to_double", "quantize_group", "quantize_rows", "quantize_fp8_rows", "dequant_rows",
     "stage_rows", "sparse_mla", "max_threads",
 ]
 
@@ -60,6 +60,9 @@ def lib():
         L.oracle_quantize_rows.restype = None
         L.oracle_quantize_rows.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p,
                                            ctypes.c_int64, ctypes.c_int64, ctypes.c_void_p]
+        L.oracle_quantize_fp8_rows.restype = None
+        L.oracle_quantize_fp8_rows.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p,
+                                               ctypes.c_int64, ctypes.c_int64, ctypes.c_void_p]
         L.oracle_dequant_row.restype = None
         L.oracle_dequant_row.argtypes = [ctypes.c_void_p, ctypes.c_void_p]
         L.oracle_stage_row.restype = None
@@ -120,6 +123,18 @@ def quantize_rows(latent_bf16_bits: np.ndarray, rope_bf16_bits: np.ndarray) -> n
     return out
 
 
+def quantize_fp8_rows(latent_bf16_bits: np.ndarray, rope_bf16_bits: np.ndarray) -> np.ndarray:
+    """BF16 bit patterns [n,512] and [n,64] -> 576-byte E4M3 rows uint8 [n,576]."""
+    lat = np.ascontiguousarray(latent_bf16_bits, dtype=np.uint16)
+    rope = np.ascontiguousarray(rope_bf16_bits, dtype=np.uint16)
+    n = lat.shape[0]
+    assert lat.shape == (n, 512) and rope.shape == (n, 64)
+    out = np.zeros((n, STAGED_ROW_BYTES), dtype=np.uint8)
+    if n:
+        lib().oracle_quantize_fp8_rows(_ptr(lat), 512, _ptr(rope), 64, n, _ptr(out))
+    return out
+
+
 def dequant_rows(rows: np.ndarray) -> np.ndarray:
     """Packed rows uint8 [n,352] -> float64 [n,576] (512 latent + 64 RoPE)."""
     rows = np.ascontiguousarray(rows, dtype=np.uint8)
@@ -144,10 +159,10 @@ def stage_rows(rows: np.ndarray) -> np.ndarray:
 
 def sparse_mla(q_nope_f16: np.ndarray, q_rope_f16: np.ndarray, cache: np.ndarray,
                indices: np.ndarray, sm_scale: float, staged: bool = False,
-               nthreads: int = 0, num_slots: int | None = None):
+               nthreads: int = 0, num_slots: int | None = None, fp8_rows: bool = False):
     """FP64 sparse MLA decode.  q: float16 [T,H,512] / [T,H,64]; cache uint8
-    [num_slots,352]; indices int32 [T,topk].  Returns (out f64 [T,H,512],
-    lse f64 [T,H])."""
+    [num_slots,352] (or [num_slots,576] E4M3 rows with fp8_rows); indices
+    int32 [T,topk].  Returns (out f64 [T,H,512], lse f64 [T,H])."""
     qn = np.ascontiguousarray(q_nope_f16, dtype=np.float16)
     qr = np.ascontiguousarray(q_rope_f16, dtype=np.float16)
     cache = np.ascontiguousarray(cache, dtype=np.uint8)
@@ -158,12 +173,13 @@ def sparse_mla(q_nope_f16: np.ndarray, q_rope_f16: np.ndarray, cache: np.ndarray
     topk = idx.shape[1]
     if num_slots is None:
         num_slots = cache.shape[0]
-    assert cache.ndim == 2 and cache.shape[1] == ROW_BYTES and cache.shape[0] >= num_slots
+    assert cache.ndim == 2 and cache.shape[1] == (STAGED_ROW_BYTES if fp8_rows else ROW_BYTES)
+    assert cache.shape[0] >= num_slots
     out = np.zeros((T, H, 512), dtype=np.float64)
     lse = np.zeros((T, H), dtype=np.float64)
     rc = lib().oracle_sparse_mla(_ptr(qn.view(np.uint16)), _ptr(qr.view(np.uint16)), _ptr(cache),
                                  int(num_slots), _ptr(idx), int(topk), int(T), int(H),
-                                 float(np.float32(sm_scale)), int(bool(staged)),
+                                 float(np.float32(sm_scale)), 2 if fp8_rows else int(bool(staged)),
                                  _ptr(out), _ptr(lse), int(nthreads))
     if rc != 0:
         raise RuntimeError("oracle_sparse_mla failed (%d)" % rc)

@@ -253,6 +253,46 @@ def test_staged_variant_equals_dense_over_e4m3_values():
                           .view(torch.uint8).numpy())
 
 
+def _bf16_rows(n, seed, scale):
+    g = torch.Generator().manual_seed(seed)
+    x = (torch.randn(n, 576, generator=g) * scale).to(torch.bfloat16)
+    lat = x[:, :512].contiguous().view(torch.int16).numpy().view(np.uint16)
+    rope = x[:, 512:].contiguous().view(torch.int16).numpy().view(np.uint16)
+    return x.to(torch.float32), lat, rope
+
+
+def test_fp8_rows_match_torch_e4m3_layout_and_saturation():
+    # one E4M3 byte per dim, latent dims first then RoPE; values spread over
+    # subnormals .. beyond the largest finite code
+    sc = torch.exp(torch.linspace(math.log(1e-3), math.log(300.0), 576))
+    x, lat, rope = _bf16_rows(64, 21, sc)
+    rows = oracle.quantize_fp8_rows(lat, rope)
+    assert rows.shape == (64, 576) and rows.dtype == np.uint8
+    xs = x.numpy()
+    inside = np.abs(xs) <= 448.0
+    ref = _torch_e4m3_code(np.where(inside, xs, 0.0))
+    assert np.array_equal(rows[inside], ref[inside])
+    big = ~inside
+    assert big.any()
+    assert np.all(rows[big & (xs > 0)] == 0x7E) and np.all(rows[big & (xs < 0)] == 0xFE)
+    assert oracle.quantize_fp8_rows(lat[:0], rope[:0]).shape == (0, 576)
+
+
+def test_fp8_row_attention_equals_dense_over_selected_rows():
+    n, H = 300, 3
+    _, lat, rope = _bf16_rows(n, 22, 0.25 + 3.75 * torch.rand(576, generator=torch.Generator().manual_seed(23)))
+    rows = oracle.quantize_fp8_rows(lat, rope)
+    qn, qr = _q(1, H, seed=24)
+    sel = np.random.default_rng(25).permutation(n)[:170].astype(np.int32)
+    idx = np.concatenate([sel, -np.ones(30, np.int32)])[None, :]
+    sm = 1 / math.sqrt(576)
+    out, lse = oracle.sparse_mla(qn, qr, rows, idx, sm, fp8_rows=True)
+    K = torch.from_numpy(rows[sel]).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    ref_o, ref_l = _dense(qn[0], qr[0], K, f32(sm))
+    np.testing.assert_allclose(out[0], ref_o, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(lse[0], ref_l, rtol=1e-12, atol=1e-12)
+
+
 def test_permutation_and_empty_entry_invariance():
     n, H, topk = 1000, 2, 2048
     cache = _cache(n, seed=2)
