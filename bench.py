@@ -43,7 +43,7 @@ def parse():
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-extras", action="store_true", help="skip staged/append/e2e/cpu legs")
     ap.add_argument("--workload", default="decode35x64",
-                    choices=["decode35x64", "sweep", "padded", "prefill", "tiny", "paged", "all-others"],
+                    choices=["decode35x64", "sweep", "padded", "prefill", "tiny", "paged", "fp8", "all-others"],
                     help="decode35x64 (default) prints the one result line; the others time the remaining "
                          "workloads and print one line per shape")
     ap.add_argument("--launch", default="graph", choices=["graph", "stream"],
@@ -335,16 +335,92 @@ def time_paged(nv, synth, args):
     torch.cuda.empty_cache()
 
 
+def cold_median_us(fn, flush, n=20):
+    """Median device time (us) of fn() over n launches, each after writing a
+    buffer larger than L2; CUDA events on the current stream."""
+    import torch
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for _ in range(3):
+        fn()
+    times = []
+    for _ in range(n):
+        flush.fill_(1)
+        e0.record(stream)
+        fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1) * 1e3)
+    return statistics.median(times)
+
+
+def time_fp8(nv, synth, args):
+    """decode35x64 over the 576-byte E4M3 row cache (the row before NVFP4)
+    against the 352-byte NVFP4 cache and the staged path, plus both append
+    kernels on the 4000 prefill rows: single launches, L2 flushed, median
+    of 20 each."""
+    import torch
+    from nvfp4_sparse_mla_decode_b200.cache import build_cache, build_fp8_cache
+    w = synth.decode35("cuda")
+    cache = build_cache(w)
+    fcache = build_fp8_cache(w)
+    rows, flop, _ = workload_stats([w.indices], w.T, w.H)
+    out = torch.empty(w.T, w.H, 512, dtype=torch.float16, device="cuda")
+    lse = torch.empty(w.T, w.H, dtype=torch.float32, device="cuda")
+    ws = torch.zeros(max(1, nv.workspace_size(w.T, w.H)), dtype=torch.uint8, device="cuda")
+    staging = torch.empty(nv.staging_size(w.T), dtype=torch.uint8, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device="cuda")
+    kw = dict(out=out, lse=lse, workspace=ws, dev_status=status)
+    us = {
+        "nvfp4_cache": cold_median_us(lambda: nv.decode(w.q_nope, w.q_rope, cache, w.indices, w.sm_scale, **kw),
+                                      flush),
+        "fp8_cache": cold_median_us(lambda: nv.fp8_decode(w.q_nope, w.q_rope, fcache, w.indices, w.sm_scale,
+                                                          **kw), flush),
+        "staged": cold_median_us(lambda: nv.staged_decode(w.q_nope, w.q_rope, cache, w.indices, w.sm_scale,
+                                                          staging=staging, **kw), flush),
+    }
+    del cache, fcache, staging
+    torch.cuda.empty_cache()
+    wa = synth.append_prefill("cuda")
+    a_us = {}
+    for name, rb, fn in (("nvfp4", nv.ROW_BYTES, nv.kv_append), ("fp8", nv.STAGED_ROW_BYTES, nv.fp8_kv_append)):
+        ac = torch.zeros(wa.num_slots, rb, dtype=torch.uint8, device="cuda")
+        a_us[name] = cold_median_us(lambda: fn(wa.new_lat, wa.new_rope, wa.new_slots, ac, status), flush)
+        del ac
+    assert int(status.item()) == 0, "device status %d" % int(status.item())
+    peaks, _ = measured_peaks()
+    line = {"metric": METRIC, "workload": "decode35x64 fp8 rows", "T": w.T, "H": w.H,
+            "valid_rows_per_launch": rows,
+            "us_per_launch": us,
+            "tflops": {k: flop / (v * 1e-6) / 1e12 for k, v in us.items()},
+            "gathered_gbs": {"nvfp4_cache": rows * nv.ROW_BYTES / (us["nvfp4_cache"] * 1e-6) / 1e9,
+                             "fp8_cache": rows * nv.STAGED_ROW_BYTES / (us["fp8_cache"] * 1e-6) / 1e9},
+            "rows_per_gb": {"nvfp4": 1e9 / nv.ROW_BYTES, "fp8": 1e9 / nv.STAGED_ROW_BYTES},
+            "capacity_ratio": nv.STAGED_ROW_BYTES / nv.ROW_BYTES,
+            "append_4000_rows_us": a_us,
+            "append_gbs": {"nvfp4": wa.T * (1152 + 352 + 4) / (a_us["nvfp4"] * 1e-6) / 1e9,
+                           "fp8": wa.T * (1152 + 576 + 4) / (a_us["fp8"] * 1e-6) / 1e9},
+            "hbm_peak_gbs": float(peaks["hbm_gbs"]),
+            "timing": "single launch, L2 flushed before it, median of 20", "data": "synthetic"}
+    print(json.dumps(line), flush=True)
+    del flush
+    torch.cuda.empty_cache()
+
+
 def other_workloads(args):
     import torch
     import nvfp4_sparse_mla_decode_b200 as nv
     from nvfp4_sparse_mla_decode_b200 import synth
     assert torch.cuda.is_available(), "bench.py needs a CUDA GPU"
     nv.lib()
-    names = ["tiny", "sweep", "padded", "prefill", "paged"] if args.workload == "all-others" else [args.workload]
+    names = (["tiny", "sweep", "padded", "prefill", "paged", "fp8"] if args.workload == "all-others"
+             else [args.workload])
     for name in names:
         if name == "paged":
             time_paged(nv, synth, args)
+        if name == "fp8":
+            time_fp8(nv, synth, args)
         if name == "tiny":
             time_other_workload("tiny1x16", synth.tiny("cuda"), nv, synth, args)
         elif name == "sweep":

@@ -92,6 +92,21 @@ nvfp4mla_status nvfp4_kv_append(const void *latent_bf16, int64_t latent_stride, 
                                 int64_t num_slots, int32_t *dev_status, void *stream);
 
 /*
+ * nvfp4mla_fp8_kv_append -- the pre-NVFP4 cache row (same page and section:
+ * a row took 576 bytes before the four-bit format): write n BF16 cache rows
+ * as 576-byte E4M3 rows at scattered slots.  Bytes [0, 512) of a row are
+ * the latent dims, [512, 576) the RoPE dims, each the E4M3 round-to-nearest-
+ * even, saturating (to +-448), of the value, with no scale.
+ *   latent_bf16, rope_bf16, slot_mapping, n, dev_status, stream: as
+ *                 nvfp4_kv_append
+ *   cache         [num_slots, 576] bytes, 16-byte aligned
+ * Same error behaviour as nvfp4_kv_append.
+ */
+nvfp4mla_status nvfp4mla_fp8_kv_append(const void *latent_bf16, int64_t latent_stride, const void *rope_bf16,
+                                       int64_t rope_stride, const int32_t *slot_mapping, int32_t n, uint8_t *cache,
+                                       int64_t num_slots, int32_t *dev_status, void *stream);
+
+/*
  * nvfp4_sparse_mla_num_splits -- how many CTAs the decode splits each
  * token's index list across: the largest power of two S <= 16 (and <= the
  * number of 128-row tiles of topk) with T * (H / min(H, 64)) * S no larger
@@ -227,7 +242,22 @@ nvfp4mla_status nvfp4_staged_fp8_mla_decode(const void *q_nope_f16, const void *
                                             uint8_t *staging, size_t staging_bytes, void *workspace,
                                             size_t workspace_bytes, int32_t *dev_status, void *stream);
 
-/* Human-readable name of a status code (static storage). */
+/*
+ * nvfp4mla_fp8_sparse_mla_decode -- the same attention as
+ * nvfp4_sparse_mla_decode over a cache of 576-byte E4M3 rows (written by
+ * nvfp4mla_fp8_kv_append): the "before" side of the 576 -> 352 byte row
+ * change on the same page and section.  List entries are slots of
+ * fp8_cache; keys are the E4M3 values of a row's 576 bytes, values its first
+ * 512.  Arguments, workspace (nvfp4_sparse_mla_workspace_size), statuses and
+ * the empty-entry rule are those of nvfp4_sparse_mla_decode, except
+ *   fp8_cache  [num_slots, 576] bytes, 16-byte aligned
+ */
+nvfp4mla_status nvfp4mla_fp8_sparse_mla_decode(const void *q_nope_f16, const void *q_rope_f16,
+                                               const uint8_t *fp8_cache, int64_t num_slots, const int32_t *indices,
+                                               int32_t topk, int32_t T, int32_t H, float sm_scale, void *out_f16,
+                                               float *lse, void *workspace, size_t workspace_bytes,
+                                               int32_t *dev_status, void *stream);
+
 /*
  * nvfp4mla_selftest_wait_timeout -- checks, on the device, that the bounded
  * waits every kernel here uses end with a status instead of hanging: one CTA
@@ -238,6 +268,7 @@ nvfp4mla_status nvfp4_staged_fp8_mla_decode(const void *q_nope_f16, const void *
  */
 nvfp4mla_status nvfp4mla_selftest_wait_timeout(uint32_t *zero_word, int32_t *dev_status, void *stream);
 
+/* Human-readable name of a status code (static storage). */
 const char *nvfp4mla_status_string(nvfp4mla_status status);
 
 /* Library ABI version: major*10000 + minor*100 + patch. */

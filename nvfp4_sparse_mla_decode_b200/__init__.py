@@ -19,7 +19,8 @@ import torch
 
 __all__ = [
     "ROW_BYTES", "STAGED_ROW_BYTES", "LATENT", "ROPE", "MAX_TOPK", "NVFP4MLAError",
-    "lib", "lib_path", "kv_append", "decode", "decode_paged", "decode_noalloc", "staged_decode", "num_splits",
+    "lib", "lib_path", "kv_append", "decode", "decode_paged", "decode_noalloc", "staged_decode",
+    "fp8_kv_append", "fp8_decode", "num_splits",
     "workspace_size", "staging_size", "status_string", "version",
     "DEV_TIMEOUT", "DEV_BAD_INDEX", "DEV_LAYOUT",
 ]
@@ -73,6 +74,11 @@ def lib() -> ctypes.CDLL:
         L.nvfp4_staged_fp8_mla_decode.restype = _i32
         L.nvfp4_staged_fp8_mla_decode.argtypes = [_vp, _vp, _vp, _i64, _vp, _i32, _i32, _i32, _f32, _vp, _vp,
                                                   _vp, _sz, _vp, _sz, _vp, _vp]
+        L.nvfp4mla_fp8_kv_append.restype = _i32
+        L.nvfp4mla_fp8_kv_append.argtypes = [_vp, _i64, _vp, _i64, _vp, _i32, _vp, _i64, _vp, _vp]
+        L.nvfp4mla_fp8_sparse_mla_decode.restype = _i32
+        L.nvfp4mla_fp8_sparse_mla_decode.argtypes = [_vp, _vp, _vp, _i64, _vp, _i32, _i32, _i32, _f32, _vp, _vp,
+                                                     _vp, _sz, _vp, _vp]
         L.nvfp4mla_selftest_wait_timeout.restype = _i32
         L.nvfp4mla_selftest_wait_timeout.argtypes = [_vp, _vp, _vp]
         L.nvfp4mla_status_string.restype = ctypes.c_char_p
@@ -124,21 +130,33 @@ def staging_size(T: int, topk: int = MAX_TOPK) -> int:
     return int(lib().nvfp4_staged_fp8_staging_size(T, topk))
 
 
-def kv_append(latent: torch.Tensor, rope: torch.Tensor, slot_mapping: torch.Tensor, cache: torch.Tensor,
-              dev_status: Optional[torch.Tensor] = None) -> None:
-    """Quantize BF16 rows latent [n, >=512] / rope [n, >=64] (row strides in
-    elements, unit inner stride) into ``cache`` uint8 [num_slots, 352] at
-    ``slot_mapping`` int32 [n]."""
+def _append(fn, name, latent, rope, slot_mapping, cache, dev_status):
     dev = _need_cuda(latent, rope, slot_mapping, cache)
     assert latent.dtype == torch.bfloat16 and rope.dtype == torch.bfloat16
     assert slot_mapping.dtype == torch.int32 and cache.dtype == torch.uint8 and cache.is_contiguous()
     assert latent.stride(-1) == 1 and rope.stride(-1) == 1 and slot_mapping.is_contiguous()
     n = slot_mapping.numel()
     assert latent.shape[0] == n and rope.shape[0] == n
-    st = lib().nvfp4_kv_append(_ptr(latent), latent.stride(0) if n else LATENT, _ptr(rope),
-                               rope.stride(0) if n else ROPE, _ptr(slot_mapping), n, _ptr(cache),
-                               cache.shape[0], _ptr(dev_status), _stream(dev))
-    _check(st, "nvfp4_kv_append")
+    st = fn(_ptr(latent), latent.stride(0) if n else LATENT, _ptr(rope), rope.stride(0) if n else ROPE,
+            _ptr(slot_mapping), n, _ptr(cache), cache.shape[0], _ptr(dev_status), _stream(dev))
+    _check(st, name)
+
+
+def kv_append(latent: torch.Tensor, rope: torch.Tensor, slot_mapping: torch.Tensor, cache: torch.Tensor,
+              dev_status: Optional[torch.Tensor] = None) -> None:
+    """Quantize BF16 rows latent [n, >=512] / rope [n, >=64] (row strides in
+    elements, unit inner stride) into ``cache`` uint8 [num_slots, 352] at
+    ``slot_mapping`` int32 [n]."""
+    assert cache.dim() == 2 and cache.shape[1] == ROW_BYTES
+    _append(lib().nvfp4_kv_append, "nvfp4_kv_append", latent, rope, slot_mapping, cache, dev_status)
+
+
+def fp8_kv_append(latent: torch.Tensor, rope: torch.Tensor, slot_mapping: torch.Tensor, cache: torch.Tensor,
+                  dev_status: Optional[torch.Tensor] = None) -> None:
+    """kv_append() into a cache of 576-byte E4M3 rows, uint8 [num_slots, 576]."""
+    assert cache.dim() == 2 and cache.shape[1] == STAGED_ROW_BYTES
+    _append(lib().nvfp4mla_fp8_kv_append, "nvfp4mla_fp8_kv_append", latent, rope, slot_mapping, cache,
+            dev_status)
 
 
 def _decode_args(q_nope, q_rope, cache, indices, out, lse):
@@ -231,6 +249,24 @@ def staged_decode(q_nope: torch.Tensor, q_rope: torch.Tensor, cache: torch.Tenso
                                            workspace.numel() if workspace is not None else 0,
                                            _ptr(dev_status), _stream(dev))
     _check(st, "nvfp4_staged_fp8_mla_decode")
+    return out, lse
+
+
+def fp8_decode(q_nope: torch.Tensor, q_rope: torch.Tensor, fp8_cache: torch.Tensor, indices: torch.Tensor,
+               sm_scale: float, out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+               workspace: Optional[torch.Tensor] = None, dev_status: Optional[torch.Tensor] = None):
+    """decode() over a cache of 576-byte E4M3 rows (uint8 [num_slots, 576])."""
+    assert fp8_cache.dim() == 2 and fp8_cache.shape[1] == STAGED_ROW_BYTES
+    dev, T, H, topk, out, lse = _decode_args(q_nope, q_rope, fp8_cache, indices, out, lse)
+    ws_need = workspace_size(T, H, topk)
+    if workspace is None and ws_need:
+        workspace = torch.zeros(ws_need, dtype=torch.uint8, device=dev)
+    st = lib().nvfp4mla_fp8_sparse_mla_decode(_ptr(q_nope), _ptr(q_rope), _ptr(fp8_cache), fp8_cache.shape[0],
+                                              _ptr(indices), topk, T, H, float(sm_scale), _ptr(out), _ptr(lse),
+                                              _ptr(workspace),
+                                              workspace.numel() * workspace.element_size()
+                                              if workspace is not None else 0, _ptr(dev_status), _stream(dev))
+    _check(st, "nvfp4mla_fp8_sparse_mla_decode")
     return out, lse
 
 

@@ -75,6 +75,20 @@ nvfp4mla_status nvfp4_kv_append(const void *latent_bf16, int64_t latent_stride, 
                                       num_slots, dev_status, static_cast<cudaStream_t>(stream)));
 }
 
+nvfp4mla_status nvfp4mla_fp8_kv_append(const void *latent_bf16, int64_t latent_stride, const void *rope_bf16,
+                                       int64_t rope_stride, const int32_t *slot_mapping, int32_t n, uint8_t *cache,
+                                       int64_t num_slots, int32_t *dev_status, void *stream) {
+    if (n < 0 || num_slots < 0 || latent_stride < NVFP4MLA_LATENT || rope_stride < NVFP4MLA_ROPE)
+        return NVFP4MLA_ERR_INVALID_ARG;
+    if (n == 0) return NVFP4MLA_OK;
+    if (!latent_bf16 || !rope_bf16 || !slot_mapping || !cache) return NVFP4MLA_ERR_INVALID_ARG;
+    if (latent_stride % 8 || rope_stride % 8 || !aligned(latent_bf16, 16) || !aligned(rope_bf16, 16) ||
+        !aligned(cache, 16) || !aligned(slot_mapping, 4))
+        return NVFP4MLA_ERR_INVALID_ARG;
+    return from_cuda(launch_fp8_kv_append(latent_bf16, latent_stride, rope_bf16, rope_stride, slot_mapping, n,
+                                          cache, num_slots, dev_status, static_cast<cudaStream_t>(stream)));
+}
+
 int32_t nvfp4_sparse_mla_num_splits(int32_t T, int32_t H, int32_t topk) {
     DecodePlan p;
     return make_decode_plan(T, H, topk, current_device_sm_count(), &p) ? p.splits : 0;
@@ -95,7 +109,7 @@ nvfp4mla_status nvfp4_sparse_mla_decode(const void *q_nope_f16, const void *q_ro
     if (st != NVFP4MLA_OK || T == 0) return st;
     if (plan.workspace_bytes > 0 && (!workspace || workspace_bytes < plan.workspace_bytes)) return NVFP4MLA_ERR_WORKSPACE;
     if (workspace && !aligned(workspace, 256)) return NVFP4MLA_ERR_INVALID_ARG;
-    return from_cuda(launch_sparse_mla_decode(false, q_nope_f16, q_rope_f16, cache, num_slots, indices, topk, T, H,
+    return from_cuda(launch_sparse_mla_decode(RowSource::kNvfp4Cache, q_nope_f16, q_rope_f16, cache, num_slots, indices, topk, T, H,
                                               sm_scale, out_f16, lse, workspace, plan, dev_status,
                                               static_cast<cudaStream_t>(stream)));
 }
@@ -119,7 +133,7 @@ nvfp4mla_status nvfp4_sparse_mla_decode_paged(const void *q_nope_f16, const void
     if (!block_table || !aligned(block_table, 4)) return NVFP4MLA_ERR_INVALID_ARG;
     if (plan.workspace_bytes > 0 && (!workspace || workspace_bytes < plan.workspace_bytes)) return NVFP4MLA_ERR_WORKSPACE;
     if (workspace && !aligned(workspace, 256)) return NVFP4MLA_ERR_INVALID_ARG;
-    return from_cuda(launch_sparse_mla_decode(false, q_nope_f16, q_rope_f16, cache, num_slots, positions, topk, T, H,
+    return from_cuda(launch_sparse_mla_decode(RowSource::kNvfp4Cache, q_nope_f16, q_rope_f16, cache, num_slots, positions, topk, T, H,
                                               sm_scale, out_f16, lse, workspace, plan, dev_status,
                                               static_cast<cudaStream_t>(stream), block_table, table_stride, shift));
 }
@@ -140,7 +154,7 @@ nvfp4mla_status nvfp4_sparse_mla_decode_noalloc(const void *q_nope_f16, const vo
         ws = noalloc_workspace(dev);
         if (!ws) return NVFP4MLA_ERR_CUDA;
     }
-    return from_cuda(launch_sparse_mla_decode(false, q_nope_f16, q_rope_f16, cache, num_slots, indices, topk, T, H,
+    return from_cuda(launch_sparse_mla_decode(RowSource::kNvfp4Cache, q_nope_f16, q_rope_f16, cache, num_slots, indices, topk, T, H,
                                               sm_scale, out_f16, lse, ws, plan, dev_status,
                                               static_cast<cudaStream_t>(stream)));
 }
@@ -166,8 +180,24 @@ nvfp4mla_status nvfp4_staged_fp8_mla_decode(const void *q_nope_f16, const void *
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     cudaError_t e = launch_stage_fp8(cache, num_slots, indices, topk, T, staging, s);
     if (e != cudaSuccess) return NVFP4MLA_ERR_CUDA;
-    return from_cuda(launch_sparse_mla_decode(true, q_nope_f16, q_rope_f16, staging, num_slots, indices, topk, T, H,
+    return from_cuda(launch_sparse_mla_decode(RowSource::kFp8Staging, q_nope_f16, q_rope_f16, staging, num_slots, indices, topk, T, H,
                                               sm_scale, out_f16, lse, workspace, plan, dev_status, s));
+}
+
+nvfp4mla_status nvfp4mla_fp8_sparse_mla_decode(const void *q_nope_f16, const void *q_rope_f16,
+                                               const uint8_t *fp8_cache, int64_t num_slots, const int32_t *indices,
+                                               int32_t topk, int32_t T, int32_t H, float sm_scale, void *out_f16,
+                                               float *lse, void *workspace, size_t workspace_bytes,
+                                               int32_t *dev_status, void *stream) {
+    DecodePlan plan;
+    nvfp4mla_status st = check_decode(q_nope_f16, q_rope_f16, fp8_cache, num_slots, indices, topk, T, H, sm_scale,
+                                      out_f16, lse, &plan);
+    if (st != NVFP4MLA_OK || T == 0) return st;
+    if (plan.workspace_bytes > 0 && (!workspace || workspace_bytes < plan.workspace_bytes)) return NVFP4MLA_ERR_WORKSPACE;
+    if (workspace && !aligned(workspace, 256)) return NVFP4MLA_ERR_INVALID_ARG;
+    return from_cuda(launch_sparse_mla_decode(RowSource::kFp8Cache, q_nope_f16, q_rope_f16, fp8_cache, num_slots,
+                                              indices, topk, T, H, sm_scale, out_f16, lse, workspace, plan,
+                                              dev_status, static_cast<cudaStream_t>(stream)));
 }
 
 nvfp4mla_status nvfp4mla_selftest_wait_timeout(uint32_t *zero_word, int32_t *dev_status, void *stream) {

@@ -374,7 +374,7 @@ __global__ void __launch_bounds__(dec::kThreads, 1)
     for (int k = 0; k < 4; ++k) {
         if (warp < 16 && ((bal[k] >> lane) & 1u)) {
             const int pos = before[k] + __popc(bal[k] & ((1u << lane) - 1u));
-            if (pos >= lo && pos < hi) idx_s[pos - lo] = kStaged ? (tid + 512 * k) : vals[k];
+            if (pos >= lo && pos < hi) idx_s[pos - lo] = (kStaged && !a.rows_by_slot) ? (tid + 512 * k) : vals[k];
         }
     }
     tc_fence_before();
@@ -741,8 +741,11 @@ __global__ void __launch_bounds__(dec::kThreads, 1)
                 slot[k] = rvalid[k] ? idx_s[e] : 0;
             }
         };
+        // FP8 rows: row `slot` of the cache, or row (t, list position) of
+        // the staging buffer.
+        const int64_t row0 = (kStaged && !a.rows_by_slot) ? (int64_t)t * a.topk : 0;
         auto row_base = [&](int k) -> const uint8_t * {
-            return kStaged ? a.src + ((int64_t)t * a.topk + slot[k]) * kStagedRowBytes
+            return kStaged ? a.src + (row0 + slot[k]) * kStagedRowBytes
                            : a.src + (int64_t)slot[k] * kRowBytes;
         };
         auto load_group = [&](int grp) {
@@ -995,7 +998,7 @@ static cudaError_t launch_hg(const DecodeArgs &a, int64_t nblocks, cudaStream_t 
     return cudaLaunchKernelEx(&cfg, kern, a, tm_qn, tm_qr);
 }
 
-cudaError_t launch_sparse_mla_decode(bool staged, const void *q_nope, const void *q_rope, const uint8_t *src,
+cudaError_t launch_sparse_mla_decode(RowSource rows, const void *q_nope, const void *q_rope, const uint8_t *src,
                                      int64_t num_slots, const int32_t *indices, int32_t topk, int32_t T,
                                      int32_t H, float sm_scale, void *out, float *lse, void *workspace,
                                      const DecodePlan &plan, int32_t *dev_status, cudaStream_t stream,
@@ -1025,6 +1028,8 @@ cudaError_t launch_sparse_mla_decode(bool staged, const void *q_nope, const void
     a.table_stride = table_stride;
     a.page_shift = page_shift;
     a.max_pos = block_table ? (table_stride << page_shift) : 0;
+    a.rows_by_slot = rows == RowSource::kFp8Cache;
+    const bool staged = rows != RowSource::kNvfp4Cache;
     const int64_t nblocks = (int64_t)T * plan.head_groups * plan.splits;
     cudaError_t e;
     switch (plan.heads_per_cta * 2 + (staged ? 1 : 0)) {

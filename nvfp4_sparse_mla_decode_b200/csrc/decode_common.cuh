@@ -31,6 +31,10 @@ struct DecodeArgs {
     int64_t table_stride;  // entries per token row of the table
     int page_shift;        // log2 of the page size
     int64_t max_pos;       // table_stride << page_shift
+    // FP8 (576-byte) rows only: true when `src` is a cache of rows addressed
+    // by slot, false when it is the staging buffer [T][topk] addressed by
+    // list position.
+    bool rows_by_slot;
 };
 
 #ifdef NVFP4MLA_TRACE

@@ -29,14 +29,23 @@ bool make_decode_plan(int32_t T, int32_t H, int32_t topk, int sm_count, DecodePl
 // (pure host use, e.g. sizing a workspace on a machine without a GPU).
 int current_device_sm_count();
 
-// Sparse MLA decode over NVFP4 rows (staged == false: `src` is the cache of
-// num_slots 352-byte rows, list entries are slots) or over the staging
-// buffer (staged == true: `src` is [T, topk, 576] E4M3 rows addressed by list
-// position; entries outside [0, num_slots) are still the empty ones).
-// block_table (optional): list entries are then request-local positions,
-// translated through table[t][pos >> page_shift] (table_stride entries per
-// token) while the list is compacted.
-cudaError_t launch_sparse_mla_decode(bool staged, const void *q_nope, const void *q_rope, const uint8_t *src,
+cudaError_t launch_fp8_kv_append(const void *latent, int64_t latent_stride, const void *rope, int64_t rope_stride,
+                                 const int32_t *slot_mapping, int32_t n, uint8_t *cache, int64_t num_slots,
+                                 int32_t *dev_status, cudaStream_t stream);
+
+// What the decode's `src` holds.
+enum class RowSource {
+    kNvfp4Cache,  // num_slots 352-byte NVFP4 rows; list entries are slots
+    kFp8Staging,  // [T, topk] 576-byte E4M3 rows addressed by list position;
+                  // entries outside [0, num_slots) are still the empty ones
+    kFp8Cache,    // num_slots 576-byte E4M3 rows; list entries are slots
+};
+
+// Sparse MLA decode over `src` (see RowSource).  block_table (optional):
+// list entries are then request-local positions, translated through
+// table[t][pos >> page_shift] (table_stride entries per token) while the
+// list is compacted.
+cudaError_t launch_sparse_mla_decode(RowSource rows, const void *q_nope, const void *q_rope, const uint8_t *src,
                                      int64_t num_slots, const int32_t *indices, int32_t topk, int32_t T,
                                      int32_t H, float sm_scale, void *out, float *lse, void *workspace,
                                      const DecodePlan &plan, int32_t *dev_status, cudaStream_t stream,

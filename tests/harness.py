@@ -18,19 +18,21 @@ def bf16_bits(t: torch.Tensor) -> np.ndarray:
     return t.detach().contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
 
 
-from nvfp4_sparse_mla_decode_b200.cache import build_cache  # noqa: E402,F401
+from nvfp4_sparse_mla_decode_b200.cache import build_cache, build_fp8_cache  # noqa: E402,F401
 
 
-def oracle_inputs(w: synth.Workload, tokens):
+def oracle_inputs(w: synth.Workload, tokens, fp8_rows=False):
     """Compact oracle problem for the given tokens: oracle-quantized rows of
-    every valid slot they reference and their lists remapped onto them."""
+    every valid slot they reference (NVFP4, or 576-byte E4M3 rows with
+    fp8_rows) and their lists remapped onto them."""
     import oracle
     tokens = list(tokens)
     idx = w.indices[tokens].cpu().numpy().astype(np.int64)
     valid = (idx >= 0) & (idx < w.num_slots)
     slots = np.unique(idx[valid])
     lat, rope = w.source_rows(torch.from_numpy(slots).to(w.indices.device))
-    rows = oracle.quantize_rows(bf16_bits(lat), bf16_bits(rope))
+    quantize = oracle.quantize_fp8_rows if fp8_rows else oracle.quantize_rows
+    rows = quantize(bf16_bits(lat), bf16_bits(rope))
     pos = np.searchsorted(slots, np.where(valid, idx, 0))
     remap = np.where(valid, pos, -1).astype(np.int32)
     qn = w.q_nope[tokens].cpu().numpy()
@@ -38,10 +40,10 @@ def oracle_inputs(w: synth.Workload, tokens):
     return qn, qr, rows, remap, slots
 
 
-def oracle_decode(w: synth.Workload, tokens, staged=False):
+def oracle_decode(w: synth.Workload, tokens, staged=False, fp8_rows=False):
     import oracle
-    qn, qr, rows, remap, _ = oracle_inputs(w, tokens)
-    return oracle.sparse_mla(qn, qr, rows, remap, w.sm_scale, staged=staged)
+    qn, qr, rows, remap, _ = oracle_inputs(w, tokens, fp8_rows=fp8_rows)
+    return oracle.sparse_mla(qn, qr, rows, remap, w.sm_scale, staged=staged, fp8_rows=fp8_rows)
 
 
 def check_close(out: torch.Tensor, lse: torch.Tensor, ref_out: np.ndarray, ref_lse: np.ndarray,

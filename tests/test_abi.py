@@ -147,3 +147,33 @@ def test_paged_argument_errors(L):
     assert call(tb=None) == INVALID
     assert call(tb=(1 << 20) + 2) == INVALID
     assert call(stride=1 << 20, page=1 << 12) == INVALID   # positions would overflow int32
+
+
+def test_fp8_append_argument_errors(L):
+    f = L.nvfp4mla_fp8_kv_append
+    assert f(None, 512, None, 64, None, 0, None, 10, None, None) == 0
+    assert f(None, 512, 1 << 20, 64, 1 << 20, 4, 1 << 20, 10, None, None) == 1
+    assert f(1 << 20, 500, 1 << 20, 64, 1 << 20, 4, 1 << 20, 10, None, None) == 1
+    assert f(1 << 20, 512, 1 << 20, 64, 1 << 20, 4, (1 << 20) + 8, 10, None, None) == 1   # cache misaligned
+    assert f(1 << 20, 512, 1 << 20, 64, 1 << 20, -1, 1 << 20, 10, None, None) == 1
+
+
+def test_fp8_decode_argument_errors(L):
+    INVALID, UNSUP, WS = 1, 2, 3
+    f = L.nvfp4mla_fp8_sparse_mla_decode
+
+    def call(**kw):
+        a = dict(q=1 << 20, qr=1 << 20, cache=1 << 20, ns=100, idx=1 << 20, topk=2048, T=1, H=64, sc=0.1,
+                 out=1 << 20, lse=1 << 20, ws=1 << 20, wsb=1 << 30, st=None, stream=None)
+        a.update(kw)
+        return f(a["q"], a["qr"], a["cache"], a["ns"], a["idx"], a["topk"], a["T"], a["H"], a["sc"], a["out"],
+                 a["lse"], a["ws"], a["wsb"], a["st"], a["stream"])
+
+    assert call(T=0) == 0
+    assert call(cache=None) == INVALID
+    assert call(cache=(1 << 20) + 4) == INVALID
+    assert call(ns=0) == INVALID
+    assert call(topk=4096) == INVALID
+    assert call(H=80) == UNSUP
+    assert call(T=35, ws=None, wsb=0) == WS
+    assert call(T=35, ws=(1 << 20) + 16) == INVALID   # workspace not 256-byte aligned
