@@ -5,3 +5,4 @@ Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
 shares no code with it.
 """
 from .oracle import *  # noqa: F401,F403
+from . import indexer  # noqa: F401,E402
