@@ -43,7 +43,8 @@ def parse():
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-extras", action="store_true", help="skip staged/append/e2e/cpu legs")
     ap.add_argument("--workload", default="decode35x64",
-                    choices=["decode35x64", "sweep", "padded", "prefill", "tiny", "paged", "fp8", "all-others"],
+                    choices=["decode35x64", "sweep", "padded", "prefill", "tiny", "paged", "fp8", "indexer",
+                             "all-others"],
                     help="decode35x64 (default) prints the one result line; the others time the remaining "
                          "workloads and print one line per shape")
     ap.add_argument("--launch", default="graph", choices=["graph", "stream"],
@@ -408,15 +409,81 @@ def time_fp8(nv, synth, args):
     torch.cuda.empty_cache()
 
 
+def time_indexer(nv, synth, args):
+    """The sparse indexer on 35 requests of 140,000 positions (page 64): the
+    score kernel, the top-k kernel and both in one call, single launches with
+    L2 flushed, median of 20 each; then the indexer followed by the paged
+    decode over its lists."""
+    import math
+    import torch
+    T, ctx, page = 35, 140_000, synth.PAGE_SIZE
+    w = synth.decode35("cuda")
+    from nvfp4_sparse_mla_decode_b200.cache import build_cache
+    cache = build_cache(w)
+    table = synth.block_table(w)
+    keys = synth.indexer_keys(w.num_slots, 1, "cuda")
+    q, wt = synth.indexer_queries(T, 1, "cuda")
+    lens = torch.tensor(w.ctx_lens, dtype=torch.int32, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    stride = nv.indexer_score_stride(ctx)
+    scores = torch.empty(T, stride, dtype=torch.float32, device="cuda")
+    pos = torch.empty(T, 2048, dtype=torch.int32, device="cuda")
+    ws_i = torch.empty(T * stride * 4, dtype=torch.uint8, device="cuda")
+    out = torch.empty(T, w.H, 512, dtype=torch.float16, device="cuda")
+    lse = torch.empty(T, w.H, dtype=torch.float32, device="cuda")
+    ws = torch.zeros(max(1, nv.workspace_size(T, w.H)), dtype=torch.uint8, device="cuda")
+    flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device="cuda")
+
+    def scores_only():
+        nv.indexer_scores(q, wt, keys, table, page, lens, ctx, scores=scores, dev_status=status)
+
+    def topk_only():
+        nv.indexer_topk(scores, lens, ctx, 2048, positions=pos, dev_status=status)
+
+    def indexer():
+        nv.sparse_indexer(q, wt, keys, table, page, lens, ctx, positions=pos, workspace=ws_i, dev_status=status)
+
+    def indexer_then_decode():
+        indexer()
+        nv.decode_paged(w.q_nope, w.q_rope, cache, pos, table, page, w.sm_scale, out=out, lse=lse, workspace=ws,
+                        dev_status=status)
+
+    us = {"scores": cold_median_us(scores_only, flush)}
+    scores_only()
+    us["topk"] = cold_median_us(topk_only, flush)
+    us["indexer"] = cold_median_us(indexer, flush)
+    us["indexer_then_decode"] = cold_median_us(indexer_then_decode, flush)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0, "device status %d" % int(status.item())
+    peaks, _ = measured_peaks()
+    positions = T * ctx
+    pages = T * math.ceil(ctx / page)
+    # algorithmic bytes of the score kernel: keys, table entries, q, w, scores written
+    score_bytes = positions * 128 + pages * 4 + T * 64 * (128 + 4) + positions * 4
+    flop = 2.0 * positions * 64 * 128
+    line = {"metric": METRIC, "workload": "indexer35x140000", "T": T, "ctx": ctx, "page_size": page,
+            "index_heads": 64, "index_dim": 128, "topk": 2048, "us_per_launch": us,
+            "score_kernel_gbs": score_bytes / (us["scores"] * 1e-6) / 1e9,
+            "score_kernel_frac_of_hbm": score_bytes / (us["scores"] * 1e-6) / 1e9 / float(peaks["hbm_gbs"]),
+            "score_kernel_alg_bytes": score_bytes, "score_kernel_tflops_fp8": flop / (us["scores"] * 1e-6) / 1e12,
+            "hbm_peak_gbs": float(peaks["hbm_gbs"]),
+            "timing": "single launch, L2 flushed before it, median of 20", "data": "synthetic"}
+    print(json.dumps(line), flush=True)
+    del cache, keys, flush
+    torch.cuda.empty_cache()
+
+
 def other_workloads(args):
     import torch
     import nvfp4_sparse_mla_decode_b200 as nv
     from nvfp4_sparse_mla_decode_b200 import synth
     assert torch.cuda.is_available(), "bench.py needs a CUDA GPU"
     nv.lib()
-    names = (["tiny", "sweep", "padded", "prefill", "paged", "fp8"] if args.workload == "all-others"
+    names = (["tiny", "sweep", "padded", "prefill", "paged", "fp8", "indexer"] if args.workload == "all-others"
              else [args.workload])
     for name in names:
+        if name == "indexer":
+            time_indexer(nv, synth, args)
         if name == "paged":
             time_paged(nv, synth, args)
         if name == "fp8":

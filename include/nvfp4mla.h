@@ -50,6 +50,8 @@ extern "C" {
 #define NVFP4MLA_GROUP 16
 #define NVFP4MLA_MAX_TOPK 2048        /* positions of one index list */
 #define NVFP4MLA_MAX_HEADS 128
+#define NVFP4MLA_INDEX_HEADS 64       /* sparse indexer heads */
+#define NVFP4MLA_INDEX_DIM 128        /* dims (= E4M3 bytes) of an indexer key or query head */
 
 typedef enum {
     NVFP4MLA_OK = 0,
@@ -257,6 +259,69 @@ nvfp4mla_status nvfp4mla_fp8_sparse_mla_decode(const void *q_nope_f16, const voi
                                                int32_t topk, int32_t T, int32_t H, float sm_scale, void *out_f16,
                                                float *lse, void *workspace, size_t workspace_bytes,
                                                int32_t *dev_status, void *stream);
+
+/*
+ * Sparse indexer: the step that produces the decode's index lists (same page
+ * and section: a sparse indexer picks the rows each token's attention reads
+ * and hands over 2,048 positions).  The page gives no scoring function; the
+ * one computed here is the lightning-indexer form of DeepSeek sparse
+ * attention:
+ *   I[t, p] = sum_h w[t, h] * max(0, sum_d q[t, h, d] * k[slot(t, p), d])
+ * over 64 heads h and 128 dims d, q and k E4M3 bytes, w FP32, for context
+ * positions 0 <= p < ctx_lens[t], slot(t, p) = block_table[t][p / page] *
+ * page + p % page.  The list of token t holds the min(topk, ctx_lens[t])
+ * positions with the largest scores (equal scores: smaller position first;
+ * -0 equals +0) in increasing position order, then -1 -- request-local
+ * positions, the input of nvfp4_sparse_mla_decode_paged.
+ *
+ * Common arguments (device pointers, caller-owned):
+ *   q_fp8        [T, 64, 128] E4M3 bytes, 16-byte aligned
+ *   weights      [T, 64] FP32
+ *   keys_fp8     [num_slots, 128] E4M3 bytes, 16-byte aligned; 1 <= num_slots <= INT32_MAX
+ *   block_table  [T, table_stride] int32 page ids (negative = no page);
+ *                a position whose page entry is negative or whose page
+ *                leaves the key cache scores -inf and sets
+ *                NVFP4MLA_DEV_BAD_INDEX
+ *   page_size    a power of two in [8, 2^20]
+ *   ctx_lens     [T] int32; a length outside [0, max_ctx] is clamped and
+ *                sets NVFP4MLA_DEV_BAD_INDEX
+ *   max_ctx      host-side bound on every ctx_lens[t];
+ *                max_ctx <= table_stride * page_size
+ *   scores       [T, score_stride] FP32, 16-byte aligned; score_stride >=
+ *                max_ctx and a multiple of 4; only positions < ctx_lens[t]
+ *                are written or read
+ *   positions    [T, topk] int32, 1 <= topk <= 2048
+ * Scores accumulate in FP32 on the tensor cores; which of two nearly equal
+ * scores ranks first may differ from an exact evaluation.  NaN scores are
+ * not supported.
+ */
+
+/* Bytes of the score buffer nvfp4mla_sparse_indexer needs:
+ * T * nvfp4mla_indexer_score_stride(max_ctx) * 4 (0 for bad arguments). */
+size_t nvfp4mla_indexer_workspace_size(int32_t T, int32_t max_ctx);
+/* The score row stride (floats) nvfp4mla_sparse_indexer uses: max_ctx rounded up to 128. */
+int64_t nvfp4mla_indexer_score_stride(int32_t max_ctx);
+
+/* Scores of every context position of every token (first half of the
+ * indexer). */
+nvfp4mla_status nvfp4mla_indexer_scores(const uint8_t *q_fp8, const float *weights, const uint8_t *keys_fp8,
+                                        int64_t num_slots, const int32_t *block_table, int32_t table_stride,
+                                        int32_t page_size, const int32_t *ctx_lens, int32_t max_ctx, int32_t T,
+                                        float *scores, int64_t score_stride, int32_t *dev_status, void *stream);
+
+/* Selection over given scores (second half): positions[t] = the list
+ * described above for scores[t, 0:ctx_lens[t]]. */
+nvfp4mla_status nvfp4mla_indexer_topk(const float *scores, int64_t score_stride, const int32_t *ctx_lens,
+                                      int32_t max_ctx, int32_t T, int32_t topk, int32_t *positions,
+                                      int32_t *dev_status, void *stream);
+
+/* Both halves; the scores go to `workspace` (at least
+ * nvfp4mla_indexer_workspace_size bytes, 16-byte aligned). */
+nvfp4mla_status nvfp4mla_sparse_indexer(const uint8_t *q_fp8, const float *weights, const uint8_t *keys_fp8,
+                                        int64_t num_slots, const int32_t *block_table, int32_t table_stride,
+                                        int32_t page_size, const int32_t *ctx_lens, int32_t max_ctx, int32_t T,
+                                        int32_t topk, int32_t *positions, void *workspace, size_t workspace_bytes,
+                                        int32_t *dev_status, void *stream);
 
 /*
  * nvfp4mla_selftest_wait_timeout -- checks, on the device, that the bounded

@@ -20,7 +20,7 @@ import torch
 __all__ = [
     "ROW_BYTES", "STAGED_ROW_BYTES", "LATENT", "ROPE", "MAX_TOPK", "NVFP4MLAError",
     "lib", "lib_path", "kv_append", "decode", "decode_paged", "decode_noalloc", "staged_decode",
-    "fp8_kv_append", "fp8_decode", "num_splits",
+    "fp8_kv_append", "fp8_decode", "indexer_scores", "indexer_topk", "sparse_indexer", "num_splits",
     "workspace_size", "staging_size", "status_string", "version",
     "DEV_TIMEOUT", "DEV_BAD_INDEX", "DEV_LAYOUT",
 ]
@@ -79,6 +79,18 @@ def lib() -> ctypes.CDLL:
         L.nvfp4mla_fp8_sparse_mla_decode.restype = _i32
         L.nvfp4mla_fp8_sparse_mla_decode.argtypes = [_vp, _vp, _vp, _i64, _vp, _i32, _i32, _i32, _f32, _vp, _vp,
                                                      _vp, _sz, _vp, _vp]
+        L.nvfp4mla_indexer_workspace_size.restype = _sz
+        L.nvfp4mla_indexer_workspace_size.argtypes = [_i32, _i32]
+        L.nvfp4mla_indexer_score_stride.restype = _i64
+        L.nvfp4mla_indexer_score_stride.argtypes = [_i32]
+        L.nvfp4mla_indexer_scores.restype = _i32
+        L.nvfp4mla_indexer_scores.argtypes = [_vp, _vp, _vp, _i64, _vp, _i32, _i32, _vp, _i32, _i32, _vp, _i64,
+                                              _vp, _vp]
+        L.nvfp4mla_indexer_topk.restype = _i32
+        L.nvfp4mla_indexer_topk.argtypes = [_vp, _i64, _vp, _i32, _i32, _i32, _vp, _vp, _vp]
+        L.nvfp4mla_sparse_indexer.restype = _i32
+        L.nvfp4mla_sparse_indexer.argtypes = [_vp, _vp, _vp, _i64, _vp, _i32, _i32, _vp, _i32, _i32, _i32, _vp,
+                                              _vp, _sz, _vp, _vp]
         L.nvfp4mla_selftest_wait_timeout.restype = _i32
         L.nvfp4mla_selftest_wait_timeout.argtypes = [_vp, _vp, _vp]
         L.nvfp4mla_status_string.restype = ctypes.c_char_p
@@ -268,6 +280,75 @@ def fp8_decode(q_nope: torch.Tensor, q_rope: torch.Tensor, fp8_cache: torch.Tens
                                               if workspace is not None else 0, _ptr(dev_status), _stream(dev))
     _check(st, "nvfp4mla_fp8_sparse_mla_decode")
     return out, lse
+
+
+def _indexer_inputs(q, w, keys, block_table, ctx_lens):
+    dev = _need_cuda(q, w, keys, block_table, ctx_lens)
+    T = q.shape[0]
+    assert q.dtype == torch.uint8 and q.shape == (T, 64, 128) and q.is_contiguous()
+    assert w.dtype == torch.float32 and w.shape == (T, 64) and w.is_contiguous()
+    assert keys.dtype == torch.uint8 and keys.dim() == 2 and keys.shape[1] == 128 and keys.is_contiguous()
+    assert block_table.dtype == torch.int32 and block_table.dim() == 2 and block_table.shape[0] == T
+    assert block_table.is_contiguous()
+    assert ctx_lens.dtype == torch.int32 and ctx_lens.shape == (T,) and ctx_lens.is_contiguous()
+    return dev, T
+
+
+def indexer_score_stride(max_ctx: int) -> int:
+    return int(lib().nvfp4mla_indexer_score_stride(max_ctx))
+
+
+def indexer_scores(q: torch.Tensor, w: torch.Tensor, keys: torch.Tensor, block_table: torch.Tensor,
+                   page_size: int, ctx_lens: torch.Tensor, max_ctx: int, scores: Optional[torch.Tensor] = None,
+                   dev_status: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Indexer scores float32 [T, stride] (positions >= ctx_lens[t] untouched).
+    q uint8 [T,64,128] E4M3, w float32 [T,64], keys uint8 [num_slots,128]
+    E4M3, block_table int32 [T, width], ctx_lens int32 [T]."""
+    dev, T = _indexer_inputs(q, w, keys, block_table, ctx_lens)
+    if scores is None:
+        scores = torch.empty(T, max(1, indexer_score_stride(max_ctx)), dtype=torch.float32, device=dev)
+    assert scores.dtype == torch.float32 and scores.dim() == 2 and scores.stride(1) == 1
+    st = lib().nvfp4mla_indexer_scores(_ptr(q), _ptr(w), _ptr(keys), keys.shape[0], _ptr(block_table),
+                                       block_table.shape[1], int(page_size), _ptr(ctx_lens), int(max_ctx), T,
+                                       _ptr(scores), scores.stride(0), _ptr(dev_status), _stream(dev))
+    _check(st, "nvfp4mla_indexer_scores")
+    return scores
+
+
+def indexer_topk(scores: torch.Tensor, ctx_lens: torch.Tensor, max_ctx: int, topk: int = MAX_TOPK,
+                 positions: Optional[torch.Tensor] = None, dev_status: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Top-k positions int32 [T, topk] of scores float32 [T, stride]."""
+    dev = _need_cuda(scores, ctx_lens)
+    T = ctx_lens.shape[0]
+    assert scores.dtype == torch.float32 and scores.dim() == 2 and scores.stride(1) == 1 and scores.shape[0] == T
+    assert ctx_lens.dtype == torch.int32 and ctx_lens.is_contiguous()
+    if positions is None:
+        positions = torch.empty(T, topk, dtype=torch.int32, device=dev)
+    st = lib().nvfp4mla_indexer_topk(_ptr(scores), scores.stride(0), _ptr(ctx_lens), int(max_ctx), T, int(topk),
+                                     _ptr(positions), _ptr(dev_status), _stream(dev))
+    _check(st, "nvfp4mla_indexer_topk")
+    return positions
+
+
+def sparse_indexer(q: torch.Tensor, w: torch.Tensor, keys: torch.Tensor, block_table: torch.Tensor,
+                   page_size: int, ctx_lens: torch.Tensor, max_ctx: int, topk: int = MAX_TOPK,
+                   positions: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                   dev_status: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Scores and selection in one call: request-local positions int32
+    [T, topk] (increasing, -1 padded), the input of decode_paged."""
+    dev, T = _indexer_inputs(q, w, keys, block_table, ctx_lens)
+    if positions is None:
+        positions = torch.empty(T, topk, dtype=torch.int32, device=dev)
+    need = int(lib().nvfp4mla_indexer_workspace_size(T, int(max_ctx)))
+    if workspace is None:
+        workspace = torch.empty(max(16, need), dtype=torch.uint8, device=dev)
+    st = lib().nvfp4mla_sparse_indexer(_ptr(q), _ptr(w), _ptr(keys), keys.shape[0], _ptr(block_table),
+                                       block_table.shape[1], int(page_size), _ptr(ctx_lens), int(max_ctx), T,
+                                       int(topk), _ptr(positions), _ptr(workspace),
+                                       workspace.numel() * workspace.element_size(), _ptr(dev_status),
+                                       _stream(dev))
+    _check(st, "nvfp4mla_sparse_indexer")
+    return positions
 
 
 def selftest_wait_timeout(device="cuda") -> int:

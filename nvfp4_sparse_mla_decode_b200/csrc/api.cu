@@ -200,6 +200,67 @@ nvfp4mla_status nvfp4mla_fp8_sparse_mla_decode(const void *q_nope_f16, const voi
                                               dev_status, static_cast<cudaStream_t>(stream)));
 }
 
+size_t nvfp4mla_indexer_workspace_size(int32_t T, int32_t max_ctx) {
+    if (T < 0 || max_ctx < 0 || max_ctx > INT32_MAX - 128) return 0;
+    return (size_t)T * (size_t)indexer_score_stride(max_ctx) * sizeof(float);
+}
+
+int64_t nvfp4mla_indexer_score_stride(int32_t max_ctx) {
+    return (max_ctx < 0 || max_ctx > INT32_MAX - 128) ? 0 : indexer_score_stride(max_ctx);
+}
+
+nvfp4mla_status nvfp4mla_indexer_scores(const uint8_t *q_fp8, const float *weights, const uint8_t *keys_fp8,
+                                        int64_t num_slots, const int32_t *block_table, int32_t table_stride,
+                                        int32_t page_size, const int32_t *ctx_lens, int32_t max_ctx, int32_t T,
+                                        float *scores, int64_t score_stride, int32_t *dev_status, void *stream) {
+    if (T < 0 || max_ctx < 0 || max_ctx > INT32_MAX - 128 || num_slots < 1 || num_slots > INT32_MAX ||
+        table_stride < 1)
+        return NVFP4MLA_ERR_INVALID_ARG;
+    int shift = 0;
+    while (shift < 21 && (1 << shift) < page_size) ++shift;
+    if (page_size < 8 || page_size > (1 << 20) || (1 << shift) != page_size ||
+        (int64_t)max_ctx > (int64_t)table_stride * page_size)
+        return NVFP4MLA_ERR_INVALID_ARG;
+    if (score_stride < max_ctx || score_stride % 4) return NVFP4MLA_ERR_INVALID_ARG;
+    if (T == 0 || max_ctx == 0) return NVFP4MLA_OK;
+    if (!q_fp8 || !weights || !keys_fp8 || !block_table || !ctx_lens || !scores) return NVFP4MLA_ERR_INVALID_ARG;
+    if (!aligned(q_fp8, 16) || !aligned(keys_fp8, 16) || !aligned(weights, 4) || !aligned(block_table, 4) ||
+        !aligned(ctx_lens, 4) || !aligned(scores, 16))
+        return NVFP4MLA_ERR_INVALID_ARG;
+    return from_cuda(launch_indexer_scores(q_fp8, weights, keys_fp8, num_slots, block_table, table_stride, shift,
+                                           ctx_lens, max_ctx, T, scores, score_stride, dev_status,
+                                           static_cast<cudaStream_t>(stream)));
+}
+
+nvfp4mla_status nvfp4mla_indexer_topk(const float *scores, int64_t score_stride, const int32_t *ctx_lens,
+                                      int32_t max_ctx, int32_t T, int32_t topk, int32_t *positions,
+                                      int32_t *dev_status, void *stream) {
+    if (T < 0 || max_ctx < 0 || max_ctx > INT32_MAX - 128 || topk < 1 || topk > NVFP4MLA_MAX_TOPK ||
+        score_stride < max_ctx || score_stride % 4)
+        return NVFP4MLA_ERR_INVALID_ARG;
+    if (T == 0) return NVFP4MLA_OK;
+    if (!ctx_lens || !positions || (max_ctx > 0 && !scores)) return NVFP4MLA_ERR_INVALID_ARG;
+    if (!aligned(scores, 16) || !aligned(ctx_lens, 4) || !aligned(positions, 4)) return NVFP4MLA_ERR_INVALID_ARG;
+    return from_cuda(launch_indexer_topk(scores, score_stride, ctx_lens, max_ctx, T, topk, positions, dev_status,
+                                         static_cast<cudaStream_t>(stream)));
+}
+
+nvfp4mla_status nvfp4mla_sparse_indexer(const uint8_t *q_fp8, const float *weights, const uint8_t *keys_fp8,
+                                        int64_t num_slots, const int32_t *block_table, int32_t table_stride,
+                                        int32_t page_size, const int32_t *ctx_lens, int32_t max_ctx, int32_t T,
+                                        int32_t topk, int32_t *positions, void *workspace, size_t workspace_bytes,
+                                        int32_t *dev_status, void *stream) {
+    if (topk < 1 || topk > NVFP4MLA_MAX_TOPK) return NVFP4MLA_ERR_INVALID_ARG;
+    const size_t need = nvfp4mla_indexer_workspace_size(T, max_ctx);
+    if (T > 0 && max_ctx > 0 && (!workspace || workspace_bytes < need)) return NVFP4MLA_ERR_WORKSPACE;
+    const int64_t stride = nvfp4mla_indexer_score_stride(max_ctx);
+    float *sc = static_cast<float *>(workspace);
+    nvfp4mla_status st = nvfp4mla_indexer_scores(q_fp8, weights, keys_fp8, num_slots, block_table, table_stride,
+                                                 page_size, ctx_lens, max_ctx, T, sc, stride, dev_status, stream);
+    if (st != NVFP4MLA_OK) return st;
+    return nvfp4mla_indexer_topk(sc, stride, ctx_lens, max_ctx, T, topk, positions, dev_status, stream);
+}
+
 nvfp4mla_status nvfp4mla_selftest_wait_timeout(uint32_t *zero_word, int32_t *dev_status, void *stream) {
     if (!zero_word || !dev_status || !aligned(zero_word, 4) || !aligned(dev_status, 4))
         return NVFP4MLA_ERR_INVALID_ARG;

@@ -55,6 +55,16 @@ cudaError_t launch_sparse_mla_decode(RowSource rows, const void *q_nope, const v
 cudaError_t launch_stage_fp8(const uint8_t *cache, int64_t num_slots, const int32_t *indices, int32_t topk,
                              int32_t T, uint8_t *staging, cudaStream_t stream);
 
+// Sparse indexer (indexer.cu).  page_shift = log2(page size) >= 3.
+int64_t indexer_score_stride(int32_t max_ctx);
+cudaError_t launch_indexer_scores(const uint8_t *q, const float *w, const uint8_t *keys, int64_t num_slots,
+                                  const int32_t *table, int64_t table_stride, int page_shift,
+                                  const int32_t *ctx_lens, int32_t max_ctx, int32_t T, float *scores,
+                                  int64_t score_stride, int32_t *dev_status, cudaStream_t stream);
+cudaError_t launch_indexer_topk(const float *scores, int64_t score_stride, const int32_t *ctx_lens, int32_t max_ctx,
+                                int32_t T, int32_t topk, int32_t *positions, int32_t *dev_status,
+                                cudaStream_t stream);
+
 // Bounded-wait self-test: a single CTA whose two waits run out (~1 ms each);
 // `counter` must point at a zero uint32 in device memory.
 cudaError_t launch_wait_timeout_selftest(uint32_t *counter, int32_t *dev_status, cudaStream_t stream);

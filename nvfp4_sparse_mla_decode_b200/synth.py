@@ -268,6 +268,32 @@ def redraw(w: Workload, seed: int) -> tuple[torch.Tensor, torch.Tensor, torch.Te
     return idx, qn, qr
 
 
+INDEX_HEADS = 64
+INDEX_DIM = 128
+
+
+def indexer_keys(num_slots: int, seed: int, device, chunk_rows: int = CHUNK_ROWS) -> torch.Tensor:
+    """Indexer key cache, uint8 [num_slots, 128]: the E4M3 bytes (torch's
+    float8_e4m3fn conversion) of N(0,1) draws, chunk c drawn from a generator
+    seeded by (seed, c)."""
+    out = torch.empty(num_slots, INDEX_DIM, dtype=torch.uint8, device=device)
+    for c, lo in enumerate(range(0, num_slots, chunk_rows)):
+        n = min(chunk_rows, num_slots - lo)
+        g = _gen(device, seed * 6151 + 37 * c + 1)
+        x = torch.randn(n, INDEX_DIM, generator=g, device=device)
+        out[lo:lo + n] = x.to(torch.float8_e4m3fn).view(torch.uint8)
+    return out
+
+
+def indexer_queries(T: int, seed: int, device) -> tuple[torch.Tensor, torch.Tensor]:
+    """Indexer queries uint8 [T, 64, 128] (E4M3 bytes of N(0,1) draws) and
+    head weights float32 [T, 64] (N(0,1) / 8, both signs)."""
+    g = _gen(device, seed * 389 + 23)
+    q = torch.randn(T, INDEX_HEADS, INDEX_DIM, generator=g, device=device)
+    w = torch.randn(T, INDEX_HEADS, generator=g, device=device) / 8
+    return q.to(torch.float8_e4m3fn).view(torch.uint8).contiguous(), w.contiguous()
+
+
 def decode35(device, seed=1, ctx=140_000, T=35, H=64) -> Workload:
     """35 query tokens from 35 requests, each with a 140,000-row context."""
     return per_request(device, [ctx] * T, H, seed, "decode35x64")

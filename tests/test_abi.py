@@ -177,3 +177,36 @@ def test_fp8_decode_argument_errors(L):
     assert call(H=80) == UNSUP
     assert call(T=35, ws=None, wsb=0) == WS
     assert call(T=35, ws=(1 << 20) + 16) == INVALID   # workspace not 256-byte aligned
+
+
+def test_indexer_argument_errors(L):
+    INVALID, WS = 1, 3
+    f = L.nvfp4mla_indexer_scores
+
+    def call(**kw):
+        a = dict(q=1 << 20, w=1 << 20, k=1 << 20, ns=4096, tb=1 << 20, tbs=64, page=64, lens=1 << 20,
+                 maxc=4096, T=2, sc=1 << 20, scs=4096, st=None, stream=None)
+        a.update(kw)
+        return f(a["q"], a["w"], a["k"], a["ns"], a["tb"], a["tbs"], a["page"], a["lens"], a["maxc"], a["T"],
+                 a["sc"], a["scs"], a["st"], a["stream"])
+
+    assert call(T=0) == 0
+    assert call(maxc=0) == 0
+    assert call(page=48) == INVALID           # not a power of two
+    assert call(page=4) == INVALID            # below the 8-row copy
+    assert call(maxc=64 * 64 + 1) == INVALID  # more positions than the table can map
+    assert call(scs=4095) == INVALID
+    assert call(scs=4098) == INVALID          # not a multiple of 4
+    assert call(k=(1 << 20) + 8) == INVALID   # key cache misaligned
+    assert call(sc=(1 << 20) + 4) == INVALID
+    assert call(q=None) == INVALID
+    t = L.nvfp4mla_indexer_topk
+    assert t(1 << 20, 4096, 1 << 20, 4096, 2, 0, 1 << 20, None, None) == INVALID       # topk 0
+    assert t(1 << 20, 4096, 1 << 20, 4096, 2, 4096, 1 << 20, None, None) == INVALID    # topk > 2048
+    assert t(1 << 20, 4096, 1 << 20, 4096, 0, 2048, 1 << 20, None, None) == 0
+    s = L.nvfp4mla_sparse_indexer
+    base = [1 << 20, 1 << 20, 1 << 20, 4096, 1 << 20, 64, 64, 1 << 20, 4096, 2, 2048, 1 << 20]
+    assert s(*base, None, 0, None, None) == WS
+    assert s(*base, 1 << 20, 1000, None, None) == WS
+    assert L.nvfp4mla_indexer_workspace_size(35, 140000) == 35 * 140032 * 4
+    assert L.nvfp4mla_indexer_score_stride(140000) == 140032
