@@ -428,7 +428,9 @@ def time_indexer(nv, synth, args):
     stride = nv.indexer_score_stride(ctx)
     scores = torch.empty(T, stride, dtype=torch.float32, device="cuda")
     pos = torch.empty(T, 2048, dtype=torch.int32, device="cuda")
-    ws_i = torch.empty(T * stride * 4, dtype=torch.uint8, device="cuda")
+    ws_i = torch.zeros(nv.lib().nvfp4mla_indexer_workspace_size(T, ctx), dtype=torch.uint8, device="cuda")
+    ws_k = torch.zeros(max(256, nv.lib().nvfp4mla_indexer_topk_workspace_size(T)), dtype=torch.uint8,
+                       device="cuda")
     out = torch.empty(T, w.H, 512, dtype=torch.float16, device="cuda")
     lse = torch.empty(T, w.H, dtype=torch.float32, device="cuda")
     ws = torch.zeros(max(1, nv.workspace_size(T, w.H)), dtype=torch.uint8, device="cuda")
@@ -438,7 +440,7 @@ def time_indexer(nv, synth, args):
         nv.indexer_scores(q, wt, keys, table, page, lens, ctx, scores=scores, dev_status=status)
 
     def topk_only():
-        nv.indexer_topk(scores, lens, ctx, 2048, positions=pos, dev_status=status)
+        nv.indexer_topk(scores, lens, ctx, 2048, positions=pos, workspace=ws_k, dev_status=status)
 
     def indexer():
         nv.sparse_indexer(q, wt, keys, table, page, lens, ctx, positions=pos, workspace=ws_i, dev_status=status)

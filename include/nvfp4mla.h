@@ -296,8 +296,17 @@ nvfp4mla_status nvfp4mla_fp8_sparse_mla_decode(const void *q_nope_f16, const voi
  * not supported.
  */
 
-/* Bytes of the score buffer nvfp4mla_sparse_indexer needs:
- * T * nvfp4mla_indexer_score_stride(max_ctx) * 4 (0 for bad arguments). */
+/* Workspace of nvfp4mla_indexer_topk for T requests on the current device:
+ * 0 when each request's row is handled by one CTA (T >= SMs / 2), else
+ * arrival counters, per-CTA candidate counts and candidate lists.  It must
+ * be zero-filled before its first use; every completed call leaves the
+ * counters at zero again. */
+size_t nvfp4mla_indexer_topk_workspace_size(int32_t T);
+
+/* Workspace of nvfp4mla_sparse_indexer: the score rows
+ * (T * nvfp4mla_indexer_score_stride(max_ctx) floats, rounded up to 256
+ * bytes) followed by nvfp4mla_indexer_topk_workspace_size(T) bytes; zero-fill
+ * it before its first use (0 is returned for bad arguments). */
 size_t nvfp4mla_indexer_workspace_size(int32_t T, int32_t max_ctx);
 /* The score row stride (floats) nvfp4mla_sparse_indexer uses: max_ctx rounded up to 128. */
 int64_t nvfp4mla_indexer_score_stride(int32_t max_ctx);
@@ -310,13 +319,16 @@ nvfp4mla_status nvfp4mla_indexer_scores(const uint8_t *q_fp8, const float *weigh
                                         float *scores, int64_t score_stride, int32_t *dev_status, void *stream);
 
 /* Selection over given scores (second half): positions[t] = the list
- * described above for scores[t, 0:ctx_lens[t]]. */
+ * described above for scores[t, 0:ctx_lens[t]].  workspace: at least
+ * nvfp4mla_indexer_topk_workspace_size(T) bytes, 256-byte aligned (NULL when
+ * that is 0); WORKSPACE when missing or too small. */
 nvfp4mla_status nvfp4mla_indexer_topk(const float *scores, int64_t score_stride, const int32_t *ctx_lens,
                                       int32_t max_ctx, int32_t T, int32_t topk, int32_t *positions,
-                                      int32_t *dev_status, void *stream);
+                                      void *workspace, size_t workspace_bytes, int32_t *dev_status, void *stream);
 
-/* Both halves; the scores go to `workspace` (at least
- * nvfp4mla_indexer_workspace_size bytes, 16-byte aligned). */
+/* Both halves; the scores and the selection's workspace live in
+ * `workspace` (at least nvfp4mla_indexer_workspace_size bytes, 256-byte
+ * aligned, zero-filled before its first use). */
 nvfp4mla_status nvfp4mla_sparse_indexer(const uint8_t *q_fp8, const float *weights, const uint8_t *keys_fp8,
                                         int64_t num_slots, const int32_t *block_table, int32_t table_stride,
                                         int32_t page_size, const int32_t *ctx_lens, int32_t max_ctx, int32_t T,

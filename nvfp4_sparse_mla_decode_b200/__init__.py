@@ -87,7 +87,9 @@ def lib() -> ctypes.CDLL:
         L.nvfp4mla_indexer_scores.argtypes = [_vp, _vp, _vp, _i64, _vp, _i32, _i32, _vp, _i32, _i32, _vp, _i64,
                                               _vp, _vp]
         L.nvfp4mla_indexer_topk.restype = _i32
-        L.nvfp4mla_indexer_topk.argtypes = [_vp, _i64, _vp, _i32, _i32, _i32, _vp, _vp, _vp]
+        L.nvfp4mla_indexer_topk.argtypes = [_vp, _i64, _vp, _i32, _i32, _i32, _vp, _vp, _sz, _vp, _vp]
+        L.nvfp4mla_indexer_topk_workspace_size.restype = _sz
+        L.nvfp4mla_indexer_topk_workspace_size.argtypes = [_i32]
         L.nvfp4mla_sparse_indexer.restype = _i32
         L.nvfp4mla_sparse_indexer.argtypes = [_vp, _vp, _vp, _i64, _vp, _i32, _i32, _vp, _i32, _i32, _i32, _vp,
                                               _vp, _sz, _vp, _vp]
@@ -316,16 +318,24 @@ def indexer_scores(q: torch.Tensor, w: torch.Tensor, keys: torch.Tensor, block_t
 
 
 def indexer_topk(scores: torch.Tensor, ctx_lens: torch.Tensor, max_ctx: int, topk: int = MAX_TOPK,
-                 positions: Optional[torch.Tensor] = None, dev_status: Optional[torch.Tensor] = None) -> torch.Tensor:
-    """Top-k positions int32 [T, topk] of scores float32 [T, stride]."""
+                 positions: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                 dev_status: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Top-k positions int32 [T, topk] of scores float32 [T, stride].  A
+    caller-supplied `workspace` must start zero-filled (completed calls leave
+    its counters at zero)."""
     dev = _need_cuda(scores, ctx_lens)
     T = ctx_lens.shape[0]
     assert scores.dtype == torch.float32 and scores.dim() == 2 and scores.stride(1) == 1 and scores.shape[0] == T
     assert ctx_lens.dtype == torch.int32 and ctx_lens.is_contiguous()
     if positions is None:
         positions = torch.empty(T, topk, dtype=torch.int32, device=dev)
+    need = int(lib().nvfp4mla_indexer_topk_workspace_size(T))
+    if workspace is None and need:
+        workspace = torch.zeros(need, dtype=torch.uint8, device=dev)
     st = lib().nvfp4mla_indexer_topk(_ptr(scores), scores.stride(0), _ptr(ctx_lens), int(max_ctx), T, int(topk),
-                                     _ptr(positions), _ptr(dev_status), _stream(dev))
+                                     _ptr(positions), _ptr(workspace),
+                                     workspace.numel() * workspace.element_size() if workspace is not None else 0,
+                                     _ptr(dev_status), _stream(dev))
     _check(st, "nvfp4mla_indexer_topk")
     return positions
 
@@ -341,7 +351,7 @@ def sparse_indexer(q: torch.Tensor, w: torch.Tensor, keys: torch.Tensor, block_t
         positions = torch.empty(T, topk, dtype=torch.int32, device=dev)
     need = int(lib().nvfp4mla_indexer_workspace_size(T, int(max_ctx)))
     if workspace is None:
-        workspace = torch.empty(max(16, need), dtype=torch.uint8, device=dev)
+        workspace = torch.zeros(max(256, need), dtype=torch.uint8, device=dev)
     st = lib().nvfp4mla_sparse_indexer(_ptr(q), _ptr(w), _ptr(keys), keys.shape[0], _ptr(block_table),
                                        block_table.shape[1], int(page_size), _ptr(ctx_lens), int(max_ctx), T,
                                        int(topk), _ptr(positions), _ptr(workspace),

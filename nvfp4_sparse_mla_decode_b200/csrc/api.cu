@@ -200,9 +200,18 @@ nvfp4mla_status nvfp4mla_fp8_sparse_mla_decode(const void *q_nope_f16, const voi
                                               dev_status, static_cast<cudaStream_t>(stream)));
 }
 
+size_t nvfp4mla_indexer_topk_workspace_size(int32_t T) {
+    return T < 0 ? 0 : indexer_topk_workspace_bytes(T, current_device_sm_count());
+}
+
+// Scores first, then the selection's workspace at a 256-byte boundary.
+static size_t indexer_scores_bytes(int32_t T, int32_t max_ctx) {
+    return ((size_t)T * (size_t)indexer_score_stride(max_ctx) * sizeof(float) + 255) / 256 * 256;
+}
+
 size_t nvfp4mla_indexer_workspace_size(int32_t T, int32_t max_ctx) {
     if (T < 0 || max_ctx < 0 || max_ctx > INT32_MAX - 128) return 0;
-    return (size_t)T * (size_t)indexer_score_stride(max_ctx) * sizeof(float);
+    return indexer_scores_bytes(T, max_ctx) + nvfp4mla_indexer_topk_workspace_size(T);
 }
 
 int64_t nvfp4mla_indexer_score_stride(int32_t max_ctx) {
@@ -234,15 +243,18 @@ nvfp4mla_status nvfp4mla_indexer_scores(const uint8_t *q_fp8, const float *weigh
 
 nvfp4mla_status nvfp4mla_indexer_topk(const float *scores, int64_t score_stride, const int32_t *ctx_lens,
                                       int32_t max_ctx, int32_t T, int32_t topk, int32_t *positions,
-                                      int32_t *dev_status, void *stream) {
+                                      void *workspace, size_t workspace_bytes, int32_t *dev_status, void *stream) {
     if (T < 0 || max_ctx < 0 || max_ctx > INT32_MAX - 128 || topk < 1 || topk > NVFP4MLA_MAX_TOPK ||
         score_stride < max_ctx || score_stride % 4)
         return NVFP4MLA_ERR_INVALID_ARG;
     if (T == 0) return NVFP4MLA_OK;
     if (!ctx_lens || !positions || (max_ctx > 0 && !scores)) return NVFP4MLA_ERR_INVALID_ARG;
     if (!aligned(scores, 16) || !aligned(ctx_lens, 4) || !aligned(positions, 4)) return NVFP4MLA_ERR_INVALID_ARG;
-    return from_cuda(launch_indexer_topk(scores, score_stride, ctx_lens, max_ctx, T, topk, positions, dev_status,
-                                         static_cast<cudaStream_t>(stream)));
+    const size_t need = nvfp4mla_indexer_topk_workspace_size(T);
+    if (need > 0 && (!workspace || workspace_bytes < need)) return NVFP4MLA_ERR_WORKSPACE;
+    if (workspace && !aligned(workspace, 256)) return NVFP4MLA_ERR_INVALID_ARG;
+    return from_cuda(launch_indexer_topk(scores, score_stride, ctx_lens, max_ctx, T, topk, positions, workspace,
+                                         dev_status, static_cast<cudaStream_t>(stream)));
 }
 
 nvfp4mla_status nvfp4mla_sparse_indexer(const uint8_t *q_fp8, const float *weights, const uint8_t *keys_fp8,
@@ -253,12 +265,16 @@ nvfp4mla_status nvfp4mla_sparse_indexer(const uint8_t *q_fp8, const float *weigh
     if (topk < 1 || topk > NVFP4MLA_MAX_TOPK) return NVFP4MLA_ERR_INVALID_ARG;
     const size_t need = nvfp4mla_indexer_workspace_size(T, max_ctx);
     if (T > 0 && max_ctx > 0 && (!workspace || workspace_bytes < need)) return NVFP4MLA_ERR_WORKSPACE;
+    if (workspace && !aligned(workspace, 256)) return NVFP4MLA_ERR_INVALID_ARG;
     const int64_t stride = nvfp4mla_indexer_score_stride(max_ctx);
     float *sc = static_cast<float *>(workspace);
     nvfp4mla_status st = nvfp4mla_indexer_scores(q_fp8, weights, keys_fp8, num_slots, block_table, table_stride,
                                                  page_size, ctx_lens, max_ctx, T, sc, stride, dev_status, stream);
     if (st != NVFP4MLA_OK) return st;
-    return nvfp4mla_indexer_topk(sc, stride, ctx_lens, max_ctx, T, topk, positions, dev_status, stream);
+    const size_t off = T > 0 ? indexer_scores_bytes(T, max_ctx) : 0;
+    uint8_t *tw = workspace ? static_cast<uint8_t *>(workspace) + off : nullptr;
+    return nvfp4mla_indexer_topk(sc, stride, ctx_lens, max_ctx, T, topk, positions, tw,
+                                 workspace_bytes > off ? workspace_bytes - off : 0, dev_status, stream);
 }
 
 nvfp4mla_status nvfp4mla_selftest_wait_timeout(uint32_t *zero_word, int32_t *dev_status, void *stream) {

@@ -24,11 +24,11 @@
 // each with a copy warp, an MMA warp and four epilogue warps, double-buffered
 // accumulators (2 x 64 TMEM columns).
 //
-// Selection (indexer_topk_kernel): one CTA per request, a three-digit radix
-// select (11 + 11 + 10 bits of an order-preserving key) for the k-th largest
-// score, then one ordered pass in which each warp owns a contiguous range of
-// positions and writes its selected positions with ballots, so the list
-// comes out in increasing position order.
+// Selection (indexer_topk_kernel): one CTA per request finds the k-th
+// largest score (a monotone binning of the score range narrows it to one
+// bin, an exact radix select finishes inside that bin), then each warp walks
+// a contiguous range of positions and writes the chosen ones with ballots,
+// so the list comes out in increasing position order.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
@@ -265,8 +265,61 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 }
 
 // ------------------------------------------------------------------ top-k
+// Each request's score row is shared by P CTAs of 1024 threads (P chosen so
+// the grid fills the SMs, at most 8); CTA p owns a contiguous range of the
+// row.  Every pass streams the CTA's range through a ring of three 32 KB
+// shared-memory buffers filled by bulk copies (one thread issues them, an
+// mbarrier per buffer counts the bytes).
+//
+// Usual path:
+//   1. each CTA draws the same sample of whole 32-position lines (at most
+//      8192 keys) and takes tau = the r-th largest, r chosen so that about
+//      1.25 x topk positions of the row should have a key >= tau;
+//   2. one streamed pass over the CTA's range collects the positions with
+//      key >= tau in position order and publishes them (and their count) in
+//      the workspace;
+//   3. the last CTA of the request to arrive on its counter (an atomic add;
+//      nobody waits) concatenates the P lists -- again in position order --
+//      and, if topk <= m <= kCandCap candidates were found, picks the topk
+//      largest with an exact radix select and writes them in order.
+// If tau missed (too few or too many candidates) that last CTA runs the
+// general path over the whole row alone:
+//   A  min and max of the finite scores;
+//   B  histogram of a linear binning of [min, max] into 2048 bins (monotone
+//      in the score: bins above the one holding the topk-th largest score,
+//      d*, are taken whole);
+//   C  the scores of bin d* are collected and an exact radix select among
+//      them gives the threshold key and the number of ties taken;
+//   D  the ordered write: per 8192-position chunk warp w takes positions
+//      256w .. 256w+255, two scans over the warps give its first tie rank
+//      and first output slot, and ballots place the chosen positions;
+// and when even that binning fails (all equal scores, fewer finite scores
+// than topk, too many in bin d*), a three-digit radix select over the whole
+// row replaces A-C.
 constexpr int kTopkThreads = 1024;
 constexpr int kTopkWarps = kTopkThreads / 32;
+constexpr int kBins = 2048;
+constexpr int kChunk = 8192;  // floats per streamed chunk
+constexpr int kRing = 3;
+constexpr int kCandCap = 12288;
+constexpr int kMaxParts = 8;
+constexpr int kTopkDynSmem = kRing * kChunk * 4 + kCandCap * 8;  // 192 KB
+static_assert(kCandCap >= 8192, "the sampled keys (at most 8192) share the candidate area");
+static_assert(kChunk == kTopkWarps * 256, "pass D gives each warp 256 positions of a chunk");
+
+struct TopkArgs {
+    const float *scores;
+    int64_t score_stride;
+    const int32_t *ctx_lens;
+    int max_ctx;
+    int topk;
+    int32_t *out;
+    int parts;           // P: CTAs per request
+    uint32_t *arrivals;  // [T] arrival counters (zero between launches)
+    uint32_t *counts;    // [T][P] candidates found by each CTA
+    uint2 *cand;         // [T][P][kCandCap] (key, position) in position order
+    int32_t *dev_status;
+};
 
 // Order-preserving unsigned key of a score; -0 is first turned into +0 so
 // the two zeros tie.
@@ -300,169 +353,477 @@ __device__ __forceinline__ uint32_t block_incl_scan(uint32_t v, uint32_t *scratc
     return v + before;
 }
 
-__global__ void __launch_bounds__(kTopkThreads, 1)
-    indexer_topk_kernel(const float *__restrict__ scores, int64_t score_stride, const int32_t *__restrict__ ctx_lens,
-                        int max_ctx, int topk, int32_t *__restrict__ out, int32_t *dev_status) {
-    __shared__ uint32_t hist[2048];
-    __shared__ uint32_t scratch[32];
-    __shared__ uint32_t found[2];
-    __shared__ uint32_t wcnt[kTopkWarps][2];
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int t = blockIdx.x;
-    int ctx = __ldg(ctx_lens + t);
-    if (ctx < 0 || ctx > max_ctx) {
-        if (tid == 0) flag(dev_status, NVFP4MLA_DEV_BAD_INDEX);
-        ctx = ctx < 0 ? 0 : max_ctx;
+// Exclusive scan of one value per warp (lane 0's `v`); returns this warp's
+// exclusive prefix and the block total.  Every thread calls it.
+__device__ __forceinline__ uint32_t warp_excl_scan(uint32_t v, uint32_t *slots, uint32_t *total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    if (lane == 0) slots[warp] = v;
+    __syncthreads();
+    if (warp == 0) {
+        const uint32_t x = slots[lane];
+        uint32_t incl = x;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+        }
+        slots[lane] = incl - x;
+        if (lane == 31) *total = incl;
     }
-    int32_t *o = out + (int64_t)t * topk;
-    if (ctx <= topk) {  // every position, then -1
-        for (int i = tid; i < topk; i += kTopkThreads) o[i] = i < ctx ? i : -1;
-        return;
-    }
-    const float *s = scores + (int64_t)t * score_stride;
+    __syncthreads();
+    return slots[warp];
+}
 
-    // Radix select of the topk-th largest key, most significant digit first.
-    uint32_t prefix = 0;        // digits found so far, in place
-    uint32_t remaining = topk;  // how many keys still to take at or below the prefix
+// Given a 1024- or 2048-bin histogram and want >= 1 items to take from the
+// top: out[0] = the bin holding the want-th largest item, out[1] = how many
+// of its items are taken, out[2] = the total count.  Every thread calls it.
+__device__ __forceinline__ void find_bin(const uint32_t *hist, int nb, uint32_t want, uint32_t *scratch,
+                                         uint32_t *out) {
+    const int tid = threadIdx.x;
+    uint32_t c_hi = 0, c_lo = 0;
+    if (2 * tid < nb) {
+        c_hi = hist[nb - 1 - 2 * tid];
+        c_lo = hist[nb - 2 - 2 * tid];
+    }
+    const uint32_t incl = block_incl_scan(c_hi + c_lo, scratch);
+    const uint32_t before = incl - c_hi - c_lo;
+    if (2 * tid < nb) {
+        if (want > before && want <= before + c_hi) {
+            out[0] = (uint32_t)(nb - 1 - 2 * tid);
+            out[1] = want - before;
+        } else if (want > before + c_hi && want <= incl) {
+            out[0] = (uint32_t)(nb - 2 - 2 * tid);
+            out[1] = want - before - c_hi;
+        }
+    }
+    if (tid == kTopkThreads - 1) out[2] = incl;
+    __syncthreads();
+}
+
+__device__ __forceinline__ void add_to_hist(uint32_t *hist, uint32_t d, int lane) {
+    // d == 0xFFFFFFFF: nothing to add; equal digits in a warp add once
+    const uint32_t peers = __match_any_sync(0xffffffffu, d);
+    if (d != 0xFFFFFFFFu && lane == __ffs(peers) - 1) atomicAdd(&hist[d], (uint32_t)__popc(peers));
+}
+
+__device__ __forceinline__ uint32_t radix_digit(uint32_t k, int pass, uint32_t prefix) {
+    const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
+    const int bits = pass == 2 ? 10 : 11;
+    const uint32_t hi_mask = pass == 0 ? 0u : (0xFFFFFFFFu << (shift + bits));
+    return (k & hi_mask) == prefix ? (k >> shift) & ((1u << bits) - 1u) : 0xFFFFFFFFu;
+}
+
+// The want-th largest of n keys in shared memory (want <= n): returns the
+// key; *ties = how many keys equal to it are taken.  Every thread calls it.
+__device__ uint32_t select_in_smem(const uint32_t *keys, uint32_t n, uint32_t want, uint32_t *hist,
+                                   uint32_t *scratch, uint32_t *found, uint32_t *ties) {
+    const int tid = threadIdx.x, lane = tid & 31;
+    uint32_t prefix = 0, remaining = want;
 #pragma unroll 1
     for (int pass = 0; pass < 3; ++pass) {
-        const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
-        const int nb = pass == 2 ? 1024 : 2048;
-        const uint32_t hi_mask = pass == 0 ? 0u : (0xFFFFFFFFu << (shift + (pass == 2 ? 10 : 11)));
-        for (int i = tid; i < 2048; i += kTopkThreads) hist[i] = 0;
+        for (int i = tid; i < kBins; i += kTopkThreads) hist[i] = 0;
         __syncthreads();
-        // every thread runs the same number of rounds, so the warp-wide
-        // match below always sees full warps
-        for (int base = 0; base < ctx; base += 4 * kTopkThreads) {
-            const int p = base + 4 * tid;  // 4 consecutive positions per thread
-            float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (p < ctx) v = __ldcg(reinterpret_cast<const float4 *>(s + p));
-            const float vv[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                uint32_t d = 0xFFFFFFFFu;
-                if (p + e < ctx) {
-                    const uint32_t k = score_key(vv[e]);
-                    if ((k & hi_mask) == prefix) d = (k >> shift) & (uint32_t)(nb - 1);
-                }
-                const uint32_t peers = __match_any_sync(0xffffffffu, d);
-                if (d != 0xFFFFFFFFu && lane == __ffs(peers) - 1) atomicAdd(&hist[d], (uint32_t)__popc(peers));
-            }
+        for (uint32_t base = 0; base < n; base += kTopkThreads) {
+            const uint32_t i = base + tid;
+            add_to_hist(hist, i < n ? radix_digit(keys[i], pass, prefix) : 0xFFFFFFFFu, lane);
         }
         __syncthreads();
-        // Thread i looks at bins nb-1-2i and nb-2-2i (descending); the
-        // running count from the top tells which bin holds the target.
-        uint32_t c_hi = 0, c_lo = 0;
-        if (2 * tid < nb) {
-            c_hi = hist[nb - 1 - 2 * tid];
-            c_lo = hist[nb - 2 - 2 * tid];
-        }
-        const uint32_t incl = block_incl_scan(c_hi + c_lo, scratch);
-        const uint32_t before = incl - c_hi - c_lo;
-        if (2 * tid < nb) {
-            if (remaining > before && remaining <= before + c_hi) {
-                found[0] = (uint32_t)(nb - 1 - 2 * tid);
-                found[1] = remaining - before;
-            } else if (remaining > before + c_hi && remaining <= incl) {
-                found[0] = (uint32_t)(nb - 2 - 2 * tid);
-                found[1] = remaining - before - c_hi;
-            }
-        }
-        __syncthreads();
-        prefix |= found[0] << shift;
+        find_bin(hist, pass == 2 ? 1024 : 2048, remaining, scratch, found);
+        prefix |= found[0] << (pass == 0 ? 21 : (pass == 1 ? 10 : 0));
         remaining = found[1];
         __syncthreads();
     }
-    const uint32_t thr = prefix;     // the topk-th largest key
-    const uint32_t need_eq = remaining;  // keys equal to thr to take, by position
+    *ties = remaining;
+    return prefix;
+}
 
-    // Each warp owns a contiguous range of positions (a multiple of 128).
-    const int seg = ((ctx + kTopkWarps * 128 - 1) / (kTopkWarps * 128)) * 128;
-    const int w_lo = warp * seg;
-    const int w_hi = min(ctx, w_lo + seg);
-    uint32_t gt = 0, eq = 0;
-    for (int base = w_lo; base < w_hi; base += 128) {
-        const int p = base + 4 * lane;
-        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (p < w_hi) v = __ldcg(reinterpret_cast<const float4 *>(s + p));
-        const float vv[4] = {v.x, v.y, v.z, v.w};
+// Write the list from m candidates held in position order: keys above thr,
+// and the first need_eq keys equal to it.
+__device__ void write_from_candidates(const uint32_t *ck, const int32_t *cp, uint32_t m, uint32_t thr,
+                                      uint32_t need_eq, int32_t *o, uint32_t *scratch) {
+    const uint32_t tid = threadIdx.x;
+    const uint32_t per = (m + kTopkThreads - 1) / kTopkThreads;  // each thread owns a contiguous run
+    const uint32_t i0 = min(m, tid * per), i1 = min(m, i0 + per);
+    uint32_t ties = 0;
+    for (uint32_t i = i0; i < i1; ++i) ties += ck[i] == thr;
+    uint32_t tie_rank = block_incl_scan(ties, scratch) - ties;
+    uint32_t sel = 0;
+    for (uint32_t i = i0; i < i1; ++i) {
+        const uint32_t k = ck[i];
+        sel += k > thr || (k == thr && tie_rank++ < need_eq);
+    }
+    uint32_t at = block_incl_scan(sel, scratch) - sel;
+    tie_rank -= ties;
+    for (uint32_t i = i0; i < i1; ++i) {
+        const uint32_t k = ck[i];
+        if (k > thr || (k == thr && tie_rank++ < need_eq)) o[at++] = cp[i];
+    }
+}
+
+__global__ void __launch_bounds__(kTopkThreads, 1) indexer_topk_kernel(const TopkArgs a) {
+    extern __shared__ __align__(128) uint8_t dyn[];
+    float *ring = reinterpret_cast<float *>(dyn);
+    uint32_t *cand_key = reinterpret_cast<uint32_t *>(dyn + kRing * kChunk * 4);
+    int32_t *cand_pos = reinterpret_cast<int32_t *>(cand_key + kCandCap);
+    __shared__ uint64_t full[kRing];
+    __shared__ uint32_t hist[kBins];
+    __shared__ uint32_t scratch[32], slots_a[32], slots_b[32];
+    __shared__ uint32_t found[3], totals[2];
+    __shared__ float red_lo[kTopkWarps], red_hi[kTopkWarps];
+    __shared__ uint32_t ncand, seg_off[kMaxParts + 1];
+    __shared__ int last;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int t = blockIdx.y, part = blockIdx.x, P = a.parts;
+    const int topk = a.topk;
+    int ctx = __ldg(a.ctx_lens + t);
+    if (ctx < 0 || ctx > a.max_ctx) {
+        if (tid == 0 && part == 0) flag(a.dev_status, NVFP4MLA_DEV_BAD_INDEX);
+        ctx = ctx < 0 ? 0 : a.max_ctx;
+    }
+    int32_t *o = a.out + (int64_t)t * topk;
+    if (ctx <= topk) {  // every position, then -1 (no counter is touched)
+        if (part == 0)
+            for (int i = tid; i < topk; i += kTopkThreads) o[i] = i < ctx ? i : -1;
+        return;
+    }
+    const float *s = a.scores + (int64_t)t * a.score_stride;
+    if (tid == 0) {
+        for (int b = 0; b < kRing; ++b) mbar_init(&full[b], 1);
+        fence_mbar_init();
+        ncand = 0;
+    }
+    __syncthreads();
+
+    // ------------------------------------------------------- streaming
+    uint32_t seq = 0;     // chunks streamed through the ring so far
+    uint32_t issued = 0;  // chunks whose copy has been issued (thread 0)
+    bool ok = true;
+    // chunk c of the range starting at r0 (r1 = its end)
+    auto issue = [&](int r0, int r1, int c) {
+        const uint32_t q = seq + (uint32_t)c;
+        const int n = min(kChunk, r1 - r0 - c * kChunk);
+        // whole 16-byte units; r0 is a multiple of kChunk and the row holds
+        // ctx rounded up to 4 floats
+        const uint32_t bytes = ((uint32_t)n * 4u + 15u) & ~15u;
+        uint64_t *bar = &full[q % kRing];
+        mbar_arrive_expect_tx(bar, bytes);
+        bulk_g2s(ring + (q % kRing) * kChunk, s + r0 + (int64_t)c * kChunk, bytes, bar);
+        issued = q + 1;
+    };
+    // One pass over [r0, r1): body(chunk data, chunk index, valid floats)
+    // for every chunk in order.  Returns false (block-uniformly) if a copy
+    // never landed within the bounded wait.
+    auto stream = [&](int r0, int r1, auto &&body) -> bool {
+        const int nchunks = r1 > r0 ? (r1 - r0 + kChunk - 1) / kChunk : 0;
+        if (tid == 0)
+            for (int c = 0; c < min(kRing, nchunks); ++c) issue(r0, r1, c);
+        for (int c = 0; c < nchunks; ++c) {
+            const uint32_t q = seq + (uint32_t)c;
+            const bool got = mbar_wait(&full[q % kRing], (q / kRing) & 1);
+            if (__syncthreads_or(!got)) {
+                seq = q;
+                return false;
+            }
+            body(ring + (q % kRing) * kChunk, c, min(kChunk, r1 - r0 - c * kChunk));
+            __syncthreads();
+            if (tid == 0 && c + kRing < nchunks) issue(r0, r1, c + kRing);
+        }
+        seq += (uint32_t)nchunks;
+        return true;
+    };
+    auto fail = [&]() {  // leave no copy in flight, report, leave
+        if (tid == 0) {
+            for (uint32_t q = seq; q < issued; ++q) (void)mbar_wait(&full[q % kRing], (q / kRing) & 1);
+            flag(a.dev_status, NVFP4MLA_DEV_TIMEOUT);
+        }
+    };
+
+    // ------------------------------------------- 1. sampled threshold tau
+    uint32_t tau;
+    {
+        const int64_t lines = ((int64_t)ctx + 31) / 32;
+        const int lstride = (int)max((int64_t)1, (lines * 32 + 8191) / 8192);
+        const int nsl = (int)((lines + lstride - 1) / lstride);  // sampled lines, <= 256
+        const int last_base = (nsl - 1) * lstride * 32;
+        const uint32_t S = (uint32_t)((nsl - 1) * 32 + min(32, ctx - last_base));
+        uint32_t *samp = cand_key;  // free until step 2
+        uint32_t sk[(8192 / 32 + kTopkWarps - 1) / kTopkWarps];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            if (p + e < w_hi) {
-                const uint32_t k = score_key(vv[e]);
-                gt += k > thr;
-                eq += k == thr;
+        for (int j = 0; j < 8; ++j) {  // all of a warp's line loads in flight at once
+            const int i = warp + kTopkWarps * j;
+            const int p = i * lstride * 32 + lane;
+            sk[j] = (i < nsl && p < ctx) ? score_key(__ldcg(s + p)) : 0u;  // 0 is below every score's key
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int i = warp + kTopkWarps * j;
+            if (i < nsl) samp[i * 32 + lane] = sk[j];
+        }
+        const uint32_t r = (uint32_t)min((int64_t)S, (int64_t)topk * S * 5 / (4 * (int64_t)ctx) + 9);
+        __syncthreads();
+        uint32_t unused;
+        tau = select_in_smem(samp, (uint32_t)nsl * 32, r, hist, scratch, found, &unused);
+    }
+
+    // ------------------------------- 2. collect this CTA's candidates
+    const int span = ((ctx + P - 1) / P + kChunk - 1) / kChunk * kChunk;
+    const int r0 = min(ctx, part * span), r1 = min(ctx, r0 + span);
+    uint32_t m = 0;  // candidates found in the range (block-uniform; may pass the cap)
+    ok = stream(r0, r1, [&](const float *buf, int c, int n) {
+        const float4 fa = reinterpret_cast<const float4 *>(buf)[warp * 64 + lane];
+        const float4 fb = reinterpret_cast<const float4 *>(buf)[warp * 64 + 32 + lane];
+        const float v[8] = {fa.x, fa.y, fa.z, fa.w, fb.x, fb.y, fb.z, fb.w};
+        const int pa = warp * 256 + 4 * lane, pb = pa + 128;  // chunk positions of fa.x and fb.x
+        uint32_t fl = 0, ca = 0, cb = 0;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const int p = (e < 4 ? pa : pb) + (e & 3);
+            const bool f = p < n && score_key(v[e]) >= tau;
+            fl |= (uint32_t)f << e;
+            if (e < 4) ca += f;
+            else cb += f;
+        }
+        // in position order a warp's 128 "a" positions precede its 128 "b"
+        // positions: scan both counts at once (16 bits each)
+        uint32_t packed = ca | (cb << 16);
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const uint32_t y = __shfl_up_sync(0xffffffffu, packed, off);
+            if (lane >= off) packed += y;
+        }
+        const uint32_t tot = __shfl_sync(0xffffffffu, packed, 31);
+        const uint32_t a_before = (packed & 0xFFFFu) - ca;
+        const uint32_t b_before = (tot & 0xFFFFu) + (packed >> 16) - cb;
+        const uint32_t wbase = m + warp_excl_scan((tot & 0xFFFFu) + (tot >> 16), slots_a, &totals[0]);
+        if (fl) {
+            uint32_t ia = wbase + a_before, ib = wbase + b_before;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                if ((fl >> e) & 1u) {
+                    const uint32_t at = e < 4 ? ia++ : ib++;
+                    if (at < (uint32_t)kCandCap) {
+                        cand_key[at] = score_key(v[e]);
+                        cand_pos[at] = r0 + c * kChunk + (e < 4 ? pa : pb) + (e & 3);
+                    }
+                }
             }
         }
+        m += totals[0];
+    });
+    if (!ok) return fail();
+
+    // ----------------------------- 3. the last CTA of the request selects
+    uint32_t mtot = m;
+    if (P > 1) {
+        const int64_t slot = (int64_t)t * P + part;
+        const uint32_t keep = min(m, (uint32_t)kCandCap);
+        uint2 *dst = a.cand + slot * kCandCap;
+        for (uint32_t i = tid; i < keep; i += kTopkThreads) dst[i] = make_uint2(cand_key[i], (uint32_t)cand_pos[i]);
+        if (tid == 0) a.counts[slot] = m;
+        __threadfence();
+        __syncthreads();
+        if (tid == 0) last = atomicAdd(a.arrivals + t, 1u) == (uint32_t)(P - 1);
+        __syncthreads();
+        if (!last) return;
+        __threadfence();
+        if (tid == 0) {
+            a.arrivals[t] = 0;  // ready for the next launch
+            uint32_t acc = 0;
+            bool fits = true;
+            for (int q = 0; q < P; ++q) {
+                const uint32_t mq = __ldcg(a.counts + (int64_t)t * P + q);
+                seg_off[q] = acc;
+                acc += mq;
+                fits &= mq <= (uint32_t)kCandCap;
+            }
+            seg_off[P] = fits ? acc : 0xFFFFFFFFu;
+        }
+        __syncthreads();
+        mtot = seg_off[P];
+        if (mtot >= (uint32_t)topk && mtot <= (uint32_t)kCandCap) {
+            for (int q = 0; q < P; ++q) {  // concatenate in part order = position order
+                const uint2 *src = a.cand + ((int64_t)t * P + q) * kCandCap;
+                const uint32_t off = seg_off[q], mq = seg_off[q + 1] - off;
+                for (uint32_t i = tid; i < mq; i += kTopkThreads) {
+                    const uint2 kp = __ldcg(src + i);
+                    cand_key[off + i] = kp.x;
+                    cand_pos[off + i] = (int32_t)kp.y;
+                }
+            }
+            __syncthreads();
+        }
     }
+    if (mtot >= (uint32_t)topk && mtot <= (uint32_t)kCandCap) {
+        uint32_t need_eq;
+        const uint32_t thr = select_in_smem(cand_key, mtot, (uint32_t)topk, hist, scratch, found, &need_eq);
+        write_from_candidates(cand_key, cand_pos, mtot, thr, need_eq, o, scratch);
+        return;
+    }
+
+    // ---------------------- tau missed: the general path over the whole row
+    for (int i = tid; i < kBins; i += kTopkThreads) hist[i] = 0;
+    if (tid == 0) ncand = 0;
+    __syncthreads();
+    // A: finite range
+    float lo = INFINITY, hi = -INFINITY;
+    ok = stream(0, ctx, [&](const float *buf, int c, int n) {
+        for (int i = tid; i < kChunk / 4; i += kTopkThreads) {
+            const float4 v4 = reinterpret_cast<const float4 *>(buf)[i];
+            const float v[4] = {v4.x, v4.y, v4.z, v4.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                if (4 * i + e < n && v[e] > -INFINITY) {
+                    lo = fminf(lo, v[e]);
+                    hi = fmaxf(hi, v[e]);
+                }
+        }
+    });
+    if (!ok) return fail();
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) {
-        gt += __shfl_xor_sync(0xffffffffu, gt, off);
-        eq += __shfl_xor_sync(0xffffffffu, eq, off);
+        lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, off));
+        hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, off));
     }
     if (lane == 0) {
-        wcnt[warp][0] = gt;
-        wcnt[warp][1] = eq;
+        red_lo[warp] = lo;
+        red_hi[warp] = hi;
     }
     __syncthreads();
-    if (warp == 0) {
-        // per warp: ties before its range, then how many it writes and where
-        const uint32_t g = wcnt[lane][0], e = wcnt[lane][1];
-        uint32_t e_incl = e;
+    lo = red_lo[lane];
+    hi = red_hi[lane];
 #pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-            const uint32_t y = __shfl_up_sync(0xffffffffu, e_incl, off);
-            if (lane >= off) e_incl += y;
-        }
-        const uint32_t e_before = e_incl - e;
-        const uint32_t take = need_eq > e_before ? min(e, need_eq - e_before) : 0u;
-        const uint32_t sel = g + take;
-        uint32_t s_incl = sel;
-#pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-            const uint32_t y = __shfl_up_sync(0xffffffffu, s_incl, off);
-            if (lane >= off) s_incl += y;
-        }
-        __syncwarp();
-        wcnt[lane][0] = s_incl - sel;  // first output slot of this warp
-        wcnt[lane][1] = e_before;      // ties before this warp's range
+    for (int off = 16; off > 0; off >>= 1) {
+        lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, off));
+        hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, off));
     }
-    __syncthreads();
-    uint32_t at = wcnt[warp][0];
-    uint32_t ties = wcnt[warp][1];
+    const float scale = (float)kBins / (hi - lo);
+    bool fast = hi > lo && scale > 0.0f && scale < INFINITY;  // block-uniform
+    // Monotone binning: x <= y gives bin(x) <= bin(y); -inf scores get -1.
+    auto bin = [&](float x) -> int {
+        if (!(x > -INFINITY)) return -1;
+        const int b = (int)((x - lo) * scale);
+        return b < kBins - 1 ? b : kBins - 1;
+    };
+    uint32_t thr = 0, need_eq = 0;  // threshold key and ties taken at it
+    int dstar = 0;                  // threshold bin
+    if (fast) {
+        // B: histogram of the bins
+        ok = stream(0, ctx, [&](const float *buf, int c, int n) {
+            for (int i = tid; i < kChunk / 4; i += kTopkThreads) {
+                const float4 v4 = reinterpret_cast<const float4 *>(buf)[i];
+                const float v[4] = {v4.x, v4.y, v4.z, v4.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int b = 4 * i + e < n ? bin(v[e]) : -1;
+                    if (b >= 0) atomicAdd(&hist[b], 1u);
+                }
+            }
+        });
+        if (!ok) return fail();
+        find_bin(hist, kBins, (uint32_t)topk, scratch, found);
+        fast = found[2] >= (uint32_t)topk;  // enough finite scores
+    }
+    if (fast) {
+        dstar = (int)found[0];
+        const uint32_t want = found[1];  // to take from bin d*
+        // C: the scores of bin d*
+        ok = stream(0, ctx, [&](const float *buf, int c, int n) {
+            for (int i = tid; i < kChunk / 4; i += kTopkThreads) {
+                const float4 v4 = reinterpret_cast<const float4 *>(buf)[i];
+                const float v[4] = {v4.x, v4.y, v4.z, v4.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const bool cnd = 4 * i + e < n && bin(v[e]) == dstar;
+                    const uint32_t cb = __ballot_sync(0xffffffffu, cnd);
+                    if (cb) {
+                        uint32_t at = 0;
+                        if (lane == 0) at = atomicAdd(&ncand, (uint32_t)__popc(cb));
+                        at = __shfl_sync(0xffffffffu, at, 0) + __popc(cb & ((1u << lane) - 1u));
+                        if (cnd && at < (uint32_t)kCandCap) cand_key[at] = score_key(v[e]);
+                    }
+                }
+            }
+        });
+        if (!ok) return fail();
+        const uint32_t mc = ncand;
+        fast = mc <= (uint32_t)kCandCap;
+        if (fast) thr = select_in_smem(cand_key, mc, want, hist, scratch, found, &need_eq);
+    }
+    if (!fast) {
+        // radix select over the whole row
+        dstar = 0;  // every position counts as "in the threshold bin"
+        uint32_t prefix = 0, remaining = (uint32_t)topk;
+#pragma unroll 1
+        for (int pass = 0; pass < 3; ++pass) {
+            for (int i = tid; i < kBins; i += kTopkThreads) hist[i] = 0;
+            __syncthreads();
+            ok = stream(0, ctx, [&](const float *buf, int c, int n) {
+                for (int i = tid; i < kChunk / 4; i += kTopkThreads) {
+                    const float4 v4 = reinterpret_cast<const float4 *>(buf)[i];
+                    const float v[4] = {v4.x, v4.y, v4.z, v4.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        add_to_hist(hist, 4 * i + e < n ? radix_digit(score_key(v[e]), pass, prefix) : 0xFFFFFFFFu,
+                                    lane);
+                }
+            });
+            if (!ok) return fail();
+            find_bin(hist, pass == 2 ? 1024 : 2048, remaining, scratch, found);
+            prefix |= found[0] << (pass == 0 ? 21 : (pass == 1 ? 10 : 0));
+            remaining = found[1];
+            __syncthreads();
+        }
+        thr = prefix;
+        need_eq = remaining;
+    }
+    // D: ordered write
+    uint32_t run_sel = 0, run_ties = 0;  // over the chunks done
     const uint32_t lt_mask = (1u << lane) - 1u;
-    for (int base = w_lo; base < w_hi; base += 128) {
-        const int p = base + 4 * lane;
-        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (p < w_hi) v = __ldcg(reinterpret_cast<const float4 *>(s + p));
-        const float vv[4] = {v.x, v.y, v.z, v.w};
-        // positions in order: element e of every lane, lanes in order, is
-        // NOT increasing position order (lane l holds p..p+3), so walk the
-        // 128 positions as 4 rounds of 32 consecutive ones via shuffles
+    ok = stream(0, ctx, [&](const float *buf, int c, int n) {
+        const float4 fa = reinterpret_cast<const float4 *>(buf)[warp * 64 + lane];
+        const float4 fb = reinterpret_cast<const float4 *>(buf)[warp * 64 + 32 + lane];
+        uint32_t eq_b[8], def_b[8];
+        uint32_t ties = 0;
 #pragma unroll
-        for (int r = 0; r < 4; ++r) {
-            // round r covers positions base + 32r .. base + 32r + 31; lane l
-            // takes position base + 32r + l, held by lane (8r + l/4) as
-            // element l%4
-            const int src = 8 * r + (lane >> 2);
+        for (int r = 0; r < 8; ++r) {
+            // round r: chunk positions 256w + 32r + lane, held by lane
+            // 8(r%4) + lane/4 of fa (r < 4) or fb as element lane%4
+            const int src = 8 * (r & 3) + (lane >> 2);
+            const float4 h = r < 4 ? fa : fb;
+            const float x0 = __shfl_sync(0xffffffffu, h.x, src);
+            const float x1 = __shfl_sync(0xffffffffu, h.y, src);
+            const float x2 = __shfl_sync(0xffffffffu, h.z, src);
+            const float x3 = __shfl_sync(0xffffffffu, h.w, src);
             const int el = lane & 3;
-            const float x0 = __shfl_sync(0xffffffffu, vv[0], src);
-            const float x1 = __shfl_sync(0xffffffffu, vv[1], src);
-            const float x2 = __shfl_sync(0xffffffffu, vv[2], src);
-            const float x3 = __shfl_sync(0xffffffffu, vv[3], src);
             const float x = el == 0 ? x0 : (el == 1 ? x1 : (el == 2 ? x2 : x3));
-            const int q = base + 32 * r + lane;
-            const bool in = q < w_hi;
-            const uint32_t k = in ? score_key(x) : 0u;
-            const bool is_eq = in && k == thr;
-            const uint32_t eq_b = __ballot_sync(0xffffffffu, is_eq);
-            const bool take = in && (k > thr || (is_eq && ties + __popc(eq_b & lt_mask) < need_eq));
-            const uint32_t sel_b = __ballot_sync(0xffffffffu, take);
-            if (take) o[at + __popc(sel_b & lt_mask)] = q;
-            at += __popc(sel_b);
-            ties += __popc(eq_b);
+            const bool in = warp * 256 + 32 * r + lane < n;
+            const uint32_t k = score_key(x);
+            const int bb = fast ? bin(x) : 0;
+            const bool at_thr = in && bb == dstar;
+            eq_b[r] = __ballot_sync(0xffffffffu, at_thr && k == thr);
+            def_b[r] = __ballot_sync(0xffffffffu, in && (bb > dstar || (at_thr && k > thr)));
+            ties += __popc(eq_b[r]);
         }
-    }
+        const uint32_t tie0 = run_ties + warp_excl_scan(ties, slots_a, &totals[0]);
+        uint32_t sel = 0, seen = 0;
+#pragma unroll
+        for (int r = 0; r < 8; ++r) {
+            const bool mine_eq = (eq_b[r] >> lane) & 1u;
+            const bool take_tie = mine_eq && tie0 + seen + __popc(eq_b[r] & lt_mask) < need_eq;
+            def_b[r] |= __ballot_sync(0xffffffffu, take_tie);
+            seen += __popc(eq_b[r]);
+            sel += __popc(def_b[r]);
+        }
+        uint32_t at = run_sel + warp_excl_scan(sel, slots_b, &totals[1]);
+#pragma unroll
+        for (int r = 0; r < 8; ++r) {
+            if ((def_b[r] >> lane) & 1u) o[at + __popc(def_b[r] & lt_mask)] = c * kChunk + warp * 256 + 32 * r + lane;
+            at += __popc(def_b[r]);
+        }
+        run_ties += totals[0];
+        run_sel += totals[1];
+    });
+    if (!ok) return fail();
 }
 
 }  // namespace idx
@@ -540,12 +901,57 @@ cudaError_t launch_indexer_scores(const uint8_t *q, const float *w, const uint8_
     return cudaGetLastError();
 }
 
+int indexer_topk_parts(int32_t T, int sm_count) {
+    if (T <= 0) return 1;
+    const int p = sm_count / T;
+    return p < 1 ? 1 : (p > idx::kMaxParts ? idx::kMaxParts : p);
+}
+
+// Workspace of a split selection: [T] arrival counters, then [T][P] counts,
+// then [T][P][kCandCap] candidates (8 bytes each); sections 256-byte aligned.
+size_t indexer_topk_workspace_bytes(int32_t T, int sm_count) {
+    const int P = indexer_topk_parts(T, sm_count);
+    if (P == 1 || T <= 0) return 0;
+    auto up = [](size_t x) { return (x + 255) / 256 * 256; };
+    return up((size_t)T * 4) + up((size_t)T * P * 4) + (size_t)T * P * idx::kCandCap * 8;
+}
+
 cudaError_t launch_indexer_topk(const float *scores, int64_t score_stride, const int32_t *ctx_lens, int32_t max_ctx,
-                                int32_t T, int32_t topk, int32_t *positions, int32_t *dev_status,
+                                int32_t T, int32_t topk, int32_t *positions, void *workspace, int32_t *dev_status,
                                 cudaStream_t stream) {
     if (T == 0) return cudaSuccess;
-    idx::indexer_topk_kernel<<<(unsigned)T, idx::kTopkThreads, 0, stream>>>(scores, score_stride, ctx_lens, max_ctx,
-                                                                           topk, positions, dev_status);
+    static bool attr_set[64] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64 || !attr_set[dev]) {
+        e = cudaFuncSetAttribute(idx::indexer_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 idx::kTopkDynSmem);
+        if (e != cudaSuccess) return e;
+        if (dev >= 0 && dev < 64) attr_set[dev] = true;
+    }
+    idx::TopkArgs a;
+    a.scores = scores;
+    a.score_stride = score_stride;
+    a.ctx_lens = ctx_lens;
+    a.max_ctx = max_ctx;
+    a.topk = topk;
+    a.out = positions;
+    a.parts = indexer_topk_parts(T, current_device_sm_count());
+    a.dev_status = dev_status;
+    a.arrivals = nullptr;
+    a.counts = nullptr;
+    a.cand = nullptr;
+    if (a.parts > 1) {
+        if (!workspace) return cudaErrorInvalidValue;
+        auto up = [](size_t x) { return (x + 255) / 256 * 256; };
+        uint8_t *w = static_cast<uint8_t *>(workspace);
+        a.arrivals = reinterpret_cast<uint32_t *>(w);
+        a.counts = reinterpret_cast<uint32_t *>(w + up((size_t)T * 4));
+        a.cand = reinterpret_cast<uint2 *>(w + up((size_t)T * 4) + up((size_t)T * a.parts * 4));
+    }
+    idx::indexer_topk_kernel<<<dim3((unsigned)a.parts, (unsigned)T), idx::kTopkThreads, idx::kTopkDynSmem, stream>>>(
+        a);
     return cudaGetLastError();
 }
 

@@ -61,8 +61,13 @@ cudaError_t launch_indexer_scores(const uint8_t *q, const float *w, const uint8_
                                   const int32_t *table, int64_t table_stride, int page_shift,
                                   const int32_t *ctx_lens, int32_t max_ctx, int32_t T, float *scores,
                                   int64_t score_stride, int32_t *dev_status, cudaStream_t stream);
+// Selection splits each request's row over indexer_topk_parts(T) CTAs; more
+// than one needs indexer_topk_workspace_bytes of workspace whose first T
+// words are zero (every completed launch leaves them so).
+int indexer_topk_parts(int32_t T, int sm_count);
+size_t indexer_topk_workspace_bytes(int32_t T, int sm_count);
 cudaError_t launch_indexer_topk(const float *scores, int64_t score_stride, const int32_t *ctx_lens, int32_t max_ctx,
-                                int32_t T, int32_t topk, int32_t *positions, int32_t *dev_status,
+                                int32_t T, int32_t topk, int32_t *positions, void *workspace, int32_t *dev_status,
                                 cudaStream_t stream);
 
 // Bounded-wait self-test: a single CTA whose two waits run out (~1 ms each);

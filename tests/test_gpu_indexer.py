@@ -43,15 +43,13 @@ def _table(ctx, page, seed, spare_pages=3):
     return table, num_pages * page
 
 
-@pytest.mark.parametrize("case", ["normal", "ties", "signed_zeros", "neg_inf"])
-@pytest.mark.parametrize("topk", [2048, 100, 1])
-def test_topk_matches_oracle(case, topk):
-    ctx = [0, 1, 99, 100, 2047, 2048, 2049, 5000, 33333, 140000]
-    T, max_ctx = len(ctx), max(ctx)
-    stride = nv.indexer_score_stride(max_ctx)
-    g = torch.Generator().manual_seed(["normal", "ties", "signed_zeros", "neg_inf"].index(case) * 10007 + topk)
+CASES = ["normal", "ties", "signed_zeros", "neg_inf", "alternating_lines", "rising"]
+
+
+def _scores(case, T, stride, seed):
+    g = torch.Generator().manual_seed(seed)
     s = torch.randn(T, stride, generator=g)
-    if case == "ties":
+    if case == "ties":                   # far more equal scores at the top than topk
         s = torch.randint(-3, 4, (T, stride), generator=g).float()
     elif case == "signed_zeros":
         s = torch.zeros(T, stride)
@@ -59,11 +57,41 @@ def test_topk_matches_oracle(case, topk):
         s[:, ::7] = 1.0
     elif case == "neg_inf":
         s[:, ::5] = -math.inf
+    elif case == "alternating_lines":    # every other 32-position line constant
+        line = torch.arange(stride) // 32
+        s = torch.where((line % 2 == 1)[None, :], torch.ones_like(s), s)
+    elif case == "rising":               # scores grow with position
+        s = s * 0.01 + torch.arange(stride, dtype=torch.float32)[None, :] / 1000
+    return s
+
+
+@pytest.mark.parametrize("case", CASES)
+@pytest.mark.parametrize("topk", [2048, 100, 1])
+def test_topk_matches_oracle(case, topk):
+    ctx = [0, 1, 99, 100, 2047, 2048, 2049, 5000, 33333, 140000]
+    T, max_ctx = len(ctx), max(ctx)
+    stride = nv.indexer_score_stride(max_ctx)
+    s = _scores(case, T, stride, CASES.index(case) * 10007 + topk)
     pos = nv.indexer_topk(s.cuda(), torch.tensor(ctx, dtype=torch.int32, device="cuda"), max_ctx, topk)
     ref = indexer.topk_positions([s[t, :ctx[t]].double().numpy() for t in range(T)], topk)
     got = pos.cpu().numpy()
     bad = [t for t in range(T) if not np.array_equal(got[t], ref[t])]
     assert not bad, "tokens %s differ" % bad
+
+
+@pytest.mark.parametrize("T", [1, 3, 35])
+def test_topk_workspace_reused_across_calls(T):
+    # rows split over several CTAs meet on counters in the workspace; every
+    # call must leave them ready for the next
+    ctx = [140000 - 977 * t for t in range(T)]
+    stride = nv.indexer_score_stride(max(ctx))
+    ws = torch.zeros(max(256, nv.lib().nvfp4mla_indexer_topk_workspace_size(T)), dtype=torch.uint8, device="cuda")
+    lens = torch.tensor(ctx, dtype=torch.int32, device="cuda")
+    for call, case in enumerate(["normal", "rising", "ties", "normal"]):
+        s = _scores(case, T, stride, 500 + call)
+        pos = nv.indexer_topk(s.cuda(), lens, max(ctx), 2048, workspace=ws).cpu().numpy()
+        ref = indexer.topk_positions([s[t, :ctx[t]].double().numpy() for t in range(T)], 2048)
+        assert np.array_equal(pos, ref), "call %d (%s)" % (call, case)
 
 
 def _check_scores(sc, ref, mag, ctx):
