@@ -6,3 +6,4 @@ shares no code with it.
 """
 from .oracle import *  # noqa: F401,F403
 from . import indexer  # noqa: F401,E402
+from . import blhnc  # noqa: F401,E402
