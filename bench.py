@@ -44,7 +44,7 @@ def parse():
     ap.add_argument("--no-extras", action="store_true", help="skip staged/append/e2e/cpu legs")
     ap.add_argument("--workload", default="decode35x64",
                     choices=["decode35x64", "sweep", "padded", "prefill", "tiny", "paged", "fp8", "indexer",
-                             "all-others"],
+                             "blhnc", "all-others"],
                     help="decode35x64 (default) prints the one result line; the others time the remaining "
                          "workloads and print one line per shape")
     ap.add_argument("--launch", default="graph", choices=["graph", "stream"],
@@ -475,15 +475,71 @@ def time_indexer(nv, synth, args):
     torch.cuda.empty_cache()
 
 
+def time_blhnc(nv, synth, args):
+    """The block-major layout conversion for one 200,000-position request
+    (page 64, 352-byte rows) over 64 layers (a representative depth; the
+    pages give none): per-layer caches -> block-major cache with blocks a
+    sixteenth of the size, and back; single launches with L2 flushed, median
+    of 20; plus the descriptor counts of moving that request."""
+    import numpy as np
+    import torch
+    L, N, C, sub, ctx = 64, synth.PAGE_SIZE, 352, 16, 200_000
+    nb = (ctx + N - 1) // N
+    num_blocks = nb + 64
+    rng = np.random.default_rng(5)
+    # the request's blocks: runs of 8 consecutive blocks in random order
+    supers = rng.permutation(num_blocks // 8)
+    ids = (supers[:, None] * 8 + np.arange(8)[None, :]).reshape(-1)[:nb].astype(np.int32)
+    # block-major ids: a packed transfer buffer, and a cache whose free
+    # blocks also come in runs of 8
+    packed = np.arange(nb * sub, dtype=np.int32)
+    nsup = (nb * sub + 7) // 8 + 8
+    frag = (rng.permutation(nsup)[:, None] * 8 + np.arange(8)[None, :]).reshape(-1)[:nb * sub].astype(np.int32)
+    g = torch.Generator(device="cuda").manual_seed(5)
+    caches = [torch.randint(0, 256, (num_blocks, N, C), generator=g, device="cuda", dtype=torch.int32)
+              .to(torch.uint8) for _ in range(L)]
+    out = torch.empty(nsup * 8, L, N // sub, C, dtype=torch.uint8, device="cuda")
+    ptrs = torch.tensor([c.data_ptr() for c in caches], dtype=torch.int64, device="cuda")
+    ids_d = torch.from_numpy(ids).cuda()
+    frag_d = torch.from_numpy(frag).cuda()
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device="cuda")
+    us = {
+        "to_block_major": cold_median_us(lambda: nv.blhnc_convert(caches, ids_d, frag_d, out, sub, True, ptrs,
+                                                                  status), flush),
+        "back": cold_median_us(lambda: nv.blhnc_convert(caches, ids_d, frag_d, out, sub, False, ptrs, status),
+                               flush),
+    }
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0, "device status %d" % int(status.item())
+    peaks, _ = measured_peaks()
+    moved = 2 * nb * N * L * C  # every byte read once and written once
+    line = {"metric": METRIC, "workload": "blhnc200000x64layers", "positions": ctx, "layers": L, "block_size": N,
+            "block_major_block_size": N // sub, "row_bytes": C, "us_per_launch": us,
+            "gbs": {k: moved / (v * 1e-6) / 1e9 for k, v in us.items()},
+            "frac_of_hbm": {k: moved / (v * 1e-6) / 1e9 / float(peaks["hbm_gbs"]) for k, v in us.items()},
+            "bytes_moved": moved,
+            "descriptors": {"per_layer_layout": nv.copy_descriptors(ids, L),
+                            "block_major_fragmented": nv.copy_descriptors(frag),
+                            "block_major_packed": nv.copy_descriptors(packed)},
+            "hbm_peak_gbs": float(peaks["hbm_gbs"]),
+            "timing": "single launch, L2 flushed before it, median of 20", "data": "synthetic"}
+    print(json.dumps(line), flush=True)
+    del caches, out, flush
+    torch.cuda.empty_cache()
+
+
 def other_workloads(args):
     import torch
     import nvfp4_sparse_mla_decode_b200 as nv
     from nvfp4_sparse_mla_decode_b200 import synth
     assert torch.cuda.is_available(), "bench.py needs a CUDA GPU"
     nv.lib()
-    names = (["tiny", "sweep", "padded", "prefill", "paged", "fp8", "indexer"] if args.workload == "all-others"
-             else [args.workload])
+    names = (["tiny", "sweep", "padded", "prefill", "paged", "fp8", "indexer", "blhnc"]
+             if args.workload == "all-others" else [args.workload])
     for name in names:
+        if name == "blhnc":
+            time_blhnc(nv, synth, args)
         if name == "indexer":
             time_indexer(nv, synth, args)
         if name == "paged":

@@ -336,6 +336,43 @@ nvfp4mla_status nvfp4mla_sparse_indexer(const uint8_t *q_fp8, const float *weigh
                                         int32_t *dev_status, void *stream);
 
 /*
+ * Block-major multi-layer layout (same page, section "Fewer copies unlock
+ * NVLink": the BLHNC layout keeps every layer of a block together, with
+ * blocks a sixteenth of the earlier size, so moving a request needs about
+ * ten times fewer copy descriptors).  The page gives no byte layout; the
+ * one used here:
+ *   per-layer caches   layer l: [num_blocks, block_size, row_bytes] bytes
+ *   block-major cache  [num_new_blocks, layers, block_size / sub, row_bytes]
+ * Positions j * (block_size/sub) .. (j+1) * (block_size/sub) - 1 of the
+ * request's i-th block block_ids[i], every layer l, correspond to
+ * block-major block new_block_ids[i * sub + j], layer slot l.
+ *
+ * nvfp4mla_blhnc_convert -- copies the request's data from the per-layer
+ * caches to the block-major cache (to_blhnc = 1) or back (to_blhnc = 0).
+ *   layer_caches   [layers] device array of the per-layer caches' device
+ *                  addresses (each 16-byte aligned)
+ *   block_ids      [nb] int32, new_block_ids [nb * sub] int32
+ *   blhnc          the block-major cache, 16-byte aligned
+ *   row_bytes      a multiple of 16; block_size a multiple of sub
+ * A block id outside [0, num_blocks), a new id outside [0, num_new_blocks)
+ * or a misaligned layer address skips that copy and sets
+ * NVFP4MLA_DEV_BAD_INDEX.  Overlapping destinations race.
+ */
+nvfp4mla_status nvfp4mla_blhnc_convert(const uint64_t *layer_caches, int32_t layers, int64_t num_blocks,
+                                       int32_t block_size, int32_t row_bytes, int32_t sub, const int32_t *block_ids,
+                                       const int32_t *new_block_ids, int32_t nb, uint8_t *blhnc,
+                                       int64_t num_new_blocks, int32_t to_blhnc, int32_t *dev_status, void *stream);
+
+/*
+ * nvfp4mla_copy_descriptors -- host-only descriptor model of a transfer:
+ * layers * (number of runs of consecutive ids in ids[0:n]).  With the
+ * request's block ids and its layer count it counts the copies of the
+ * per-layer layout; with its block-major ids and layers = 1, those of the
+ * block-major layout.  ids is a HOST pointer; returns -1 for bad arguments.
+ */
+int64_t nvfp4mla_copy_descriptors(const int32_t *ids, int32_t n, int32_t layers);
+
+/*
  * nvfp4mla_selftest_wait_timeout -- checks, on the device, that the bounded
  * waits every kernel here uses end with a status instead of hanging: one CTA
  * waits on an mbarrier nothing arrives on and on *zero_word (which must stay

@@ -20,7 +20,8 @@ import torch
 __all__ = [
     "ROW_BYTES", "STAGED_ROW_BYTES", "LATENT", "ROPE", "MAX_TOPK", "NVFP4MLAError",
     "lib", "lib_path", "kv_append", "decode", "decode_paged", "decode_noalloc", "staged_decode",
-    "fp8_kv_append", "fp8_decode", "indexer_scores", "indexer_topk", "sparse_indexer", "num_splits",
+    "fp8_kv_append", "fp8_decode", "indexer_scores", "indexer_topk", "sparse_indexer", "blhnc_convert",
+    "copy_descriptors", "num_splits",
     "workspace_size", "staging_size", "status_string", "version",
     "DEV_TIMEOUT", "DEV_BAD_INDEX", "DEV_LAYOUT",
 ]
@@ -93,6 +94,11 @@ def lib() -> ctypes.CDLL:
         L.nvfp4mla_sparse_indexer.restype = _i32
         L.nvfp4mla_sparse_indexer.argtypes = [_vp, _vp, _vp, _i64, _vp, _i32, _i32, _vp, _i32, _i32, _i32, _vp,
                                               _vp, _sz, _vp, _vp]
+        L.nvfp4mla_blhnc_convert.restype = _i32
+        L.nvfp4mla_blhnc_convert.argtypes = [_vp, _i32, _i64, _i32, _i32, _i32, _vp, _vp, _i32, _vp, _i64, _i32,
+                                             _vp, _vp]
+        L.nvfp4mla_copy_descriptors.restype = _i64
+        L.nvfp4mla_copy_descriptors.argtypes = [_vp, _i32, _i32]
         L.nvfp4mla_selftest_wait_timeout.restype = _i32
         L.nvfp4mla_selftest_wait_timeout.argtypes = [_vp, _vp, _vp]
         L.nvfp4mla_status_string.restype = ctypes.c_char_p
@@ -359,6 +365,39 @@ def sparse_indexer(q: torch.Tensor, w: torch.Tensor, keys: torch.Tensor, block_t
                                        _stream(dev))
     _check(st, "nvfp4mla_sparse_indexer")
     return positions
+
+
+def blhnc_convert(layer_caches, block_ids: torch.Tensor, new_block_ids: torch.Tensor, blhnc: torch.Tensor,
+                  sub: int, to_blhnc: bool = True, layer_ptrs: Optional[torch.Tensor] = None,
+                  dev_status: Optional[torch.Tensor] = None) -> None:
+    """Per-layer caches (list of uint8 [num_blocks, N, C] tensors, equal
+    shapes) <-> block-major cache uint8 [num_new, L, N // sub, C] for the
+    request's blocks.  `layer_ptrs` (int64 device tensor of the caches'
+    addresses) may be passed to avoid rebuilding it per call."""
+    dev = _need_cuda(block_ids, new_block_ids, blhnc, *layer_caches)
+    L = len(layer_caches)
+    nblk, N, C = layer_caches[0].shape
+    assert all(c.shape == (nblk, N, C) and c.dtype == torch.uint8 and c.is_contiguous() for c in layer_caches)
+    assert blhnc.dtype == torch.uint8 and blhnc.is_contiguous() and blhnc.shape[1:] == (L, N // sub, C)
+    assert block_ids.dtype == torch.int32 and new_block_ids.dtype == torch.int32
+    assert block_ids.is_contiguous() and new_block_ids.is_contiguous()
+    assert new_block_ids.numel() == block_ids.numel() * sub
+    if layer_ptrs is None:
+        layer_ptrs = torch.tensor([c.data_ptr() for c in layer_caches], dtype=torch.int64, device=dev)
+    st = lib().nvfp4mla_blhnc_convert(_ptr(layer_ptrs), L, nblk, N, C, int(sub), _ptr(block_ids),
+                                      _ptr(new_block_ids), block_ids.numel(), _ptr(blhnc), blhnc.shape[0],
+                                      1 if to_blhnc else 0, _ptr(dev_status), _stream(dev))
+    _check(st, "nvfp4mla_blhnc_convert")
+
+
+def copy_descriptors(ids, layers: int = 1) -> int:
+    """Host-side descriptor model: layers x runs of consecutive ids."""
+    import numpy as np
+    a = np.ascontiguousarray(np.asarray(ids, dtype=np.int32))
+    r = lib().nvfp4mla_copy_descriptors(a.ctypes.data if a.size else None, a.size, int(layers))
+    if r < 0:
+        raise ValueError("bad arguments")
+    return int(r)
 
 
 def selftest_wait_timeout(device="cuda") -> int:

@@ -277,6 +277,31 @@ nvfp4mla_status nvfp4mla_sparse_indexer(const uint8_t *q_fp8, const float *weigh
                                  workspace_bytes > off ? workspace_bytes - off : 0, dev_status, stream);
 }
 
+nvfp4mla_status nvfp4mla_blhnc_convert(const uint64_t *layer_caches, int32_t layers, int64_t num_blocks,
+                                       int32_t block_size, int32_t row_bytes, int32_t sub, const int32_t *block_ids,
+                                       const int32_t *new_block_ids, int32_t nb, uint8_t *blhnc,
+                                       int64_t num_new_blocks, int32_t to_blhnc, int32_t *dev_status, void *stream) {
+    if (layers < 1 || num_blocks < 1 || block_size < 1 || sub < 1 || block_size % sub || row_bytes < 16 ||
+        row_bytes % 16 || nb < 0 || num_new_blocks < 1 || (to_blhnc != 0 && to_blhnc != 1))
+        return NVFP4MLA_ERR_INVALID_ARG;
+    if ((int64_t)block_size * row_bytes > INT32_MAX) return NVFP4MLA_ERR_INVALID_ARG;
+    if (nb == 0) return NVFP4MLA_OK;
+    if (!layer_caches || !block_ids || !new_block_ids || !blhnc) return NVFP4MLA_ERR_INVALID_ARG;
+    if (!aligned(layer_caches, 8) || !aligned(block_ids, 4) || !aligned(new_block_ids, 4) || !aligned(blhnc, 16))
+        return NVFP4MLA_ERR_INVALID_ARG;
+    return from_cuda(launch_blhnc_convert(layer_caches, layers, num_blocks, block_size, row_bytes, sub, block_ids,
+                                          new_block_ids, nb, blhnc, num_new_blocks, to_blhnc != 0, dev_status,
+                                          static_cast<cudaStream_t>(stream)));
+}
+
+int64_t nvfp4mla_copy_descriptors(const int32_t *ids, int32_t n, int32_t layers) {
+    if (n < 0 || layers < 1 || (n > 0 && !ids)) return -1;
+    int64_t runs = 0;
+    for (int32_t k = 0; k < n; ++k)
+        if (k == 0 || (int64_t)ids[k] != (int64_t)ids[k - 1] + 1) ++runs;
+    return runs * layers;
+}
+
 nvfp4mla_status nvfp4mla_selftest_wait_timeout(uint32_t *zero_word, int32_t *dev_status, void *stream) {
     if (!zero_word || !dev_status || !aligned(zero_word, 4) || !aligned(dev_status, 4))
         return NVFP4MLA_ERR_INVALID_ARG;

@@ -70,6 +70,12 @@ cudaError_t launch_indexer_topk(const float *scores, int64_t score_stride, const
                                 int32_t T, int32_t topk, int32_t *positions, void *workspace, int32_t *dev_status,
                                 cudaStream_t stream);
 
+// Per-layer paged caches <-> block-major multi-layer cache (blhnc.cu).
+cudaError_t launch_blhnc_convert(const uint64_t *layer_ptrs, int32_t layers, int64_t num_blocks, int32_t block_size,
+                                 int32_t row_bytes, int32_t sub, const int32_t *block_ids, const int32_t *new_ids,
+                                 int32_t nb, uint8_t *blhnc, int64_t num_new, bool to_blhnc, int32_t *dev_status,
+                                 cudaStream_t stream);
+
 // Bounded-wait self-test: a single CTA whose two waits run out (~1 ms each);
 // `counter` must point at a zero uint32 in device memory.
 cudaError_t launch_wait_timeout_selftest(uint32_t *counter, int32_t *dev_status, cudaStream_t stream);

@@ -221,3 +221,34 @@ def test_indexer_argument_errors(L):
     # 35 requests x 4 CTAs: counters (140 B -> 256), counts (560 B -> 768), candidates
     assert L.nvfp4mla_indexer_topk_workspace_size(35) == 256 + 768 + 35 * 4 * 12288 * 8
     assert L.nvfp4mla_indexer_score_stride(140000) == 140032
+
+
+def test_blhnc_argument_errors(L):
+    INVALID = 1
+    f = L.nvfp4mla_blhnc_convert
+
+    def call(**kw):
+        a = dict(lp=1 << 20, L=4, nblk=100, N=64, C=352, sub=16, ids=1 << 20, nids=1 << 20, nb=5, out=1 << 20,
+                 nnew=1000, dirn=1, st=None, stream=None)
+        a.update(kw)
+        return f(a["lp"], a["L"], a["nblk"], a["N"], a["C"], a["sub"], a["ids"], a["nids"], a["nb"], a["out"],
+                 a["nnew"], a["dirn"], a["st"], a["stream"])
+
+    assert call(nb=0) == 0
+    assert call(sub=3) == INVALID           # 64 positions do not split in 3
+    assert call(C=350) == INVALID           # rows must be whole 16-byte units
+    assert call(L=0) == INVALID
+    assert call(dirn=2) == INVALID
+    assert call(out=(1 << 20) + 8) == INVALID
+    assert call(lp=None) == INVALID
+
+
+def test_copy_descriptor_model_matches_oracle():
+    import numpy as np
+    from oracle import blhnc
+    rng = np.random.default_rng(3)
+    for _ in range(50):
+        ids = rng.integers(0, 50, size=int(rng.integers(0, 40)))
+        layers = int(rng.integers(1, 100))
+        assert nv.copy_descriptors(ids, layers) == blhnc.descriptors_layer_major(ids, layers)
+        assert nv.copy_descriptors(ids) == blhnc.descriptors_block_major(ids)
