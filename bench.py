@@ -47,6 +47,8 @@ def parse():
                              "blhnc", "all-others"],
                     help="decode35x64 (default) prints the one result line; the others time the remaining "
                          "workloads and print one line per shape")
+    ap.add_argument("--layers", type=int, default=64,
+                    help="layers of the request converted by --workload blhnc")
     ap.add_argument("--launch", default="graph", choices=["graph", "stream"],
                     help="time the K launches replayed from a captured CUDA graph (default) or issued one by one")
     return ap.parse_args()
@@ -477,13 +479,14 @@ def time_indexer(nv, synth, args):
 
 def time_blhnc(nv, synth, args):
     """The block-major layout conversion for one 200,000-position request
-    (page 64, 352-byte rows) over 64 layers (a representative depth; the
-    pages give none): per-layer caches -> block-major cache with blocks a
+    (page 64, 352-byte rows) over --layers layers (64 by default, a
+    representative depth; the pages give none): per-layer caches ->
+    block-major cache with blocks a
     sixteenth of the size, and back; single launches with L2 flushed, median
     of 20; plus the descriptor counts of moving that request."""
     import numpy as np
     import torch
-    L, N, C, sub, ctx = 64, synth.PAGE_SIZE, 352, 16, 200_000
+    L, N, C, sub, ctx = args.layers, synth.PAGE_SIZE, 352, 16, 200_000
     nb = (ctx + N - 1) // N
     num_blocks = nb + 64
     rng = np.random.default_rng(5)
@@ -514,7 +517,7 @@ def time_blhnc(nv, synth, args):
     assert int(status.item()) == 0, "device status %d" % int(status.item())
     peaks, _ = measured_peaks()
     moved = 2 * nb * N * L * C  # every byte read once and written once
-    line = {"metric": METRIC, "workload": "blhnc200000x64layers", "positions": ctx, "layers": L, "block_size": N,
+    line = {"metric": METRIC, "workload": "blhnc200000x%dlayers" % L, "positions": ctx, "layers": L, "block_size": N,
             "block_major_block_size": N // sub, "row_bytes": C, "us_per_launch": us,
             "gbs": {k: moved / (v * 1e-6) / 1e9 for k, v in us.items()},
             "frac_of_hbm": {k: moved / (v * 1e-6) / 1e9 / float(peaks["hbm_gbs"]) for k, v in us.items()},
