@@ -17,12 +17,13 @@
 // (N = 64), the 128 dims the K dimension (four K = 32 steps):
 //   S^T[p, h] = K[p, 0:128] . Q[h, 0:128]      (E4M3 x E4M3 -> FP32 in TMEM)
 // Key pages arrive by TMA (box = min(page, 128) rows x 128 bytes, 128-byte
-// swizzle) into a 4-stage ring; the epilogue reads one TMEM lane (one
+// swizzle) into a 2-stage ring; the epilogue reads one TMEM lane (one
 // position) per thread and folds the 64 heads with ReLU and the weights.
-// The work is HBM-bound (128 key bytes per position against 16K FLOP), so
-// the design goal is to keep every SM streaming keys: several CTAs per SM,
-// each with a copy warp, an MMA warp and four epilogue warps, double-buffered
-// accumulators (2 x 64 TMEM columns).
+// The work is HBM-bound (128 key bytes per position against 16K FLOP), but
+// each CTA's chain (copy -> MMA -> epilogue) handles about one tile per
+// microsecond whatever its depth, so the keys stream best from many short
+// pipelines: four CTAs per SM, each with a copy warp, an MMA warp and four
+// epilogue warps and double-buffered accumulators (2 x 64 TMEM columns).
 //
 // Selection (indexer_topk_kernel): one CTA per request finds the k-th
 // largest score (a monotone binning of the score range narrows it to one
@@ -47,9 +48,9 @@ using namespace ptx;
 constexpr int kHeads = NVFP4MLA_INDEX_HEADS;   // 64
 constexpr int kDimI = NVFP4MLA_INDEX_DIM;      // 128 (bytes per key row)
 constexpr int kTile = 128;                     // positions per tile (MMA M)
-constexpr int kStages = 4;
+constexpr int kStages = 2;
 constexpr int kThreads = 192;                  // warp 0 copies, warp 1 MMA + TMEM, warps 2-5 epilogue
-constexpr int kCtasPerSm = 3;
+constexpr int kCtasPerSm = 4;                  // 4 x 128 TMEM columns = all 512
 constexpr int kStageBytes = kTile * kDimI;     // 16 KB
 constexpr int kOffQ = 0;                       // 64 x 128 B
 constexpr int kOffStage = 8192;
@@ -213,8 +214,17 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         const int row = 32 * wq + lane;
         const uint32_t lane_base = (uint32_t)(32 * wq) << 16;
         const int box = 1 << a.box_shift;
+        const int32_t *trow = a.table + (int64_t)t * a.table_stride;
+        // block-table entry of this thread's position in tile i, read one
+        // tile ahead so the load is off the per-tile critical path
+        auto entry = [&](int i) -> int32_t {
+            const int p = (first + i * (int)gridDim.x) * kTile + row;
+            return (i < n && p < ctx) ? __ldg(trow + (p >> a.page_shift)) : -1;
+        };
+        int32_t blk = entry(0);
         for (int i = 0; i < n; ++i) {
             const int b = i & 1;
+            const int32_t blk_next = entry(i + 1);
             const bool got = mbar_wait(&bars[BAR_TFULL + b], (i >> 1) & 1);
             if (!__all_sync(0xffffffffu, got)) {
                 ok = false;
@@ -228,30 +238,35 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars[BAR_TEMPTY + b]);
-            float acc = 0.0f;
+            // four independent accumulation chains over the heads
+            float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
             for (int h = 0; h < 32; h += 4) {
                 const float4 wv = *reinterpret_cast<const float4 *>(w_s + h);
-                acc = fmaf(wv.x, fmaxf(__uint_as_float(r0[h]), 0.0f), acc);
-                acc = fmaf(wv.y, fmaxf(__uint_as_float(r0[h + 1]), 0.0f), acc);
-                acc = fmaf(wv.z, fmaxf(__uint_as_float(r0[h + 2]), 0.0f), acc);
-                acc = fmaf(wv.w, fmaxf(__uint_as_float(r0[h + 3]), 0.0f), acc);
+                acc[0] = fmaf(wv.x, fmaxf(__uint_as_float(r0[h]), 0.0f), acc[0]);
+                acc[1] = fmaf(wv.y, fmaxf(__uint_as_float(r0[h + 1]), 0.0f), acc[1]);
+                acc[2] = fmaf(wv.z, fmaxf(__uint_as_float(r0[h + 2]), 0.0f), acc[2]);
+                acc[3] = fmaf(wv.w, fmaxf(__uint_as_float(r0[h + 3]), 0.0f), acc[3]);
             }
 #pragma unroll
             for (int h = 0; h < 32; h += 4) {
                 const float4 wv = *reinterpret_cast<const float4 *>(w_s + 32 + h);
-                acc = fmaf(wv.x, fmaxf(__uint_as_float(r1[h]), 0.0f), acc);
-                acc = fmaf(wv.y, fmaxf(__uint_as_float(r1[h + 1]), 0.0f), acc);
-                acc = fmaf(wv.z, fmaxf(__uint_as_float(r1[h + 2]), 0.0f), acc);
-                acc = fmaf(wv.w, fmaxf(__uint_as_float(r1[h + 3]), 0.0f), acc);
+                acc[0] = fmaf(wv.x, fmaxf(__uint_as_float(r1[h]), 0.0f), acc[0]);
+                acc[1] = fmaf(wv.y, fmaxf(__uint_as_float(r1[h + 1]), 0.0f), acc[1]);
+                acc[2] = fmaf(wv.z, fmaxf(__uint_as_float(r1[h + 2]), 0.0f), acc[2]);
+                acc[3] = fmaf(wv.w, fmaxf(__uint_as_float(r1[h + 3]), 0.0f), acc[3]);
             }
+            const float score = (acc[0] + acc[1]) + (acc[2] + acc[3]);
             const int p = (first + i * (int)gridDim.x) * kTile + row;
             if (p < ctx) {
                 // a position whose key copy was refused (empty table entry or
                 // a page outside the cache) scores -inf
-                const bool valid = copy_row(a, t, p & ~(box - 1)) >= 0;
-                a.scores[(int64_t)t * a.score_stride + p] = valid ? acc : -INFINITY;
+                const int p0 = p & ~(box - 1);
+                const int64_t y = ((int64_t)blk << a.page_shift) + (p0 & ((1 << a.page_shift) - 1));
+                const bool valid = blk >= 0 && y + box <= a.num_slots;
+                a.scores[(int64_t)t * a.score_stride + p] = valid ? score : -INFINITY;
             }
+            blk = blk_next;
         }
     }
 
