@@ -25,11 +25,12 @@
 // pipelines: four CTAs per SM, each with a copy warp, an MMA warp and four
 // epilogue warps and double-buffered accumulators (2 x 64 TMEM columns).
 //
-// Selection (indexer_topk_kernel): one CTA per request finds the k-th
-// largest score (a monotone binning of the score range narrows it to one
-// bin, an exact radix select finishes inside that bin), then each warp walks
-// a contiguous range of positions and writes the chosen ones with ballots,
-// so the list comes out in increasing position order.
+// Selection (indexer_topk_kernel): up to 8 CTAs share a request's score row.
+// Each takes a threshold from a sample of the row, streams its part once and
+// publishes the positions at or above it in position order; the last CTA to
+// arrive (an atomic counter, nobody waits) selects exactly among them and
+// writes the list in increasing position order.  If the threshold missed,
+// that CTA falls back to binned or radix passes over the whole row.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
