@@ -2,6 +2,7 @@
 // argument checks, work planning, launches.  Nothing here allocates memory.
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cstdint>
 
 #include "../../include/nvfp4mla.h"
@@ -24,19 +25,24 @@ static_assert(kSplitCounterBytes + size_t(148) * 64 * (NVFP4MLA_LATENT + 2) * 4 
               "the no-allocation scratch must hold every plan on a 148-SM device");
 static __device__ __align__(256) uint8_t g_noalloc_workspace[kNoAllocWorkspaceBytes];
 
-// Device address of the scratch on `dev`, looked up once per device.
+// Device address of the scratch on `dev`, looked up once per device.  The
+// cache is read and written with acquire/release atomics, so first calls from
+// several host threads at once are well defined (they may each look the
+// address up; all of them store the same value).
 void *noalloc_workspace(int dev) {
-    static void *addr[64] = {};
+    static std::atomic<void *> addr[64] = {};
     if (dev < 0 || dev >= 64) return nullptr;
-    if (!addr[dev]) {
+    void *cached = addr[dev].load(std::memory_order_acquire);
+    if (!cached) {
         void *p = nullptr;
         if (cudaGetSymbolAddress(&p, g_noalloc_workspace) != cudaSuccess) {
             (void)cudaGetLastError();
             return nullptr;
         }
-        addr[dev] = p;
+        addr[dev].store(p, std::memory_order_release);
+        cached = p;
     }
-    return addr[dev];
+    return cached;
 }
 
 nvfp4mla_status from_cuda(cudaError_t e) { return e == cudaSuccess ? NVFP4MLA_OK : NVFP4MLA_ERR_CUDA; }

@@ -63,26 +63,28 @@ def test_staged_tiny():
 
 @pytest.mark.parametrize("T", [1, 8, 32, 64, 128, 256])
 def test_sweep_h128(T):
+    # every token and both head groups of every token are compared
     w = synth.sweep("cuda", T)
     cache = build_cache(w)
-    tokens = sorted(set([0, T - 1, T // 2]))
-    run(w, cache, tokens=tokens)
+    run(w, cache)
     del cache
     torch.cuda.empty_cache()
 
 
 def test_padded_lists_256x64():
+    # all 256 tokens: half the lists sorted (empty entries first), half in
+    # random order, lengths from 16 to 2048 valid entries
     w = synth.padded("cuda")
     cache = build_cache(w)
-    tokens = list(range(0, 256, 11)) + [127, 128, 255]
-    run(w, cache, tokens=sorted(set(tokens)))
+    run(w, cache)
 
 
 def test_append_then_prefill_4000x64():
+    # all 4000 tokens of the prefill budget (about 1.1 TFLOP of FP64 work
+    # for the oracle)
     w = synth.append_prefill("cuda")
     cache = build_cache(w)
-    tokens = [0, 1, 2, 999, 2000, 3998, 3999]
-    run(w, cache, tokens=tokens)
+    run(w, cache)
 
 
 def test_all_empty_and_out_of_range_entries():
