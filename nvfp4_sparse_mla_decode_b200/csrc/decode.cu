@@ -409,7 +409,7 @@ __global__ void __launch_bounds__(dec::kThreads, 1)
             const uint64_t dQ0 = smem_desc(smem_u32(smem + kOffQ), 16, 1024);
             const uint64_t dV0 = smem_desc(smem_u32(smem), kChunkBytes, 1024);
             const uint64_t dP0 = smem_desc(smem_u32(smem + 8 * kChunkBytes), kChunkBytes, 1024);
-            bool ok = ntiles == 0 || mbar_wait(&bars[BAR_Q_FULL], 0);
+            bool ok = mbar_wait(&bars[BAR_Q_FULL], 0);  // always: the Q copies must land before the CTA exits
             // Descriptors advance by adding (byte offset >> 4) to the start
             // address field; the chunk and block loops stay rolled so the
             // compiler keeps a handful of descriptors live, not one per MMA.
@@ -484,7 +484,9 @@ __global__ void __launch_bounds__(dec::kThreads, 1)
         for (int i = 0; i < ntiles; ++i) {
             // S_FULL(i) also covers PV(i-1): the MMA thread issued it earlier,
             // so O^T is quiescent and may be rescaled here.
-            if (!mbar_wait(&bars[BAR_S_FULL], i & 1)) {
+            // the wait's outcome is agreed by the whole warpgroup, so its four
+            // warps always meet at the same named barriers
+            if (named_bar_or(bar_id, 128, !mbar_wait(&bars[BAR_S_FULL], i & 1))) {
                 ok = false;
                 break;
             }
@@ -928,7 +930,7 @@ static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 // Encoded maps are kept in a small per-thread cache keyed by (address, rows,
 // cols, box rows), so a caller that reuses its query buffers pays for the
 // encoding once.
-static bool make_q_map(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+bool make_q_map(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
     struct Entry {
         const void *base;
         uint64_t rows, cols;
@@ -1031,6 +1033,7 @@ cudaError_t launch_sparse_mla_decode(RowSource rows, const void *q_nope, const v
     a.rows_by_slot = rows == RowSource::kFp8Cache;
     const bool staged = rows != RowSource::kNvfp4Cache;
     const int64_t nblocks = (int64_t)T * plan.head_groups * plan.splits;
+    if (!staged) return launch_nvfp4_decode(a, plan.heads_per_cta, nblocks, stream);
     cudaError_t e;
     switch (plan.heads_per_cta * 2 + (staged ? 1 : 0)) {
         case 32: e = launch_hg<16, false>(a, nblocks, stream); break;

@@ -2,6 +2,7 @@
 // arguments, base-2 exp/log instructions, softmax-warp barriers, the in-warp
 // transpose reduction and debug-only tracing.
 #pragma once
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <cmath>
@@ -122,6 +123,13 @@ __device__ __forceinline__ int transposed_col(int lane, int j) {
 }
 __host__ __device__ constexpr int cols_per_lane(int W) { return W >= 32 ? W / 32 : 1; }
 
+
+// Tensor map for Q: a 2-D FP16 view [rows = T*H, cols] of q_nope (cols 512)
+// or q_rope (cols 64), box 64 cols x box_rows rows, 128-byte swizzle; encoded
+// maps are cached per host thread, keyed by (address, rows, cols, box rows).
+bool make_q_map(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols, uint32_t box_rows);
+// Launch of the pipelined NVFP4 decode kernel (decode_nvfp4.cu).
+cudaError_t launch_nvfp4_decode(const DecodeArgs &a, int heads_per_cta, int64_t nblocks, cudaStream_t stream);
 
 // N consecutive TMEM columns (32 lanes x 32 bit) in one instruction.
 template <int N>

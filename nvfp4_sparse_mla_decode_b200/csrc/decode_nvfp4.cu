@@ -1,0 +1,905 @@
+// decode_nvfp4.cu -- sparse MLA decode over 352-byte NVFP4 cache rows on the
+// fifth-generation tensor cores of B200 (sm_100a), pipelined so that row
+// gather, on-chip unpack, the score MMAs, the softmax and the output MMAs of
+// neighbouring tiles overlap.
+//
+// What it computes (page "Prime Intellect Launches Prime Inference, Serving
+// 600B Tokens Daily", section "Four-bit caches make room"): each query token
+// attends only to the cache rows its sparse-indexer list names; the rows are
+// unpacked on chip from NVFP4 to FP16; q.k and p.V run with FP16 operands and
+// FP32 accumulation; list entries that name no row take no part.  The same
+// section credits a multi-stage pipeline in which one group of warps unpacks
+// rows while others score and accumulate; this kernel is that idea laid out
+// for sm_100a: every stage has its own warps and its own ring.
+//
+// Work decomposition: one CTA per (token t, head group g of HG <= 64 heads,
+// split s of the token's valid list entries).  The list is compacted once per
+// CTA (empty entries dropped, order kept), so every 128-row tile is full
+// except the last one.
+//
+// Per tile j (rows = the M dimension, heads = N):
+//   S^T[row, h]  = K[row, 0:576] . Q[h, 0:576]      A = K from tensor memory
+//   O^T[dv, h]  += V^T[dv, row] . P^T[row, h]       A = V^T, B = P^T in shared
+// The score MMA reads its K operand from tensor memory (a ring of four
+// 64-dim chunks written by the unpack warps with tcgen05.st), so only Q
+// streams from shared memory.  V is the latent part of the same rows; it is
+// decoded a second time, 16 rows at a time, into a two-slot shared-memory
+// ring in the MN-major layout the output MMA reads.  The MMA warp issues the
+// score MMAs of tile j+1 before the output MMAs of tile j, so the softmax of
+// tile j runs while the tensor core scores the next tile.
+//
+// Warp roles (640 threads, five warpgroups):
+//   warp 0      MMA issue (whole warp, one elected lane issues)
+//   warp 1      gather: the CTA's Q by tensor copies, then one 352-byte bulk
+//               copy per valid row into a two-tile raw ring (rows padded to
+//               368 bytes so the unpack warps read them without bank
+//               conflicts)
+//   warp 2      tensor-memory allocation and release
+//   warps 4-11  K unpack: thread = tile row = TMEM lane; warps 4-7 take the
+//               even 64-dim chunks, warps 8-11 the odd ones (and RoPE)
+//   warps 12-15 softmax (thread = tile row), then the epilogue and the split
+//               merge
+//   warps 16-19 V unpack: 16 rows x 8 dv groups per ring slot, rows read
+//               again from L2 (they arrived one tile earlier)
+//
+// Tensor memory (512 columns): O^T at 0 (four 128-dv blocks of HG columns),
+// S^T double-buffered at 256 and 320, the K ring at 384 (4 x 32 columns).
+//
+// Online softmax in base 2 with a lazily updated reference max: a head's
+// reference moves (and O^T and the row sums are rescaled) only when a score
+// exceeds it by more than 8, so p = 2^(s - m) <= 256 fits FP16.
+//
+// Splits: when T * G alone would leave SMs idle, S CTAs share a token's list;
+// each writes its unnormalised FP32 partial and (max, row sum), the S CTAs
+// meet on a counter (cooperative launch, bounded wait) and each merges one
+// 512/S-wide dv slice of every head.  A CTA whose wait runs out marks the
+// counter poisoned, so later launches on the same workspace report the
+// timeout instead of merging stale partials.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cmath>
+
+#include "common.cuh"
+#include "decode_common.cuh"
+#include "kernels.h"
+#include "ptx.cuh"
+
+namespace nvfp4mla {
+using namespace ptx;
+
+namespace nv4 {
+constexpr int kTileRows = 128;
+constexpr int kMaxHG = 64;
+constexpr int kRawStride = 368;                            // 352-byte row + 16 bytes of padding
+constexpr int kRawSlotBytes = kTileRows * kRawStride;      // 47104
+constexpr int kVRows = 16;                                 // rows per V ring slot (one MMA K step)
+constexpr int kVSlotBytes = kVRows * kLatent * 2;          // 16384
+constexpr int kVGroups = kTileRows / kVRows;               // 8
+constexpr int kKChunks = 9;                                // 8 latent chunks of 64 dims + RoPE
+constexpr int kKSlots = 4;
+constexpr int kOffQ = 0;                                   // 9 chunks x HG rows x 128 B
+constexpr int kOffP = kOffQ + kKChunks * kMaxHG * 128;     // 73728: P^T, 128 rows x 128 B
+constexpr int kOffV = kOffP + kTileRows * 128;             // 90112: two V slots
+constexpr int kOffRaw = kOffV + 2 * kVSlotBytes;           // 122880: two raw tiles
+constexpr int kOffIdx = kOffRaw + 2 * kRawSlotBytes;       // 217088: compacted list share
+constexpr int kOffM = kOffIdx + kMaxTopk * 4;              // reference max per head (log2 units)
+constexpr int kOffAux = kOffM + kMaxHG * 4;                // rescale factors, then 1/l
+constexpr int kOffRed = kOffAux + kMaxHG * 4;              // 4 warps x 64 floats
+constexpr int kOffBar = kOffRed + 4 * kMaxHG * 4;
+constexpr int kNumBars = 24;
+constexpr int kOffMisc = kOffBar + kNumBars * 8;
+constexpr int kSmemBytes = kOffMisc + 64;
+static_assert(kSmemBytes <= 232448, "shared memory budget");
+static_assert(kOffP % 1024 == 0 && kOffV % 1024 == 0, "swizzled operands need 1 KB alignment");
+static_assert(kMaxHG * kLatent * 2 <= 2 * kRawSlotBytes, "output staging must fit in the raw ring");
+static_assert(kMaxHG * (kLatent / 2) * 4 <= 2 * kRawSlotBytes, "own merge slice must fit in the raw ring");
+constexpr int kThreads = 640;
+constexpr int kKWarp0 = 4;
+constexpr int kSoftWarp0 = 12;
+constexpr int kVWarp0 = 16;
+// Register budgets per warpgroup (setmaxnreg): launched with 96 per thread
+// (65536 / 640 rounded down to a multiple of 8); the control warpgroup and
+// the K-unpack warps give registers to the softmax warps, whose threads hold
+// a score and a running row sum per head.
+constexpr int kRegsLaunch = 96;
+constexpr int kRegsCtl = 56;
+constexpr int kRegsK = 72;
+constexpr int kRegsSoft = 184;
+static_assert(128 * kRegsCtl + 256 * kRegsK + 128 * kRegsSoft + 128 * kRegsLaunch <= kThreads * kRegsLaunch,
+              "register split exceeds the launch budget");
+
+// mbarriers
+constexpr int BAR_Q = 0;           // Q tensor copies (expect_tx)
+constexpr int BAR_RAW_FULL = 1;    // [2] raw tile landed (expect_tx)
+constexpr int BAR_RAW_FREE = 3;    // [2] raw tile read by the 8 K-unpack warps
+constexpr int BAR_K_FULL = 5;      // [4] K chunk in TMEM (4 warps)
+constexpr int BAR_K_FREE = 9;      // [4] score MMAs of the chunk done (commit)
+constexpr int BAR_V_FULL = 13;     // [2] V slot written (4 warps)
+constexpr int BAR_V_FREE = 15;     // [2] output MMAs of the slot done (commit)
+constexpr int BAR_S_FULL = 17;     // [2] score MMAs of a tile done (commit)
+constexpr int BAR_P_FULL = 19;     // P^T written, O^T rescaled (4 softmax warps)
+constexpr int BAR_PV_DONE = 20;    // output MMAs of a tile done (commit)
+constexpr int BAR_DRAIN = 21;      // every MMA issued so far done
+constexpr int kBarsUsed = 22;
+static_assert(kBarsUsed <= kNumBars, "barrier slots");
+
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColO = 0;
+constexpr uint32_t kColS = 256;
+constexpr uint32_t kColK = 384;
+constexpr float kRescaleThreshold = 8.0f;
+constexpr int kMaxSplits = 16;
+constexpr uint32_t kPoison = 0x80000000u;
+}  // namespace nv4
+
+// Whole-warp bounded wait: every lane polls, the result is agreed by vote
+// so the warp stays converged for the elected-lane instructions after it.
+__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity) {
+    return __all_sync(0xffffffffu, mbar_wait(bar, parity));
+}
+
+__device__ __forceinline__ uint4 lds128(const uint8_t *p) { return *reinterpret_cast<const uint4 *>(p); }
+__device__ __forceinline__ uint32_t lds32(const uint8_t *p) { return *reinterpret_cast<const uint32_t *>(p); }
+
+// 64 latent dims of one row: 32 nibble bytes (two 16-byte words) and the
+// four E4M3 scales of its 16-dim groups -> 32 f16x2 words, dims 2i, 2i+1 in
+// word i (low half = even dim).  Exact: e2m1 x e4m3 has at most 6
+// significant bits and lies inside FP16's range.
+__device__ __forceinline__ void unpack_latent64(uint4 w0, uint4 w1, uint32_t scales, uint32_t (&o)[32]) {
+    const uint32_t w[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const uint32_t sb = (scales >> (8 * k)) & 0xFFu;
+        const uint32_t s2 = e4m3x2_to_f16x2(sb | (sb << 8));
+        uint32_t lo[4], hi[4];
+        e2m1x8_to_f16x8(w[2 * k], lo);
+        e2m1x8_to_f16x8(w[2 * k + 1], hi);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            o[8 * k + i] = hmul2_u32(lo[i], s2);
+            o[8 * k + 4 + i] = hmul2_u32(hi[i], s2);
+        }
+    }
+}
+
+// Split merge, run by the 128 softmax threads of each of the S CTAs of a
+// (token, head group) once its partial is written: announce the partial on
+// the group's arrival counter (release), wait (bounded) until all S have,
+// then combine dv slice [split*512/S, (split+1)*512/S) of every head:
+//   out = sum_s w_s O_s / sum_s w_s l_s,  w_s = 2^(m_s - max m)
+// over the splits with rows (l_s > 0); split 0 also writes
+// lse = (max m + log2 of the denominator) ln 2.  With S <= 4 the CTA's own
+// slice is in shared memory.  The last CTA to leave resets the counters.  A
+// wait that runs out sets the counter's poison bit: that CTA and every later
+// one on the same counter report NVFP4MLA_DEV_TIMEOUT and write NaN to their
+// slice instead of merging partials that were never written.
+template <int HG, int S>
+__device__ __forceinline__ void merge_splits_nv4(const DecodeArgs &a, int t, int g, int split, uint8_t *smem, int mt) {
+    using namespace nv4;
+    constexpr int kMergeThreads = 128;
+    constexpr int D = kLatent / S;
+    constexpr int NQ = D / 4;
+    constexpr int ITEMS = HG * NQ;
+    constexpr bool kOwnInSmem = S <= 4;
+    constexpr int kGlobal = kOwnInSmem ? S - 1 : S;
+    constexpr int kPerThread = (ITEMS + kMergeThreads - 1) / kMergeThreads;
+    constexpr int B = (24 / kGlobal) < 1 ? 1 : ((24 / kGlobal) > kPerThread ? kPerThread : (24 / kGlobal));
+    uint32_t *arrive = a.counters + 2 * ((int64_t)t * a.G + g);
+    uint32_t *depart = arrive + 1;
+    uint32_t *flag = reinterpret_cast<uint32_t *>(smem + kOffMisc) + 1;
+    float *w_s = reinterpret_cast<float *>(smem + kOffV);   // [S][HG]
+    float *inv_den = w_s + kMaxSplits * HG;                  // [HG]
+    const float *own = reinterpret_cast<const float *>(smem + kOffRaw);  // [HG][D]
+    named_bar(1, kMergeThreads);  // every partial store of this CTA precedes the release
+    if (mt == 0) {
+        __threadfence();
+        const uint32_t old = atomicAdd(arrive, 1u);  // relaxed add; the fence above orders the partials
+        bool ok = (old & kPoison) == 0;
+        if (ok) {
+            const unsigned long long t0 = clock64();
+            while (true) {
+                const uint32_t v = ld_acquire_gpu(arrive);
+                if (v & kPoison) { ok = false; break; }
+                if (v >= (uint32_t)S) break;
+                if (clock64() - t0 > kWaitCycles) { ok = false; break; }
+                __nanosleep(64);
+            }
+        }
+        if (!ok) {
+            atomicOr(arrive, kPoison);
+            if (a.dev_status) atomicOr(a.dev_status, NVFP4MLA_DEV_TIMEOUT);
+        }
+        *flag = ok ? 1u : 0u;
+    }
+    named_bar(1, kMergeThreads);
+    const int dv0 = split * D;
+    __half *dst = a.out + ((int64_t)t * a.H + (int64_t)g * HG) * kLatent + dv0;
+    if (!*flag) {  // poisoned: make the failure visible in the output
+        for (int item = mt; item < HG * D; item += kMergeThreads) {
+            const int h = item / D, d = item - h * D;
+            dst[(int64_t)h * kLatent + d] = __float2half_rn(NAN);
+        }
+        if (split == 0 && mt < HG) a.lse[(int64_t)t * a.H + (int64_t)g * HG + mt] = NAN;
+        return;
+    }
+    const int64_t part = (int64_t)a.H * kLatent;
+    const float *src = a.ws_o + ((int64_t)t * S * a.H + (int64_t)g * HG) * kLatent + dv0;
+    float4 o[B][kGlobal];
+    auto load_batch = [&](int base) {
+#pragma unroll
+        for (int b = 0; b < B; ++b) {
+            const int item = base + b * kMergeThreads;
+            const int h = item / NQ, q = item - h * NQ;
+#pragma unroll
+            for (int j = 0; j < kGlobal; ++j) {
+                const int s = kOwnInSmem && j >= split ? j + 1 : j;
+                o[b][j] = item < ITEMS
+                              ? __ldcg(reinterpret_cast<const float4 *>(src + (int64_t)h * kLatent + 4 * q + s * part))
+                              : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+            }
+        }
+    };
+    auto combine_batch = [&](int base) {
+#pragma unroll
+        for (int b = 0; b < B; ++b) {
+            const int item = base + b * kMergeThreads;
+            if (item < ITEMS) {
+                const int h = item / NQ, q = item - h * NQ;
+                float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+                if (kOwnInSmem) {
+                    const float w = w_s[split * HG + h];
+                    const float4 v = *reinterpret_cast<const float4 *>(own + h * D + 4 * q);
+                    acc.x = w * v.x;
+                    acc.y = w * v.y;
+                    acc.z = w * v.z;
+                    acc.w = w * v.w;
+                }
+#pragma unroll
+                for (int j = 0; j < kGlobal; ++j) {
+                    const int s = kOwnInSmem && j >= split ? j + 1 : j;
+                    const float w = w_s[s * HG + h];
+                    acc.x += w * o[b][j].x;
+                    acc.y += w * o[b][j].y;
+                    acc.z += w * o[b][j].z;
+                    acc.w += w * o[b][j].w;
+                }
+                const float r = inv_den[h];
+                __half2 *d2 = reinterpret_cast<__half2 *>(dst + (int64_t)h * kLatent + 4 * q);
+                d2[0] = __floats2half2_rn(acc.x * r, acc.y * r);
+                d2[1] = __floats2half2_rn(acc.z * r, acc.w * r);
+            }
+        }
+    };
+    load_batch(mt);
+    if (mt < HG) {
+        const float *ml = a.ws_ml + 2 * ((int64_t)t * S * a.H + (int64_t)g * HG + mt);
+        float2 v[S];
+#pragma unroll
+        for (int s = 0; s < S; ++s) v[s] = __ldcg(reinterpret_cast<const float2 *>(ml + 2 * (int64_t)s * a.H));
+        float mmax = -INFINITY;
+#pragma unroll
+        for (int s = 0; s < S; ++s)
+            if (v[s].y > 0.0f) mmax = fmaxf(mmax, v[s].x);
+        float den = 0.0f;
+#pragma unroll
+        for (int s = 0; s < S; ++s) {
+            const float w = v[s].y > 0.0f ? ex2(v[s].x - mmax) : 0.0f;
+            w_s[s * HG + mt] = w;
+            den += w * v[s].y;
+        }
+        inv_den[mt] = den > 0.0f ? 1.0f / den : 0.0f;
+        if (split == 0)
+            a.lse[(int64_t)t * a.H + (int64_t)g * HG + mt] =
+                den > 0.0f ? (mmax + lg2(den)) * 0.69314718055994531f : -INFINITY;
+    }
+    named_bar(1, kMergeThreads);
+    combine_batch(mt);
+    for (int base = mt + kMergeThreads * B; base < ITEMS; base += kMergeThreads * B) {
+        load_batch(base);
+        combine_batch(base);
+    }
+    named_bar(1, kMergeThreads);
+    if (mt == 0) {
+        const uint32_t old = atomicAdd(depart, 1u);
+        if (old == (uint32_t)S - 1u) {  // every CTA of the group is past its wait
+            atomicExch(arrive, 0u);
+            atomicExch(depart, 0u);
+        }
+    }
+}
+
+template <int HG>
+__global__ void __launch_bounds__(nv4::kThreads, 1)
+    nvfp4_decode_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_qn,
+                        const __grid_constant__ CUtensorMap tm_qr) {
+    using namespace nv4;
+    extern __shared__ __align__(1024) uint8_t smem[];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int split = blockIdx.x % a.S;
+    const int rest = blockIdx.x / a.S;
+    const int g = rest % a.G;
+    const int t = rest / a.G;
+
+    if (smem_u32(smem) & 1023u) {  // the swizzled operand layouts need a 1 KB aligned base
+        if (tid == 0 && a.dev_status) atomicOr(a.dev_status, NVFP4MLA_DEV_LAYOUT);
+        return;
+    }
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kOffBar);
+    uint32_t *misc = reinterpret_cast<uint32_t *>(smem + kOffMisc);
+    int32_t *idx_s = reinterpret_cast<int32_t *>(smem + kOffIdx);
+    float *m_s = reinterpret_cast<float *>(smem + kOffM);
+    float *aux_s = reinterpret_cast<float *>(smem + kOffAux);
+    float *red_s = reinterpret_cast<float *>(smem + kOffRed);
+    uint32_t *cnt_s = reinterpret_cast<uint32_t *>(smem + kOffRed);  // reused before the softmax starts
+
+    // ---------------------------------------------------------------- setup
+    if (warp == 1 && lane == 0) {
+        for (int b = 0; b < kBarsUsed; ++b) {
+            uint32_t count = 1;
+            if (b == BAR_RAW_FREE || b == BAR_RAW_FREE + 1) count = 8;
+            else if (b >= BAR_K_FULL && b < BAR_K_FULL + kKSlots) count = 4;
+            else if (b == BAR_V_FULL || b == BAR_V_FULL + 1) count = 4;
+            else if (b == BAR_P_FULL) count = 4;
+            mbar_init(&bars[b], count);
+        }
+        fence_mbar_init();
+        // Q of (t, heads g*HG ..): nine tensor copies (box 64 dims x HG heads,
+        // 128-byte swizzle) straight into the K-major operand layout.
+        const int32_t row = t * a.H + g * HG;
+        mbar_arrive_expect_tx(&bars[BAR_Q], (uint32_t)(HG * kDim * 2));
+#pragma unroll 1
+        for (int c = 0; c < 8; ++c) tma_load_2d(smem + kOffQ + c * (HG * 128), &tm_qn, 64 * c, row, &bars[BAR_Q]);
+        tma_load_2d(smem + kOffQ + 8 * (HG * 128), &tm_qr, 0, row, &bars[BAR_Q]);
+    }
+    if (warp == 2) {
+        tmem_alloc(&misc[0], kTmemCols);
+        tmem_relinquish();
+    }
+    if (tid < HG) m_s[tid] = -INFINITY;
+
+    // Compact the token's list: keep valid entries in list order; this CTA
+    // keeps entries [lo, hi) of the compacted order.
+    const int32_t *lst = a.indices + (int64_t)t * a.topk;
+    int32_t vals[4];
+    uint32_t bal[4];
+    bool bad = false;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const int p = tid + 512 * k;  // warps 16.. hold no list entries (p >= 2048)
+        int32_t v = (p < a.topk && tid < 512) ? __ldg(lst + p) : -1;
+        bool entry_bad = false;
+        if (a.block_table && v >= 0) {  // request-local position -> slot through the block table
+            int64_t slot = -1;
+            if ((int64_t)v < a.max_pos) {
+                const int32_t blk = __ldg(a.block_table + (int64_t)t * a.table_stride + (v >> a.page_shift));
+                if (blk >= 0) slot = ((int64_t)blk << a.page_shift) + (v & ((1 << a.page_shift) - 1));
+            }
+            entry_bad = slot < 0 || slot >= a.num_slots;
+            v = entry_bad ? -1 : (int32_t)slot;
+        }
+        const bool ok = v >= 0 && (int64_t)v < a.num_slots;
+        bad |= (p < a.topk) && (entry_bad || v < -1 || (int64_t)v >= a.num_slots);
+        vals[k] = v;
+        bal[k] = __ballot_sync(0xffffffffu, ok);
+        if (lane == 0 && warp < 16) cnt_s[k * 16 + warp] = __popc(bal[k]);
+    }
+    if (__any_sync(0xffffffffu, bad) && lane == 0 && split == 0 && g == 0 && a.dev_status)
+        atomicOr(a.dev_status, NVFP4MLA_DEV_BAD_INDEX);
+    __syncthreads();
+    int before[4];
+    int n_valid;
+    {
+        const uint32_t c0 = cnt_s[2 * lane], c1 = cnt_s[2 * lane + 1];
+        uint32_t incl = c0 + c1;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+        }
+        const uint32_t excl = incl - c0 - c1;
+        n_valid = (int)__shfl_sync(0xffffffffu, incl, 31);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const int j = k * 16 + (warp & 15);
+            const uint32_t mine = (j & 1) ? excl + c0 : excl;
+            const uint32_t b = __shfl_sync(0xffffffffu, mine, j >> 1);
+            before[k] = warp < 16 ? (int)b : 0;
+        }
+    }
+    const int per = (n_valid + a.S - 1) / a.S;
+    const int lo = split * per;
+    const int hi = min(n_valid, lo + per);
+    const int n_mine = max(0, hi - lo);
+    const int ntiles = (n_mine + kTileRows - 1) / kTileRows;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        if (warp < 16 && ((bal[k] >> lane) & 1u)) {
+            const int pos = before[k] + __popc(bal[k] & ((1u << lane) - 1u));
+            if (pos >= lo && pos < hi) idx_s[pos - lo] = vals[k];
+        }
+    }
+    tc_fence_before();
+    __syncthreads();  // also orders cnt_s reads before the softmax reuses the region
+    tc_fence_after();
+    const uint32_t tmem = misc[0];
+    auto tile_rows = [&](int j) { return min(kTileRows, n_mine - kTileRows * j); };
+
+    if (warp < 4) {
+        regs_dec<kRegsCtl>();
+        if (warp == 0) {
+            // ------------------------------------------------------- MMA
+            const uint32_t id_qk = idesc_f16_f32(128, HG, false, false);
+            const uint32_t id_pv = idesc_f16_f32(128, HG, true, true);
+            const uint64_t dQ0 = smem_desc(smem_u32(smem + kOffQ), 16, 1024);
+            const uint64_t dV0 = smem_desc(smem_u32(smem + kOffV), 2048, 1024);
+            const uint64_t dP0 = smem_desc(smem_u32(smem + kOffP), 2048, 1024);
+            bool ok = warp_wait(&bars[BAR_Q], 0);  // always: the copies must land before the CTA may exit
+            uint32_t kn = 0, vn = 0;
+            auto score = [&](int j) -> bool {
+                const uint32_t dS = tmem + kColS + 64u * (uint32_t)(j & 1);
+                uint64_t dq = dQ0;
+#pragma unroll 1
+                for (int c = 0; c < kKChunks; ++c) {
+                    const uint32_t slot = kn & 3u;
+                    if (!warp_wait(&bars[BAR_K_FULL + slot], (kn >> 2) & 1u)) return false;
+                    tc_fence_after();
+                    const uint32_t ak = tmem + kColK + 32u * slot;
+                    mma_ts_warp(dS, ak, dq, id_qk, c != 0);
+                    mma_ts_warp(dS, ak + 8, dq + 2, id_qk, 1u);
+                    mma_ts_warp(dS, ak + 16, dq + 4, id_qk, 1u);
+                    mma_ts_warp(dS, ak + 24, dq + 6, id_qk, 1u);
+                    mma_commit_warp(&bars[BAR_K_FREE + slot]);
+                    dq += (uint64_t)((HG * 128) >> 4);
+                    ++kn;
+                }
+                mma_commit_warp(&bars[BAR_S_FULL + (j & 1)]);
+                return true;
+            };
+            if (ok && ntiles > 0) ok = score(0);
+            for (int j = 0; j < ntiles && ok; ++j) {
+                if (j + 1 < ntiles && !(ok = score(j + 1))) break;
+                if (!warp_wait(&bars[BAR_P_FULL], j & 1)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                uint64_t dp = dP0;
+#pragma unroll 1
+                for (int gi = 0; gi < kVGroups; ++gi) {
+                    const uint32_t slot = vn & 1u;
+                    if (!warp_wait(&bars[BAR_V_FULL + slot], (vn >> 1) & 1u)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint64_t dv = dV0 + (uint64_t)(slot * (kVSlotBytes >> 4));
+                    const uint32_t acc = (j > 0 || gi > 0) ? 1u : 0u;
+#pragma unroll
+                    for (int b = 0; b < 4; ++b)
+                        mma_ss_warp(tmem + kColO + b * HG, dv + (uint64_t)(b * (4096 >> 4)), dp, id_pv, acc);
+                    mma_commit_warp(&bars[BAR_V_FREE + slot]);
+                    dp += (uint64_t)(2048 >> 4);
+                    ++vn;
+                }
+                if (!ok) break;
+                mma_commit_warp(&bars[BAR_PV_DONE]);
+            }
+            if (!ok && lane == 0 && a.dev_status) atomicOr(a.dev_status, NVFP4MLA_DEV_TIMEOUT);
+            mma_commit_warp(&bars[BAR_DRAIN]);  // nothing may still read or write TMEM at teardown
+            warp_wait(&bars[BAR_DRAIN], 0);
+        } else if (warp == 1) {
+            // ---------------------------------------------------- gather
+            int issued = 0;
+            bool ok = true;
+            for (int j = 0; j < ntiles; ++j) {
+                const int slot = j & 1;
+                if (j >= 2 && !warp_wait(&bars[BAR_RAW_FREE + slot], ((j >> 1) - 1) & 1)) {
+                    ok = false;
+                    break;
+                }
+                const int nrows = tile_rows(j);
+                if (lane == 0) mbar_arrive_expect_tx(&bars[BAR_RAW_FULL + slot], (uint32_t)(nrows * kRowBytes));
+                __syncwarp();
+                uint8_t *dst = smem + kOffRaw + slot * kRawSlotBytes;
+                const int32_t *ids = idx_s + kTileRows * j;
+                for (int r = lane; r < nrows; r += 32)
+                    bulk_g2s(dst + r * kRawStride, a.src + (int64_t)ids[r] * kRowBytes, kRowBytes,
+                             &bars[BAR_RAW_FULL + slot]);
+                ++issued;
+            }
+            // Copies still in flight must land before the CTA may exit (the
+            // consumers wait for them too unless a wait ran out).
+            for (int j = max(0, issued - 2); j < issued; ++j) warp_wait(&bars[BAR_RAW_FULL + (j & 1)], (j >> 1) & 1);
+            if (!ok && lane == 0 && a.dev_status) atomicOr(a.dev_status, NVFP4MLA_DEV_TIMEOUT);
+        }
+        __syncwarp();
+    } else if (warp < kSoftWarp0) {
+        // ------------------------------------------------------- K unpack
+        regs_dec<kRegsK>();
+        const int kw = warp - kKWarp0;  // 0..7
+        const int quarter = warp & 3;   // TMEM lanes this warp may reach
+        const int half = kw >> 2;       // even or odd chunks
+        const int r = 32 * quarter + lane;
+        const uint32_t lane_base = (uint32_t)(32 * quarter) << 16;
+        bool ok = true;
+        for (int j = 0; j < ntiles && ok; ++j) {
+            const int rslot = j & 1;
+            if (!warp_wait(&bars[BAR_RAW_FULL + rslot], (j >> 1) & 1)) {
+                ok = false;
+                break;
+            }
+            const bool valid = r < tile_rows(j);
+            const uint8_t *row = smem + kOffRaw + rslot * kRawSlotBytes + r * kRawStride;
+#pragma unroll 1
+            for (int c = half; c < kKChunks; c += 2) {
+                const uint32_t n = (uint32_t)(kKChunks * j + c);
+                const uint32_t slot = n & 3u;
+                uint32_t o[32];
+                if (valid) {
+                    if (c < 8) {
+                        unpack_latent64(lds128(row + 32 * c), lds128(row + 32 * c + 16), lds32(row + kScaleOff + 4 * c), o);
+                    } else {
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            const uint4 w = lds128(row + kRopeOff + 16 * q);
+                            uint32_t e[4];
+                            e4m3x8_to_f16x8(w.x, w.y, e);
+                            o[8 * q + 0] = e[0];
+                            o[8 * q + 1] = e[1];
+                            o[8 * q + 2] = e[2];
+                            o[8 * q + 3] = e[3];
+                            e4m3x8_to_f16x8(w.z, w.w, e);
+                            o[8 * q + 4] = e[0];
+                            o[8 * q + 5] = e[1];
+                            o[8 * q + 6] = e[2];
+                            o[8 * q + 7] = e[3];
+                        }
+                    }
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) o[i] = 0u;
+                }
+                if (n >= 4 && !warp_wait(&bars[BAR_K_FREE + slot], ((n >> 2) - 1) & 1u)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                tmem_st32(tmem + lane_base + kColK + 32u * slot, o);
+                tmem_st_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bars[BAR_K_FULL + slot]);
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars[BAR_RAW_FREE + rslot]);
+        }
+        if (!ok && lane == 0 && a.dev_status) atomicOr(a.dev_status, NVFP4MLA_DEV_TIMEOUT);
+    } else if (warp < kVWarp0) {
+        // -------------------------------------------------------- softmax
+        regs_inc<kRegsSoft>();
+        const int st = tid - 32 * kSoftWarp0;  // tile row == TMEM lane
+        const int wq = st >> 5;
+        const uint32_t lane_base = (uint32_t)(32 * wq) << 16;
+        uint8_t *p_tile = smem + kOffP;
+        // Running row sums: each tile's per-row values are folded across the
+        // warp (transpose reduction), so a lane keeps the sums of the warp's
+        // 32 rows for only cols_per_lane(HG) heads: heads lp_head(k).
+        constexpr int NL = cols_per_lane(HG);
+        auto lp_head = [&](int k) { return HG >= 32 ? lane * NL + k : (lane >> 1); };
+        float lp[NL];
+#pragma unroll
+        for (int k = 0; k < NL; ++k) lp[k] = 0.0f;
+        bool ok = true;
+        // Every wait's outcome is agreed by all 128 threads (bar.red.or), so
+        // the four warps always meet at the same named barriers.
+        for (int j = 0; j < ntiles; ++j) {
+            if (named_bar_or(1, 128, !warp_wait(&bars[BAR_S_FULL + (j & 1)], (j >> 1) & 1))) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            float sv[HG];
+            {
+                uint32_t rs[HG];
+                tmem_ld_cols<HG>(tmem + lane_base + kColS + 64u * (uint32_t)(j & 1), rs);
+                tmem_ld_wait();
+#pragma unroll
+                for (int h = 0; h < HG; ++h) sv[h] = __uint_as_float(rs[h]) * a.scale_log2;
+            }
+            const bool valid = st < tile_rows(j);
+            bool need = false;
+            if (valid) {
+#pragma unroll
+                for (int h = 0; h < HG; ++h) need |= sv[h] > m_s[h] + kRescaleThreshold;
+            }
+            const bool rescale = named_bar_or(1, 128, need);
+            if (rescale) {
+#pragma unroll
+                for (int c0 = 0; c0 < HG; c0 += 16) {  // column max, 16 heads at a time
+                    float mx[16];
+#pragma unroll
+                    for (int h = 0; h < 16; ++h) mx[h] = valid ? sv[c0 + h] : -INFINITY;
+                    warp_transpose_reduce<16, true>(mx, lane);
+                    if (!(lane & 1)) red_s[wq * 64 + c0 + transposed_col<16>(lane, 0)] = mx[0];
+                }
+                named_bar(1, 128);
+                if (st < HG) {
+                    const float old = m_s[st];
+                    float nm = old;
+#pragma unroll
+                    for (int w = 0; w < 4; ++w) nm = fmaxf(nm, red_s[w * 64 + st]);
+                    aux_s[st] = (old == -INFINITY) ? 0.0f : ex2(old - nm);
+                    m_s[st] = nm;
+                }
+                named_bar(1, 128);
+#pragma unroll
+                for (int k = 0; k < NL; ++k) lp[k] *= aux_s[lp_head(k)];
+            }
+            // O^T and P^T belong to the output MMAs of the previous tile
+            // until they are done.
+            if (j > 0) {
+                if (named_bar_or(1, 128, !warp_wait(&bars[BAR_PV_DONE], (j - 1) & 1))) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                if (rescale) {
+#pragma unroll 1
+                    for (int b = 0; b < 4; ++b) {
+#pragma unroll
+                        for (int cb = 0; cb < HG; cb += 16) {
+                            uint32_t rr[16];
+                            const uint32_t addr = tmem + lane_base + kColO + b * HG + cb;
+                            tmem_ld16(addr, rr);
+                            tmem_ld_wait();
+#pragma unroll
+                            for (int h = 0; h < 16; ++h) rr[h] = __float_as_uint(__uint_as_float(rr[h]) * aux_s[cb + h]);
+                            tmem_st16(addr, rr);
+                        }
+                    }
+                    tmem_st_wait();
+                }
+            }
+#pragma unroll
+            for (int h = 0; h < HG; ++h) sv[h] = valid ? ex2(sv[h] - m_s[h]) : 0.0f;
+#pragma unroll
+            for (int jj = 0; jj < HG / 8; ++jj) {
+                uint4 pk;
+                pk.x = pack_half2(sv[8 * jj + 0], sv[8 * jj + 1]);
+                pk.y = pack_half2(sv[8 * jj + 2], sv[8 * jj + 3]);
+                pk.z = pack_half2(sv[8 * jj + 4], sv[8 * jj + 5]);
+                pk.w = pack_half2(sv[8 * jj + 6], sv[8 * jj + 7]);
+                *reinterpret_cast<uint4 *>(p_tile + sw128_offset(st, jj)) = pk;
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars[BAR_P_FULL]);
+            // row sums of this tile (FP32 values, as the FP16 P rounds them
+            // only for the MMA), folded over the warp's rows
+            warp_transpose_reduce<HG, false>(sv, lane);
+#pragma unroll
+            for (int k = 0; k < NL; ++k) lp[k] += sv[k];
+        }
+        if (!ok && a.dev_status && lane == 0) atomicOr(a.dev_status, NVFP4MLA_DEV_TIMEOUT);
+        // ---------------------------------------------------------- epilogue
+        const bool have = ok && ntiles > 0;
+        if (HG >= 32 || !(lane & 1)) {  // row sums: one partial per warp and head
+#pragma unroll
+            for (int k = 0; k < NL; ++k) red_s[wq * 64 + lp_head(k)] = lp[k];
+        }
+        named_bar(1, 128);
+        if (st < HG) {
+            const float l = have ? red_s[st] + red_s[64 + st] + red_s[128 + st] + red_s[192 + st] : 0.0f;
+            const float m = m_s[st];
+            aux_s[st] = l > 0.0f ? 1.0f / l : 0.0f;
+            const int64_t hrow = (int64_t)t * a.H + (int64_t)g * HG + st;
+            if (a.S == 1) {
+                a.lse[hrow] = l > 0.0f ? (m + lg2(l)) * 0.69314718055994531f : -INFINITY;
+            } else {
+                const int64_t prow = ((int64_t)t * a.S + split) * a.H + (int64_t)g * HG + st;
+                a.ws_ml[2 * prow] = l > 0.0f ? m : -INFINITY;
+                a.ws_ml[2 * prow + 1] = l;
+            }
+        }
+        named_bar(1, 128);
+        bool fin = have;
+        if (have) {  // O^T is final once the last tile's output MMAs are done
+            fin = !named_bar_or(1, 128, !warp_wait(&bars[BAR_PV_DONE], (ntiles - 1) & 1));
+            if (!fin && st == 0 && a.dev_status) atomicOr(a.dev_status, NVFP4MLA_DEV_TIMEOUT);
+            tc_fence_after();
+        }
+        // Every K-unpack warp is past its last raw tile once the last output
+        // MMAs are done (they needed every chunk), so the raw ring is free.
+        uint8_t *stage = smem + kOffRaw;
+        if (a.S == 1) {
+            // O^T (TMEM lanes = dv) -> normalised FP16 rows [HG][512] staged
+            // in the raw ring, then one bulk copy of HG x 1 KB.
+            constexpr int HC = HG > 32 ? 32 : HG;  // columns per TMEM load
+#pragma unroll 1
+            for (int b = 0; b < 4; ++b) {
+                const int dv = 128 * b + st;
+#pragma unroll
+                for (int h0 = 0; h0 < HG; h0 += HC) {
+                    uint32_t rr[HC];
+                    if (fin) {
+                        tmem_ld_cols<HC>(tmem + lane_base + kColO + b * HG + h0, rr);
+                        tmem_ld_wait();
+                    } else {
+#pragma unroll
+                        for (int h = 0; h < HC; ++h) rr[h] = 0u;
+                    }
+#pragma unroll
+                    for (int h = 0; h < HC; ++h)
+                        reinterpret_cast<__half *>(stage)[(h0 + h) * kLatent + dv] =
+                            __float2half_rn(__uint_as_float(rr[h]) * aux_s[h0 + h]);
+                }
+            }
+            fence_proxy_async_smem();
+            named_bar(1, 128);
+            if (st == 0) {
+                bulk_s2g(a.out + ((int64_t)t * a.H + (int64_t)g * HG) * kLatent, stage, HG * kLatent * 2);
+                bulk_commit_wait_read();
+            }
+        } else {
+            // Unnormalised partial O of this split: blocks inside the CTA's
+            // own merge slice (S <= 4) stay in shared memory, the others go
+            // to the workspace (for each head a warp writes 32 consecutive
+            // dv, one 128-byte segment).
+            float *dst = a.ws_o + (((int64_t)t * a.S + split) * a.H + (int64_t)g * HG) * kLatent + st;
+            const int own_n = a.S <= 4 ? 4 / a.S : 0;
+            const int own_b0 = split * own_n;
+            const int own_d = kLatent / a.S;
+            float *own = reinterpret_cast<float *>(stage) + st;
+            constexpr int HC = HG > 32 ? 32 : HG;
+#pragma unroll 1
+            for (int b = 0; b < 4; ++b) {
+                const bool mine = b >= own_b0 && b < own_b0 + own_n;
+#pragma unroll
+                for (int h0 = 0; h0 < HG; h0 += HC) {
+                    uint32_t rr[HC];
+                    if (fin) {
+                        tmem_ld_cols<HC>(tmem + lane_base + kColO + b * HG + h0, rr);
+                        tmem_ld_wait();
+                    } else {
+#pragma unroll
+                        for (int h = 0; h < HC; ++h) rr[h] = 0u;
+                    }
+                    if (mine) {
+#pragma unroll
+                        for (int h = 0; h < HC; ++h) own[(h0 + h) * own_d + 128 * (b - own_b0)] = __uint_as_float(rr[h]);
+                    } else {
+#pragma unroll
+                        for (int h = 0; h < HC; ++h)
+                            __stcg(dst + (int64_t)(h0 + h) * kLatent + 128 * b, __uint_as_float(rr[h]));
+                    }
+                }
+            }
+            switch (a.S) {
+                case 2: merge_splits_nv4<HG, 2>(a, t, g, split, smem, st); break;
+                case 4: merge_splits_nv4<HG, 4>(a, t, g, split, smem, st); break;
+                case 8: merge_splits_nv4<HG, 8>(a, t, g, split, smem, st); break;
+                default: merge_splits_nv4<HG, 16>(a, t, g, split, smem, st); break;
+            }
+        }
+    } else {
+        // -------------------------------------------------------- V unpack
+        // Slot layout (MN-major A operand of the output MMA): dv group dg
+        // (64 dims) at dg * 2048, row r of the 16 at r * 128, 16-byte chunk
+        // jj swizzled by the row.  Thread = (row r, dv group dg); the rows
+        // are read from L2 (the gather brought them in a tile earlier).
+        const int vw = warp - kVWarp0;  // 0..3
+        const int r = lane & 15;
+        const int dg = 2 * vw + (lane >> 4);
+        bool ok = true;
+        uint32_t vn = 0;
+        for (int j = 0; j < ntiles && ok; ++j) {
+            // The tile's rows are in L2 once its score MMAs are done; that
+            // also keeps these loads from racing the gather to HBM.
+            if (!warp_wait(&bars[BAR_S_FULL + (j & 1)], (j >> 1) & 1)) {
+                ok = false;
+                break;
+            }
+            const int nrows = tile_rows(j);
+            const int32_t *ids = idx_s + kTileRows * j;
+            auto load = [&](int gi, uint4 &w0, uint4 &w1, uint32_t &sc) {
+                const int e = kVRows * gi + r;
+                if (e < nrows) {
+                    const uint8_t *rp = a.src + (int64_t)ids[e] * kRowBytes;
+                    w0 = __ldg(reinterpret_cast<const uint4 *>(rp + 32 * dg));
+                    w1 = __ldg(reinterpret_cast<const uint4 *>(rp + 32 * dg + 16));
+                    sc = __ldg(reinterpret_cast<const uint32_t *>(rp + kScaleOff + 4 * dg));
+                } else {
+                    w0 = w1 = make_uint4(0u, 0u, 0u, 0u);
+                    sc = 0u;
+                }
+            };
+            uint4 a0, a1, b0, b1;
+            uint32_t as, bs;
+            load(0, a0, a1, as);
+            load(1, b0, b1, bs);
+#pragma unroll 1
+            for (int gi = 0; gi < kVGroups; ++gi) {
+                uint32_t o[32];
+                unpack_latent64(a0, a1, as, o);
+                a0 = b0;
+                a1 = b1;
+                as = bs;
+                if (gi + 2 < kVGroups) load(gi + 2, b0, b1, bs);
+                const uint32_t slot = vn & 1u;
+                if (vn >= 2 && !warp_wait(&bars[BAR_V_FREE + slot], ((vn >> 1) - 1) & 1u)) {
+                    ok = false;
+                    break;
+                }
+                uint8_t *base = smem + kOffV + slot * kVSlotBytes + dg * 2048;
+#pragma unroll
+                for (int jj = 0; jj < 8; ++jj)
+                    *reinterpret_cast<uint4 *>(base + sw128_offset(r, jj)) =
+                        make_uint4(o[4 * jj], o[4 * jj + 1], o[4 * jj + 2], o[4 * jj + 3]);
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bars[BAR_V_FULL + slot]);
+                ++vn;
+            }
+        }
+        if (!ok && lane == 0 && a.dev_status) atomicOr(a.dev_status, NVFP4MLA_DEV_TIMEOUT);
+    }
+
+    // ---------------------------------------------------------------- teardown
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 2) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+template <int HG>
+static cudaError_t launch_nv4(const DecodeArgs &a, int64_t nblocks, cudaStream_t stream) {
+    auto kern = nvfp4_decode_kernel<HG>;
+    static std::atomic<bool> attr_set[64] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64 || !attr_set[dev].load(std::memory_order_acquire)) {
+        // The per-role register split (setmaxnreg) assumes the block starts
+        // with kRegsLaunch registers per thread; with fewer, an increase
+        // could never be granted, so refuse to launch.
+        cudaFuncAttributes fa;
+        e = cudaFuncGetAttributes(&fa, kern);
+        if (e != cudaSuccess) return e;
+        if (fa.numRegs != nv4::kRegsLaunch || fa.maxThreadsPerBlock < nv4::kThreads) return cudaErrorInvalidConfiguration;
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, nv4::kSmemBytes);
+        if (e != cudaSuccess) return e;
+        if (dev >= 0 && dev < 64) attr_set[dev].store(true, std::memory_order_release);
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)nblocks);
+    cfg.blockDim = dim3(nv4::kThreads);
+    cfg.dynamicSmemBytes = nv4::kSmemBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = a.S > 1 ? 1 : 0;  // split launches need every CTA resident at once
+    CUtensorMap tm_qn, tm_qr;
+    const uint64_t rows = (uint64_t)a.T * (uint64_t)a.H;
+    if (!make_q_map(&tm_qn, a.q_nope, rows, kLatent, HG) || !make_q_map(&tm_qr, a.q_rope, rows, kRope, HG))
+        return cudaErrorInvalidValue;
+    return cudaLaunchKernelEx(&cfg, kern, a, tm_qn, tm_qr);
+}
+
+cudaError_t launch_nvfp4_decode(const DecodeArgs &a, int heads_per_cta, int64_t nblocks, cudaStream_t stream) {
+    switch (heads_per_cta) {
+        case 16: return launch_nv4<16>(a, nblocks, stream);
+        case 32: return launch_nv4<32>(a, nblocks, stream);
+        case 64: return launch_nv4<64>(a, nblocks, stream);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace nvfp4mla
