@@ -22,24 +22,27 @@
 //   O^T[dv, h]  += V^T[dv, row] . P^T[row, h]       A = V^T, B = P^T in shared
 // The score MMA reads its K operand from tensor memory (a ring of four
 // 64-dim chunks written by the unpack warps with tcgen05.st), so only Q
-// streams from shared memory.  V is the latent part of the same rows; it is
+// streams from shared memory.  Score and output MMAs are issued by two
+// different warps, so the barrier waits of one stream overlap the MMAs of
+// the other.  V is the latent part of the same rows; it is
 // decoded a second time, 16 rows at a time, into a two-slot shared-memory
-// ring in the MN-major layout the output MMA reads.  The MMA warp issues the
-// score MMAs of tile j+1 before the output MMAs of tile j, so the softmax of
-// tile j runs while the tensor core scores the next tile.
+// ring in the MN-major layout the output MMA reads.  The score MMAs of tile
+// j+1 need only the K ring and a free S buffer (S is double-buffered), so
+// they run while the softmax of tile j is still working.
 //
-// Warp roles (640 threads, five warpgroups):
-//   warp 0      MMA issue (whole warp, one elected lane issues)
-//   warp 1      gather: the CTA's Q by tensor copies, then one 352-byte bulk
-//               copy per valid row into a two-tile raw ring (rows padded to
-//               368 bytes so the unpack warps read them without bank
-//               conflicts)
-//   warp 2      tensor-memory allocation and release
+// Warp roles (768 threads, six warpgroups):
+//   warp 0      score MMA issue (whole warp, one elected lane issues)
+//   warps 1, 3  gather: the CTA's Q by tensor copies (warp 1), then the
+//               valid rows in 16-byte cp.async pieces into a two-tile raw
+//               ring (rows padded to 368 bytes so the unpack warps read
+//               them without bank conflicts)
+//   warp 2      tensor-memory allocation and release; output MMA issue
 //   warps 4-11  K unpack: thread = tile row = TMEM lane; warps 4-7 take the
 //               even 64-dim chunks, warps 8-11 the odd ones (and RoPE)
 //   warps 12-15 softmax (thread = tile row), then the epilogue and the split
 //               merge
-//   warps 16-19 V unpack: 16 rows x 8 dv groups per ring slot, rows read
+//   warps 16-23 V unpack, two sets of four alternating the 16-row groups
+//               of a tile (16 rows x 8 dv groups per ring slot), rows read
 //               again from L2 (they arrived one tile earlier)
 //
 // Tensor memory (512 columns): O^T at 0 (four 128-dv blocks of HG columns),
@@ -69,6 +72,9 @@
 
 namespace nvfp4mla {
 using namespace ptx;
+#ifdef NVFP4MLA_TRACE
+void set_trace_buffer_nv4(unsigned long long *p) { set_trace_local(p); }
+#endif
 
 namespace nv4 {
 constexpr int kTileRows = 128;
@@ -77,53 +83,62 @@ constexpr int kRawStride = 368;                            // 352-byte row + 16 
 constexpr int kRawSlotBytes = kTileRows * kRawStride;      // 47104
 constexpr int kVRows = 16;                                 // rows per V ring slot (one MMA K step)
 constexpr int kVSlotBytes = kVRows * kLatent * 2;          // 16384
+constexpr int kVSlots = 2;                                 // V ring depth
+constexpr int kRawSlots = 2;                               // raw tiles in shared memory
+constexpr int kPrefetchAhead = 0;                          // tiles brought into L2 ahead of their copy (0: none)
 constexpr int kVGroups = kTileRows / kVRows;               // 8
 constexpr int kKChunks = 9;                                // 8 latent chunks of 64 dims + RoPE
 constexpr int kKSlots = 4;
 constexpr int kOffQ = 0;                                   // 9 chunks x HG rows x 128 B
 constexpr int kOffP = kOffQ + kKChunks * kMaxHG * 128;     // 73728: P^T, 128 rows x 128 B
-constexpr int kOffV = kOffP + kTileRows * 128;             // 90112: two V slots
-constexpr int kOffRaw = kOffV + 2 * kVSlotBytes;           // 122880: two raw tiles
-constexpr int kOffIdx = kOffRaw + 2 * kRawSlotBytes;       // 217088: compacted list share
+constexpr int kOffV = kOffP + kTileRows * 128;             // 90112: V ring
+constexpr int kOffRaw = kOffV + kVSlots * kVSlotBytes;     // 155648: raw ring
+constexpr int kOffIdx = kOffRaw + kRawSlots * kRawSlotBytes;  // compacted list share
 constexpr int kOffM = kOffIdx + kMaxTopk * 4;              // reference max per head (log2 units)
 constexpr int kOffAux = kOffM + kMaxHG * 4;                // rescale factors, then 1/l
 constexpr int kOffRed = kOffAux + kMaxHG * 4;              // 4 warps x 64 floats
 constexpr int kOffBar = kOffRed + 4 * kMaxHG * 4;
-constexpr int kNumBars = 24;
+constexpr int kNumBars = 28;
 constexpr int kOffMisc = kOffBar + kNumBars * 8;
 constexpr int kSmemBytes = kOffMisc + 64;
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 static_assert(kOffP % 1024 == 0 && kOffV % 1024 == 0, "swizzled operands need 1 KB alignment");
-static_assert(kMaxHG * kLatent * 2 <= 2 * kRawSlotBytes, "output staging must fit in the raw ring");
-static_assert(kMaxHG * (kLatent / 2) * 4 <= 2 * kRawSlotBytes, "own merge slice must fit in the raw ring");
-constexpr int kThreads = 640;
+// the epilogue stages its output (or its own merge slice) over the V and raw
+// rings, which are free by then; the merge weights go to the P^T region
+constexpr int kOffStage = kOffV;
+static_assert(kMaxHG * kLatent * 2 <= kOffIdx - kOffStage, "output staging must fit over the rings");
+static_assert(kMaxHG * (kLatent / 2) * 4 <= kOffIdx - kOffStage, "own merge slice must fit over the rings");
+constexpr int kThreads = 768;
 constexpr int kKWarp0 = 4;
 constexpr int kSoftWarp0 = 12;
 constexpr int kVWarp0 = 16;
-// Register budgets per warpgroup (setmaxnreg): launched with 96 per thread
-// (65536 / 640 rounded down to a multiple of 8); the control warpgroup and
-// the K-unpack warps give registers to the softmax warps, whose threads hold
-// a score and a running row sum per head.
-constexpr int kRegsLaunch = 96;
-constexpr int kRegsCtl = 56;
-constexpr int kRegsK = 72;
-constexpr int kRegsSoft = 184;
-static_assert(128 * kRegsCtl + 256 * kRegsK + 128 * kRegsSoft + 128 * kRegsLaunch <= kThreads * kRegsLaunch,
+// Register budgets per warpgroup (setmaxnreg): launched with 80 per thread
+// (65536 / 768 rounded down to a multiple of 8); the control and K-unpack
+// warpgroups give registers to the softmax warps, whose threads hold a row of
+// scores and of P.
+constexpr int kRegsLaunch = 80;
+constexpr int kRegsCtl = 48;
+constexpr int kRegsK = 64;
+constexpr int kRegsV = 80;
+constexpr int kRegsSoft = 144;
+static_assert(128 * kRegsCtl + 256 * kRegsK + 128 * kRegsSoft + 256 * kRegsV <= kThreads * kRegsLaunch,
               "register split exceeds the launch budget");
 
 // mbarriers
-constexpr int BAR_Q = 0;           // Q tensor copies (expect_tx)
-constexpr int BAR_RAW_FULL = 1;    // [2] raw tile landed (expect_tx)
-constexpr int BAR_RAW_FREE = 3;    // [2] raw tile read by the 8 K-unpack warps
-constexpr int BAR_K_FULL = 5;      // [4] K chunk in TMEM (4 warps)
-constexpr int BAR_K_FREE = 9;      // [4] score MMAs of the chunk done (commit)
-constexpr int BAR_V_FULL = 13;     // [2] V slot written (4 warps)
-constexpr int BAR_V_FREE = 15;     // [2] output MMAs of the slot done (commit)
-constexpr int BAR_S_FULL = 17;     // [2] score MMAs of a tile done (commit)
-constexpr int BAR_P_FULL = 19;     // P^T written, O^T rescaled (4 softmax warps)
-constexpr int BAR_PV_DONE = 20;    // output MMAs of a tile done (commit)
-constexpr int BAR_DRAIN = 21;      // every MMA issued so far done
-constexpr int kBarsUsed = 22;
+constexpr int BAR_Q = 0;                           // Q tensor copies (expect_tx)
+constexpr int BAR_RAW_FULL = 1;                    // [kRawSlots] raw tile landed (cp.async arrivals of 64 threads)
+constexpr int BAR_RAW_FREE = BAR_RAW_FULL + kRawSlots;  // [kRawSlots] raw tile read by the 8 K-unpack warps
+constexpr int BAR_K_FULL = BAR_RAW_FREE + kRawSlots;    // [4] K chunk in TMEM (4 warps)
+constexpr int BAR_K_FREE = BAR_K_FULL + kKSlots;        // [4] score MMAs of the chunk done (commit)
+constexpr int BAR_V_FULL = BAR_K_FREE + kKSlots;        // [kVSlots] V slot written (the 4 warps of a V set)
+constexpr int BAR_V_FREE = BAR_V_FULL + kVSlots;        // [kVSlots] output MMAs of the slot done (commit)
+constexpr int BAR_S_FULL = BAR_V_FREE + kVSlots;        // [2] score MMAs of a tile done (commit)
+constexpr int BAR_P_FULL = BAR_S_FULL + 2;              // P^T written, O^T rescaled (4 softmax warps)
+constexpr int BAR_PV_DONE = BAR_P_FULL + 1;             // output MMAs of a tile done (commit)
+constexpr int BAR_DRAIN = BAR_PV_DONE + 1;              // every score MMA issued so far done
+constexpr int BAR_S_FREE = BAR_DRAIN + 1;               // [2] softmax done reading an S buffer (4 softmax warps)
+constexpr int BAR_DRAIN_PV = BAR_S_FREE + 2;            // every output MMA issued so far done
+constexpr int kBarsUsed = BAR_DRAIN_PV + 1;
 static_assert(kBarsUsed <= kNumBars, "barrier slots");
 
 constexpr uint32_t kTmemCols = 512;
@@ -150,10 +165,13 @@ __device__ __forceinline__ uint32_t lds32(const uint8_t *p) { return *reinterpre
 // significant bits and lies inside FP16's range.
 __device__ __forceinline__ void unpack_latent64(uint4 w0, uint4 w1, uint32_t scales, uint32_t (&o)[32]) {
     const uint32_t w[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+    // the four scales as two f16x2 pairs, then each broadcast to both halves
+    const uint32_t s01 = e4m3x2_to_f16x2(scales & 0xFFFFu), s23 = e4m3x2_to_f16x2(scales >> 16);
+    const uint32_t sc2[4] = {__byte_perm(s01, 0u, 0x1010), __byte_perm(s01, 0u, 0x3232), __byte_perm(s23, 0u, 0x1010),
+                             __byte_perm(s23, 0u, 0x3232)};
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
-        const uint32_t sb = (scales >> (8 * k)) & 0xFFu;
-        const uint32_t s2 = e4m3x2_to_f16x2(sb | (sb << 8));
+        const uint32_t s2 = sc2[k];
         uint32_t lo[4], hi[4];
         e2m1x8_to_f16x8(w[2 * k], lo);
         e2m1x8_to_f16x8(w[2 * k + 1], hi);
@@ -177,7 +195,8 @@ __device__ __forceinline__ void unpack_latent64(uint4 w0, uint4 w1, uint32_t sca
 // one on the same counter report NVFP4MLA_DEV_TIMEOUT and write NaN to their
 // slice instead of merging partials that were never written.
 template <int HG, int S>
-__device__ __forceinline__ void merge_splits_nv4(const DecodeArgs &a, int t, int g, int split, uint8_t *smem, int mt) {
+__device__ __forceinline__ void merge_splits_nv4(const DecodeArgs &a, int t, int g, int split, uint8_t *smem, int mt,
+                                                 [[maybe_unused]] unsigned long long t_start) {
     using namespace nv4;
     constexpr int kMergeThreads = 128;
     constexpr int D = kLatent / S;
@@ -190,12 +209,14 @@ __device__ __forceinline__ void merge_splits_nv4(const DecodeArgs &a, int t, int
     uint32_t *arrive = a.counters + 2 * ((int64_t)t * a.G + g);
     uint32_t *depart = arrive + 1;
     uint32_t *flag = reinterpret_cast<uint32_t *>(smem + kOffMisc) + 1;
-    float *w_s = reinterpret_cast<float *>(smem + kOffV);   // [S][HG]
+    float *w_s = reinterpret_cast<float *>(smem + kOffP);   // [S][HG]
     float *inv_den = w_s + kMaxSplits * HG;                  // [HG]
-    const float *own = reinterpret_cast<const float *>(smem + kOffRaw);  // [HG][D]
+    const float *own = reinterpret_cast<const float *>(smem + kOffStage);  // [HG][D]
     named_bar(1, kMergeThreads);  // every partial store of this CTA precedes the release
     if (mt == 0) {
+        TRACE(190);
         __threadfence();
+        TRACE(191);
         const uint32_t old = atomicAdd(arrive, 1u);  // relaxed add; the fence above orders the partials
         bool ok = (old & kPoison) == 0;
         if (ok) {
@@ -213,6 +234,7 @@ __device__ __forceinline__ void merge_splits_nv4(const DecodeArgs &a, int t, int
             if (a.dev_status) atomicOr(a.dev_status, NVFP4MLA_DEV_TIMEOUT);
         }
         *flag = ok ? 1u : 0u;
+        TRACE(192);
     }
     named_bar(1, kMergeThreads);
     const int dv0 = split * D;
@@ -296,6 +318,7 @@ __device__ __forceinline__ void merge_splits_nv4(const DecodeArgs &a, int t, int
                 den > 0.0f ? (mmax + lg2(den)) * 0.69314718055994531f : -INFINITY;
     }
     named_bar(1, kMergeThreads);
+    if (mt == 0) TRACE(193);
     combine_batch(mt);
     for (int base = mt + kMergeThreads * B; base < ITEMS; base += kMergeThreads * B) {
         load_batch(base);
@@ -303,6 +326,7 @@ __device__ __forceinline__ void merge_splits_nv4(const DecodeArgs &a, int t, int
     }
     named_bar(1, kMergeThreads);
     if (mt == 0) {
+        TRACE(194);
         const uint32_t old = atomicAdd(depart, 1u);
         if (old == (uint32_t)S - 1u) {  // every CTA of the group is past its wait
             atomicExch(arrive, 0u);
@@ -322,6 +346,11 @@ __global__ void __launch_bounds__(nv4::kThreads, 1)
     const int rest = blockIdx.x / a.S;
     const int g = rest % a.G;
     const int t = rest / a.G;
+#ifdef NVFP4MLA_TRACE
+    const unsigned long long t_start = clock64();
+#else
+    const unsigned long long t_start = 0;  // timestamps exist only in trace builds
+#endif
 
     if (smem_u32(smem) & 1023u) {  // the swizzled operand layouts need a 1 KB aligned base
         if (tid == 0 && a.dev_status) atomicOr(a.dev_status, NVFP4MLA_DEV_LAYOUT);
@@ -339,10 +368,11 @@ __global__ void __launch_bounds__(nv4::kThreads, 1)
     if (warp == 1 && lane == 0) {
         for (int b = 0; b < kBarsUsed; ++b) {
             uint32_t count = 1;
-            if (b == BAR_RAW_FREE || b == BAR_RAW_FREE + 1) count = 8;
+            if (b >= BAR_RAW_FULL && b < BAR_RAW_FULL + kRawSlots) count = 64;  // cp.async arrivals
+            else if (b >= BAR_RAW_FREE && b < BAR_RAW_FREE + kRawSlots) count = 8;
             else if (b >= BAR_K_FULL && b < BAR_K_FULL + kKSlots) count = 4;
-            else if (b == BAR_V_FULL || b == BAR_V_FULL + 1) count = 4;
-            else if (b == BAR_P_FULL) count = 4;
+            else if (b >= BAR_V_FULL && b < BAR_V_FULL + kVSlots) count = 4;
+            else if (b == BAR_P_FULL || b == BAR_S_FREE || b == BAR_S_FREE + 1) count = 4;
             mbar_init(&bars[b], count);
         }
         fence_mbar_init();
@@ -426,25 +456,35 @@ __global__ void __launch_bounds__(nv4::kThreads, 1)
     tc_fence_after();
     const uint32_t tmem = misc[0];
     auto tile_rows = [&](int j) { return min(kTileRows, n_mine - kTileRows * j); };
+    if (tid == 0) TRACE(0);
 
     if (warp < 4) {
         regs_dec<kRegsCtl>();
         if (warp == 0) {
-            // ------------------------------------------------------- MMA
+            // ------------------------------------------------- score MMAs
+            // S^T(j) = K(j) Q^T into S buffer j & 1, chunk by chunk as the K
+            // ring fills; buffer j & 1 is reused once the softmax of tile
+            // j - 2 has read it.
             const uint32_t id_qk = idesc_f16_f32(128, HG, false, false);
-            const uint32_t id_pv = idesc_f16_f32(128, HG, true, true);
             const uint64_t dQ0 = smem_desc(smem_u32(smem + kOffQ), 16, 1024);
-            const uint64_t dV0 = smem_desc(smem_u32(smem + kOffV), 2048, 1024);
-            const uint64_t dP0 = smem_desc(smem_u32(smem + kOffP), 2048, 1024);
             bool ok = warp_wait(&bars[BAR_Q], 0);  // always: the copies must land before the CTA may exit
-            uint32_t kn = 0, vn = 0;
-            auto score = [&](int j) -> bool {
+            if (lane == 0) TRACE(1);
+            uint32_t kn = 0;
+            for (int j = 0; j < ntiles && ok; ++j) {
+                if (j >= 2 && !warp_wait(&bars[BAR_S_FREE + (j & 1)], ((j >> 1) - 1) & 1)) {
+                    ok = false;
+                    break;
+                }
                 const uint32_t dS = tmem + kColS + 64u * (uint32_t)(j & 1);
+                if (lane == 0 && j < 8) TRACE(10 + 8 * j);
                 uint64_t dq = dQ0;
 #pragma unroll 1
                 for (int c = 0; c < kKChunks; ++c) {
                     const uint32_t slot = kn & 3u;
-                    if (!warp_wait(&bars[BAR_K_FULL + slot], (kn >> 2) & 1u)) return false;
+                    if (!warp_wait(&bars[BAR_K_FULL + slot], (kn >> 2) & 1u)) {
+                        ok = false;
+                        break;
+                    }
                     tc_fence_after();
                     const uint32_t ak = tmem + kColK + 32u * slot;
                     mma_ts_warp(dS, ak, dq, id_qk, c != 0);
@@ -452,67 +492,104 @@ __global__ void __launch_bounds__(nv4::kThreads, 1)
                     mma_ts_warp(dS, ak + 16, dq + 4, id_qk, 1u);
                     mma_ts_warp(dS, ak + 24, dq + 6, id_qk, 1u);
                     mma_commit_warp(&bars[BAR_K_FREE + slot]);
+                    if (lane == 0 && j == 1) TRACE(240 + c);
                     dq += (uint64_t)((HG * 128) >> 4);
                     ++kn;
                 }
+                if (!ok) break;
                 mma_commit_warp(&bars[BAR_S_FULL + (j & 1)]);
-                return true;
-            };
-            if (ok && ntiles > 0) ok = score(0);
+                if (lane == 0 && j < 8) TRACE(11 + 8 * j);
+            }
+            if (!ok && lane == 0 && a.dev_status) atomicOr(a.dev_status, NVFP4MLA_DEV_TIMEOUT);
+            mma_commit_warp(&bars[BAR_DRAIN]);  // nothing may still read or write TMEM at teardown
+            warp_wait(&bars[BAR_DRAIN], 0);
+        } else if (warp == 2) {
+            // ------------------------------------------------ output MMAs
+            // O^T += V^T(j) P^T(j), one 16-row V ring slot at a time, once the
+            // softmax has written P^T(j) (and rescaled O^T if it had to).
+            const uint32_t id_pv = idesc_f16_f32(128, HG, true, true);
+            const uint64_t dV0 = smem_desc(smem_u32(smem + kOffV), 2048, 1024);
+            const uint64_t dP0 = smem_desc(smem_u32(smem + kOffP), 2048, 1024);
+            bool ok = true;
+            uint32_t vn = 0;
             for (int j = 0; j < ntiles && ok; ++j) {
-                if (j + 1 < ntiles && !(ok = score(j + 1))) break;
                 if (!warp_wait(&bars[BAR_P_FULL], j & 1)) {
                     ok = false;
                     break;
                 }
+                if (lane == 0 && j < 8) TRACE(12 + 8 * j);
                 tc_fence_after();
                 uint64_t dp = dP0;
 #pragma unroll 1
                 for (int gi = 0; gi < kVGroups; ++gi) {
-                    const uint32_t slot = vn & 1u;
-                    if (!warp_wait(&bars[BAR_V_FULL + slot], (vn >> 1) & 1u)) {
+                    const uint32_t slot = vn % kVSlots;
+                    if (!warp_wait(&bars[BAR_V_FULL + slot], (vn / kVSlots) & 1u)) {
                         ok = false;
                         break;
                     }
+                    if (lane == 0 && j == 1) TRACE(340 + gi);
                     tc_fence_after();
                     const uint64_t dv = dV0 + (uint64_t)(slot * (kVSlotBytes >> 4));
                     const uint32_t acc = (j > 0 || gi > 0) ? 1u : 0u;
-#pragma unroll
-                    for (int b = 0; b < 4; ++b)
-                        mma_ss_warp(tmem + kColO + b * HG, dv + (uint64_t)(b * (4096 >> 4)), dp, id_pv, acc);
+                    if (lane == 0 && j == 1) TRACE(350 + gi);
+                    mma_ss_warp(tmem + kColO, dv, dp, id_pv, acc);
+                    if (lane == 0 && j == 1) TRACE(360 + gi);
+                    mma_ss_warp(tmem + kColO + HG, dv + (uint64_t)(4096 >> 4), dp, id_pv, acc);
+                    mma_ss_warp(tmem + kColO + 2 * HG, dv + (uint64_t)(2 * (4096 >> 4)), dp, id_pv, acc);
+                    mma_ss_warp(tmem + kColO + 3 * HG, dv + (uint64_t)(3 * (4096 >> 4)), dp, id_pv, acc);
+                    if (lane == 0 && j == 1) TRACE(370 + gi);
                     mma_commit_warp(&bars[BAR_V_FREE + slot]);
+                    if (lane == 0 && j == 1) TRACE(260 + gi);
                     dp += (uint64_t)(2048 >> 4);
                     ++vn;
                 }
                 if (!ok) break;
                 mma_commit_warp(&bars[BAR_PV_DONE]);
+                if (lane == 0 && j < 8) TRACE(13 + 8 * j);
             }
             if (!ok && lane == 0 && a.dev_status) atomicOr(a.dev_status, NVFP4MLA_DEV_TIMEOUT);
-            mma_commit_warp(&bars[BAR_DRAIN]);  // nothing may still read or write TMEM at teardown
-            warp_wait(&bars[BAR_DRAIN], 0);
-        } else if (warp == 1) {
+            mma_commit_warp(&bars[BAR_DRAIN_PV]);  // nothing may still read or write TMEM at teardown
+            warp_wait(&bars[BAR_DRAIN_PV], 0);
+        } else if (warp == 1 || warp == 3) {
             // ---------------------------------------------------- gather
-            int issued = 0;
+            // 64 threads copy the tile's rows in 16-byte pieces (22 per row)
+            // with cp.async; each thread's arrival on RAW_FULL fires when its
+            // own copies have landed.
+            const int gt = (warp == 1 ? 0 : 32) + lane;
             bool ok = true;
+            // rows of the first tiles go to L2 at once; later tiles are
+            // prefetched kPrefetchAhead tiles ahead of their copy, so the copy
+            // into the (single) raw slot costs an L2 round trip, not HBM's
+            auto prefetch_tile = [&](int jt) {  // every 128-byte line a row touches (4 probes cover 352 bytes)
+                const int32_t *pids = idx_s + kTileRows * jt;
+                const int n = tile_rows(jt) * 4;
+                for (int it = gt; it < n; it += 64) {
+                    const int r = it >> 2, q = it & 3;
+                    prefetch_l2(a.src + (int64_t)pids[r] * kRowBytes + (q < 3 ? 128 * q : kRowBytes - 1));
+                }
+            };
+            for (int jt = 0; jt < kPrefetchAhead && jt < ntiles; ++jt) prefetch_tile(jt);
             for (int j = 0; j < ntiles; ++j) {
-                const int slot = j & 1;
-                if (j >= 2 && !warp_wait(&bars[BAR_RAW_FREE + slot], ((j >> 1) - 1) & 1)) {
+                if (kPrefetchAhead > 0 && j + kPrefetchAhead < ntiles) prefetch_tile(j + kPrefetchAhead);
+                const int slot = j % kRawSlots;
+                if (j >= kRawSlots && !warp_wait(&bars[BAR_RAW_FREE + slot], ((j / kRawSlots) - 1) & 1)) {
                     ok = false;
                     break;
                 }
                 const int nrows = tile_rows(j);
-                if (lane == 0) mbar_arrive_expect_tx(&bars[BAR_RAW_FULL + slot], (uint32_t)(nrows * kRowBytes));
-                __syncwarp();
                 uint8_t *dst = smem + kOffRaw + slot * kRawSlotBytes;
                 const int32_t *ids = idx_s + kTileRows * j;
-                for (int r = lane; r < nrows; r += 32)
-                    bulk_g2s(dst + r * kRawStride, a.src + (int64_t)ids[r] * kRowBytes, kRowBytes,
-                             &bars[BAR_RAW_FULL + slot]);
-                ++issued;
+                const int items = nrows * (kRowBytes / 16);
+#pragma unroll 4
+                for (int it = gt; it < items; it += 64) {
+                    const int r = it / (kRowBytes / 16), k = it - r * (kRowBytes / 16);
+                    cp_async16(dst + r * kRawStride + 16 * k, a.src + (int64_t)ids[r] * kRowBytes + 16 * k);
+                }
+                cp_async_mbar_arrive(&bars[BAR_RAW_FULL + slot]);
+                if (gt == 0 && j < 8) TRACE(80 + j);
             }
-            // Copies still in flight must land before the CTA may exit (the
-            // consumers wait for them too unless a wait ran out).
-            for (int j = max(0, issued - 2); j < issued; ++j) warp_wait(&bars[BAR_RAW_FULL + (j & 1)], (j >> 1) & 1);
+            // copies still in flight land before the CTA may exit
+            asm volatile("cp.async.wait_all;" ::: "memory");
             if (!ok && lane == 0 && a.dev_status) atomicOr(a.dev_status, NVFP4MLA_DEV_TIMEOUT);
         }
         __syncwarp();
@@ -526,11 +603,12 @@ __global__ void __launch_bounds__(nv4::kThreads, 1)
         const uint32_t lane_base = (uint32_t)(32 * quarter) << 16;
         bool ok = true;
         for (int j = 0; j < ntiles && ok; ++j) {
-            const int rslot = j & 1;
-            if (!warp_wait(&bars[BAR_RAW_FULL + rslot], (j >> 1) & 1)) {
+            const int rslot = j % kRawSlots;
+            if (!warp_wait(&bars[BAR_RAW_FULL + rslot], (j / kRawSlots) & 1)) {
                 ok = false;
                 break;
             }
+            if (kw == 0 && lane == 0 && j < 8) TRACE(100 + j);
             const bool valid = r < tile_rows(j);
             const uint8_t *row = smem + kOffRaw + rslot * kRawSlotBytes + r * kRawStride;
 #pragma unroll 1
@@ -572,9 +650,11 @@ __global__ void __launch_bounds__(nv4::kThreads, 1)
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&bars[BAR_K_FULL + slot]);
+                if ((kw & 3) == 0 && lane == 0 && j == 1) TRACE(200 + c);
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars[BAR_RAW_FREE + rslot]);
+            if (kw == 0 && lane == 0 && j < 8) TRACE(110 + j);
         }
         if (!ok && lane == 0 && a.dev_status) atomicOr(a.dev_status, NVFP4MLA_DEV_TIMEOUT);
     } else if (warp < kVWarp0) {
@@ -584,11 +664,16 @@ __global__ void __launch_bounds__(nv4::kThreads, 1)
         const int wq = st >> 5;
         const uint32_t lane_base = (uint32_t)(32 * wq) << 16;
         uint8_t *p_tile = smem + kOffP;
-        // Running row sums: each tile's per-row values are folded across the
-        // warp (transpose reduction), so a lane keeps the sums of the warp's
-        // 32 rows for only cols_per_lane(HG) heads: heads lp_head(k).
-        constexpr int NL = cols_per_lane(HG);
-        auto lp_head = [&](int k) { return HG >= 32 ? lane * NL + k : (lane >> 1); };
+        // Scores are read from tensor memory twice, HC columns at a time:
+        // once to decide whether any head's reference max must move, once to
+        // form P.  The reference max is read from shared memory with 16-byte
+        // broadcast loads.  Row sums: each HC-column block of P is folded
+        // over the warp's 32 rows (transpose reduction) once P^T is
+        // published, so a lane keeps only the sums of NL heads, lp_head(k).
+        constexpr int HC = HG > 32 ? 32 : HG;
+        constexpr int NB = HG / HC;            // column blocks
+        constexpr int NL = NB * (HC >= 32 ? 1 : 1);
+        auto lp_head = [&](int k) { return HC >= 32 ? HC * k + lane : (lane >> 1); };
         float lp[NL];
 #pragma unroll
         for (int k = 0; k < NL; ++k) lp[k] = 0.0f;
@@ -600,28 +685,35 @@ __global__ void __launch_bounds__(nv4::kThreads, 1)
                 ok = false;
                 break;
             }
+            if (st == 0 && j < 8) TRACE(120 + j);
             tc_fence_after();
-            float sv[HG];
-            {
-                uint32_t rs[HG];
-                tmem_ld_cols<HG>(tmem + lane_base + kColS + 64u * (uint32_t)(j & 1), rs);
-                tmem_ld_wait();
-#pragma unroll
-                for (int h = 0; h < HG; ++h) sv[h] = __uint_as_float(rs[h]) * a.scale_log2;
-            }
+            const uint32_t s_addr = tmem + lane_base + kColS + 64u * (uint32_t)(j & 1);
             const bool valid = st < tile_rows(j);
             bool need = false;
-            if (valid) {
 #pragma unroll
-                for (int h = 0; h < HG; ++h) need |= sv[h] > m_s[h] + kRescaleThreshold;
+            for (int c0 = 0; c0 < HG; c0 += HC) {
+                uint32_t rs[HC];
+                tmem_ld_cols<HC>(s_addr + c0, rs);
+                tmem_ld_wait();
+#pragma unroll
+                for (int h = 0; h < HC; h += 4) {
+                    const float4 m4 = *reinterpret_cast<const float4 *>(m_s + c0 + h);
+                    need |= __uint_as_float(rs[h + 0]) * a.scale_log2 > m4.x + kRescaleThreshold;
+                    need |= __uint_as_float(rs[h + 1]) * a.scale_log2 > m4.y + kRescaleThreshold;
+                    need |= __uint_as_float(rs[h + 2]) * a.scale_log2 > m4.z + kRescaleThreshold;
+                    need |= __uint_as_float(rs[h + 3]) * a.scale_log2 > m4.w + kRescaleThreshold;
+                }
             }
-            const bool rescale = named_bar_or(1, 128, need);
+            const bool rescale = named_bar_or(1, 128, valid && need);
             if (rescale) {
 #pragma unroll
                 for (int c0 = 0; c0 < HG; c0 += 16) {  // column max, 16 heads at a time
+                    uint32_t rs[16];
+                    tmem_ld16(s_addr + c0, rs);
+                    tmem_ld_wait();
                     float mx[16];
 #pragma unroll
-                    for (int h = 0; h < 16; ++h) mx[h] = valid ? sv[c0 + h] : -INFINITY;
+                    for (int h = 0; h < 16; ++h) mx[h] = valid ? __uint_as_float(rs[h]) * a.scale_log2 : -INFINITY;
                     warp_transpose_reduce<16, true>(mx, lane);
                     if (!(lane & 1)) red_s[wq * 64 + c0 + transposed_col<16>(lane, 0)] = mx[0];
                 }
@@ -638,6 +730,35 @@ __global__ void __launch_bounds__(nv4::kThreads, 1)
 #pragma unroll
                 for (int k = 0; k < NL; ++k) lp[k] *= aux_s[lp_head(k)];
             }
+            // P (FP16, packed in registers) and this tile's row sums need
+            // neither O^T nor the P^T buffer, so they are formed while the
+            // output MMAs of the previous tile may still run; only the P^T
+            // stores (and a rare O^T rescale) wait for those to finish.
+            uint32_t pk[HG / 2];
+#pragma unroll
+            for (int c0 = 0; c0 < HG; c0 += HC) {
+                float pv[HC];
+                {
+                    uint32_t rs[HC];
+                    tmem_ld_cols<HC>(s_addr + c0, rs);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int h = 0; h < HC; h += 4) {
+                        const float4 m4 = *reinterpret_cast<const float4 *>(m_s + c0 + h);
+                        pv[h + 0] = valid ? ex2(__uint_as_float(rs[h + 0]) * a.scale_log2 - m4.x) : 0.0f;
+                        pv[h + 1] = valid ? ex2(__uint_as_float(rs[h + 1]) * a.scale_log2 - m4.y) : 0.0f;
+                        pv[h + 2] = valid ? ex2(__uint_as_float(rs[h + 2]) * a.scale_log2 - m4.z) : 0.0f;
+                        pv[h + 3] = valid ? ex2(__uint_as_float(rs[h + 3]) * a.scale_log2 - m4.w) : 0.0f;
+                    }
+                }
+#pragma unroll
+                for (int h = 0; h < HC; h += 2) pk[(c0 + h) / 2] = pack_half2(pv[h], pv[h + 1]);
+                warp_transpose_reduce<HC, false>(pv, lane);
+                lp[c0 / HC] += pv[0];
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars[BAR_S_FREE + (j & 1)]);  // this warp's reads of S(j) are done
             // O^T and P^T belong to the output MMAs of the previous tile
             // until they are done.
             if (j > 0) {
@@ -645,6 +766,7 @@ __global__ void __launch_bounds__(nv4::kThreads, 1)
                     ok = false;
                     break;
                 }
+                if (st == 0 && j < 8) TRACE(130 + j);
                 tc_fence_after();
                 if (rescale) {
 #pragma unroll 1
@@ -664,30 +786,20 @@ __global__ void __launch_bounds__(nv4::kThreads, 1)
                 }
             }
 #pragma unroll
-            for (int h = 0; h < HG; ++h) sv[h] = valid ? ex2(sv[h] - m_s[h]) : 0.0f;
-#pragma unroll
-            for (int jj = 0; jj < HG / 8; ++jj) {
-                uint4 pk;
-                pk.x = pack_half2(sv[8 * jj + 0], sv[8 * jj + 1]);
-                pk.y = pack_half2(sv[8 * jj + 2], sv[8 * jj + 3]);
-                pk.z = pack_half2(sv[8 * jj + 4], sv[8 * jj + 5]);
-                pk.w = pack_half2(sv[8 * jj + 6], sv[8 * jj + 7]);
-                *reinterpret_cast<uint4 *>(p_tile + sw128_offset(st, jj)) = pk;
-            }
+            for (int jj = 0; jj < HG / 8; ++jj)
+                *reinterpret_cast<uint4 *>(p_tile + sw128_offset(st, jj)) =
+                    make_uint4(pk[4 * jj], pk[4 * jj + 1], pk[4 * jj + 2], pk[4 * jj + 3]);
             fence_proxy_async_smem();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars[BAR_P_FULL]);
-            // row sums of this tile (FP32 values, as the FP16 P rounds them
-            // only for the MMA), folded over the warp's rows
-            warp_transpose_reduce<HG, false>(sv, lane);
-#pragma unroll
-            for (int k = 0; k < NL; ++k) lp[k] += sv[k];
+            if (st == 0 && j < 8) TRACE(140 + j);
         }
         if (!ok && a.dev_status && lane == 0) atomicOr(a.dev_status, NVFP4MLA_DEV_TIMEOUT);
         // ---------------------------------------------------------- epilogue
+        if (st == 0) TRACE(170);
         const bool have = ok && ntiles > 0;
-        if (HG >= 32 || !(lane & 1)) {  // row sums: one partial per warp and head
+        if (HC >= 32 || !(lane & 1)) {  // row sums: one partial per warp and head
 #pragma unroll
             for (int k = 0; k < NL; ++k) red_s[wq * 64 + lp_head(k)] = lp[k];
         }
@@ -712,9 +824,10 @@ __global__ void __launch_bounds__(nv4::kThreads, 1)
             if (!fin && st == 0 && a.dev_status) atomicOr(a.dev_status, NVFP4MLA_DEV_TIMEOUT);
             tc_fence_after();
         }
+        if (st == 0) TRACE(171);
         // Every K-unpack warp is past its last raw tile once the last output
         // MMAs are done (they needed every chunk), so the raw ring is free.
-        uint8_t *stage = smem + kOffRaw;
+        uint8_t *stage = smem + kOffStage;
         if (a.S == 1) {
             // O^T (TMEM lanes = dv) -> normalised FP16 rows [HG][512] staged
             // in the raw ring, then one bulk copy of HG x 1 KB.
@@ -778,24 +891,31 @@ __global__ void __launch_bounds__(nv4::kThreads, 1)
                     }
                 }
             }
+            if (st == 0) TRACE(172);
             switch (a.S) {
-                case 2: merge_splits_nv4<HG, 2>(a, t, g, split, smem, st); break;
-                case 4: merge_splits_nv4<HG, 4>(a, t, g, split, smem, st); break;
-                case 8: merge_splits_nv4<HG, 8>(a, t, g, split, smem, st); break;
-                default: merge_splits_nv4<HG, 16>(a, t, g, split, smem, st); break;
+                case 2: merge_splits_nv4<HG, 2>(a, t, g, split, smem, st, t_start); break;
+                case 4: merge_splits_nv4<HG, 4>(a, t, g, split, smem, st, t_start); break;
+                case 8: merge_splits_nv4<HG, 8>(a, t, g, split, smem, st, t_start); break;
+                default: merge_splits_nv4<HG, 16>(a, t, g, split, smem, st, t_start); break;
             }
+            if (st == 0) TRACE(174);
         }
     } else {
         // -------------------------------------------------------- V unpack
-        // Slot layout (MN-major A operand of the output MMA): dv group dg
-        // (64 dims) at dg * 2048, row r of the 16 at r * 128, 16-byte chunk
-        // jj swizzled by the row.  Thread = (row r, dv group dg); the rows
-        // are read from L2 (the gather brought them in a tile earlier).
-        const int vw = warp - kVWarp0;  // 0..3
+        // Two sets of four warps alternate the 16-row groups of a tile: set
+        // vs converts groups vs, vs + 2, ... into ring slot vs, so each set
+        // has two group periods for its own convert-and-store work.  Slot
+        // layout (MN-major A operand of the output MMA): dv group dg (64
+        // dims) at dg * 2048, row r of the 16 at r * 128, 16-byte chunk jj
+        // swizzled by the row.  Thread = (row r, dv group dg); the rows are
+        // read from L2 (the gather brought them in a tile earlier).
+        if (kRegsV < kRegsLaunch) regs_dec<kRegsV < kRegsLaunch ? kRegsV : kRegsLaunch - 8>();
+        const int vs = (warp - kVWarp0) >> 2;  // V set: 0 or 1
+        const int vw = (warp - kVWarp0) & 3;
         const int r = lane & 15;
         const int dg = 2 * vw + (lane >> 4);
         bool ok = true;
-        uint32_t vn = 0;
+        uint32_t vn = (uint32_t)vs;  // ring position of this set's next group (groups alternate sets)
         for (int j = 0; j < ntiles && ok; ++j) {
             // The tile's rows are in L2 once its score MMAs are done; that
             // also keeps these loads from racing the gather to HBM.
@@ -803,6 +923,7 @@ __global__ void __launch_bounds__(nv4::kThreads, 1)
                 ok = false;
                 break;
             }
+            if (vs == 0 && vw == 0 && lane == 0 && j < 8) TRACE(150 + j);
             const int nrows = tile_rows(j);
             const int32_t *ids = idx_s + kTileRows * j;
             auto load = [&](int gi, uint4 &w0, uint4 &w1, uint32_t &sc) {
@@ -817,38 +938,45 @@ __global__ void __launch_bounds__(nv4::kThreads, 1)
                     sc = 0u;
                 }
             };
-            uint4 a0, a1, b0, b1;
-            uint32_t as, bs;
-            load(0, a0, a1, as);
-            load(1, b0, b1, bs);
-#pragma unroll 1
-            for (int gi = 0; gi < kVGroups; ++gi) {
+            // this set's next two groups are in flight ahead of the one
+            // being converted
+            constexpr int kMine = kVGroups / 2;
+            constexpr int kDepth = 2;
+            uint4 w0[kDepth], w1[kDepth];
+            uint32_t sc[kDepth];
+#pragma unroll
+            for (int d = 0; d < kDepth; ++d) load(vs + 2 * d, w0[d], w1[d], sc[d]);
+#pragma unroll
+            for (int m = 0; m < kMine; ++m) {
+                const uint32_t slot = vn % kVSlots;
+                uint8_t *base = smem + kOffV + slot * kVSlotBytes + dg * 2048;
                 uint32_t o[32];
-                unpack_latent64(a0, a1, as, o);
-                a0 = b0;
-                a1 = b1;
-                as = bs;
-                if (gi + 2 < kVGroups) load(gi + 2, b0, b1, bs);
-                const uint32_t slot = vn & 1u;
-                if (vn >= 2 && !warp_wait(&bars[BAR_V_FREE + slot], ((vn >> 1) - 1) & 1u)) {
+                unpack_latent64(w0[m % kDepth], w1[m % kDepth], sc[m % kDepth], o);
+                if (m + kDepth < kMine) load(vs + 2 * (m + kDepth), w0[m % kDepth], w1[m % kDepth], sc[m % kDepth]);
+                if (vw == 0 && lane == 0 && j == 1) TRACE(300 + 20 * vs + 4 * m);
+                if (vn >= kVSlots && !warp_wait(&bars[BAR_V_FREE + slot], ((vn / kVSlots) - 1) & 1u)) {
                     ok = false;
                     break;
                 }
-                uint8_t *base = smem + kOffV + slot * kVSlotBytes + dg * 2048;
+                if (vw == 0 && lane == 0 && j == 1) TRACE(301 + 20 * vs + 4 * m);
 #pragma unroll
                 for (int jj = 0; jj < 8; ++jj)
                     *reinterpret_cast<uint4 *>(base + sw128_offset(r, jj)) =
                         make_uint4(o[4 * jj], o[4 * jj + 1], o[4 * jj + 2], o[4 * jj + 3]);
                 fence_proxy_async_smem();
+                if (vw == 0 && lane == 0 && j == 1) TRACE(302 + 20 * vs + 4 * m);
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&bars[BAR_V_FULL + slot]);
-                ++vn;
+                if (vw == 0 && lane == 0 && j == 1) TRACE(220 + vs + 2 * m);
+                vn += 2;
             }
+            if (vs == 0 && vw == 0 && lane == 0 && j < 8) TRACE(160 + j);
         }
         if (!ok && lane == 0 && a.dev_status) atomicOr(a.dev_status, NVFP4MLA_DEV_TIMEOUT);
     }
 
     // ---------------------------------------------------------------- teardown
+    if (tid == 32 * kSoftWarp0) TRACE(180);
     tc_fence_before();
     __syncthreads();
     if (warp == 2) {
