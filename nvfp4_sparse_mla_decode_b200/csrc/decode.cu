@@ -962,6 +962,40 @@ bool make_q_map(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols, 
     return true;
 }
 
+// Tensor map for the FP32 split partials: a 2-D view [rows, 512] of
+// ws_o, box box_cols x box_rows, no swizzle; cached like the Q maps.
+bool make_partial_map(CUtensorMap *m, const void *base, uint64_t rows, uint32_t box_cols, uint32_t box_rows) {
+    struct Entry {
+        const void *base;
+        uint64_t rows;
+        uint32_t box_cols, box_rows;
+        CUtensorMap map;
+    };
+    constexpr int kEntries = 8;
+    thread_local Entry cache[kEntries] = {};
+    thread_local int next = 0;
+    for (int i = 0; i < kEntries; ++i) {
+        const Entry &e = cache[i];
+        if (e.base == base && e.rows == rows && e.box_cols == box_cols && e.box_rows == box_rows) {
+            *m = e.map;
+            return true;
+        }
+    }
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    const cuuint64_t dims[2] = {(cuuint64_t)kLatent, rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)kLatent * 4};
+    const cuuint32_t box[2] = {box_cols, box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    if (enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void *>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return false;
+    cache[next] = Entry{base, rows, box_cols, box_rows, *m};
+    next = (next + 1) % kEntries;
+    return true;
+}
+
 template <int HG, bool kStaged>
 static cudaError_t launch_hg(const DecodeArgs &a, int64_t nblocks, cudaStream_t stream) {
     auto kern = sparse_mla_decode_kernel<HG, kStaged>;

@@ -128,6 +128,9 @@ __host__ __device__ constexpr int cols_per_lane(int W) { return W >= 32 ? W / 32
 // or q_rope (cols 64), box 64 cols x box_rows rows, 128-byte swizzle; encoded
 // maps are cached per host thread, keyed by (address, rows, cols, box rows).
 bool make_q_map(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols, uint32_t box_rows);
+// Tensor map over the FP32 split partials [rows, 512] (box box_cols x box_rows,
+// no swizzle), cached per host thread like the Q maps.
+bool make_partial_map(CUtensorMap *m, const void *base, uint64_t rows, uint32_t box_cols, uint32_t box_rows);
 // Launch of the pipelined NVFP4 decode kernel (decode_nvfp4.cu).
 cudaError_t launch_nvfp4_decode(const DecodeArgs &a, int heads_per_cta, int64_t nblocks, cudaStream_t stream);
 

@@ -106,6 +106,9 @@ static_assert(kOffP % 1024 == 0 && kOffV % 1024 == 0, "swizzled operands need 1 
 // the epilogue stages its output (or its own merge slice) over the V and raw
 // rings, which are free by then; the merge weights go to the P^T region
 constexpr int kOffStage = kOffV;
+constexpr int kOffPartial = kOffP;  // split partial boxes [S][HG][512/S] FP32 over P^T and the rings
+constexpr int kOffMergeW = kOffPartial + kMaxHG * kLatent * 4;  // merge weights, after the boxes
+static_assert(kOffMergeW + (16 * kMaxHG + kMaxHG) * 4 <= kOffIdx, "partial boxes and weights must fit before the list");
 static_assert(kMaxHG * kLatent * 2 <= kOffIdx - kOffStage, "output staging must fit over the rings");
 static_assert(kMaxHG * (kLatent / 2) * 4 <= kOffIdx - kOffStage, "own merge slice must fit over the rings");
 constexpr int kThreads = 768;
@@ -147,6 +150,7 @@ constexpr uint32_t kColS = 256;
 constexpr uint32_t kColK = 384;
 constexpr float kRescaleThreshold = 8.0f;
 constexpr int kMaxSplits = 16;
+static_assert(kMaxSplits == 16, "merge weight area sized for 16 splits");
 constexpr uint32_t kPoison = 0x80000000u;
 }  // namespace nv4
 
@@ -184,54 +188,82 @@ __device__ __forceinline__ void unpack_latent64(uint4 w0, uint4 w1, uint32_t sca
 }
 
 // Split merge, run by the 128 softmax threads of each of the S CTAs of a
-// (token, head group) once its partial is written: announce the partial on
-// the group's arrival counter (release), wait (bounded) until all S have,
-// then combine dv slice [split*512/S, (split+1)*512/S) of every head:
+// (token, head group) once this CTA's unnormalised partial O sits in shared
+// memory as S boxes of [HG heads][D = 512/S dims] FP32 (box k = dims
+// k*D .. k*D+D-1).  Thread 0 sends every box but the CTA's own (box `split`)
+// to the workspace with 2-D tensor copies, waits until they have landed and
+// announces them on the group's arrival counter (release).  Once all S have
+// arrived (bounded wait), it fetches the other splits' copies of box `split`
+// into the places the sent boxes occupied, and the 128 threads combine dims
+// [split*D, split*D + D) of every head:
 //   out = sum_s w_s O_s / sum_s w_s l_s,  w_s = 2^(m_s - max m)
 // over the splits with rows (l_s > 0); split 0 also writes
-// lse = (max m + log2 of the denominator) ln 2.  With S <= 4 the CTA's own
-// slice is in shared memory.  The last CTA to leave resets the counters.  A
-// wait that runs out sets the counter's poison bit: that CTA and every later
-// one on the same counter report NVFP4MLA_DEV_TIMEOUT and write NaN to their
-// slice instead of merging partials that were never written.
+// lse = (max m + log2 of the denominator) ln 2.  The last CTA to leave resets
+// the counters.  A wait that runs out sets the counter's poison bit: that CTA
+// and every later one on the same counter report NVFP4MLA_DEV_TIMEOUT and
+// write NaN to their slice instead of merging partials that were never
+// written.
 template <int HG, int S>
-__device__ __forceinline__ void merge_splits_nv4(const DecodeArgs &a, int t, int g, int split, uint8_t *smem, int mt,
+__device__ __forceinline__ void merge_splits_nv4(const DecodeArgs &a, const CUtensorMap *tm_ws, int t, int g,
+                                                 int split, uint8_t *smem, uint64_t *bar, int mt,
                                                  [[maybe_unused]] unsigned long long t_start) {
     using namespace nv4;
     constexpr int kMergeThreads = 128;
     constexpr int D = kLatent / S;
+    constexpr int kBoxBytes = HG * D * 4;
     constexpr int NQ = D / 4;
     constexpr int ITEMS = HG * NQ;
-    constexpr bool kOwnInSmem = S <= 4;
-    constexpr int kGlobal = kOwnInSmem ? S - 1 : S;
-    constexpr int kPerThread = (ITEMS + kMergeThreads - 1) / kMergeThreads;
-    constexpr int B = (24 / kGlobal) < 1 ? 1 : ((24 / kGlobal) > kPerThread ? kPerThread : (24 / kGlobal));
     uint32_t *arrive = a.counters + 2 * ((int64_t)t * a.G + g);
     uint32_t *depart = arrive + 1;
     uint32_t *flag = reinterpret_cast<uint32_t *>(smem + kOffMisc) + 1;
-    float *w_s = reinterpret_cast<float *>(smem + kOffP);   // [S][HG]
-    float *inv_den = w_s + kMaxSplits * HG;                  // [HG]
-    const float *own = reinterpret_cast<const float *>(smem + kOffStage);  // [HG][D]
-    named_bar(1, kMergeThreads);  // every partial store of this CTA precedes the release
+    const float *stage = reinterpret_cast<const float *>(smem + kOffPartial);  // [S][HG][D]
+    float *w_s = reinterpret_cast<float *>(smem + kOffMergeW);               // [S][HG]
+    float *inv_den = w_s + nv4::kMaxSplits * HG;                              // [HG]
+    const int32_t row0 = (t * S + split) * a.H + g * HG;  // this split's partial rows
+    fence_proxy_async_smem();       // the drained boxes are visible to the copy engine
+    named_bar(1, kMergeThreads);    // ... and to thread 0, with the statistics stores
     if (mt == 0) {
         TRACE(190);
-        __threadfence();
+#pragma unroll 1
+        for (int k = 0; k < S; ++k)
+            if (k != split) tma_store_2d(tm_ws, smem + kOffPartial + k * kBoxBytes, k * D, row0);
+        bulk_commit_wait_all();     // the partial boxes have reached global memory
+        fence_proxy_async_global();
+        __threadfence();            // ... and, with the statistics, are ordered before the arrival
         TRACE(191);
-        const uint32_t old = atomicAdd(arrive, 1u);  // relaxed add; the fence above orders the partials
+        const uint32_t old = atomicAdd(arrive, 1u);
         bool ok = (old & kPoison) == 0;
         if (ok) {
             const unsigned long long t0 = clock64();
             while (true) {
                 const uint32_t v = ld_acquire_gpu(arrive);
-                if (v & kPoison) { ok = false; break; }
+                if (v & kPoison) {
+                    ok = false;
+                    break;
+                }
                 if (v >= (uint32_t)S) break;
-                if (clock64() - t0 > kWaitCycles) { ok = false; break; }
-                __nanosleep(64);
+                if (clock64() - t0 > kWaitCycles) {
+                    ok = false;
+                    break;
+                }
+                __nanosleep(32);
             }
         }
         if (!ok) {
             atomicOr(arrive, kPoison);
             if (a.dev_status) atomicOr(a.dev_status, NVFP4MLA_DEV_TIMEOUT);
+        } else {
+            // the other splits' copies of this CTA's box, into the places of
+            // the boxes just sent (their copies have read them)
+            fence_proxy_async_global();
+            // this barrier's first phase tracked the Q copies; they have
+            // landed before its second phase is armed
+            if (!mbar_wait(bar, 0) && a.dev_status) atomicOr(a.dev_status, NVFP4MLA_DEV_TIMEOUT);
+            mbar_arrive_expect_tx(bar, (uint32_t)((S - 1) * kBoxBytes));
+#pragma unroll 1
+            for (int s = 0; s < S; ++s)
+                if (s != split)
+                    tma_load_2d(smem + kOffPartial + s * kBoxBytes, tm_ws, split * D, (t * S + s) * a.H + g * HG, bar);
         }
         *flag = ok ? 1u : 0u;
         TRACE(192);
@@ -247,56 +279,7 @@ __device__ __forceinline__ void merge_splits_nv4(const DecodeArgs &a, int t, int
         if (split == 0 && mt < HG) a.lse[(int64_t)t * a.H + (int64_t)g * HG + mt] = NAN;
         return;
     }
-    const int64_t part = (int64_t)a.H * kLatent;
-    const float *src = a.ws_o + ((int64_t)t * S * a.H + (int64_t)g * HG) * kLatent + dv0;
-    float4 o[B][kGlobal];
-    auto load_batch = [&](int base) {
-#pragma unroll
-        for (int b = 0; b < B; ++b) {
-            const int item = base + b * kMergeThreads;
-            const int h = item / NQ, q = item - h * NQ;
-#pragma unroll
-            for (int j = 0; j < kGlobal; ++j) {
-                const int s = kOwnInSmem && j >= split ? j + 1 : j;
-                o[b][j] = item < ITEMS
-                              ? __ldcg(reinterpret_cast<const float4 *>(src + (int64_t)h * kLatent + 4 * q + s * part))
-                              : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-            }
-        }
-    };
-    auto combine_batch = [&](int base) {
-#pragma unroll
-        for (int b = 0; b < B; ++b) {
-            const int item = base + b * kMergeThreads;
-            if (item < ITEMS) {
-                const int h = item / NQ, q = item - h * NQ;
-                float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-                if (kOwnInSmem) {
-                    const float w = w_s[split * HG + h];
-                    const float4 v = *reinterpret_cast<const float4 *>(own + h * D + 4 * q);
-                    acc.x = w * v.x;
-                    acc.y = w * v.y;
-                    acc.z = w * v.z;
-                    acc.w = w * v.w;
-                }
-#pragma unroll
-                for (int j = 0; j < kGlobal; ++j) {
-                    const int s = kOwnInSmem && j >= split ? j + 1 : j;
-                    const float w = w_s[s * HG + h];
-                    acc.x += w * o[b][j].x;
-                    acc.y += w * o[b][j].y;
-                    acc.z += w * o[b][j].z;
-                    acc.w += w * o[b][j].w;
-                }
-                const float r = inv_den[h];
-                __half2 *d2 = reinterpret_cast<__half2 *>(dst + (int64_t)h * kLatent + 4 * q);
-                d2[0] = __floats2half2_rn(acc.x * r, acc.y * r);
-                d2[1] = __floats2half2_rn(acc.z * r, acc.w * r);
-            }
-        }
-    };
-    load_batch(mt);
-    if (mt < HG) {
+    if (mt < HG) {  // split weights from the statistics while the boxes travel
         const float *ml = a.ws_ml + 2 * ((int64_t)t * S * a.H + (int64_t)g * HG + mt);
         float2 v[S];
 #pragma unroll
@@ -317,12 +300,26 @@ __device__ __forceinline__ void merge_splits_nv4(const DecodeArgs &a, int t, int
             a.lse[(int64_t)t * a.H + (int64_t)g * HG + mt] =
                 den > 0.0f ? (mmax + lg2(den)) * 0.69314718055994531f : -INFINITY;
     }
+    const bool landed = mbar_wait(bar, 1);  // the box copies (phase 1 of the Q barrier)
+    if (!landed && a.dev_status) atomicOr(a.dev_status, NVFP4MLA_DEV_TIMEOUT);
     named_bar(1, kMergeThreads);
     if (mt == 0) TRACE(193);
-    combine_batch(mt);
-    for (int base = mt + kMergeThreads * B; base < ITEMS; base += kMergeThreads * B) {
-        load_batch(base);
-        combine_batch(base);
+    for (int item = mt; item < ITEMS; item += kMergeThreads) {
+        const int h = item / NQ, q = item - h * NQ;
+        float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+#pragma unroll
+        for (int s = 0; s < S; ++s) {
+            const float w = w_s[s * HG + h];
+            const float4 v = *reinterpret_cast<const float4 *>(stage + (s * HG + h) * D + 4 * q);
+            acc.x += w * v.x;
+            acc.y += w * v.y;
+            acc.z += w * v.z;
+            acc.w += w * v.w;
+        }
+        const float r = inv_den[h];
+        __half2 *d2 = reinterpret_cast<__half2 *>(dst + (int64_t)h * kLatent + 4 * q);
+        d2[0] = __floats2half2_rn(acc.x * r, acc.y * r);
+        d2[1] = __floats2half2_rn(acc.z * r, acc.w * r);
     }
     named_bar(1, kMergeThreads);
     if (mt == 0) {
@@ -338,7 +335,7 @@ __device__ __forceinline__ void merge_splits_nv4(const DecodeArgs &a, int t, int
 template <int HG>
 __global__ void __launch_bounds__(nv4::kThreads, 1)
     nvfp4_decode_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_qn,
-                        const __grid_constant__ CUtensorMap tm_qr) {
+                        const __grid_constant__ CUtensorMap tm_qr, const __grid_constant__ CUtensorMap tm_ws) {
     using namespace nv4;
     extern __shared__ __align__(1024) uint8_t smem[];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -858,19 +855,19 @@ __global__ void __launch_bounds__(nv4::kThreads, 1)
                 bulk_commit_wait_read();
             }
         } else {
-            // Unnormalised partial O of this split: blocks inside the CTA's
-            // own merge slice (S <= 4) stay in shared memory, the others go
-            // to the workspace (for each head a warp writes 32 consecutive
-            // dv, one 128-byte segment).
-            float *dst = a.ws_o + (((int64_t)t * a.S + split) * a.H + (int64_t)g * HG) * kLatent + st;
-            const int own_n = a.S <= 4 ? 4 / a.S : 0;
-            const int own_b0 = split * own_n;
-            const int own_d = kLatent / a.S;
-            float *own = reinterpret_cast<float *>(stage) + st;
+            // Unnormalised partial O of this split into shared memory as S
+            // boxes [HG][D] (box k = dims k*D ..), over the P^T and ring
+            // regions, which no MMA or copy uses any more; for each head a
+            // warp writes 32 consecutive dims.  The merge sends the boxes out
+            // with tensor copies.
+            const int D = kLatent / a.S;
+            float *box = reinterpret_cast<float *>(smem + kOffPartial);
             constexpr int HC = HG > 32 ? 32 : HG;
 #pragma unroll 1
             for (int b = 0; b < 4; ++b) {
-                const bool mine = b >= own_b0 && b < own_b0 + own_n;
+                const int dv = 128 * b + st;
+                const int k = dv / D, d = dv - k * D;
+                float *dst = box + (k * HG) * D + d;
 #pragma unroll
                 for (int h0 = 0; h0 < HG; h0 += HC) {
                     uint32_t rr[HC];
@@ -881,22 +878,17 @@ __global__ void __launch_bounds__(nv4::kThreads, 1)
 #pragma unroll
                         for (int h = 0; h < HC; ++h) rr[h] = 0u;
                     }
-                    if (mine) {
 #pragma unroll
-                        for (int h = 0; h < HC; ++h) own[(h0 + h) * own_d + 128 * (b - own_b0)] = __uint_as_float(rr[h]);
-                    } else {
-#pragma unroll
-                        for (int h = 0; h < HC; ++h)
-                            __stcg(dst + (int64_t)(h0 + h) * kLatent + 128 * b, __uint_as_float(rr[h]));
-                    }
+                    for (int h = 0; h < HC; ++h) dst[(h0 + h) * D] = __uint_as_float(rr[h]);
                 }
             }
             if (st == 0) TRACE(172);
+            uint64_t *mbar = &bars[BAR_Q];  // its second phase tracks the merge's box copies
             switch (a.S) {
-                case 2: merge_splits_nv4<HG, 2>(a, t, g, split, smem, st, t_start); break;
-                case 4: merge_splits_nv4<HG, 4>(a, t, g, split, smem, st, t_start); break;
-                case 8: merge_splits_nv4<HG, 8>(a, t, g, split, smem, st, t_start); break;
-                default: merge_splits_nv4<HG, 16>(a, t, g, split, smem, st, t_start); break;
+                case 2: merge_splits_nv4<HG, 2>(a, &tm_ws, t, g, split, smem, mbar, st, t_start); break;
+                case 4: merge_splits_nv4<HG, 4>(a, &tm_ws, t, g, split, smem, mbar, st, t_start); break;
+                case 8: merge_splits_nv4<HG, 8>(a, &tm_ws, t, g, split, smem, mbar, st, t_start); break;
+                default: merge_splits_nv4<HG, 16>(a, &tm_ws, t, g, split, smem, mbar, st, t_start); break;
             }
             if (st == 0) TRACE(174);
         }
@@ -1014,11 +1006,17 @@ static cudaError_t launch_nv4(const DecodeArgs &a, int64_t nblocks, cudaStream_t
     attr[0].val.cooperative = 1;
     cfg.attrs = attr;
     cfg.numAttrs = a.S > 1 ? 1 : 0;  // split launches need every CTA resident at once
-    CUtensorMap tm_qn, tm_qr;
+    CUtensorMap tm_qn, tm_qr, tm_ws;
     const uint64_t rows = (uint64_t)a.T * (uint64_t)a.H;
     if (!make_q_map(&tm_qn, a.q_nope, rows, kLatent, HG) || !make_q_map(&tm_qr, a.q_rope, rows, kRope, HG))
         return cudaErrorInvalidValue;
-    return cudaLaunchKernelEx(&cfg, kern, a, tm_qn, tm_qr);
+    if (a.S > 1) {  // split partials [T * S * H, 512], one box = HG heads x 512/S dims
+        if (!make_partial_map(&tm_ws, a.ws_o, rows * (uint64_t)a.S, (uint32_t)(kLatent / a.S), HG))
+            return cudaErrorInvalidValue;
+    } else {
+        tm_ws = tm_qn;  // unused without splits
+    }
+    return cudaLaunchKernelEx(&cfg, kern, a, tm_qn, tm_qr, tm_ws);
 }
 
 cudaError_t launch_nvfp4_decode(const DecodeArgs &a, int heads_per_cta, int64_t nblocks, cudaStream_t stream) {

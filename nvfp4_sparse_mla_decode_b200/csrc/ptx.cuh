@@ -107,6 +107,25 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const void *tmap, int32_t
         : "memory");
 }
 
+// Tiled 2-D tensor copy from this CTA's shared memory to global memory
+// (bulk-group completion; see bulk_commit_wait_all / bulk_commit_wait_read).
+__device__ __forceinline__ void tma_store_2d(const void *tmap, const void *src, int32_t x, int32_t y) {
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                     reinterpret_cast<uint64_t>(tmap)),
+                 "r"(smem_u32(src)), "r"(x), "r"(y)
+                 : "memory");
+}
+// Commit the bulk copies issued so far and wait until they have completed
+// (their global writes done, not only their shared-memory reads).
+__device__ __forceinline__ void bulk_commit_wait_all() {
+    asm volatile("cp.async.bulk.commit_group;\n\tcp.async.bulk.wait_group 0;" ::: "memory");
+}
+// Order this thread's async-proxy accesses to global memory with its generic
+// ones (both directions), e.g. between tensor copies and a release/acquire.
+__device__ __forceinline__ void fence_proxy_async_global() {
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
 // 16-byte asynchronous copy global -> shared (no register staging); the
 // copies of a thread complete at cp_async_wait_all().
 __device__ __forceinline__ void cp_async16(void *dst, const void *src) {
