@@ -163,7 +163,7 @@ def kernel_traffic(kernel_file: str):
         return None
     with open(path) as f:
         d = json.load(f)
-    if d.get("decode_cu_code_sha256") != code_fingerprint(kernel_file):
+    if d.get("kernel_code_sha256") != code_fingerprint(kernel_file):
         return None
     return d.get("dram_bytes_per_launch")
 
@@ -284,9 +284,21 @@ def time_other_workload(name, w, nv, synth, args):
             "tflops": flop / (us * 1e-6) / 1e12, "gathered_gbs": rows * ROW_BYTES / (us * 1e-6) / 1e9,
             "roofline_us": t_roof * 1e6, "frac_of_roofline": t_roof / (us * 1e-6),
             "timing": "single launch, L2 flushed before it, median of 20", "data": "synthetic"}
-    print(json.dumps(line), flush=True)
     del cache, flush
     torch.cuda.empty_cache()
+    return line
+
+
+def config_workloads(synth):
+    """The parity configurations other than the headline launch, as
+    (name, workload factory) pairs: the tiny case, the H=128 decode sweep at
+    every token count, the padded-list stress and the 4000-token prefill."""
+    items = [("tiny1x16", lambda: synth.tiny("cuda"))]
+    for T in (1, 8, 32, 64, 128, 256):
+        items.append(("sweep%dx128" % T, lambda T=T: synth.sweep("cuda", T)))
+    items.append(("padded256x64", lambda: synth.padded("cuda")))
+    items.append(("prefill4000x64", lambda: synth.append_prefill("cuda")))
+    return items
 
 
 def time_paged(nv, synth, args):
@@ -549,15 +561,129 @@ def other_workloads(args):
             time_paged(nv, synth, args)
         if name == "fp8":
             time_fp8(nv, synth, args)
-        if name == "tiny":
-            time_other_workload("tiny1x16", synth.tiny("cuda"), nv, synth, args)
-        elif name == "sweep":
-            for T in (1, 8, 32, 64, 128, 256):
-                time_other_workload("sweep%dx128" % T, synth.sweep("cuda", T), nv, synth, args)
-        elif name == "padded":
-            time_other_workload("padded256x64", synth.padded("cuda"), nv, synth, args)
-        elif name == "prefill":
-            time_other_workload("prefill4000x64", synth.append_prefill("cuda"), nv, synth, args)
+        for cname, make in config_workloads(synth):
+            if (name == "tiny" and cname.startswith("tiny")) or (name == "sweep" and cname.startswith("sweep")) or \
+                    (name == "padded" and cname.startswith("padded")) or (name == "prefill" and cname.startswith("prefill")):
+                print(json.dumps(time_other_workload(cname, make(), nv, synth, args)), flush=True)
+
+
+def graph_us(fns, n):
+    """Device time per call (us) of the callables in fns, captured once in a
+    CUDA graph (one call each) and replayed until n calls have run; CUDA
+    events on the launching stream around the replays."""
+    import torch
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for fn in fns:
+            fn()
+    g.replay()
+    torch.cuda.synchronize()
+    reps = max(1, n // len(fns))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    stream = torch.cuda.current_stream()
+    e0.record(stream)
+    for _ in range(reps):
+        g.replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    us = e0.elapsed_time(e1) * 1e3 / (reps * len(fns))
+    del g
+    return us
+
+
+def staged_leg(nv, w, cache, sets, rows, flop, native_us, peak_bw, args):
+    """The staged FP8 path on the same rotating sets, each step timed alone
+    and both together, every figure from CUDA-graph replays like the native
+    launch: step 1 writes the E4M3 rows of the valid entries to HBM, step 2
+    runs attention over them."""
+    import torch
+    T, H, topk = w.T, w.H, sets[0][0].shape[1]
+    staging = torch.empty(nv.staging_size(T, topk), dtype=torch.uint8, device="cuda")
+    out = torch.empty(T, H, 512, dtype=torch.float16, device="cuda")
+    lse = torch.empty(T, H, dtype=torch.float32, device="cuda")
+    ws = torch.zeros(max(1, nv.workspace_size(T, H, topk)), dtype=torch.uint8, device="cuda")
+    n = max(80, min(4000, args.steps // 4))
+    stage = [lambda ix=ix: nv.staged_stage(cache, ix, staging) for ix, _, _ in sets]
+    attend = [lambda ix=ix, qn=qn, qr=qr: nv.staged_attend(qn, qr, cache.shape[0], ix, staging, w.sm_scale, out=out,
+                                                           lse=lse, workspace=ws) for ix, qn, qr in sets]
+    both = [lambda ix=ix, qn=qn, qr=qr: nv.staged_decode(qn, qr, cache, ix, w.sm_scale, out=out, lse=lse,
+                                                         staging=staging, workspace=ws) for ix, qn, qr in sets]
+    for f in both:
+        f()
+    us_stage, us_attend, us_both = graph_us(stage, n), graph_us(attend, n), graph_us(both, n)
+    stage_bytes = rows * (ROW_BYTES + nv.STAGED_ROW_BYTES) + T * topk * 4
+    del staging
+    return {"us_per_launch": us_both, "tflops": flop / (us_both * 1e-6) / 1e12, "native_speedup": us_both / native_us,
+            "stage_us": us_stage, "stage_gbs": stage_bytes / (us_stage * 1e-6) / 1e9,
+            "stage_frac_of_hbm": stage_bytes / (us_stage * 1e-6) / 1e9 / peak_bw, "stage_bytes": stage_bytes,
+            "attend_us": us_attend, "attend_tflops": flop / (us_attend * 1e-6) / 1e12, "launches": 2,
+            "staging_bytes": nv.staging_size(T, topk), "timing": "CUDA graph replays, %d calls each" % n}
+
+
+def e2e_leg(nv, w, cache, sets, flop, world, args):
+    """End to end through the host-buffer C-ABI call: each step copies its
+    queries and lists from pinned host memory, decodes, and copies out and
+    lse back; consecutive steps alternate two streams (each with its own
+    device buffers and workspace) so one step's copies overlap the other's
+    kernel.  Device time from the first copy to the last result."""
+    import torch
+    T, H, topk = w.T, w.H, sets[0][0].shape[1]
+    h_sets = [(ix.cpu().pin_memory(), qn.cpu().pin_memory(), qr.cpu().pin_memory()) for ix, qn, qr in sets]
+    streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+    bufs = []
+    for _ in streams:
+        bufs.append(dict(d_q_nope=torch.empty_like(sets[0][1]), d_q_rope=torch.empty_like(sets[0][2]),
+                         d_indices=torch.empty_like(sets[0][0]),
+                         d_out=torch.empty(T, H, 512, dtype=torch.float16, device="cuda"),
+                         d_lse=torch.empty(T, H, dtype=torch.float32, device="cuda"),
+                         h_out=torch.empty(T, H, 512, dtype=torch.float16).pin_memory(),
+                         h_lse=torch.empty(T, H, dtype=torch.float32).pin_memory(),
+                         workspace=torch.zeros(max(1, nv.workspace_size(T, H, topk)), dtype=torch.uint8,
+                                               device="cuda")))
+
+    def step(k):
+        b = bufs[k % 2]
+        ix, qn, qr = h_sets[k % len(h_sets)]
+        nv.decode_host(qn, qr, ix, b["h_out"], b["h_lse"], b["d_q_nope"], b["d_q_rope"], b["d_indices"], b["d_out"],
+                       b["d_lse"], cache, w.sm_scale, workspace=b["workspace"], stream=streams[k % 2])
+
+    for k in range(6):
+        step(k)
+    torch.cuda.synchronize()
+    ne = max(40, min(2000, args.steps // 10))
+    cur = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(cur)
+    for s in streams:
+        s.wait_stream(cur)
+    for k in range(ne):
+        step(k)
+    for s in streams:
+        cur.wait_stream(s)
+    e1.record(cur)
+    torch.cuda.synchronize()
+    eus = e0.elapsed_time(e1) * 1e3 / ne
+    h2d = sets[0][0].numel() * 4 + sets[0][1].numel() * 2 + sets[0][2].numel() * 2
+    d2h = T * H * 512 * 2 + T * H * 4
+    return {"value": flop / (eus * 1e-6) / 1e12 * world, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "us_per_step": eus, "copies_declared": True,
+            "api": "nvfp4_sparse_mla_decode_host (pinned host in/out, copies inside the call)",
+            "overlap": "two streams, double-buffered device buffers"}
+
+
+def configs_leg(nv, synth, args):
+    """Every other parity configuration, timed as single launches with L2
+    flushed before each (median of 20): us/launch, TFLOP/s, gathered GB/s and
+    the fraction of the roofline at the measured peaks."""
+    import torch
+    res = {}
+    for name, make in config_workloads(synth):
+        r = time_other_workload(name, make(), nv, synth, args)
+        res[name] = {k: r[k] for k in ("T", "H", "valid_rows_per_launch", "splits", "us_per_launch", "tflops",
+                                        "gathered_gbs", "roofline_us", "frac_of_roofline")}
+        torch.cuda.empty_cache()
+    return res
 
 
 def main():
@@ -680,7 +806,7 @@ def main():
         "alg_bytes_per_launch": alg_bytes, "alg_flop_per_launch": flop,
         "roofline": {"bound": "tensor", "achieved": flop / sec_per / 1e12, "peak": peak_tf, "unit": "TFLOP/s",
                      "frac": (flop / sec_per / 1e12) / peak_tf,
-                     "traffic": kernel_traffic(os.path.join(ROOT, "nvfp4_sparse_mla_decode_b200", "csrc", "decode.cu")),
+                     "traffic": kernel_traffic(os.path.join(ROOT, "nvfp4_sparse_mla_decode_b200", "csrc", "decode_nvfp4.cu")),
                      "peak_source": "%s bf16_tflops (burst) from MEASURED_PEAKS.json" % peak_kind
                                     if peak_kind == "measured" else "fallback 1590 TFLOP/s",
                      "roofline_us": t_roof * 1e6, "frac_of_roofline_time": t_roof / sec_per,
@@ -691,61 +817,8 @@ def main():
     }
 
     if not args.no_extras:
-        # ----------------------------------------------------- staged path
-        staging = torch.empty(nv.staging_size(T, topk), dtype=torch.uint8, device="cuda")
-        nst = max(20, min(2000, args.steps // 10))
-
-        def sstep(k):
-            ix, qn, qr = sets[k % N_SETS]
-            nv.staged_decode(qn, qr, cache, ix, w.sm_scale, out=out, lse=lse, staging=staging, workspace=ws,
-                             dev_status=status)
-
-        for k in range(5):
-            sstep(k)
-        torch.cuda.synchronize()
-        e0.record(stream)
-        for k in range(nst):
-            sstep(k)
-        e1.record(stream)
-        torch.cuda.synchronize()
-        sus = e0.elapsed_time(e1) * 1e3 / nst
-        line["staged_fp8"] = {"us_per_launch": sus, "tflops": flop / (sus * 1e-6) / 1e12,
-                              "native_speedup": sus / us, "launches": 2,
-                              "staging_bytes": staging.numel()}
-        del staging
-        # ------------------------------------------------------------ e2e
-        h_sets = []
-        for ix, qn, qr in sets:
-            h_sets.append((ix.cpu().pin_memory(), qn.cpu().pin_memory(), qr.cpu().pin_memory()))
-        d_ix = torch.empty_like(sets[0][0])
-        d_qn = torch.empty_like(sets[0][1])
-        d_qr = torch.empty_like(sets[0][2])
-        h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-        h_lse = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
-        ne = max(20, min(2000, args.steps // 10))
-
-        def estep(k):
-            ix, qn, qr = h_sets[k % N_SETS]
-            d_ix.copy_(ix, non_blocking=True)
-            d_qn.copy_(qn, non_blocking=True)
-            d_qr.copy_(qr, non_blocking=True)
-            nv.decode(d_qn, d_qr, cache, d_ix, w.sm_scale, out=out, lse=lse, workspace=ws, dev_status=status)
-            h_out.copy_(out, non_blocking=True)
-            h_lse.copy_(lse, non_blocking=True)
-
-        for k in range(5):
-            estep(k)
-        torch.cuda.synchronize()
-        e0.record(stream)
-        for k in range(ne):
-            estep(k)
-        e1.record(stream)
-        torch.cuda.synchronize()
-        eus = e0.elapsed_time(e1) * 1e3 / ne
-        h2d = d_ix.numel() * 4 + d_qn.numel() * 2 + d_qr.numel() * 2
-        d2h = out.numel() * 2 + lse.numel() * 4
-        line["e2e"] = {"value": flop / (eus * 1e-6) / 1e12 * world, "unit": "TFLOP/s",
-                       "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "us_per_step": eus}
+        line["staged_fp8"] = staged_leg(nv, w, cache, sets, rows, flop, us, peak_bw, args)
+        line["e2e"] = e2e_leg(nv, w, cache, sets, flop, world, args)
         # ----------------------------------------------------------- append
         wa = synth.append_prefill("cuda")
         acache = torch.zeros(wa.num_slots, nv.ROW_BYTES, dtype=torch.uint8, device="cuda")
@@ -776,6 +849,9 @@ def main():
             except Exception as e:  # noqa: BLE001
                 line["cpu_baseline"] = {"value": None, "unit": "TFLOP/s", "cores": None, "kind": "oracle",
                                         "sample": "oracle unavailable: %s" % e}
+    if not args.no_extras and rank == 0:
+        line["configs"] = configs_leg(nv, synth, args)
+        line["configs_timing"] = "single launch per config, L2 flushed before it, median of 20"
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -165,6 +165,32 @@ nvfp4mla_status nvfp4_sparse_mla_decode(const void *q_nope_f16, const void *q_ro
                                         size_t workspace_bytes, int32_t *dev_status, void *stream);
 
 /*
+ * nvfp4_sparse_mla_decode_host -- nvfp4_sparse_mla_decode for inputs and
+ * outputs in host memory: on `stream` it copies q_nope, q_rope and indices
+ * from the host into the caller's device buffers (one cudaMemcpyAsync each),
+ * runs the decode, and copies out and lse back to the host.  The pages'
+ * serving loop moves each decode step's queries and lists to the GPU and its
+ * results back; this call keeps those copies on the same stream as the
+ * kernel, so a caller that alternates two streams (each with its own device
+ * buffers and workspace) overlaps one step's copies with the other's kernel.
+ *   *_host     host buffers with the shapes of nvfp4_sparse_mla_decode's
+ *              arguments; page-locked memory (cudaHostAlloc) is needed for
+ *              the copies to run asynchronously
+ *   *_dev      device buffers of the same shapes, owned by the caller,
+ *              16-byte aligned (lse_dev 4-byte)
+ * The host output buffers are written when `stream` reaches the end of the
+ * call; synchronize before reading them.  Other arguments, the workspace
+ * contract and errors are those of nvfp4_sparse_mla_decode; a failed copy
+ * returns NVFP4MLA_ERR_CUDA.
+ */
+nvfp4mla_status nvfp4_sparse_mla_decode_host(const void *q_nope_host, const void *q_rope_host,
+                                             const int32_t *indices_host, void *out_host, float *lse_host,
+                                             void *q_nope_dev, void *q_rope_dev, int32_t *indices_dev, void *out_dev,
+                                             float *lse_dev, const uint8_t *cache, int64_t num_slots, int32_t topk,
+                                             int32_t T, int32_t H, float sm_scale, void *workspace,
+                                             size_t workspace_bytes, int32_t *dev_status, void *stream);
+
+/*
  * nvfp4_sparse_mla_decode_paged -- nvfp4_sparse_mla_decode for lists of
  * request-local token positions instead of slot ids: the position -> slot
  * translation through each request's page table (the paged cache the pages'
@@ -243,6 +269,28 @@ nvfp4mla_status nvfp4_staged_fp8_mla_decode(const void *q_nope_f16, const void *
                                             int32_t H, float sm_scale, void *out_f16, float *lse,
                                             uint8_t *staging, size_t staging_bytes, void *workspace,
                                             size_t workspace_bytes, int32_t *dev_status, void *stream);
+
+/*
+ * nvfp4_staged_fp8_stage, nvfp4_staged_fp8_attend -- the two steps of
+ * nvfp4_staged_fp8_mla_decode as separate calls (same page and section), so
+ * each step can be launched, captured and timed on its own.  Calling
+ * nvfp4_staged_fp8_stage and then nvfp4_staged_fp8_attend on the same
+ * stream with the same arguments gives the result of
+ * nvfp4_staged_fp8_mla_decode.
+ *   stage:  cache, num_slots, indices, topk, T, staging, staging_bytes,
+ *           stream as nvfp4_staged_fp8_mla_decode; writes the E4M3 rows of
+ *           the valid entries into staging[t, j, 0:576]
+ *   attend: every argument of nvfp4_staged_fp8_mla_decode except cache;
+ *           reads staging[t, j] for the entries with 0 <= indices[t, j] <
+ *           num_slots (the rows the stage step wrote)
+ * Errors as nvfp4_staged_fp8_mla_decode.
+ */
+nvfp4mla_status nvfp4_staged_fp8_stage(const uint8_t *cache, int64_t num_slots, const int32_t *indices, int32_t topk,
+                                       int32_t T, uint8_t *staging, size_t staging_bytes, void *stream);
+nvfp4mla_status nvfp4_staged_fp8_attend(const void *q_nope_f16, const void *q_rope_f16, int64_t num_slots,
+                                        const int32_t *indices, int32_t topk, int32_t T, int32_t H, float sm_scale,
+                                        void *out_f16, float *lse, const uint8_t *staging, size_t staging_bytes,
+                                        void *workspace, size_t workspace_bytes, int32_t *dev_status, void *stream);
 
 /*
  * nvfp4mla_fp8_sparse_mla_decode -- the same attention as

@@ -19,7 +19,8 @@ import torch
 
 __all__ = [
     "ROW_BYTES", "STAGED_ROW_BYTES", "LATENT", "ROPE", "MAX_TOPK", "NVFP4MLAError",
-    "lib", "lib_path", "kv_append", "decode", "decode_paged", "decode_noalloc", "staged_decode",
+    "lib", "lib_path", "kv_append", "decode", "decode_host", "decode_paged", "decode_noalloc", "staged_decode", "staged_stage",
+    "staged_attend",
     "fp8_kv_append", "fp8_decode", "indexer_scores", "indexer_topk", "sparse_indexer", "blhnc_convert",
     "copy_descriptors", "num_splits",
     "workspace_size", "staging_size", "status_string", "version",
@@ -75,6 +76,14 @@ def lib() -> ctypes.CDLL:
         L.nvfp4_staged_fp8_mla_decode.restype = _i32
         L.nvfp4_staged_fp8_mla_decode.argtypes = [_vp, _vp, _vp, _i64, _vp, _i32, _i32, _i32, _f32, _vp, _vp,
                                                   _vp, _sz, _vp, _sz, _vp, _vp]
+        L.nvfp4_sparse_mla_decode_host.restype = _i32
+        L.nvfp4_sparse_mla_decode_host.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i32,
+                                                   _i32, _i32, _f32, _vp, _sz, _vp, _vp]
+        L.nvfp4_staged_fp8_stage.restype = _i32
+        L.nvfp4_staged_fp8_stage.argtypes = [_vp, _i64, _vp, _i32, _i32, _vp, _sz, _vp]
+        L.nvfp4_staged_fp8_attend.restype = _i32
+        L.nvfp4_staged_fp8_attend.argtypes = [_vp, _vp, _i64, _vp, _i32, _i32, _i32, _f32, _vp, _vp, _vp, _sz, _vp,
+                                              _sz, _vp, _vp]
         L.nvfp4mla_fp8_kv_append.restype = _i32
         L.nvfp4mla_fp8_kv_append.argtypes = [_vp, _i64, _vp, _i64, _vp, _i32, _vp, _i64, _vp, _vp]
         L.nvfp4mla_fp8_sparse_mla_decode.restype = _i32
@@ -215,6 +224,31 @@ def decode(q_nope: torch.Tensor, q_rope: torch.Tensor, cache: torch.Tensor, indi
     return out, lse
 
 
+def decode_host(h_q_nope: torch.Tensor, h_q_rope: torch.Tensor, h_indices: torch.Tensor, h_out: torch.Tensor,
+                h_lse: torch.Tensor, d_q_nope: torch.Tensor, d_q_rope: torch.Tensor, d_indices: torch.Tensor,
+                d_out: torch.Tensor, d_lse: torch.Tensor, cache: torch.Tensor, sm_scale: float,
+                workspace: Optional[torch.Tensor] = None, dev_status: Optional[torch.Tensor] = None,
+                stream: Optional[torch.cuda.Stream] = None) -> None:
+    """decode() with inputs and outputs in (pinned) host tensors; the library
+    copies them to and from the given device tensors on `stream` around the
+    kernel.  Host outputs are valid once the stream has been synchronized."""
+    for h in (h_q_nope, h_q_rope, h_indices, h_out, h_lse):
+        assert h.device.type == "cpu" and h.is_contiguous()
+    dev, T, H, topk, d_out, d_lse = _decode_args(d_q_nope, d_q_rope, cache, d_indices, d_out, d_lse)
+    assert h_q_nope.shape == d_q_nope.shape and h_q_rope.shape == d_q_rope.shape
+    assert h_indices.shape == d_indices.shape and h_out.shape == d_out.shape and h_lse.shape == d_lse.shape
+    ws_need = workspace_size(T, H, topk)
+    if workspace is None and ws_need:
+        workspace = torch.zeros(ws_need, dtype=torch.uint8, device=dev)
+    s = stream.cuda_stream if stream is not None else _stream(dev)
+    st = lib().nvfp4_sparse_mla_decode_host(
+        h_q_nope.data_ptr(), h_q_rope.data_ptr(), h_indices.data_ptr(), h_out.data_ptr(), h_lse.data_ptr(),
+        _ptr(d_q_nope), _ptr(d_q_rope), _ptr(d_indices), _ptr(d_out), _ptr(d_lse), _ptr(cache), cache.shape[0],
+        topk, T, H, float(sm_scale), _ptr(workspace),
+        workspace.numel() * workspace.element_size() if workspace is not None else 0, _ptr(dev_status), s)
+    _check(st, "nvfp4_sparse_mla_decode_host")
+
+
 def decode_paged(q_nope: torch.Tensor, q_rope: torch.Tensor, cache: torch.Tensor, positions: torch.Tensor,
                  block_table: torch.Tensor, page_size: int, sm_scale: float, out: Optional[torch.Tensor] = None,
                  lse: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
@@ -269,6 +303,32 @@ def staged_decode(q_nope: torch.Tensor, q_rope: torch.Tensor, cache: torch.Tenso
                                            workspace.numel() if workspace is not None else 0,
                                            _ptr(dev_status), _stream(dev))
     _check(st, "nvfp4_staged_fp8_mla_decode")
+    return out, lse
+
+
+def staged_stage(cache: torch.Tensor, indices: torch.Tensor, staging: torch.Tensor) -> None:
+    """Step 1 of the staged path: E4M3 rows of the valid entries into staging."""
+    assert indices.dtype == torch.int32 and indices.dim() == 2 and indices.is_contiguous()
+    T, topk = indices.shape
+    st = lib().nvfp4_staged_fp8_stage(_ptr(cache), cache.shape[0], _ptr(indices), topk, T, _ptr(staging),
+                                      staging.numel(), _stream(cache.device))
+    _check(st, "nvfp4_staged_fp8_stage")
+
+
+def staged_attend(q_nope: torch.Tensor, q_rope: torch.Tensor, num_slots: int, indices: torch.Tensor,
+                  staging: torch.Tensor, sm_scale: float, out: Optional[torch.Tensor] = None,
+                  lse: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                  dev_status: Optional[torch.Tensor] = None):
+    """Step 2 of the staged path: attention over the staged E4M3 rows."""
+    dev, T, H, topk, out, lse = _decode_args(q_nope, q_rope, staging, indices, out, lse)
+    ws_need = workspace_size(T, H, topk)
+    if workspace is None and ws_need:
+        workspace = torch.zeros(ws_need, dtype=torch.uint8, device=dev)
+    st = lib().nvfp4_staged_fp8_attend(_ptr(q_nope), _ptr(q_rope), num_slots, _ptr(indices), topk, T, H,
+                                       float(sm_scale), _ptr(out), _ptr(lse), _ptr(staging), staging.numel(),
+                                       _ptr(workspace), workspace.numel() if workspace is not None else 0,
+                                       _ptr(dev_status), _stream(dev))
+    _check(st, "nvfp4_staged_fp8_attend")
     return out, lse
 
 

@@ -120,6 +120,34 @@ nvfp4mla_status nvfp4_sparse_mla_decode(const void *q_nope_f16, const void *q_ro
                                               static_cast<cudaStream_t>(stream)));
 }
 
+nvfp4mla_status nvfp4_sparse_mla_decode_host(const void *q_nope_host, const void *q_rope_host,
+                                             const int32_t *indices_host, void *out_host, float *lse_host,
+                                             void *q_nope_dev, void *q_rope_dev, int32_t *indices_dev, void *out_dev,
+                                             float *lse_dev, const uint8_t *cache, int64_t num_slots, int32_t topk,
+                                             int32_t T, int32_t H, float sm_scale, void *workspace,
+                                             size_t workspace_bytes, int32_t *dev_status, void *stream) {
+    DecodePlan plan;
+    nvfp4mla_status st = check_decode(q_nope_dev, q_rope_dev, cache, num_slots, indices_dev, topk, T, H, sm_scale,
+                                      out_dev, lse_dev, &plan);
+    if (st != NVFP4MLA_OK || T == 0) return st;
+    if (!q_nope_host || !q_rope_host || !indices_host || !out_host || !lse_host) return NVFP4MLA_ERR_INVALID_ARG;
+    if (plan.workspace_bytes > 0 && (!workspace || workspace_bytes < plan.workspace_bytes)) return NVFP4MLA_ERR_WORKSPACE;
+    if (workspace && !aligned(workspace, 256)) return NVFP4MLA_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const size_t th = (size_t)T * (size_t)H;
+    if (cudaMemcpyAsync(q_nope_dev, q_nope_host, th * NVFP4MLA_LATENT * 2, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+        cudaMemcpyAsync(q_rope_dev, q_rope_host, th * NVFP4MLA_ROPE * 2, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+        cudaMemcpyAsync(indices_dev, indices_host, (size_t)T * topk * 4, cudaMemcpyHostToDevice, s) != cudaSuccess)
+        return NVFP4MLA_ERR_CUDA;
+    if (launch_sparse_mla_decode(RowSource::kNvfp4Cache, q_nope_dev, q_rope_dev, cache, num_slots, indices_dev, topk,
+                                 T, H, sm_scale, out_dev, lse_dev, workspace, plan, dev_status, s) != cudaSuccess)
+        return NVFP4MLA_ERR_CUDA;
+    if (cudaMemcpyAsync(out_host, out_dev, th * NVFP4MLA_LATENT * 2, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+        cudaMemcpyAsync(lse_host, lse_dev, th * 4, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+        return NVFP4MLA_ERR_CUDA;
+    return NVFP4MLA_OK;
+}
+
 nvfp4mla_status nvfp4_sparse_mla_decode_paged(const void *q_nope_f16, const void *q_rope_f16, const uint8_t *cache,
                                               int64_t num_slots, const int32_t *positions, int32_t topk,
                                               const int32_t *block_table, int32_t table_stride, int32_t page_size,
@@ -188,6 +216,33 @@ nvfp4mla_status nvfp4_staged_fp8_mla_decode(const void *q_nope_f16, const void *
     if (e != cudaSuccess) return NVFP4MLA_ERR_CUDA;
     return from_cuda(launch_sparse_mla_decode(RowSource::kFp8Staging, q_nope_f16, q_rope_f16, staging, num_slots, indices, topk, T, H,
                                               sm_scale, out_f16, lse, workspace, plan, dev_status, s));
+}
+
+nvfp4mla_status nvfp4_staged_fp8_stage(const uint8_t *cache, int64_t num_slots, const int32_t *indices, int32_t topk,
+                                       int32_t T, uint8_t *staging, size_t staging_bytes, void *stream) {
+    if (T < 0 || topk < 1 || topk > NVFP4MLA_MAX_TOPK || num_slots < 1 || num_slots > INT32_MAX)
+        return NVFP4MLA_ERR_INVALID_ARG;
+    if (T == 0) return NVFP4MLA_OK;
+    if (!cache || !indices || !staging) return NVFP4MLA_ERR_INVALID_ARG;
+    if (!aligned(cache, 16) || !aligned(indices, 4) || !aligned(staging, 16)) return NVFP4MLA_ERR_INVALID_ARG;
+    if (staging_bytes < nvfp4_staged_fp8_staging_size(T, topk)) return NVFP4MLA_ERR_WORKSPACE;
+    return from_cuda(launch_stage_fp8(cache, num_slots, indices, topk, T, staging, static_cast<cudaStream_t>(stream)));
+}
+
+nvfp4mla_status nvfp4_staged_fp8_attend(const void *q_nope_f16, const void *q_rope_f16, int64_t num_slots,
+                                        const int32_t *indices, int32_t topk, int32_t T, int32_t H, float sm_scale,
+                                        void *out_f16, float *lse, const uint8_t *staging, size_t staging_bytes,
+                                        void *workspace, size_t workspace_bytes, int32_t *dev_status, void *stream) {
+    DecodePlan plan;
+    nvfp4mla_status st = check_decode(q_nope_f16, q_rope_f16, staging, num_slots, indices, topk, T, H, sm_scale,
+                                      out_f16, lse, &plan);
+    if (st != NVFP4MLA_OK || T == 0) return st;
+    if (staging_bytes < nvfp4_staged_fp8_staging_size(T, topk)) return NVFP4MLA_ERR_WORKSPACE;
+    if (plan.workspace_bytes > 0 && (!workspace || workspace_bytes < plan.workspace_bytes)) return NVFP4MLA_ERR_WORKSPACE;
+    if (workspace && !aligned(workspace, 256)) return NVFP4MLA_ERR_INVALID_ARG;
+    return from_cuda(launch_sparse_mla_decode(RowSource::kFp8Staging, q_nope_f16, q_rope_f16, staging, num_slots,
+                                              indices, topk, T, H, sm_scale, out_f16, lse, workspace, plan,
+                                              dev_status, static_cast<cudaStream_t>(stream)));
 }
 
 nvfp4mla_status nvfp4mla_fp8_sparse_mla_decode(const void *q_nope_f16, const void *q_rope_f16,

@@ -13,7 +13,7 @@ import torch
 import oracle
 import nvfp4_sparse_mla_decode_b200 as nv
 from nvfp4_sparse_mla_decode_b200 import synth
-from harness import build_cache, check_close, oracle_decode
+from harness import build_cache, check_close, oracle_decode, oracle_inputs
 
 pytestmark = pytest.mark.gpu
 
@@ -54,6 +54,43 @@ def test_decode35x64_full():
 def test_staged_path_matches_staged_oracle():
     w = synth.decode35("cuda", T=6, ctx=20000)
     run(w, build_cache(w), staged=True)
+
+
+def test_staged_rows_bit_exact_against_oracle():
+    # the stage kernel's 576-byte E4M3 rows, entry by entry, equal the
+    # oracle's re-encoding of its own dequantized rows; empty entries are
+    # left untouched
+    w = synth.decode35("cuda", T=5, ctx=20000)
+    w.indices[1, 1500:] = -1
+    w.indices[3, ::3] = -1
+    cache = build_cache(w)
+    topk = w.indices.shape[1]
+    staging = torch.full((nv.staging_size(w.T, topk),), 0xA5, dtype=torch.uint8, device="cuda")
+    nv.staged_decode(w.q_nope, w.q_rope, cache, w.indices, w.sm_scale, staging=staging)
+    torch.cuda.synchronize()
+    _, _, rows, remap, _ = oracle_inputs(w, range(w.T))
+    ref = oracle.stage_rows(rows)
+    got = staging.view(w.T * topk, nv.STAGED_ROW_BYTES).cpu().numpy()
+    flat = remap.reshape(-1)
+    valid = flat >= 0
+    assert np.array_equal(got[valid], ref[flat[valid]])
+    assert np.all(got[~valid] == 0xA5)
+
+
+def test_staged_two_steps_equal_one_call():
+    # stage + attend as separate calls reproduce the one-call staged path bit for bit
+    w = synth.decode35("cuda", T=6, ctx=20000)
+    w.indices[2, 700:] = -1
+    cache = build_cache(w)
+    topk = w.indices.shape[1]
+    staging = torch.empty(nv.staging_size(w.T, topk), dtype=torch.uint8, device="cuda")
+    out1, lse1 = nv.staged_decode(w.q_nope, w.q_rope, cache, w.indices, w.sm_scale, staging=staging)
+    out1, lse1 = out1.clone(), lse1.clone()
+    staging2 = torch.empty_like(staging)
+    nv.staged_stage(cache, w.indices, staging2)
+    out2, lse2 = nv.staged_attend(w.q_nope, w.q_rope, cache.shape[0], w.indices, staging2, w.sm_scale)
+    torch.cuda.synchronize()
+    assert torch.equal(out1, out2) and torch.equal(lse1, lse2)
 
 
 def test_staged_tiny():
@@ -153,3 +190,29 @@ def test_split_workspace_reused_across_shapes_and_calls():
         ref_o, ref_l = oracle_decode(w, tokens)
         check_close(out[tokens], lse[tokens], ref_o, ref_l)
         del cache
+
+
+def test_host_buffer_call_matches_device_call():
+    # the call that copies host inputs in and results out on its stream gives
+    # the device call's results bit for bit, on two streams with their own
+    # device buffers and workspaces
+    w = synth.decode35("cuda", T=6, ctx=20000)
+    cache = build_cache(w)
+    ref_out, ref_lse = nv.decode(w.q_nope, w.q_rope, cache, w.indices, w.sm_scale)
+    torch.cuda.synchronize()
+    h_qn, h_qr, h_ix = w.q_nope.cpu().pin_memory(), w.q_rope.cpu().pin_memory(), w.indices.cpu().pin_memory()
+    streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+    outs = []
+    for s in streams:
+        d = dict(d_q_nope=torch.empty_like(w.q_nope), d_q_rope=torch.empty_like(w.q_rope),
+                 d_indices=torch.empty_like(w.indices), d_out=torch.empty(w.T, w.H, 512, dtype=torch.float16,
+                                                                          device="cuda"),
+                 d_lse=torch.empty(w.T, w.H, dtype=torch.float32, device="cuda"))
+        h_out = torch.empty(w.T, w.H, 512, dtype=torch.float16).pin_memory()
+        h_lse = torch.empty(w.T, w.H, dtype=torch.float32).pin_memory()
+        ws = torch.zeros(max(1, nv.workspace_size(w.T, w.H)), dtype=torch.uint8, device="cuda")
+        nv.decode_host(h_qn, h_qr, h_ix, h_out, h_lse, cache=cache, sm_scale=w.sm_scale, workspace=ws, stream=s, **d)
+        outs.append((h_out, h_lse))
+    torch.cuda.synchronize()
+    for h_out, h_lse in outs:
+        assert torch.equal(h_out, ref_out.cpu()) and torch.equal(h_lse, ref_lse.cpu())
