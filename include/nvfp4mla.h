@@ -430,6 +430,13 @@ int64_t nvfp4mla_copy_descriptors(const int32_t *ids, int32_t n, int32_t layers)
  */
 nvfp4mla_status nvfp4mla_selftest_wait_timeout(uint32_t *zero_word, int32_t *dev_status, void *stream);
 
+/* The CUDA runtime error (a cudaError_t value) behind the last
+ * NVFP4MLA_ERR_CUDA that a call of this library returned on the calling host
+ * thread, or 0 if none has; and its description (static storage).  Neither
+ * is reset by later successful calls. */
+int32_t nvfp4mla_last_cuda_error(void);
+const char *nvfp4mla_last_cuda_error_string(void);
+
 /* Human-readable name of a status code (static storage). */
 const char *nvfp4mla_status_string(nvfp4mla_status status);
 

@@ -44,9 +44,11 @@ _vp, _i32, _i64, _f32, _sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ct
 
 
 class NVFP4MLAError(RuntimeError):
-    def __init__(self, status: int, what: str):
-        super().__init__("%s: %s (status %d)" % (what, status_string(status), status))
+    def __init__(self, status: int, what: str, detail: str | None = None):
+        msg = "%s: %s (status %d)" % (what, status_string(status), status)
+        super().__init__(msg + (": " + detail if detail else ""))
         self.status = status
+        self.detail = detail
 
 
 def lib() -> ctypes.CDLL:
@@ -112,6 +114,10 @@ def lib() -> ctypes.CDLL:
         L.nvfp4mla_selftest_wait_timeout.argtypes = [_vp, _vp, _vp]
         L.nvfp4mla_status_string.restype = ctypes.c_char_p
         L.nvfp4mla_status_string.argtypes = [_i32]
+        L.nvfp4mla_last_cuda_error.restype = _i32
+        L.nvfp4mla_last_cuda_error.argtypes = []
+        L.nvfp4mla_last_cuda_error_string.restype = ctypes.c_char_p
+        L.nvfp4mla_last_cuda_error_string.argtypes = []
         L.nvfp4mla_version.restype = _i32
         L.nvfp4mla_version.argtypes = []
         _lib = L
@@ -144,7 +150,10 @@ def _need_cuda(*ts: torch.Tensor) -> torch.device:
 
 def _check(status: int, what: str) -> None:
     if status != 0:
-        raise NVFP4MLAError(status, what)
+        detail = None
+        if status == 4:  # NVFP4MLA_ERR_CUDA: name the CUDA error behind it
+            detail = lib().nvfp4mla_last_cuda_error_string().decode()
+        raise NVFP4MLAError(status, what, detail)
 
 
 def num_splits(T: int, H: int, topk: int = MAX_TOPK) -> int:

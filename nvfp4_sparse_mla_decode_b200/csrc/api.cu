@@ -6,6 +6,7 @@
 #include <cstdint>
 
 #include "../../include/nvfp4mla.h"
+#include "decode_common.cuh"
 #include "kernels.h"
 
 using namespace nvfp4mla;
@@ -45,7 +46,14 @@ void *noalloc_workspace(int dev) {
     return cached;
 }
 
-nvfp4mla_status from_cuda(cudaError_t e) { return e == cudaSuccess ? NVFP4MLA_OK : NVFP4MLA_ERR_CUDA; }
+// The CUDA error behind the last NVFP4MLA_ERR_CUDA this host thread got.
+thread_local cudaError_t g_last_cuda_error = cudaSuccess;
+
+nvfp4mla_status from_cuda(cudaError_t e) {
+    if (e == cudaSuccess) return NVFP4MLA_OK;
+    g_last_cuda_error = e;
+    return NVFP4MLA_ERR_CUDA;
+}
 
 // Checks shared by the native and staged decode entry points.
 nvfp4mla_status check_decode(const void *q_nope, const void *q_rope, const uint8_t *cache, int64_t num_slots,
@@ -120,6 +128,29 @@ nvfp4mla_status nvfp4_sparse_mla_decode(const void *q_nope_f16, const void *q_ro
                                               static_cast<cudaStream_t>(stream)));
 }
 
+// Test-only (not in the public header): the NVFP4 decode with a chosen wait
+// bound (SM clock cycles, > 0) and one arrival withheld (1: P^T is never
+// published; 2: split 0 never arrives on the merge counter), so that tests
+// can drive the kernel's timeout paths and check that it reports
+// NVFP4MLA_DEV_TIMEOUT through dev_status and leaves the context usable.
+nvfp4mla_status nvfp4mla_test_decode_hooks(const void *q_nope_f16, const void *q_rope_f16, const uint8_t *cache,
+                                           int64_t num_slots, const int32_t *indices, int32_t topk, int32_t T,
+                                           int32_t H, float sm_scale, void *out_f16, float *lse, void *workspace,
+                                           size_t workspace_bytes, int32_t *dev_status, uint64_t wait_cycles,
+                                           int32_t withhold, void *stream) {
+    DecodePlan plan;
+    nvfp4mla_status st =
+        check_decode(q_nope_f16, q_rope_f16, cache, num_slots, indices, topk, T, H, sm_scale, out_f16, lse, &plan);
+    if (st != NVFP4MLA_OK || T == 0) return st;
+    if (wait_cycles == 0 || withhold < 0 || withhold > 2) return NVFP4MLA_ERR_INVALID_ARG;
+    if (plan.workspace_bytes > 0 && (!workspace || workspace_bytes < plan.workspace_bytes)) return NVFP4MLA_ERR_WORKSPACE;
+    if (workspace && !aligned(workspace, 256)) return NVFP4MLA_ERR_INVALID_ARG;
+    DecodeTestHooks hooks{wait_cycles, withhold};
+    return from_cuda(launch_sparse_mla_decode(RowSource::kNvfp4Cache, q_nope_f16, q_rope_f16, cache, num_slots, indices,
+                                              topk, T, H, sm_scale, out_f16, lse, workspace, plan, dev_status,
+                                              static_cast<cudaStream_t>(stream), nullptr, 0, 0, &hooks));
+}
+
 nvfp4mla_status nvfp4_sparse_mla_decode_host(const void *q_nope_host, const void *q_rope_host,
                                              const int32_t *indices_host, void *out_host, float *lse_host,
                                              void *q_nope_dev, void *q_rope_dev, int32_t *indices_dev, void *out_dev,
@@ -135,17 +166,15 @@ nvfp4mla_status nvfp4_sparse_mla_decode_host(const void *q_nope_host, const void
     if (workspace && !aligned(workspace, 256)) return NVFP4MLA_ERR_INVALID_ARG;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const size_t th = (size_t)T * (size_t)H;
-    if (cudaMemcpyAsync(q_nope_dev, q_nope_host, th * NVFP4MLA_LATENT * 2, cudaMemcpyHostToDevice, s) != cudaSuccess ||
-        cudaMemcpyAsync(q_rope_dev, q_rope_host, th * NVFP4MLA_ROPE * 2, cudaMemcpyHostToDevice, s) != cudaSuccess ||
-        cudaMemcpyAsync(indices_dev, indices_host, (size_t)T * topk * 4, cudaMemcpyHostToDevice, s) != cudaSuccess)
-        return NVFP4MLA_ERR_CUDA;
-    if (launch_sparse_mla_decode(RowSource::kNvfp4Cache, q_nope_dev, q_rope_dev, cache, num_slots, indices_dev, topk,
-                                 T, H, sm_scale, out_dev, lse_dev, workspace, plan, dev_status, s) != cudaSuccess)
-        return NVFP4MLA_ERR_CUDA;
-    if (cudaMemcpyAsync(out_host, out_dev, th * NVFP4MLA_LATENT * 2, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
-        cudaMemcpyAsync(lse_host, lse_dev, th * 4, cudaMemcpyDeviceToHost, s) != cudaSuccess)
-        return NVFP4MLA_ERR_CUDA;
-    return NVFP4MLA_OK;
+    cudaError_t e = cudaMemcpyAsync(q_nope_dev, q_nope_host, th * NVFP4MLA_LATENT * 2, cudaMemcpyHostToDevice, s);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(q_rope_dev, q_rope_host, th * NVFP4MLA_ROPE * 2, cudaMemcpyHostToDevice, s);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(indices_dev, indices_host, (size_t)T * topk * 4, cudaMemcpyHostToDevice, s);
+    if (e == cudaSuccess)
+        e = launch_sparse_mla_decode(RowSource::kNvfp4Cache, q_nope_dev, q_rope_dev, cache, num_slots, indices_dev, topk,
+                                     T, H, sm_scale, out_dev, lse_dev, workspace, plan, dev_status, s);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(out_host, out_dev, th * NVFP4MLA_LATENT * 2, cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(lse_host, lse_dev, th * 4, cudaMemcpyDeviceToHost, s);
+    return from_cuda(e);
 }
 
 nvfp4mla_status nvfp4_sparse_mla_decode_paged(const void *q_nope_f16, const void *q_rope_f16, const uint8_t *cache,
@@ -184,9 +213,10 @@ nvfp4mla_status nvfp4_sparse_mla_decode_noalloc(const void *q_nope_f16, const vo
     void *ws = nullptr;
     if (plan.workspace_bytes > 0) {
         int dev = 0;
-        if (cudaGetDevice(&dev) != cudaSuccess) return NVFP4MLA_ERR_CUDA;
+        const cudaError_t e = cudaGetDevice(&dev);
+        if (e != cudaSuccess) return from_cuda(e);
         ws = noalloc_workspace(dev);
-        if (!ws) return NVFP4MLA_ERR_CUDA;
+        if (!ws) return from_cuda(cudaErrorMemoryAllocation);
     }
     return from_cuda(launch_sparse_mla_decode(RowSource::kNvfp4Cache, q_nope_f16, q_rope_f16, cache, num_slots, indices, topk, T, H,
                                               sm_scale, out_f16, lse, ws, plan, dev_status,
@@ -213,7 +243,7 @@ nvfp4mla_status nvfp4_staged_fp8_mla_decode(const void *q_nope_f16, const void *
     if (workspace && !aligned(workspace, 256)) return NVFP4MLA_ERR_INVALID_ARG;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     cudaError_t e = launch_stage_fp8(cache, num_slots, indices, topk, T, staging, s);
-    if (e != cudaSuccess) return NVFP4MLA_ERR_CUDA;
+    if (e != cudaSuccess) return from_cuda(e);
     return from_cuda(launch_sparse_mla_decode(RowSource::kFp8Staging, q_nope_f16, q_rope_f16, staging, num_slots, indices, topk, T, H,
                                               sm_scale, out_f16, lse, workspace, plan, dev_status, s));
 }
@@ -368,6 +398,10 @@ nvfp4mla_status nvfp4mla_selftest_wait_timeout(uint32_t *zero_word, int32_t *dev
         return NVFP4MLA_ERR_INVALID_ARG;
     return from_cuda(launch_wait_timeout_selftest(zero_word, dev_status, static_cast<cudaStream_t>(stream)));
 }
+
+int32_t nvfp4mla_last_cuda_error(void) { return (int32_t)g_last_cuda_error; }
+
+const char *nvfp4mla_last_cuda_error_string(void) { return cudaGetErrorString(g_last_cuda_error); }
 
 const char *nvfp4mla_status_string(nvfp4mla_status status) {
     switch (status) {

@@ -48,6 +48,8 @@
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
+
 #include <cmath>
 
 #include "common.cuh"
@@ -139,6 +141,7 @@ static_assert(kOffOwn + kMaxHG * (kLatent / 2) * 4 <= kTileBytes, "own slice mus
 template <int HG, int S>
 __device__ __forceinline__ void merge_splits(const DecodeArgs &a, int t, int g, int split, uint8_t *smem, int mt,
                                              [[maybe_unused]] unsigned long long t_start) {
+    TRACE_SETUP();
     using namespace dec;
     constexpr int kMergeThreads = 256;
     constexpr int D = kLatent / S;           // dv per CTA
@@ -276,6 +279,7 @@ __global__ void __launch_bounds__(dec::kThreads, 1)
 #else
     const unsigned long long t_start = 0;  // timestamps exist only in trace builds
 #endif
+    TRACE_SETUP();
     const int split = blockIdx.x % a.S;
     const int rest = blockIdx.x / a.S;
     const int g = rest % a.G;
@@ -962,13 +966,15 @@ bool make_q_map(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols, 
     return true;
 }
 
-// Tensor map for the FP32 split partials: a 2-D view [rows, 512] of
-// ws_o, box box_cols x box_rows, no swizzle; cached like the Q maps.
-bool make_partial_map(CUtensorMap *m, const void *base, uint64_t rows, uint32_t box_cols, uint32_t box_rows) {
+// Tensor map for the NVFP4 kernel's split exchange area: a 2-D FP32 view
+// [rows, 2048] of ws_o (row = one 4-head piece of one split's partial, 512 dv
+// x 4 heads), box box_x floats x box_rows rows, no swizzle; cached per host
+// thread like the Q maps.
+bool make_xch_map(CUtensorMap *m, const void *base, uint64_t rows, uint32_t box_x, uint32_t box_rows) {
     struct Entry {
         const void *base;
         uint64_t rows;
-        uint32_t box_cols, box_rows;
+        uint32_t box_x, box_rows;
         CUtensorMap map;
     };
     constexpr int kEntries = 8;
@@ -976,22 +982,22 @@ bool make_partial_map(CUtensorMap *m, const void *base, uint64_t rows, uint32_t 
     thread_local int next = 0;
     for (int i = 0; i < kEntries; ++i) {
         const Entry &e = cache[i];
-        if (e.base == base && e.rows == rows && e.box_cols == box_cols && e.box_rows == box_rows) {
+        if (e.base == base && e.rows == rows && e.box_x == box_x && e.box_rows == box_rows) {
             *m = e.map;
             return true;
         }
     }
     auto enc = tensor_map_encoder();
     if (!enc) return false;
-    const cuuint64_t dims[2] = {(cuuint64_t)kLatent, rows};
-    const cuuint64_t strides[1] = {(cuuint64_t)kLatent * 4};
-    const cuuint32_t box[2] = {box_cols, box_rows};
+    const cuuint64_t dims[2] = {(cuuint64_t)kLatent * 4, rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)kLatent * 16};
+    const cuuint32_t box[2] = {box_x, box_rows};
     const cuuint32_t estr[2] = {1, 1};
     if (enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void *>(base), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
         return false;
-    cache[next] = Entry{base, rows, box_cols, box_rows, *m};
+    cache[next] = Entry{base, rows, box_x, box_rows, *m};
     next = (next + 1) % kEntries;
     return true;
 }
@@ -999,11 +1005,11 @@ bool make_partial_map(CUtensorMap *m, const void *base, uint64_t rows, uint32_t 
 template <int HG, bool kStaged>
 static cudaError_t launch_hg(const DecodeArgs &a, int64_t nblocks, cudaStream_t stream) {
     auto kern = sparse_mla_decode_kernel<HG, kStaged>;
-    static bool attr_set[64] = {};
+    static std::atomic<bool> attr_set[64] = {};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= 64 || !attr_set[dev]) {
+    if (dev < 0 || dev >= 64 || !attr_set[dev].load(std::memory_order_acquire)) {
         // The per-role register split (setmaxnreg) assumes the block starts
         // with kRegsLaunch registers per thread; with fewer, a role's
         // increase could never be granted, so refuse to launch.
@@ -1013,7 +1019,7 @@ static cudaError_t launch_hg(const DecodeArgs &a, int64_t nblocks, cudaStream_t 
         if (fa.numRegs != dec::kRegsLaunch || fa.maxThreadsPerBlock < dec::kThreads) return cudaErrorInvalidConfiguration;
         e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, dec::kSmemBytes);
         if (e != cudaSuccess) return e;
-        if (dev >= 0 && dev < 64) attr_set[dev] = true;
+        if (dev >= 0 && dev < 64) attr_set[dev].store(true, std::memory_order_release);
     }
     // Split launches are cooperative: the runtime refuses the launch unless
     // every CTA can be resident at once, which the merge's wait relies on.
@@ -1038,7 +1044,8 @@ cudaError_t launch_sparse_mla_decode(RowSource rows, const void *q_nope, const v
                                      int64_t num_slots, const int32_t *indices, int32_t topk, int32_t T,
                                      int32_t H, float sm_scale, void *out, float *lse, void *workspace,
                                      const DecodePlan &plan, int32_t *dev_status, cudaStream_t stream,
-                                     const int32_t *block_table, int64_t table_stride, int page_shift) {
+                                     const int32_t *block_table, int64_t table_stride, int page_shift,
+                                     const DecodeTestHooks *hooks) {
     if (T == 0) return cudaSuccess;
     DecodeArgs a;
     a.q_nope = static_cast<const __half *>(q_nope);
@@ -1065,6 +1072,8 @@ cudaError_t launch_sparse_mla_decode(RowSource rows, const void *q_nope, const v
     a.page_shift = page_shift;
     a.max_pos = block_table ? (table_stride << page_shift) : 0;
     a.rows_by_slot = rows == RowSource::kFp8Cache;
+    a.wait_cycles = hooks ? hooks->wait_cycles : ptx::kWaitCycles;
+    a.test_withhold = hooks ? hooks->withhold : 0;
     const bool staged = rows != RowSource::kNvfp4Cache;
     const int64_t nblocks = (int64_t)T * plan.head_groups * plan.splits;
     if (!staged) return launch_nvfp4_decode(a, plan.heads_per_cta, nblocks, stream);

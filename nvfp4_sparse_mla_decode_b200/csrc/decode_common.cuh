@@ -22,7 +22,8 @@ struct DecodeArgs {
     float scale_log2;
     __half *out;
     float *lse;
-    float *ws_o;        // split partials: [T][S][H][512] FP32, unnormalised
+    float *ws_o;        // split partials, unnormalised FP32: [T][S][H][512] (FP8-row kernel) or
+                        // [T][G][S][HG/4][512][4] (NVFP4 kernel: 4-head pieces, dv-major)
     float *ws_ml;       // split statistics: [T][S][H] x (max in log2 units, row sum)
     uint32_t *counters; // per (token, head group): arrivals, departures
     int32_t *dev_status;
@@ -36,15 +37,34 @@ struct DecodeArgs {
     // by slot, false when it is the staging buffer [T][topk] addressed by
     // list position.
     bool rows_by_slot;
+    // NVFP4 kernel: SM clock cycles after which any one wait gives up
+    // (about a second by default), and a test hook that withholds one
+    // arrival so that tests can drive the timeout paths (0 in every
+    // product call; see DecodeTestHooks).
+    unsigned long long wait_cycles;
+    int test_withhold;
+};
+
+// Test-only settings for a decode launch (never set by the public API):
+// withhold = 1: the softmax warps never publish P^T, so the output MMAs'
+// wait runs out and every role that depends on it follows;
+// withhold = 2: split 0 of each group never arrives on the merge counter, so
+// the group's merge wait runs out and poisons the counter.
+struct DecodeTestHooks {
+    unsigned long long wait_cycles;
+    int withhold;
 };
 
 #ifdef NVFP4MLA_TRACE
 // Debug builds only: per-CTA phase timestamps (clock64 deltas) for the
 // first 16 CTAs, 512 slots each.
+// TRACE_SETUP() reads the buffer pointer once, so a stamp is a clock read
+// and a store, not a global load after every wait.
 static __device__ unsigned long long *g_trace;
-#define TRACE(slot)                                                                  \
-    do {                                                                             \
-        if (g_trace && blockIdx.x < 16) g_trace[blockIdx.x * 512 + (slot)] = clock64() - t_start; \
+#define TRACE_SETUP() unsigned long long *const trace_buf_ = blockIdx.x < 16 && g_trace ? g_trace + blockIdx.x * 512 : nullptr
+#define TRACE(slot)                                                   \
+    do {                                                              \
+        if (trace_buf_) trace_buf_[(slot)] = clock64() - t_start;     \
     } while (0)
 static inline void set_trace_local(unsigned long long *p) { cudaMemcpyToSymbol(g_trace, &p, sizeof(p)); }
 // Every CTA: [start ns, end ns, SM id] from the global timer (comparable
@@ -62,6 +82,9 @@ __device__ __forceinline__ unsigned sm_id() {
     return r;
 }
 #else
+#define TRACE_SETUP() \
+    do {              \
+    } while (0)
 #define TRACE(slot) \
     do {            \
     } while (0)
@@ -128,9 +151,9 @@ __host__ __device__ constexpr int cols_per_lane(int W) { return W >= 32 ? W / 32
 // or q_rope (cols 64), box 64 cols x box_rows rows, 128-byte swizzle; encoded
 // maps are cached per host thread, keyed by (address, rows, cols, box rows).
 bool make_q_map(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols, uint32_t box_rows);
-// Tensor map over the FP32 split partials [rows, 512] (box box_cols x box_rows,
-// no swizzle), cached per host thread like the Q maps.
-bool make_partial_map(CUtensorMap *m, const void *base, uint64_t rows, uint32_t box_cols, uint32_t box_rows);
+// Tensor map over the NVFP4 kernel's split exchange area: FP32 rows of 2048
+// (512 dv x 4 heads), box box_x floats x box_rows rows, no swizzle.
+bool make_xch_map(CUtensorMap *m, const void *base, uint64_t rows, uint32_t box_x, uint32_t box_rows);
 // Launch of the pipelined NVFP4 decode kernel (decode_nvfp4.cu).
 cudaError_t launch_nvfp4_decode(const DecodeArgs &a, int heads_per_cta, int64_t nblocks, cudaStream_t stream);
 

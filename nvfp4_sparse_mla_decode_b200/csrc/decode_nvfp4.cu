@@ -106,11 +106,13 @@ static_assert(kOffP % 1024 == 0 && kOffV % 1024 == 0, "swizzled operands need 1 
 // the epilogue stages its output (or its own merge slice) over the V and raw
 // rings, which are free by then; the merge weights go to the P^T region
 constexpr int kOffStage = kOffV;
-constexpr int kOffPartial = kOffP;  // split partial boxes [S][HG][512/S] FP32 over P^T and the rings
-constexpr int kOffMergeW = kOffPartial + kMaxHG * kLatent * 4;  // merge weights, after the boxes
-static_assert(kOffMergeW + (16 * kMaxHG + kMaxHG) * 4 <= kOffIdx, "partial boxes and weights must fit before the list");
+// split merge: S boxes of D dv x HG heads FP32 (HG x 2 KB in all) over P^T
+// and the rings, then the merge weights
+constexpr int kOffPartial = kOffP;
+constexpr int kOffMergeW = kOffPartial + kMaxHG * kLatent * 4;
+static_assert(kOffMergeW + (16 * kMaxHG + kMaxHG) * 4 <= kOffIdx, "merge areas must fit before the list");
+static_assert(kOffPartial % 128 == 0 && kOffMergeW % 16 == 0, "merge areas take tensor copies and 16-byte accesses");
 static_assert(kMaxHG * kLatent * 2 <= kOffIdx - kOffStage, "output staging must fit over the rings");
-static_assert(kMaxHG * (kLatent / 2) * 4 <= kOffIdx - kOffStage, "own merge slice must fit over the rings");
 constexpr int kThreads = 768;
 constexpr int kKWarp0 = 4;
 constexpr int kSoftWarp0 = 12;
@@ -156,8 +158,10 @@ constexpr uint32_t kPoison = 0x80000000u;
 
 // Whole-warp bounded wait: every lane polls, the result is agreed by vote
 // so the warp stays converged for the elected-lane instructions after it.
-__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity) {
-    return __all_sync(0xffffffffu, mbar_wait(bar, parity));
+// Whole-warp bounded wait (the warp agrees on the outcome); `lim` is the
+// launch's wait bound in SM clock cycles.
+__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, unsigned long long lim) {
+    return __all_sync(0xffffffffu, mbar_wait(bar, parity, lim));
 }
 
 __device__ __forceinline__ uint4 lds128(const uint8_t *p) { return *reinterpret_cast<const uint4 *>(p); }
@@ -188,14 +192,20 @@ __device__ __forceinline__ void unpack_latent64(uint4 w0, uint4 w1, uint32_t sca
 }
 
 // Split merge, run by the 128 softmax threads of each of the S CTAs of a
-// (token, head group) once this CTA's unnormalised partial O sits in shared
-// memory as S boxes of [HG heads][D = 512/S dims] FP32 (box k = dims
-// k*D .. k*D+D-1).  Thread 0 sends every box but the CTA's own (box `split`)
-// to the workspace with 2-D tensor copies, waits until they have landed and
-// announces them on the group's arrival counter (release).  Once all S have
-// arrived (bounded wait), it fetches the other splits' copies of box `split`
-// into the places the sent boxes occupied, and the 128 threads combine dims
-// [split*D, split*D + D) of every head:
+// (token t, head group g).  Exchange area for the group (FP32): S partials,
+// each [HG/4 pieces][512 dv][4 heads] (piece q = heads 4q .. 4q+3); split s
+// owns dims [s*D, s*D + D), D = 512/S.  Before the merge every thread has
+// written its dv rows of the partial straight from tensor memory (a warp
+// store covers 32 consecutive dv of one piece, 512 contiguous bytes): rows
+// owned by other splits to this split's partial in the exchange area, its
+// own rows to shared memory box `split`.  Box layout (D dv x HG heads):
+// chunks of C = min(D, 64) dv, each [HG/4][C][4] -- the shape of a tensor
+// copy of C*4 floats x HG/4 rows of the exchange area.  Thread 0 announces
+// the rows on the group's arrival counter (release, cumulative over the 128
+// threads through the barrier before it), waits, bounded, until all S have
+// arrived, then fetches the other splits' rows of this slice into boxes s !=
+// split with tensor copies.  The threads combine dims [split*D, split*D + D)
+// of every head:
 //   out = sum_s w_s O_s / sum_s w_s l_s,  w_s = 2^(m_s - max m)
 // over the splits with rows (l_s > 0); split 0 also writes
 // lse = (max m + log2 of the denominator) ln 2.  The last CTA to leave resets
@@ -204,34 +214,28 @@ __device__ __forceinline__ void unpack_latent64(uint4 w0, uint4 w1, uint32_t sca
 // write NaN to their slice instead of merging partials that were never
 // written.
 template <int HG, int S>
-__device__ __forceinline__ void merge_splits_nv4(const DecodeArgs &a, const CUtensorMap *tm_ws, int t, int g,
+__device__ __forceinline__ void merge_splits_nv4(const DecodeArgs &a, const CUtensorMap *tm_xch, int t, int g,
                                                  int split, uint8_t *smem, uint64_t *bar, int mt,
                                                  [[maybe_unused]] unsigned long long t_start) {
+    TRACE_SETUP();
     using namespace nv4;
     constexpr int kMergeThreads = 128;
+    constexpr int NQ = HG / 4;
     constexpr int D = kLatent / S;
-    constexpr int kBoxBytes = HG * D * 4;
-    constexpr int NQ = D / 4;
-    constexpr int ITEMS = HG * NQ;
+    constexpr int C = D < 64 ? D : 64;  // dv per tensor copy
+    constexpr int box_bytes = D * HG * 4;
     uint32_t *arrive = a.counters + 2 * ((int64_t)t * a.G + g);
     uint32_t *depart = arrive + 1;
     uint32_t *flag = reinterpret_cast<uint32_t *>(smem + kOffMisc) + 1;
-    const float *stage = reinterpret_cast<const float *>(smem + kOffPartial);  // [S][HG][D]
-    float *w_s = reinterpret_cast<float *>(smem + kOffMergeW);               // [S][HG]
-    float *inv_den = w_s + nv4::kMaxSplits * HG;                              // [HG]
-    const int32_t row0 = (t * S + split) * a.H + g * HG;  // this split's partial rows
-    fence_proxy_async_smem();       // the drained boxes are visible to the copy engine
-    named_bar(1, kMergeThreads);    // ... and to thread 0, with the statistics stores
+    float *w_s = reinterpret_cast<float *>(smem + kOffMergeW);  // [S][HG]
+    float *inv_den = w_s + kMaxSplits * HG;                      // [HG]
+    const int dv0 = split * D;
+    named_bar(1, kMergeThreads);  // every thread's partial rows and statistics are written
     if (mt == 0) {
         TRACE(190);
-#pragma unroll 1
-        for (int k = 0; k < S; ++k)
-            if (k != split) tma_store_2d(tm_ws, smem + kOffPartial + k * kBoxBytes, k * D, row0);
-        bulk_commit_wait_all();     // the partial boxes have reached global memory
-        fence_proxy_async_global();
-        __threadfence();            // ... and, with the statistics, are ordered before the arrival
+        __threadfence();
         TRACE(191);
-        const uint32_t old = atomicAdd(arrive, 1u);
+        const uint32_t old = (a.test_withhold == 2 && split == 0) ? 0u : atomicAdd(arrive, 1u);
         bool ok = (old & kPoison) == 0;
         if (ok) {
             const unsigned long long t0 = clock64();
@@ -242,7 +246,7 @@ __device__ __forceinline__ void merge_splits_nv4(const DecodeArgs &a, const CUte
                     break;
                 }
                 if (v >= (uint32_t)S) break;
-                if (clock64() - t0 > kWaitCycles) {
+                if (clock64() - t0 > a.wait_cycles) {
                     ok = false;
                     break;
                 }
@@ -253,23 +257,25 @@ __device__ __forceinline__ void merge_splits_nv4(const DecodeArgs &a, const CUte
             atomicOr(arrive, kPoison);
             if (a.dev_status) atomicOr(a.dev_status, NVFP4MLA_DEV_TIMEOUT);
         } else {
-            // the other splits' copies of this CTA's box, into the places of
-            // the boxes just sent (their copies have read them)
-            fence_proxy_async_global();
+            fence_proxy_async_global();  // the other splits' rows, seen through the counter, to the copy engine
             // this barrier's first phase tracked the Q copies; they have
             // landed before its second phase is armed
-            if (!mbar_wait(bar, 0) && a.dev_status) atomicOr(a.dev_status, NVFP4MLA_DEV_TIMEOUT);
-            mbar_arrive_expect_tx(bar, (uint32_t)((S - 1) * kBoxBytes));
+            if (!mbar_wait(bar, 0, a.wait_cycles) && a.dev_status) atomicOr(a.dev_status, NVFP4MLA_DEV_TIMEOUT);
+            mbar_arrive_expect_tx(bar, (uint32_t)((S - 1) * box_bytes));
+            const int32_t row_g = ((t * a.G + g) * S) * NQ;  // first exchange row of the group
 #pragma unroll 1
-            for (int s = 0; s < S; ++s)
-                if (s != split)
-                    tma_load_2d(smem + kOffPartial + s * kBoxBytes, tm_ws, split * D, (t * S + s) * a.H + g * HG, bar);
+            for (int s = 0; s < S; ++s) {
+                if (s == split) continue;
+#pragma unroll
+                for (int c = 0; c < D / C; ++c)
+                    tma_load_2d(smem + kOffPartial + s * box_bytes + c * (NQ * C * 16), tm_xch, (dv0 + c * C) * 4,
+                                row_g + s * NQ, bar);
+            }
         }
         *flag = ok ? 1u : 0u;
         TRACE(192);
     }
     named_bar(1, kMergeThreads);
-    const int dv0 = split * D;
     __half *dst = a.out + ((int64_t)t * a.H + (int64_t)g * HG) * kLatent + dv0;
     if (!*flag) {  // poisoned: make the failure visible in the output
         for (int item = mt; item < HG * D; item += kMergeThreads) {
@@ -279,7 +285,7 @@ __device__ __forceinline__ void merge_splits_nv4(const DecodeArgs &a, const CUte
         if (split == 0 && mt < HG) a.lse[(int64_t)t * a.H + (int64_t)g * HG + mt] = NAN;
         return;
     }
-    if (mt < HG) {  // split weights from the statistics while the boxes travel
+    if (mt < HG) {  // split weights from the statistics while the rows travel
         const float *ml = a.ws_ml + 2 * ((int64_t)t * S * a.H + (int64_t)g * HG + mt);
         float2 v[S];
 #pragma unroll
@@ -300,26 +306,51 @@ __device__ __forceinline__ void merge_splits_nv4(const DecodeArgs &a, const CUte
             a.lse[(int64_t)t * a.H + (int64_t)g * HG + mt] =
                 den > 0.0f ? (mmax + lg2(den)) * 0.69314718055994531f : -INFINITY;
     }
-    const bool landed = mbar_wait(bar, 1);  // the box copies (phase 1 of the Q barrier)
+    const bool landed = mbar_wait(bar, 1, a.wait_cycles);  // the tensor copies (phase 1 of the Q barrier)
     if (!landed && a.dev_status) atomicOr(a.dev_status, NVFP4MLA_DEV_TIMEOUT);
     named_bar(1, kMergeThreads);
     if (mt == 0) TRACE(193);
-    for (int item = mt; item < ITEMS; item += kMergeThreads) {
-        const int h = item / NQ, q = item - h * NQ;
+    // item = (piece q, dv d): neighbouring threads take neighbouring dv, so
+    // the box reads are conflict-free; neighbouring lanes then swap halves
+    // so that each stores two adjacent dv of one head (4 bytes; a warp store
+    // covers 32 consecutive dv of two heads)
+    const float *boxes = reinterpret_cast<const float *>(smem + kOffPartial);
+    const bool odd = mt & 1;
+    constexpr int kItems = D * NQ / kMergeThreads;  // D * NQ is a multiple of 128
+    static_assert(D * NQ % kMergeThreads == 0, "merge items per thread");
+#pragma unroll 2
+    for (int k = 0; k < kItems; ++k) {
+        const int item = mt + kMergeThreads * k;
+        const int q = item / D, d = item - q * D;
+        const int c = d / C, dd = d - c * C;
+        const int off = c * (NQ * C * 4) + (q * C + dd) * 4;  // floats, within a box
         float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
 #pragma unroll
         for (int s = 0; s < S; ++s) {
-            const float w = w_s[s * HG + h];
-            const float4 v = *reinterpret_cast<const float4 *>(stage + (s * HG + h) * D + 4 * q);
-            acc.x += w * v.x;
-            acc.y += w * v.y;
-            acc.z += w * v.z;
-            acc.w += w * v.w;
+            const float4 v = *reinterpret_cast<const float4 *>(boxes + s * (box_bytes / 4) + off);
+            const float4 w = *reinterpret_cast<const float4 *>(w_s + s * HG + 4 * q);
+            acc.x += w.x * v.x;
+            acc.y += w.y * v.y;
+            acc.z += w.z * v.z;
+            acc.w += w.w * v.w;
         }
-        const float r = inv_den[h];
-        __half2 *d2 = reinterpret_cast<__half2 *>(dst + (int64_t)h * kLatent + 4 * q);
-        d2[0] = __floats2half2_rn(acc.x * r, acc.y * r);
-        d2[1] = __floats2half2_rn(acc.z * r, acc.w * r);
+        const float4 r = *reinterpret_cast<const float4 *>(inv_den + 4 * q);
+        acc.x *= r.x;
+        acc.y *= r.y;
+        acc.z *= r.z;
+        acc.w *= r.w;
+        // even lane keeps heads 4q, 4q+1 and takes its neighbour's; odd lane
+        // keeps heads 4q+2, 4q+3 and takes its neighbour's
+        const float s0 = odd ? acc.x : acc.z, s1 = odd ? acc.y : acc.w;
+        const float r0 = __shfl_xor_sync(0xffffffffu, s0, 1), r1 = __shfl_xor_sync(0xffffffffu, s1, 1);
+        const float k0 = odd ? acc.z : acc.x, k1 = odd ? acc.w : acc.y;
+        const int h = 4 * q + (odd ? 2 : 0);
+        const int de = d & ~1;  // the pair's even dv
+        // (own value, neighbour's value) in dv order
+        const __half2 p0 = odd ? __floats2half2_rn(r0, k0) : __floats2half2_rn(k0, r0);
+        const __half2 p1 = odd ? __floats2half2_rn(r1, k1) : __floats2half2_rn(k1, r1);
+        *reinterpret_cast<__half2 *>(dst + (int64_t)h * kLatent + de) = p0;
+        *reinterpret_cast<__half2 *>(dst + (int64_t)(h + 1) * kLatent + de) = p1;
     }
     named_bar(1, kMergeThreads);
     if (mt == 0) {
@@ -335,7 +366,7 @@ __device__ __forceinline__ void merge_splits_nv4(const DecodeArgs &a, const CUte
 template <int HG>
 __global__ void __launch_bounds__(nv4::kThreads, 1)
     nvfp4_decode_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_qn,
-                        const __grid_constant__ CUtensorMap tm_qr, const __grid_constant__ CUtensorMap tm_ws) {
+                        const __grid_constant__ CUtensorMap tm_qr, const __grid_constant__ CUtensorMap tm_xch) {
     using namespace nv4;
     extern __shared__ __align__(1024) uint8_t smem[];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -348,6 +379,7 @@ __global__ void __launch_bounds__(nv4::kThreads, 1)
 #else
     const unsigned long long t_start = 0;  // timestamps exist only in trace builds
 #endif
+    TRACE_SETUP();
 
     if (smem_u32(smem) & 1023u) {  // the swizzled operand layouts need a 1 KB aligned base
         if (tid == 0 && a.dev_status) atomicOr(a.dev_status, NVFP4MLA_DEV_LAYOUT);
@@ -464,11 +496,11 @@ __global__ void __launch_bounds__(nv4::kThreads, 1)
             // j - 2 has read it.
             const uint32_t id_qk = idesc_f16_f32(128, HG, false, false);
             const uint64_t dQ0 = smem_desc(smem_u32(smem + kOffQ), 16, 1024);
-            bool ok = warp_wait(&bars[BAR_Q], 0);  // always: the copies must land before the CTA may exit
+            bool ok = warp_wait(&bars[BAR_Q], 0, a.wait_cycles);  // always: the copies must land before the CTA may exit
             if (lane == 0) TRACE(1);
             uint32_t kn = 0;
             for (int j = 0; j < ntiles && ok; ++j) {
-                if (j >= 2 && !warp_wait(&bars[BAR_S_FREE + (j & 1)], ((j >> 1) - 1) & 1)) {
+                if (j >= 2 && !warp_wait(&bars[BAR_S_FREE + (j & 1)], ((j >> 1) - 1) & 1, a.wait_cycles)) {
                     ok = false;
                     break;
                 }
@@ -478,7 +510,7 @@ __global__ void __launch_bounds__(nv4::kThreads, 1)
 #pragma unroll 1
                 for (int c = 0; c < kKChunks; ++c) {
                     const uint32_t slot = kn & 3u;
-                    if (!warp_wait(&bars[BAR_K_FULL + slot], (kn >> 2) & 1u)) {
+                    if (!warp_wait(&bars[BAR_K_FULL + slot], (kn >> 2) & 1u, a.wait_cycles)) {
                         ok = false;
                         break;
                     }
@@ -499,7 +531,7 @@ __global__ void __launch_bounds__(nv4::kThreads, 1)
             }
             if (!ok && lane == 0 && a.dev_status) atomicOr(a.dev_status, NVFP4MLA_DEV_TIMEOUT);
             mma_commit_warp(&bars[BAR_DRAIN]);  // nothing may still read or write TMEM at teardown
-            warp_wait(&bars[BAR_DRAIN], 0);
+            warp_wait(&bars[BAR_DRAIN], 0, a.wait_cycles);
         } else if (warp == 2) {
             // ------------------------------------------------ output MMAs
             // O^T += V^T(j) P^T(j), one 16-row V ring slot at a time, once the
@@ -510,7 +542,7 @@ __global__ void __launch_bounds__(nv4::kThreads, 1)
             bool ok = true;
             uint32_t vn = 0;
             for (int j = 0; j < ntiles && ok; ++j) {
-                if (!warp_wait(&bars[BAR_P_FULL], j & 1)) {
+                if (!warp_wait(&bars[BAR_P_FULL], j & 1, a.wait_cycles)) {
                     ok = false;
                     break;
                 }
@@ -520,7 +552,7 @@ __global__ void __launch_bounds__(nv4::kThreads, 1)
 #pragma unroll 1
                 for (int gi = 0; gi < kVGroups; ++gi) {
                     const uint32_t slot = vn % kVSlots;
-                    if (!warp_wait(&bars[BAR_V_FULL + slot], (vn / kVSlots) & 1u)) {
+                    if (!warp_wait(&bars[BAR_V_FULL + slot], (vn / kVSlots) & 1u, a.wait_cycles)) {
                         ok = false;
                         break;
                     }
@@ -546,7 +578,7 @@ __global__ void __launch_bounds__(nv4::kThreads, 1)
             }
             if (!ok && lane == 0 && a.dev_status) atomicOr(a.dev_status, NVFP4MLA_DEV_TIMEOUT);
             mma_commit_warp(&bars[BAR_DRAIN_PV]);  // nothing may still read or write TMEM at teardown
-            warp_wait(&bars[BAR_DRAIN_PV], 0);
+            warp_wait(&bars[BAR_DRAIN_PV], 0, a.wait_cycles);
         } else if (warp == 1 || warp == 3) {
             // ---------------------------------------------------- gather
             // 64 threads copy the tile's rows in 16-byte pieces (22 per row)
@@ -569,7 +601,7 @@ __global__ void __launch_bounds__(nv4::kThreads, 1)
             for (int j = 0; j < ntiles; ++j) {
                 if (kPrefetchAhead > 0 && j + kPrefetchAhead < ntiles) prefetch_tile(j + kPrefetchAhead);
                 const int slot = j % kRawSlots;
-                if (j >= kRawSlots && !warp_wait(&bars[BAR_RAW_FREE + slot], ((j / kRawSlots) - 1) & 1)) {
+                if (j >= kRawSlots && !warp_wait(&bars[BAR_RAW_FREE + slot], ((j / kRawSlots) - 1) & 1, a.wait_cycles)) {
                     ok = false;
                     break;
                 }
@@ -601,7 +633,7 @@ __global__ void __launch_bounds__(nv4::kThreads, 1)
         bool ok = true;
         for (int j = 0; j < ntiles && ok; ++j) {
             const int rslot = j % kRawSlots;
-            if (!warp_wait(&bars[BAR_RAW_FULL + rslot], (j / kRawSlots) & 1)) {
+            if (!warp_wait(&bars[BAR_RAW_FULL + rslot], (j / kRawSlots) & 1, a.wait_cycles)) {
                 ok = false;
                 break;
             }
@@ -637,7 +669,7 @@ __global__ void __launch_bounds__(nv4::kThreads, 1)
 #pragma unroll
                     for (int i = 0; i < 32; ++i) o[i] = 0u;
                 }
-                if (n >= 4 && !warp_wait(&bars[BAR_K_FREE + slot], ((n >> 2) - 1) & 1u)) {
+                if (n >= 4 && !warp_wait(&bars[BAR_K_FREE + slot], ((n >> 2) - 1) & 1u, a.wait_cycles)) {
                     ok = false;
                     break;
                 }
@@ -678,7 +710,7 @@ __global__ void __launch_bounds__(nv4::kThreads, 1)
         // Every wait's outcome is agreed by all 128 threads (bar.red.or), so
         // the four warps always meet at the same named barriers.
         for (int j = 0; j < ntiles; ++j) {
-            if (named_bar_or(1, 128, !warp_wait(&bars[BAR_S_FULL + (j & 1)], (j >> 1) & 1))) {
+            if (named_bar_or(1, 128, !warp_wait(&bars[BAR_S_FULL + (j & 1)], (j >> 1) & 1, a.wait_cycles))) {
                 ok = false;
                 break;
             }
@@ -759,7 +791,7 @@ __global__ void __launch_bounds__(nv4::kThreads, 1)
             // O^T and P^T belong to the output MMAs of the previous tile
             // until they are done.
             if (j > 0) {
-                if (named_bar_or(1, 128, !warp_wait(&bars[BAR_PV_DONE], (j - 1) & 1))) {
+                if (named_bar_or(1, 128, !warp_wait(&bars[BAR_PV_DONE], (j - 1) & 1, a.wait_cycles))) {
                     ok = false;
                     break;
                 }
@@ -789,7 +821,7 @@ __global__ void __launch_bounds__(nv4::kThreads, 1)
             fence_proxy_async_smem();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&bars[BAR_P_FULL]);
+            if (lane == 0 && a.test_withhold != 1) mbar_arrive(&bars[BAR_P_FULL]);
             if (st == 0 && j < 8) TRACE(140 + j);
         }
         if (!ok && a.dev_status && lane == 0) atomicOr(a.dev_status, NVFP4MLA_DEV_TIMEOUT);
@@ -817,7 +849,7 @@ __global__ void __launch_bounds__(nv4::kThreads, 1)
         named_bar(1, 128);
         bool fin = have;
         if (have) {  // O^T is final once the last tile's output MMAs are done
-            fin = !named_bar_or(1, 128, !warp_wait(&bars[BAR_PV_DONE], (ntiles - 1) & 1));
+            fin = !named_bar_or(1, 128, !warp_wait(&bars[BAR_PV_DONE], (ntiles - 1) & 1, a.wait_cycles));
             if (!fin && st == 0 && a.dev_status) atomicOr(a.dev_status, NVFP4MLA_DEV_TIMEOUT);
             tc_fence_after();
         }
@@ -855,40 +887,52 @@ __global__ void __launch_bounds__(nv4::kThreads, 1)
                 bulk_commit_wait_read();
             }
         } else {
-            // Unnormalised partial O of this split into shared memory as S
-            // boxes [HG][D] (box k = dims k*D ..), over the P^T and ring
-            // regions, which no MMA or copy uses any more; for each head a
-            // warp writes 32 consecutive dims.  The merge sends the boxes out
-            // with tensor copies.
+            // Unnormalised partial O of this split, row dv = this thread's
+            // TMEM lane in each 128-dv block, as 4-head pieces: rows owned by
+            // another split go straight to this split's partial in the
+            // exchange area ([HG/4][512][4]; a warp store covers 32
+            // consecutive dv of a piece), this split's own rows to shared
+            // box `split` (chunks of C dv, [HG/4][C][4] each), over the P^T
+            // and ring regions, which no MMA or copy uses any more.  A warp's
+            // 32 rows never straddle two owners (D = 512/S is a multiple of
+            // 32).
             const int D = kLatent / a.S;
-            float *box = reinterpret_cast<float *>(smem + kOffPartial);
+            const int C = D < 64 ? D : 64;
+            constexpr int NQ = HG / 4;
+            float *own = reinterpret_cast<float *>(smem + kOffPartial + split * (D * HG * 4));
+            float *xch = a.ws_o + (((int64_t)t * a.G + g) * a.S + split) * (int64_t)NQ * kLatent * 4;
             constexpr int HC = HG > 32 ? 32 : HG;
 #pragma unroll 1
             for (int b = 0; b < 4; ++b) {
                 const int dv = 128 * b + st;
-                const int k = dv / D, d = dv - k * D;
-                float *dst = box + (k * HG) * D + d;
+                const bool mine = dv / D == split;
+                const int d = dv - split * D, c = d / C, dd = d - (d / C) * C;
+                uint32_t rr[HG];  // every head of row dv: all loads issued, one wait
+                if (fin) {
 #pragma unroll
-                for (int h0 = 0; h0 < HG; h0 += HC) {
-                    uint32_t rr[HC];
-                    if (fin) {
-                        tmem_ld_cols<HC>(tmem + lane_base + kColO + b * HG + h0, rr);
-                        tmem_ld_wait();
-                    } else {
+                    for (int h0 = 0; h0 < HG; h0 += HC)
+                        tmem_ld_cols<HC>(tmem + lane_base + kColO + b * HG + h0, *reinterpret_cast<uint32_t(*)[HC]>(rr + h0));
+                    tmem_ld_wait();
+                } else {
 #pragma unroll
-                        for (int h = 0; h < HC; ++h) rr[h] = 0u;
-                    }
+                    for (int h = 0; h < HG; ++h) rr[h] = 0u;
+                }
 #pragma unroll
-                    for (int h = 0; h < HC; ++h) dst[(h0 + h) * D] = __uint_as_float(rr[h]);
+                for (int q = 0; q < NQ; ++q) {
+                    const float4 v = make_float4(__uint_as_float(rr[4 * q]), __uint_as_float(rr[4 * q + 1]),
+                                                 __uint_as_float(rr[4 * q + 2]), __uint_as_float(rr[4 * q + 3]));
+                    if (mine)
+                        *reinterpret_cast<float4 *>(own + c * (NQ * C * 4) + (q * C + dd) * 4) = v;
+                    else
+                        __stcg(reinterpret_cast<float4 *>(xch + ((int64_t)q * kLatent + dv) * 4), v);
                 }
             }
             if (st == 0) TRACE(172);
-            uint64_t *mbar = &bars[BAR_Q];  // its second phase tracks the merge's box copies
             switch (a.S) {
-                case 2: merge_splits_nv4<HG, 2>(a, &tm_ws, t, g, split, smem, mbar, st, t_start); break;
-                case 4: merge_splits_nv4<HG, 4>(a, &tm_ws, t, g, split, smem, mbar, st, t_start); break;
-                case 8: merge_splits_nv4<HG, 8>(a, &tm_ws, t, g, split, smem, mbar, st, t_start); break;
-                default: merge_splits_nv4<HG, 16>(a, &tm_ws, t, g, split, smem, mbar, st, t_start); break;
+                case 2: merge_splits_nv4<HG, 2>(a, &tm_xch, t, g, split, smem, &bars[BAR_Q], st, t_start); break;
+                case 4: merge_splits_nv4<HG, 4>(a, &tm_xch, t, g, split, smem, &bars[BAR_Q], st, t_start); break;
+                case 8: merge_splits_nv4<HG, 8>(a, &tm_xch, t, g, split, smem, &bars[BAR_Q], st, t_start); break;
+                default: merge_splits_nv4<HG, 16>(a, &tm_xch, t, g, split, smem, &bars[BAR_Q], st, t_start); break;
             }
             if (st == 0) TRACE(174);
         }
@@ -909,9 +953,13 @@ __global__ void __launch_bounds__(nv4::kThreads, 1)
         bool ok = true;
         uint32_t vn = (uint32_t)vs;  // ring position of this set's next group (groups alternate sets)
         for (int j = 0; j < ntiles && ok; ++j) {
-            // The tile's rows are in L2 once its score MMAs are done; that
-            // also keeps these loads from racing the gather to HBM.
-            if (!warp_wait(&bars[BAR_S_FULL + (j & 1)], (j >> 1) & 1)) {
+            // The tile's rows are in L2 once the softmax has read its
+            // scores; that also keeps these loads from racing the gather to
+            // HBM.  (S_FREE, unlike S_FULL, cannot complete this buffer's
+            // next phase, tile j + 2, before these warps finish tile j: the
+            // softmax reaches tile j + 2 only after the output MMAs of tile
+            // j, which need every V group of it.)
+            if (!warp_wait(&bars[BAR_S_FREE + (j & 1)], (j >> 1) & 1, a.wait_cycles)) {
                 ok = false;
                 break;
             }
@@ -946,7 +994,7 @@ __global__ void __launch_bounds__(nv4::kThreads, 1)
                 unpack_latent64(w0[m % kDepth], w1[m % kDepth], sc[m % kDepth], o);
                 if (m + kDepth < kMine) load(vs + 2 * (m + kDepth), w0[m % kDepth], w1[m % kDepth], sc[m % kDepth]);
                 if (vw == 0 && lane == 0 && j == 1) TRACE(300 + 20 * vs + 4 * m);
-                if (vn >= kVSlots && !warp_wait(&bars[BAR_V_FREE + slot], ((vn / kVSlots) - 1) & 1u)) {
+                if (vn >= kVSlots && !warp_wait(&bars[BAR_V_FREE + slot], ((vn / kVSlots) - 1) & 1u, a.wait_cycles)) {
                     ok = false;
                     break;
                 }
@@ -1006,17 +1054,18 @@ static cudaError_t launch_nv4(const DecodeArgs &a, int64_t nblocks, cudaStream_t
     attr[0].val.cooperative = 1;
     cfg.attrs = attr;
     cfg.numAttrs = a.S > 1 ? 1 : 0;  // split launches need every CTA resident at once
-    CUtensorMap tm_qn, tm_qr, tm_ws;
+    CUtensorMap tm_qn, tm_qr, tm_xch;
     const uint64_t rows = (uint64_t)a.T * (uint64_t)a.H;
     if (!make_q_map(&tm_qn, a.q_nope, rows, kLatent, HG) || !make_q_map(&tm_qr, a.q_rope, rows, kRope, HG))
         return cudaErrorInvalidValue;
-    if (a.S > 1) {  // split partials [T * S * H, 512], one box = HG heads x 512/S dims
-        if (!make_partial_map(&tm_ws, a.ws_o, rows * (uint64_t)a.S, (uint32_t)(kLatent / a.S), HG))
+    if (a.S > 1) {  // exchange rows: T * H * S / 4 pieces of 2048 floats; one copy = C dv x HG/4 pieces
+        const int D = kLatent / a.S, C = D < 64 ? D : 64;
+        if (!make_xch_map(&tm_xch, a.ws_o, rows * (uint64_t)a.S / 4, (uint32_t)(C * 4), HG / 4))
             return cudaErrorInvalidValue;
     } else {
-        tm_ws = tm_qn;  // unused without splits
+        tm_xch = tm_qn;  // unused without splits
     }
-    return cudaLaunchKernelEx(&cfg, kern, a, tm_qn, tm_qr, tm_ws);
+    return cudaLaunchKernelEx(&cfg, kern, a, tm_qn, tm_qr, tm_xch);
 }
 
 cudaError_t launch_nvfp4_decode(const DecodeArgs &a, int heads_per_cta, int64_t nblocks, cudaStream_t stream) {

@@ -33,6 +33,8 @@ cudaError_t launch_fp8_kv_append(const void *latent, int64_t latent_stride, cons
                                  const int32_t *slot_mapping, int32_t n, uint8_t *cache, int64_t num_slots,
                                  int32_t *dev_status, cudaStream_t stream);
 
+struct DecodeTestHooks;  // test-only launch settings (decode_common.cuh)
+
 // What the decode's `src` holds.
 enum class RowSource {
     kNvfp4Cache,  // num_slots 352-byte NVFP4 rows; list entries are slots
@@ -50,7 +52,7 @@ cudaError_t launch_sparse_mla_decode(RowSource rows, const void *q_nope, const v
                                      int32_t H, float sm_scale, void *out, float *lse, void *workspace,
                                      const DecodePlan &plan, int32_t *dev_status, cudaStream_t stream,
                                      const int32_t *block_table = nullptr, int64_t table_stride = 0,
-                                     int page_shift = 0);
+                                     int page_shift = 0, const DecodeTestHooks *hooks = nullptr);
 
 cudaError_t launch_stage_fp8(const uint8_t *cache, int64_t num_slots, const int32_t *indices, int32_t topk,
                              int32_t T, uint8_t *staging, cudaStream_t stream);
