@@ -143,7 +143,8 @@ constexpr int BAR_PV_DONE = BAR_P_FULL + 1;             // output MMAs of a tile
 constexpr int BAR_DRAIN = BAR_PV_DONE + 1;              // every score MMA issued so far done
 constexpr int BAR_S_FREE = BAR_DRAIN + 1;               // [2] softmax done reading an S buffer (4 softmax warps)
 constexpr int BAR_DRAIN_PV = BAR_S_FREE + 2;            // every output MMA issued so far done
-constexpr int kBarsUsed = BAR_DRAIN_PV + 1;
+constexpr int BAR_ROWS0 = BAR_DRAIN_PV + 1;             // the first tile's rows landed (cp.async arrivals of 64 threads)
+constexpr int kBarsUsed = BAR_ROWS0 + 1;
 static_assert(kBarsUsed <= kNumBars, "barrier slots");
 
 constexpr uint32_t kTmemCols = 512;
@@ -397,7 +398,7 @@ __global__ void __launch_bounds__(nv4::kThreads, 1)
     if (warp == 1 && lane == 0) {
         for (int b = 0; b < kBarsUsed; ++b) {
             uint32_t count = 1;
-            if (b >= BAR_RAW_FULL && b < BAR_RAW_FULL + kRawSlots) count = 64;  // cp.async arrivals
+            if ((b >= BAR_RAW_FULL && b < BAR_RAW_FULL + kRawSlots) || b == BAR_ROWS0) count = 64;  // cp.async arrivals
             else if (b >= BAR_RAW_FREE && b < BAR_RAW_FREE + kRawSlots) count = 8;
             else if (b >= BAR_K_FULL && b < BAR_K_FULL + kKSlots) count = 4;
             else if (b >= BAR_V_FULL && b < BAR_V_FULL + kVSlots) count = 4;
@@ -615,6 +616,7 @@ __global__ void __launch_bounds__(nv4::kThreads, 1)
                     cp_async16(dst + r * kRawStride + 16 * k, a.src + (int64_t)ids[r] * kRowBytes + 16 * k);
                 }
                 cp_async_mbar_arrive(&bars[BAR_RAW_FULL + slot]);
+                if (j == 0) cp_async_mbar_arrive(&bars[BAR_ROWS0]);
                 if (gt == 0 && j < 8) TRACE(80 + j);
             }
             // copies still in flight land before the CTA may exit
@@ -953,13 +955,17 @@ __global__ void __launch_bounds__(nv4::kThreads, 1)
         bool ok = true;
         uint32_t vn = (uint32_t)vs;  // ring position of this set's next group (groups alternate sets)
         for (int j = 0; j < ntiles && ok; ++j) {
-            // The tile's rows are in L2 once the softmax has read its
-            // scores; that also keeps these loads from racing the gather to
-            // HBM.  (S_FREE, unlike S_FULL, cannot complete this buffer's
-            // next phase, tile j + 2, before these warps finish tile j: the
-            // softmax reaches tile j + 2 only after the output MMAs of tile
-            // j, which need every V group of it.)
-            if (!warp_wait(&bars[BAR_S_FREE + (j & 1)], (j >> 1) & 1, a.wait_cycles)) {
+            // Rows are read once they are in L2, which also keeps these loads
+            // from racing the gather to HBM: the first tile's once its copies
+            // have landed (a barrier that completes only once), later tiles'
+            // once the softmax has read their scores.  (S_FREE, unlike S_FULL
+            // or the raw ring, cannot complete this buffer's next phase, tile
+            // j + 2, before these warps finish tile j: the softmax reaches
+            // tile j + 2 only after the output MMAs of tile j, which need
+            // every V group of it.)
+            const bool rows_in = j == 0 ? warp_wait(&bars[BAR_ROWS0], 0, a.wait_cycles)
+                                        : warp_wait(&bars[BAR_S_FREE + (j & 1)], (j >> 1) & 1, a.wait_cycles);
+            if (!rows_in) {
                 ok = false;
                 break;
             }
@@ -980,19 +986,22 @@ __global__ void __launch_bounds__(nv4::kThreads, 1)
             };
             // this set's next two groups are in flight ahead of the one
             // being converted
+            // (a rolled loop: this role's code stays small)
             constexpr int kMine = kVGroups / 2;
-            constexpr int kDepth = 2;
-            uint4 w0[kDepth], w1[kDepth];
-            uint32_t sc[kDepth];
-#pragma unroll
-            for (int d = 0; d < kDepth; ++d) load(vs + 2 * d, w0[d], w1[d], sc[d]);
-#pragma unroll
+            uint4 a0, a1, b0, b1;  // rows of this set's current and next group
+            uint32_t as, bs;
+            load(vs, a0, a1, as);
+            load(vs + 2, b0, b1, bs);
+#pragma unroll 1
             for (int m = 0; m < kMine; ++m) {
                 const uint32_t slot = vn % kVSlots;
                 uint8_t *base = smem + kOffV + slot * kVSlotBytes + dg * 2048;
                 uint32_t o[32];
-                unpack_latent64(w0[m % kDepth], w1[m % kDepth], sc[m % kDepth], o);
-                if (m + kDepth < kMine) load(vs + 2 * (m + kDepth), w0[m % kDepth], w1[m % kDepth], sc[m % kDepth]);
+                unpack_latent64(a0, a1, as, o);
+                a0 = b0;
+                a1 = b1;
+                as = bs;
+                if (m + 2 < kMine) load(vs + 2 * (m + 2), b0, b1, bs);
                 if (vw == 0 && lane == 0 && j == 1) TRACE(300 + 20 * vs + 4 * m);
                 if (vn >= kVSlots && !warp_wait(&bars[BAR_V_FREE + slot], ((vn / kVSlots) - 1) & 1u, a.wait_cycles)) {
                     ok = false;

@@ -33,16 +33,15 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t by
                  "r"(bytes)
                  : "memory");
 }
-// One bounded probe of the phase: the thread may be suspended in hardware
-// until the phase completes or about kSuspendNs nanoseconds pass, so waiting
-// warps do not take issue slots from working ones by spinning.
-constexpr uint32_t kSuspendNs = 100000;
+// One bounded probe of the phase (the hardware's own short wait, no
+// suspend-time hint: a hinted wait measured slower to wake on the decode
+// kernel's hand-offs).
 __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
-        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\tselp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity), "n"(kSuspendNs)
+        : "r"(smem_u32(bar)), "r"(parity)
         : "memory");
     return ok != 0;
 }
