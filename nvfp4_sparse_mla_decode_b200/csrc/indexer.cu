@@ -314,6 +314,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 // row replaces A-C.
 constexpr int kTopkThreads = 1024;
 constexpr int kTopkWarps = kTopkThreads / 32;
+static_assert(kTopkWarps == 32, "one warp reduces the per-warp minima and maxima");
 constexpr int kBins = 2048;
 constexpr int kChunk = 8192;  // floats per streamed chunk
 constexpr int kRing = 3;
@@ -453,6 +454,188 @@ __device__ uint32_t select_in_smem(const uint32_t *keys, uint32_t n, uint32_t wa
     return prefix;
 }
 
+// The want-th largest of n keys in shared memory (1 <= want <= n), exactly
+// as select_in_smem gives it, usually in one histogram pass: keys are binned
+// by (key - min) >> shift, a monotone map onto at most 2048 bins, so every
+// bin above the one holding the want-th largest key, b*, is taken whole; the
+// few keys of b* (at most 32) are then ranked by one warp.  When b* holds
+// more than 32 keys it falls back to the radix select.  Every thread calls
+// it; `sub` is 32 words of scratch, `mm` 2.
+__device__ uint32_t select_fast(const uint32_t *keys, uint32_t n, uint32_t want, uint32_t *hist, uint32_t *scratch,
+                                uint32_t *found, uint32_t *ties, uint32_t *sub, uint32_t *mm) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    uint32_t lo = 0xFFFFFFFFu, hi = 0u;
+    for (uint32_t i = tid; i < n; i += kTopkThreads) {
+        const uint32_t k = keys[i];
+        lo = min(lo, k);
+        hi = max(hi, k);
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+        lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, off));
+        hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, off));
+    }
+    if (lane == 0) {  // per-warp minima and maxima (kTopkWarps == 32)
+        scratch[warp] = lo;
+        sub[warp] = hi;
+    }
+    if (tid == 0) found[0] = 0;  // keys of b* collected so far (below)
+    for (int i = tid; i < kBins; i += kTopkThreads) hist[i] = 0;
+    __syncthreads();
+    if (warp == 0) {
+        lo = scratch[lane];
+        hi = sub[lane];
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, off));
+            hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, off));
+        }
+        if (lane == 0) {
+            mm[0] = lo;
+            mm[1] = hi;
+        }
+    }
+    __syncthreads();
+    lo = mm[0];
+    hi = mm[1];
+    if (lo == hi) {  // all keys equal: the threshold is that key, want of them taken
+        *ties = want;
+        return lo;
+    }
+    const uint32_t range = hi - lo;
+    const int shift = max(0, 32 - __clz(range) - 11);  // range >> shift < 2048
+    for (uint32_t i = tid; i < n; i += kTopkThreads) atomicAdd(&hist[(keys[i] - lo) >> shift], 1u);
+    __syncthreads();
+    find_bin(hist, kBins, want, scratch, found + 1);  // found[1] = b*, found[2] = taken from b*
+    const uint32_t bstar = found[1], within = found[2], cnt = hist[bstar];
+    if (cnt > 32u) {  // too many keys share b*: the radix select
+        __syncthreads();
+        return select_in_smem(keys, n, want, hist, scratch, found, ties);
+    }
+    for (uint32_t i = tid; i < n; i += kTopkThreads) {
+        const uint32_t k = keys[i];
+        if (((k - lo) >> shift) == bstar) sub[atomicAdd(&found[0], 1u)] = k;
+    }
+    __syncthreads();
+    if (warp == 0) {
+        // lane i holds key i of b* (if any); the want-th largest overall is
+        // the within-th largest of b*: the key v with #(> v) < within <= #(>= v)
+        const uint32_t v = lane < (int)cnt ? sub[lane] : 0u;
+        uint32_t gt = 0, ge = 0;
+        for (uint32_t j = 0; j < cnt; ++j) {
+            const uint32_t u = __shfl_sync(0xffffffffu, v, j);
+            gt += u > v;
+            ge += u >= v;
+        }
+        const bool hit = lane < (int)cnt && gt < within && within <= ge;
+        const uint32_t who = __ballot_sync(0xffffffffu, hit);
+        if (lane == __ffs(who) - 1) {
+            mm[0] = v;
+            mm[1] = within - gt;
+        }
+    }
+    __syncthreads();
+    *ties = mm[1];
+    const uint32_t thr = mm[0];
+    __syncthreads();  // mm, sub and found may be reused right after
+    return thr;
+}
+
+// Score of a key (inverse of score_key).
+__device__ __forceinline__ float key_score(uint32_t k) {
+    return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
+}
+
+// A sampling threshold: a key tau with at least r of the n keys >= tau and
+// few more (key 0 marks an empty sample and is never counted).  One pass
+// over a linear binning of the scores' range into 2048 bins (monotone in the
+// score), tau = the smallest key in the bin holding the r-th largest score,
+// so every key of that bin and the bins above is >= tau.  Falls back to the
+// exact radix select when the binning cannot be formed (fewer than r finite
+// scores, all equal).  Every thread calls it; `sub` is 32 words, `mm` 2.
+__device__ uint32_t sample_threshold(const uint32_t *keys, uint32_t n, uint32_t r, uint32_t *hist,
+                                     uint32_t *scratch, uint32_t *found, uint32_t *sub, uint32_t *mm) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    float lo = INFINITY, hi = -INFINITY;
+    for (uint32_t i = tid; i < n; i += kTopkThreads) {
+        const uint32_t k = keys[i];
+        const float x = key_score(k);
+        if (k != 0u && x > -INFINITY && x < INFINITY) {
+            lo = fminf(lo, x);
+            hi = fmaxf(hi, x);
+        }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+        lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, off));
+        hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, off));
+    }
+    if (lane == 0) {
+        scratch[warp] = __float_as_uint(lo);
+        sub[warp] = __float_as_uint(hi);
+    }
+    for (int i = tid; i < kBins; i += kTopkThreads) hist[i] = 0;
+    __syncthreads();
+    if (warp == 0) {
+        lo = __uint_as_float(scratch[lane]);
+        hi = __uint_as_float(sub[lane]);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, off));
+            hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, off));
+        }
+        if (lane == 0) {
+            mm[0] = __float_as_uint(lo);
+            mm[1] = __float_as_uint(hi);
+        }
+    }
+    __syncthreads();
+    lo = __uint_as_float(mm[0]);
+    hi = __uint_as_float(mm[1]);
+    const float scale = (float)kBins / (hi - lo);
+    const bool binned = hi > lo && scale > 0.0f && scale < INFINITY;  // block-uniform
+    auto bin = [&](uint32_t k) -> int {
+        const float x = key_score(k);
+        if (k == 0u || !(x > -INFINITY && x < INFINITY)) return -1;
+        const int b = (int)((x - lo) * scale);
+        return b < kBins - 1 ? b : kBins - 1;
+    };
+    if (binned) {
+        for (uint32_t i = tid; i < n; i += kTopkThreads) {
+            const int b = bin(keys[i]);
+            if (b >= 0) atomicAdd(&hist[b], 1u);
+        }
+        __syncthreads();
+        find_bin(hist, kBins, r, scratch, found);
+    }
+    if (!binned || found[2] < r) {  // block-uniform: the exact select
+        __syncthreads();
+        uint32_t unused;
+        return select_in_smem(keys, n, r, hist, scratch, found, &unused);
+    }
+    const int bstar = (int)found[0];
+    uint32_t kmin = 0xFFFFFFFFu;
+    for (uint32_t i = tid; i < n; i += kTopkThreads) {
+        const uint32_t k = keys[i];
+        if (bin(k) == bstar) kmin = min(kmin, k);
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, off));
+    __syncthreads();  // find_bin's readers of scratch are done
+    if (lane == 0) scratch[warp] = kmin;
+    __syncthreads();
+    if (warp == 0) {
+        kmin = scratch[lane];
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, off));
+        if (lane == 0) mm[0] = kmin;
+    }
+    __syncthreads();
+    const uint32_t tau = mm[0];
+    __syncthreads();  // mm and scratch may be reused right after
+    return tau;
+}
+
 // Write the list from m candidates held in position order: keys above thr,
 // and the first need_eq keys equal to it.
 __device__ void write_from_candidates(const uint32_t *ck, const int32_t *cp, uint32_t m, uint32_t thr,
@@ -484,7 +667,7 @@ __global__ void __launch_bounds__(kTopkThreads, 1) indexer_topk_kernel(const Top
     __shared__ uint64_t full[kRing];
     __shared__ uint32_t hist[kBins];
     __shared__ uint32_t scratch[32], slots_a[32], slots_b[32];
-    __shared__ uint32_t found[3], totals[2];
+    __shared__ uint32_t found[4], totals[2], sub32[32], mm2[2];
     __shared__ float red_lo[kTopkWarps], red_hi[kTopkWarps];
     __shared__ uint32_t ncand, seg_off[kMaxParts + 1];
     __shared__ int last;
@@ -578,55 +761,87 @@ __global__ void __launch_bounds__(kTopkThreads, 1) indexer_topk_kernel(const Top
         const uint32_t r = (uint32_t)min((int64_t)S, (int64_t)topk * S * 5 / (4 * (int64_t)ctx) + 9);
         __syncthreads();
         uint32_t unused;
-        tau = select_in_smem(samp, (uint32_t)nsl * 32, r, hist, scratch, found, &unused);
+        (void)unused;
+        tau = sample_threshold(samp, (uint32_t)nsl * 32, r, hist, scratch, found, sub32, mm2);
     }
 
     // ------------------------------- 2. collect this CTA's candidates
     const int span = ((ctx + P - 1) / P + kChunk - 1) / kChunk * kChunk;
     const int r0 = min(ctx, part * span), r1 = min(ctx, r0 + span);
     uint32_t m = 0;  // candidates found in the range (block-uniform; may pass the cap)
-    ok = stream(r0, r1, [&](const float *buf, int c, int n) {
-        const float4 fa = reinterpret_cast<const float4 *>(buf)[warp * 64 + lane];
-        const float4 fb = reinterpret_cast<const float4 *>(buf)[warp * 64 + 32 + lane];
-        const float v[8] = {fa.x, fa.y, fa.z, fa.w, fb.x, fb.y, fb.z, fb.w};
-        const int pa = warp * 256 + 4 * lane, pb = pa + 128;  // chunk positions of fa.x and fb.x
-        uint32_t fl = 0, ca = 0, cb = 0;
+    // Straight from global memory (the row was just written and sits in L2),
+    // in batches of 16K positions: warp w takes the 512 positions
+    // [b0 + 512w, b0 + 512w + 512) as J = 4 float4 per lane, load j of lane
+    // l covering positions 128j + 4l .. +3 (each load instruction reads 512
+    // contiguous bytes; all of a lane's loads are in flight at once).
+    // Position order inside a warp is (j, lane, element): the per-lane counts
+    // of the four loads, packed 8 bits each into one word, take one warp
+    // scan; one block scan of the warp totals places the warps.  A float4
+    // that starts below r1 lies in the row, which holds ctx rounded up to 4
+    // floats (r0 and span are multiples of 4).
+    {
+        constexpr int J = 4;
+        float4 nx[J];  // the next batch's loads, in flight while this one is scanned
+        auto load_batch = [&](int b0, float4 (&d)[J]) {
+            const int wb = b0 + warp * (32 * 4 * J);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-            const int p = (e < 4 ? pa : pb) + (e & 3);
-            const bool f = p < n && score_key(v[e]) >= tau;
-            fl |= (uint32_t)f << e;
-            if (e < 4) ca += f;
-            else cb += f;
-        }
-        // in position order a warp's 128 "a" positions precede its 128 "b"
-        // positions: scan both counts at once (16 bits each)
-        uint32_t packed = ca | (cb << 16);
+            for (int j = 0; j < J; ++j) {
+                const int p = wb + 128 * j + 4 * lane;
+                d[j] = p < r1 ? __ldcg(reinterpret_cast<const float4 *>(s + p))
+                              : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+            }
+        };
+        if (r0 < r1) load_batch(r0, nx);
+#pragma unroll 1
+        for (int b0 = r0; b0 < r1; b0 += kTopkThreads * 4 * J) {
+            const int wb = b0 + warp * (32 * 4 * J);
+            float4 v4[J];
 #pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-            const uint32_t y = __shfl_up_sync(0xffffffffu, packed, off);
-            if (lane >= off) packed += y;
-        }
-        const uint32_t tot = __shfl_sync(0xffffffffu, packed, 31);
-        const uint32_t a_before = (packed & 0xFFFFu) - ca;
-        const uint32_t b_before = (tot & 0xFFFFu) + (packed >> 16) - cb;
-        const uint32_t wbase = m + warp_excl_scan((tot & 0xFFFFu) + (tot >> 16), slots_a, &totals[0]);
-        if (fl) {
-            uint32_t ia = wbase + a_before, ib = wbase + b_before;
+            for (int j = 0; j < J; ++j) v4[j] = nx[j];
+            if (b0 + kTopkThreads * 4 * J < r1) load_batch(b0 + kTopkThreads * 4 * J, nx);
+            uint32_t sel = 0;  // bit 4j+e: position wb + 128j + 4*lane + e is a candidate
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                if ((fl >> e) & 1u) {
-                    const uint32_t at = e < 4 ? ia++ : ib++;
-                    if (at < (uint32_t)kCandCap) {
-                        cand_key[at] = score_key(v[e]);
-                        cand_pos[at] = r0 + c * kChunk + (e < 4 ? pa : pb) + (e & 3);
+            for (int j = 0; j < J; ++j) {
+                const int p = wb + 128 * j + 4 * lane;
+                sel |= (p + 0 < r1 && score_key(v4[j].x) >= tau ? 1u : 0u) << (4 * j + 0);
+                sel |= (p + 1 < r1 && score_key(v4[j].y) >= tau ? 1u : 0u) << (4 * j + 1);
+                sel |= (p + 2 < r1 && score_key(v4[j].z) >= tau ? 1u : 0u) << (4 * j + 2);
+                sel |= (p + 3 < r1 && score_key(v4[j].w) >= tau ? 1u : 0u) << (4 * j + 3);
+            }
+            uint32_t pc = 0;  // count of load j in byte j (<= 4 per lane, <= 128 per warp)
+#pragma unroll
+            for (int j = 0; j < J; ++j) pc |= (uint32_t)__popc((sel >> (4 * j)) & 0xFu) << (8 * j);
+            uint32_t inc = pc;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const uint32_t y = __shfl_up_sync(0xffffffffu, inc, off);
+                if (lane >= off) inc += y;
+            }
+            const uint32_t tot = __shfl_sync(0xffffffffu, inc, 31);
+            const uint32_t exc = inc - pc;
+            const uint32_t wtot = (tot & 0xFFu) + ((tot >> 8) & 0xFFu) + ((tot >> 16) & 0xFFu) + (tot >> 24);
+            uint32_t at_j = m + warp_excl_scan(wtot, slots_a, &totals[0]);  // first slot of load 0's candidates
+#pragma unroll
+            for (int j = 0; j < J; ++j) {
+                uint32_t at = at_j + ((exc >> (8 * j)) & 0xFFu);
+                const int p = wb + 128 * j + 4 * lane;
+                const float v[4] = {v4[j].x, v4[j].y, v4[j].z, v4[j].w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    if ((sel >> (4 * j + e)) & 1u) {
+                        if (at < (uint32_t)kCandCap) {
+                            cand_key[at] = score_key(v[e]);
+                            cand_pos[at] = p + e;
+                        }
+                        ++at;
                     }
                 }
+                at_j += (tot >> (8 * j)) & 0xFFu;
             }
+            m += totals[0];
         }
-        m += totals[0];
-    });
-    if (!ok) return fail();
+        __syncthreads();  // every thread's candidates are written before anyone reads them
+    }
 
     // ----------------------------- 3. the last CTA of the request selects
     uint32_t mtot = m;
@@ -657,13 +872,26 @@ __global__ void __launch_bounds__(kTopkThreads, 1) indexer_topk_kernel(const Top
         __syncthreads();
         mtot = seg_off[P];
         if (mtot >= (uint32_t)topk && mtot <= (uint32_t)kCandCap) {
-            for (int q = 0; q < P; ++q) {  // concatenate in part order = position order
-                const uint2 *src = a.cand + ((int64_t)t * P + q) * kCandCap;
-                const uint32_t off = seg_off[q], mq = seg_off[q + 1] - off;
-                for (uint32_t i = tid; i < mq; i += kTopkThreads) {
-                    const uint2 kp = __ldcg(src + i);
-                    cand_key[off + i] = kp.x;
-                    cand_pos[off + i] = (int32_t)kp.y;
+            // concatenate in part order = position order; slot i of the
+            // joined list belongs to the part q with seg_off[q] <= i <
+            // seg_off[q + 1], so every load is independent of the others
+            constexpr int kPer = (kCandCap + kTopkThreads - 1) / kTopkThreads;
+            uint2 kp[kPer];
+#pragma unroll
+            for (int k = 0; k < kPer; ++k) {
+                const uint32_t i = tid + (uint32_t)k * kTopkThreads;
+                if (i < mtot) {
+                    int q = 0;
+                    while (q + 1 < P && seg_off[q + 1] <= i) ++q;
+                    kp[k] = __ldcg(a.cand + ((int64_t)t * P + q) * kCandCap + (i - seg_off[q]));
+                }
+            }
+#pragma unroll
+            for (int k = 0; k < kPer; ++k) {
+                const uint32_t i = tid + (uint32_t)k * kTopkThreads;
+                if (i < mtot) {
+                    cand_key[i] = kp[k].x;
+                    cand_pos[i] = (int32_t)kp[k].y;
                 }
             }
             __syncthreads();
@@ -671,7 +899,7 @@ __global__ void __launch_bounds__(kTopkThreads, 1) indexer_topk_kernel(const Top
     }
     if (mtot >= (uint32_t)topk && mtot <= (uint32_t)kCandCap) {
         uint32_t need_eq;
-        const uint32_t thr = select_in_smem(cand_key, mtot, (uint32_t)topk, hist, scratch, found, &need_eq);
+        const uint32_t thr = select_fast(cand_key, mtot, (uint32_t)topk, hist, scratch, found, &need_eq, sub32, mm2);
         write_from_candidates(cand_key, cand_pos, mtot, thr, need_eq, o, scratch);
         return;
     }

@@ -64,3 +64,22 @@ def check_close(out: torch.Tensor, lse: torch.Tensor, ref_out: np.ndarray, ref_l
     assert not np.any(np.isnan(lerr)), "lse: one side -inf, the other finite" 
     assert np.all(lerr <= lse_tol), "lse mismatch: max %.3g" % np.nanmax(lerr)
     return worst, float(lerr.max())
+
+
+def translate(positions: np.ndarray, table: np.ndarray, page: int, num_slots: int) -> np.ndarray:
+    """Plain definition: slot = table[t, pos // page] * page + pos % page;
+    -1, out-of-range positions and missing pages give -1."""
+    T, K = positions.shape
+    out = np.full((T, K), -1, dtype=np.int64)
+    for t in range(T):
+        for j in range(K):
+            p = int(positions[t, j])
+            if p < 0 or p >= table.shape[1] * page:
+                continue
+            blk = int(table[t, p // page])
+            if blk < 0:
+                continue
+            slot = blk * page + p % page
+            if slot < num_slots:
+                out[t, j] = slot
+    return out

@@ -204,9 +204,13 @@ def test_sparse_indexer_short_and_ragged_contexts():
 
 
 def test_indexer_lists_feed_the_paged_decode():
-    # the indexer's positions are the paged decode's input as they stand
+    # the indexer's positions are the paged decode's input as they stand: the
+    # list is a valid top-k of the oracle's scores, and the decode over it
+    # matches the oracle's decode over the same positions, translated to
+    # slots through the block table by the plain definition
     w = synth.decode35("cuda", T=4, ctx=20000)
     from nvfp4_sparse_mla_decode_b200.cache import build_cache
+    from harness import check_close, oracle_decode, translate
     cache = build_cache(w)
     table = synth.block_table(w)
     keys = synth.indexer_keys(w.num_slots, 81, "cuda")
@@ -218,4 +222,12 @@ def test_indexer_lists_feed_the_paged_decode():
                                dev_status=status)
     torch.cuda.synchronize()
     assert int(status.item()) == 0
-    assert torch.all(torch.isfinite(lse)) and torch.all(torch.isfinite(out.float()))
+    pos_h = pos.cpu().numpy()
+    ref, mag = indexer.indexer_scores(q.cpu().numpy(), wt.cpu().numpy(), keys.cpu().numpy(), table.cpu().numpy(),
+                                      list(w.ctx_lens), synth.PAGE_SIZE, magnitude=True)
+    for t in range(w.T):
+        _valid_topk(pos_h[t], ref[t], mag[t], w.ctx_lens[t], 2048)
+    slots = translate(pos_h, table.cpu().numpy(), synth.PAGE_SIZE, w.num_slots)
+    w.indices = torch.from_numpy(slots.astype(np.int32)).to("cuda")
+    ref_o, ref_l = oracle_decode(w, range(w.T))
+    check_close(out, lse, ref_o, ref_l)

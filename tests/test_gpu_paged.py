@@ -8,29 +8,10 @@ import torch
 
 import nvfp4_sparse_mla_decode_b200 as nv
 from nvfp4_sparse_mla_decode_b200 import synth
-from harness import build_cache, check_close, oracle_decode
+from harness import build_cache, check_close, oracle_decode, translate
 
 pytestmark = pytest.mark.gpu
 PAGE = synth.PAGE_SIZE
-
-
-def translate(positions: np.ndarray, table: np.ndarray, page: int, num_slots: int) -> np.ndarray:
-    """Plain definition: slot = table[t, pos // page] * page + pos % page;
-    -1, out-of-range positions and missing pages give -1."""
-    T, K = positions.shape
-    out = np.full((T, K), -1, dtype=np.int64)
-    for t in range(T):
-        for j in range(K):
-            p = int(positions[t, j])
-            if p < 0 or p >= table.shape[1] * page:
-                continue
-            blk = int(table[t, p // page])
-            if blk < 0:
-                continue
-            slot = blk * page + p % page
-            if slot < num_slots:
-                out[t, j] = slot
-    return out
 
 
 def run_paged(w, cache, positions, table, page):
