@@ -47,6 +47,9 @@ def parse():
                              "blhnc", "all-others"],
                     help="decode35x64 (default) prints the one result line; the others time the remaining "
                          "workloads and print one line per shape")
+    ap.add_argument("--ctx", type=int, default=140_000,
+                    help="context rows per request of the decode35x64 leg (smaller values give a small case "
+                         "of the same kernel, e.g. for a profiler capture)")
     ap.add_argument("--layers", type=int, default=64,
                     help="layers of the request converted by --workload blhnc")
     ap.add_argument("--launch", default="graph", choices=["graph", "stream"],
@@ -707,7 +710,7 @@ def main():
     nv.lib()  # fails loudly if the library is missing
 
     # ------------------------------------------------------------ workload
-    w = synth.decode35("cuda", seed=1 + 1000 * rank)
+    w = synth.decode35("cuda", seed=1 + 1000 * rank, ctx=args.ctx)
     from nvfp4_sparse_mla_decode_b200.cache import build_cache
     t_build = time.perf_counter()
     cache = build_cache(w)
@@ -794,7 +797,7 @@ def main():
         "metric": METRIC, "value": tflops, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f16", "data": "synthetic",
-        "config": {"workload": "decode35x64", "T": T, "H": H, "topk": topk, "ctx_rows": 140000,
+        "config": {"workload": "decode35x64", "T": T, "H": H, "topk": topk, "ctx_rows": args.ctx,
                    "cache_rows": w.num_slots, "valid_rows_per_launch": rows, "splits": nv.num_splits(T, H, topk),
                    "l2": "inputs larger than L2: %d rotating index/query sets, %.0f MB gathered per cycle > %d MB L2"
                          % (N_SETS, N_SETS * rows * ROW_BYTES / 1e6, L2_BYTES >> 20),
