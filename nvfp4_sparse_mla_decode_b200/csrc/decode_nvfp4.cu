@@ -114,6 +114,9 @@ static_assert(kOffMergeW + (16 * kMaxHG + kMaxHG) * 4 <= kOffIdx, "merge areas m
 static_assert(kOffPartial % 128 == 0 && kOffMergeW % 16 == 0, "merge areas take tensor copies and 16-byte accesses");
 static_assert(kMaxHG * kLatent * 2 <= kOffIdx - kOffStage, "output staging must fit over the rings");
 constexpr int kThreads = 768;
+// the first tile's rows are copied by the gather warps and the eight V-unpack
+// warps together (the V warps have nothing to do until those rows land)
+constexpr int kTile0Threads = 64 + 256;
 constexpr int kKWarp0 = 4;
 constexpr int kSoftWarp0 = 12;
 constexpr int kVWarp0 = 16;
@@ -143,8 +146,9 @@ constexpr int BAR_PV_DONE = BAR_P_FULL + 1;             // output MMAs of a tile
 constexpr int BAR_DRAIN = BAR_PV_DONE + 1;              // every score MMA issued so far done
 constexpr int BAR_S_FREE = BAR_DRAIN + 1;               // [2] softmax done reading an S buffer (4 softmax warps)
 constexpr int BAR_DRAIN_PV = BAR_S_FREE + 2;            // every output MMA issued so far done
-constexpr int BAR_ROWS0 = BAR_DRAIN_PV + 1;             // the first tile's rows landed (cp.async arrivals of 64 threads)
-constexpr int kBarsUsed = BAR_ROWS0 + 1;
+constexpr int BAR_ROWS0 = BAR_DRAIN_PV + 1;             // the first tile's rows landed (cp.async arrivals of kTile0Threads)
+constexpr int BAR_K0DONE = BAR_ROWS0 + 1;              // the first tile's K unpacked (8 K-unpack warps)
+constexpr int kBarsUsed = BAR_K0DONE + 1;
 static_assert(kBarsUsed <= kNumBars, "barrier slots");
 
 constexpr uint32_t kTmemCols = 512;
@@ -398,7 +402,9 @@ __global__ void __launch_bounds__(nv4::kThreads, 1)
     if (warp == 1 && lane == 0) {
         for (int b = 0; b < kBarsUsed; ++b) {
             uint32_t count = 1;
-            if ((b >= BAR_RAW_FULL && b < BAR_RAW_FULL + kRawSlots) || b == BAR_ROWS0) count = 64;  // cp.async arrivals
+            if (b >= BAR_RAW_FULL && b < BAR_RAW_FULL + kRawSlots) count = 64;  // cp.async arrivals
+            else if (b == BAR_ROWS0) count = kTile0Threads;
+            else if (b == BAR_K0DONE) count = 8;
             else if (b >= BAR_RAW_FREE && b < BAR_RAW_FREE + kRawSlots) count = 8;
             else if (b >= BAR_K_FULL && b < BAR_K_FULL + kKSlots) count = 4;
             else if (b >= BAR_V_FULL && b < BAR_V_FULL + kVSlots) count = 4;
@@ -610,8 +616,10 @@ __global__ void __launch_bounds__(nv4::kThreads, 1)
                 uint8_t *dst = smem + kOffRaw + slot * kRawSlotBytes;
                 const int32_t *ids = idx_s + kTileRows * j;
                 const int items = nrows * (kRowBytes / 16);
+                // the first tile is shared with the V warps (items gt, gt + 320, ...)
+                const int step = j == 0 ? kTile0Threads : 64;
 #pragma unroll 4
-                for (int it = gt; it < items; it += 64) {
+                for (int it = gt; it < items; it += step) {
                     const int r = it / (kRowBytes / 16), k = it - r * (kRowBytes / 16);
                     cp_async16(dst + r * kRawStride + 16 * k, a.src + (int64_t)ids[r] * kRowBytes + 16 * k);
                 }
@@ -635,7 +643,12 @@ __global__ void __launch_bounds__(nv4::kThreads, 1)
         bool ok = true;
         for (int j = 0; j < ntiles && ok; ++j) {
             const int rslot = j % kRawSlots;
-            if (!warp_wait(&bars[BAR_RAW_FULL + rslot], (j / kRawSlots) & 1, a.wait_cycles)) {
+            // the first tile's rows are complete once all kTile0Threads
+            // copiers' copies have landed (ROWS0); RAW_FULL's first phase
+            // tracks only the gather warps' share and nobody waits on it
+            const bool landed = j == 0 ? warp_wait(&bars[BAR_ROWS0], 0, a.wait_cycles)
+                                       : warp_wait(&bars[BAR_RAW_FULL + rslot], (j / kRawSlots) & 1, a.wait_cycles);
+            if (!landed) {
                 ok = false;
                 break;
             }
@@ -685,6 +698,7 @@ __global__ void __launch_bounds__(nv4::kThreads, 1)
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars[BAR_RAW_FREE + rslot]);
+            if (j == 0 && lane == 0) mbar_arrive(&bars[BAR_K0DONE]);
             if (kw == 0 && lane == 0 && j < 8) TRACE(110 + j);
         }
         if (!ok && lane == 0 && a.dev_status) atomicOr(a.dev_status, NVFP4MLA_DEV_TIMEOUT);
@@ -720,9 +734,11 @@ __global__ void __launch_bounds__(nv4::kThreads, 1)
             tc_fence_after();
             const uint32_t s_addr = tmem + lane_base + kColS + 64u * (uint32_t)(j & 1);
             const bool valid = st < tile_rows(j);
-            bool need = false;
+            // the first tile always moves every reference max (they start at
+            // -inf), so only later tiles read the scores for the check
+            bool need = j == 0;
 #pragma unroll
-            for (int c0 = 0; c0 < HG; c0 += HC) {
+            for (int c0 = 0; c0 < (j > 0 ? HG : 0); c0 += HC) {
                 uint32_t rs[HC];
                 tmem_ld_cols<HC>(s_addr + c0, rs);
                 tmem_ld_wait();
@@ -948,6 +964,16 @@ __global__ void __launch_bounds__(nv4::kThreads, 1)
         // swizzled by the row.  Thread = (row r, dv group dg); the rows are
         // read from L2 (the gather brought them in a tile earlier).
         if (kRegsV < kRegsLaunch) regs_dec<kRegsV < kRegsLaunch ? kRegsV : kRegsLaunch - 8>();
+        if (ntiles > 0) {  // this thread's share of the first tile's row copies (items 64 + v, 64 + v + 320, ...)
+            const int items = tile_rows(0) * (kRowBytes / 16);
+            uint8_t *dst = smem + kOffRaw;
+#pragma unroll 4
+            for (int it = 64 + (tid - 32 * kVWarp0); it < items; it += kTile0Threads) {
+                const int r = it / (kRowBytes / 16), k = it - r * (kRowBytes / 16);
+                cp_async16(dst + r * kRawStride + 16 * k, a.src + (int64_t)idx_s[r] * kRowBytes + 16 * k);
+            }
+            cp_async_mbar_arrive(&bars[BAR_ROWS0]);
+        }
         const int vs = (warp - kVWarp0) >> 2;  // V set: 0 or 1
         const int vw = (warp - kVWarp0) & 3;
         const int r = lane & 15;
@@ -956,14 +982,15 @@ __global__ void __launch_bounds__(nv4::kThreads, 1)
         uint32_t vn = (uint32_t)vs;  // ring position of this set's next group (groups alternate sets)
         for (int j = 0; j < ntiles && ok; ++j) {
             // Rows are read once they are in L2, which also keeps these loads
-            // from racing the gather to HBM: the first tile's once its copies
-            // have landed (a barrier that completes only once), later tiles'
-            // once the softmax has read their scores.  (S_FREE, unlike S_FULL
-            // or the raw ring, cannot complete this buffer's next phase, tile
-            // j + 2, before these warps finish tile j: the softmax reaches
-            // tile j + 2 only after the output MMAs of tile j, which need
-            // every V group of it.)
-            const bool rows_in = j == 0 ? warp_wait(&bars[BAR_ROWS0], 0, a.wait_cycles)
+            // from racing the gather to HBM: the first tile's once its K has
+            // been unpacked (a barrier that completes only once; V is needed
+            // only after the tile's scores, and starting earlier would take
+            // issue slots from that unpack), later tiles' once the softmax has
+            // read their scores.  (S_FREE, unlike S_FULL or the raw ring,
+            // cannot complete this buffer's next phase, tile j + 2, before
+            // these warps finish tile j: the softmax reaches tile j + 2 only
+            // after the output MMAs of tile j, which need every V group of it.)
+            const bool rows_in = j == 0 ? warp_wait(&bars[BAR_K0DONE], 0, a.wait_cycles)
                                         : warp_wait(&bars[BAR_S_FREE + (j & 1)], (j >> 1) & 1, a.wait_cycles);
             if (!rows_in) {
                 ok = false;
@@ -1021,6 +1048,7 @@ __global__ void __launch_bounds__(nv4::kThreads, 1)
             }
             if (vs == 0 && vw == 0 && lane == 0 && j < 8) TRACE(160 + j);
         }
+        asm volatile("cp.async.wait_all;" ::: "memory");  // its first-tile copies land before the CTA may exit
         if (!ok && lane == 0 && a.dev_status) atomicOr(a.dev_status, NVFP4MLA_DEV_TIMEOUT);
     }
 
