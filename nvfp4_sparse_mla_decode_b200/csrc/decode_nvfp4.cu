@@ -432,23 +432,36 @@ __global__ void __launch_bounds__(nv4::kThreads, 1)
     int32_t vals[4];
     uint32_t bal[4];
     bool bad = false;
+    // all of a thread's list loads (and then its block-table loads) are in
+    // flight together; entries 512k + tid, warps 16.. hold none (p >= 2048)
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
-        const int p = tid + 512 * k;  // warps 16.. hold no list entries (p >= 2048)
-        int32_t v = (p < a.topk && tid < 512) ? __ldg(lst + p) : -1;
-        bool entry_bad = false;
-        if (a.block_table && v >= 0) {  // request-local position -> slot through the block table
-            int64_t slot = -1;
-            if ((int64_t)v < a.max_pos) {
-                const int32_t blk = __ldg(a.block_table + (int64_t)t * a.table_stride + (v >> a.page_shift));
-                if (blk >= 0) slot = ((int64_t)blk << a.page_shift) + (v & ((1 << a.page_shift) - 1));
-            }
-            entry_bad = slot < 0 || slot >= a.num_slots;
-            v = entry_bad ? -1 : (int32_t)slot;
+        const int p = tid + 512 * k;
+        vals[k] = (p < a.topk && tid < 512) ? __ldg(lst + p) : -1;
+    }
+    bool entry_bad[4] = {false, false, false, false};
+    if (a.block_table) {  // request-local position -> slot through the block table
+        int32_t blk[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+            blk[k] = (vals[k] >= 0 && (int64_t)vals[k] < a.max_pos)
+                         ? __ldg(a.block_table + (int64_t)t * a.table_stride + (vals[k] >> a.page_shift))
+                         : -1;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            if (vals[k] < 0) continue;
+            const int64_t slot = blk[k] >= 0 ? ((int64_t)blk[k] << a.page_shift) + (vals[k] & ((1 << a.page_shift) - 1))
+                                             : -1;
+            entry_bad[k] = slot < 0 || slot >= a.num_slots;
+            vals[k] = entry_bad[k] ? -1 : (int32_t)slot;
         }
+    }
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const int p = tid + 512 * k;
+        const int32_t v = vals[k];
         const bool ok = v >= 0 && (int64_t)v < a.num_slots;
-        bad |= (p < a.topk) && (entry_bad || v < -1 || (int64_t)v >= a.num_slots);
-        vals[k] = v;
+        bad |= (p < a.topk) && (entry_bad[k] || v < -1 || (int64_t)v >= a.num_slots);
         bal[k] = __ballot_sync(0xffffffffu, ok);
         if (lane == 0 && warp < 16) cnt_s[k * 16 + warp] = __popc(bal[k]);
     }
