@@ -750,14 +750,14 @@ __global__ void __launch_bounds__(nv4::kThreads, 1)
             // the first tile always moves every reference max (they start at
             // -inf), so only later tiles read the scores for the check
             bool need = j == 0;
+            if (j > 0) {
+                uint32_t rs[HG];  // every score of the row: all loads in flight, one wait
 #pragma unroll
-            for (int c0 = 0; c0 < (j > 0 ? HG : 0); c0 += HC) {
-                uint32_t rs[HC];
-                tmem_ld_cols<HC>(s_addr + c0, rs);
+                for (int c0 = 0; c0 < HG; c0 += HC) tmem_ld_cols<HC>(s_addr + c0, *reinterpret_cast<uint32_t(*)[HC]>(rs + c0));
                 tmem_ld_wait();
 #pragma unroll
-                for (int h = 0; h < HC; h += 4) {
-                    const float4 m4 = *reinterpret_cast<const float4 *>(m_s + c0 + h);
+                for (int h = 0; h < HG; h += 4) {
+                    const float4 m4 = *reinterpret_cast<const float4 *>(m_s + h);
                     need |= __uint_as_float(rs[h + 0]) * a.scale_log2 > m4.x + kRescaleThreshold;
                     need |= __uint_as_float(rs[h + 1]) * a.scale_log2 > m4.y + kRescaleThreshold;
                     need |= __uint_as_float(rs[h + 2]) * a.scale_log2 > m4.z + kRescaleThreshold;
@@ -766,14 +766,15 @@ __global__ void __launch_bounds__(nv4::kThreads, 1)
             }
             const bool rescale = named_bar_or(1, 128, valid && need);
             if (rescale) {
+                uint32_t rsa[HG];  // every score of the row: all loads in flight, one wait
+#pragma unroll
+                for (int c0 = 0; c0 < HG; c0 += 16) tmem_ld16(s_addr + c0, *reinterpret_cast<uint32_t(*)[16]>(rsa + c0));
+                tmem_ld_wait();
 #pragma unroll
                 for (int c0 = 0; c0 < HG; c0 += 16) {  // column max, 16 heads at a time
-                    uint32_t rs[16];
-                    tmem_ld16(s_addr + c0, rs);
-                    tmem_ld_wait();
                     float mx[16];
 #pragma unroll
-                    for (int h = 0; h < 16; ++h) mx[h] = valid ? __uint_as_float(rs[h]) * a.scale_log2 : -INFINITY;
+                    for (int h = 0; h < 16; ++h) mx[h] = valid ? __uint_as_float(rsa[c0 + h]) * a.scale_log2 : -INFINITY;
                     warp_transpose_reduce<16, true>(mx, lane);
                     if (!(lane & 1)) red_s[wq * 64 + c0 + transposed_col<16>(lane, 0)] = mx[0];
                 }
@@ -795,13 +796,15 @@ __global__ void __launch_bounds__(nv4::kThreads, 1)
             // output MMAs of the previous tile may still run; only the P^T
             // stores (and a rare O^T rescale) wait for those to finish.
             uint32_t pk[HG / 2];
+            uint32_t rsp[HG];  // every score of the row: all loads in flight, one wait
+#pragma unroll
+            for (int c0 = 0; c0 < HG; c0 += HC) tmem_ld_cols<HC>(s_addr + c0, *reinterpret_cast<uint32_t(*)[HC]>(rsp + c0));
+            tmem_ld_wait();
 #pragma unroll
             for (int c0 = 0; c0 < HG; c0 += HC) {
                 float pv[HC];
                 {
-                    uint32_t rs[HC];
-                    tmem_ld_cols<HC>(s_addr + c0, rs);
-                    tmem_ld_wait();
+                    const uint32_t *rs = rsp + c0;
 #pragma unroll
                     for (int h = 0; h < HC; h += 4) {
                         const float4 m4 = *reinterpret_cast<const float4 *>(m_s + c0 + h);
