@@ -117,6 +117,10 @@ constexpr int kThreads = 768;
 // the first tile's rows are copied by the gather warps and the eight V-unpack
 // warps together (the V warps have nothing to do until those rows land)
 constexpr int kTile0Threads = 64 + 256;
+// the split merge's combine runs on the softmax and V-unpack threads, which
+// meet at named barrier kMergeBar (barrier 1 is the softmax warps' own)
+constexpr int kCombineThreads = 128 + 256;
+constexpr int kMergeBar = 2;
 constexpr int kKWarp0 = 4;
 constexpr int kSoftWarp0 = 12;
 constexpr int kVWarp0 = 16;
@@ -194,6 +198,84 @@ __device__ __forceinline__ void unpack_latent64(uint4 w0, uint4 w1, uint32_t sca
             o[8 * k + 4 + i] = hmul2_u32(hi[i], s2);
         }
     }
+}
+
+// The combine of the split merge, run by kCombineThreads threads (the 128
+// softmax threads and the 256 V-unpack threads, which are idle by then);
+// ct = 0 .. kCombineThreads-1.  The rows of every split's partial for this
+// CTA's dv slice are in the shared boxes, the weights in w_s and inv_den.
+template <int HG, int S>
+__device__ __forceinline__ void merge_combine(const DecodeArgs &a, int t, int g, int split, const uint8_t *smem,
+                                              int ct) {
+    using namespace nv4;
+    constexpr int NQ = HG / 4;
+    constexpr int D = kLatent / S;
+    constexpr int C = D < 64 ? D : 64;
+    constexpr int box_bytes = D * HG * 4;
+    const float *w_s = reinterpret_cast<const float *>(smem + kOffMergeW);
+    const float *inv_den = w_s + kMaxSplits * HG;
+    __half *dst = a.out + ((int64_t)t * a.H + (int64_t)g * HG) * kLatent + split * D;
+    // item = (piece q, dv d): neighbouring threads take neighbouring dv, so
+    // the box reads are conflict-free; neighbouring lanes then swap halves
+    // so that each stores two adjacent dv of one head (4 bytes; a warp store
+    // covers 32 consecutive dv of two heads)
+    const float *boxes = reinterpret_cast<const float *>(smem + kOffPartial);
+    const bool odd = ct & 1;
+    constexpr int kAll = D * NQ;  // even, so the two lanes of a pair are both in range or both out
+    constexpr int kRounds = (kAll + kCombineThreads - 1) / kCombineThreads;
+#pragma unroll 2
+    for (int k = 0; k < kRounds; ++k) {
+        const int item0 = ct + kCombineThreads * k;
+        const bool in = item0 < kAll;
+        const int item = in ? item0 : kAll - 1;  // out-of-range lanes still take part in the swap
+        const int q = item / D, d = item - q * D;
+        const int c = d / C, dd = d - c * C;
+        const int off = c * (NQ * C * 4) + (q * C + dd) * 4;  // floats, within a box
+        float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+#pragma unroll
+        for (int s = 0; s < S; ++s) {
+            const float4 v = *reinterpret_cast<const float4 *>(boxes + s * (box_bytes / 4) + off);
+            const float4 w = *reinterpret_cast<const float4 *>(w_s + s * HG + 4 * q);
+            acc.x += w.x * v.x;
+            acc.y += w.y * v.y;
+            acc.z += w.z * v.z;
+            acc.w += w.w * v.w;
+        }
+        const float4 r = *reinterpret_cast<const float4 *>(inv_den + 4 * q);
+        acc.x *= r.x;
+        acc.y *= r.y;
+        acc.z *= r.z;
+        acc.w *= r.w;
+        // even lane keeps heads 4q, 4q+1 and takes its neighbour's; odd lane
+        // keeps heads 4q+2, 4q+3 and takes its neighbour's
+        const float s0 = odd ? acc.x : acc.z, s1 = odd ? acc.y : acc.w;
+        const float r0 = __shfl_xor_sync(0xffffffffu, s0, 1), r1 = __shfl_xor_sync(0xffffffffu, s1, 1);
+        const float k0 = odd ? acc.z : acc.x, k1 = odd ? acc.w : acc.y;
+        const int h = 4 * q + (odd ? 2 : 0);
+        const int de = d & ~1;  // the pair's even dv
+        // (own value, neighbour's value) in dv order
+        const __half2 p0 = odd ? __floats2half2_rn(r0, k0) : __floats2half2_rn(k0, r0);
+        const __half2 p1 = odd ? __floats2half2_rn(r1, k1) : __floats2half2_rn(k1, r1);
+        if (in) {
+            *reinterpret_cast<__half2 *>(dst + (int64_t)h * kLatent + de) = p0;
+            *reinterpret_cast<__half2 *>(dst + (int64_t)(h + 1) * kLatent + de) = p1;
+        }
+    }
+}
+
+// The V-unpack threads' part in the split merge (vt = 0..255): they meet the
+// softmax threads at the merge's named barriers and take items 128 + vt, ...
+// of the combine.
+template <int HG, int S>
+__device__ __forceinline__ void merge_join_v(const DecodeArgs &a, int t, int g, int split, const uint8_t *smem,
+                                             int vt) {
+    using namespace nv4;
+    const uint32_t *flag = reinterpret_cast<const uint32_t *>(smem + kOffMisc) + 1;
+    named_bar(kMergeBar, kCombineThreads);  // the arrival wait is over and *flag set
+    if (!*flag) return;                     // poisoned: the softmax threads write NaN
+    named_bar(kMergeBar, kCombineThreads);  // weights computed, the other splits' rows landed
+    merge_combine<HG, S>(a, t, g, split, smem, 128 + vt);
+    named_bar(kMergeBar, kCombineThreads);
 }
 
 // Split merge, run by the 128 softmax threads of each of the S CTAs of a
@@ -280,7 +362,7 @@ __device__ __forceinline__ void merge_splits_nv4(const DecodeArgs &a, const CUte
         *flag = ok ? 1u : 0u;
         TRACE(192);
     }
-    named_bar(1, kMergeThreads);
+    named_bar(kMergeBar, kCombineThreads);  // with the V-unpack threads (merge_join_v)
     __half *dst = a.out + ((int64_t)t * a.H + (int64_t)g * HG) * kLatent + dv0;
     if (!*flag) {  // poisoned: make the failure visible in the output
         for (int item = mt; item < HG * D; item += kMergeThreads) {
@@ -313,51 +395,10 @@ __device__ __forceinline__ void merge_splits_nv4(const DecodeArgs &a, const CUte
     }
     const bool landed = mbar_wait(bar, 1, a.wait_cycles);  // the tensor copies (phase 1 of the Q barrier)
     if (!landed && a.dev_status) atomicOr(a.dev_status, NVFP4MLA_DEV_TIMEOUT);
-    named_bar(1, kMergeThreads);
+    named_bar(kMergeBar, kCombineThreads);
     if (mt == 0) TRACE(193);
-    // item = (piece q, dv d): neighbouring threads take neighbouring dv, so
-    // the box reads are conflict-free; neighbouring lanes then swap halves
-    // so that each stores two adjacent dv of one head (4 bytes; a warp store
-    // covers 32 consecutive dv of two heads)
-    const float *boxes = reinterpret_cast<const float *>(smem + kOffPartial);
-    const bool odd = mt & 1;
-    constexpr int kItems = D * NQ / kMergeThreads;  // D * NQ is a multiple of 128
-    static_assert(D * NQ % kMergeThreads == 0, "merge items per thread");
-#pragma unroll 2
-    for (int k = 0; k < kItems; ++k) {
-        const int item = mt + kMergeThreads * k;
-        const int q = item / D, d = item - q * D;
-        const int c = d / C, dd = d - c * C;
-        const int off = c * (NQ * C * 4) + (q * C + dd) * 4;  // floats, within a box
-        float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-#pragma unroll
-        for (int s = 0; s < S; ++s) {
-            const float4 v = *reinterpret_cast<const float4 *>(boxes + s * (box_bytes / 4) + off);
-            const float4 w = *reinterpret_cast<const float4 *>(w_s + s * HG + 4 * q);
-            acc.x += w.x * v.x;
-            acc.y += w.y * v.y;
-            acc.z += w.z * v.z;
-            acc.w += w.w * v.w;
-        }
-        const float4 r = *reinterpret_cast<const float4 *>(inv_den + 4 * q);
-        acc.x *= r.x;
-        acc.y *= r.y;
-        acc.z *= r.z;
-        acc.w *= r.w;
-        // even lane keeps heads 4q, 4q+1 and takes its neighbour's; odd lane
-        // keeps heads 4q+2, 4q+3 and takes its neighbour's
-        const float s0 = odd ? acc.x : acc.z, s1 = odd ? acc.y : acc.w;
-        const float r0 = __shfl_xor_sync(0xffffffffu, s0, 1), r1 = __shfl_xor_sync(0xffffffffu, s1, 1);
-        const float k0 = odd ? acc.z : acc.x, k1 = odd ? acc.w : acc.y;
-        const int h = 4 * q + (odd ? 2 : 0);
-        const int de = d & ~1;  // the pair's even dv
-        // (own value, neighbour's value) in dv order
-        const __half2 p0 = odd ? __floats2half2_rn(r0, k0) : __floats2half2_rn(k0, r0);
-        const __half2 p1 = odd ? __floats2half2_rn(r1, k1) : __floats2half2_rn(k1, r1);
-        *reinterpret_cast<__half2 *>(dst + (int64_t)h * kLatent + de) = p0;
-        *reinterpret_cast<__half2 *>(dst + (int64_t)(h + 1) * kLatent + de) = p1;
-    }
-    named_bar(1, kMergeThreads);
+    merge_combine<HG, S>(a, t, g, split, smem, mt);
+    named_bar(kMergeBar, kCombineThreads);
     if (mt == 0) {
         TRACE(194);
         const uint32_t old = atomicAdd(depart, 1u);
@@ -1066,6 +1107,14 @@ __global__ void __launch_bounds__(nv4::kThreads, 1)
         }
         asm volatile("cp.async.wait_all;" ::: "memory");  // its first-tile copies land before the CTA may exit
         if (!ok && lane == 0 && a.dev_status) atomicOr(a.dev_status, NVFP4MLA_DEV_TIMEOUT);
+        const int vt = tid - 32 * kVWarp0;
+        switch (a.S) {  // the split merge's combine (the softmax warps run the rest of it)
+            case 1: break;
+            case 2: merge_join_v<HG, 2>(a, t, g, split, smem, vt); break;
+            case 4: merge_join_v<HG, 4>(a, t, g, split, smem, vt); break;
+            case 8: merge_join_v<HG, 8>(a, t, g, split, smem, vt); break;
+            default: merge_join_v<HG, 16>(a, t, g, split, smem, vt); break;
+        }
     }
 
     // ---------------------------------------------------------------- teardown
