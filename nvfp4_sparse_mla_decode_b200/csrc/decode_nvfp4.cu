@@ -85,7 +85,6 @@ constexpr int kVRows = 16;                                 // rows per V ring sl
 constexpr int kVSlotBytes = kVRows * kLatent * 2;          // 16384
 constexpr int kVSlots = 2;                                 // V ring depth
 constexpr int kRawSlots = 2;                               // raw tiles in shared memory
-constexpr int kPrefetchAhead = 0;                          // tiles brought into L2 ahead of their copy (0: none)
 constexpr int kVGroups = kTileRows / kVRows;               // 8
 constexpr int kKChunks = 9;                                // 8 latent chunks of 64 dims + RoPE
 constexpr int kKSlots = 4;
@@ -647,20 +646,7 @@ __global__ void __launch_bounds__(nv4::kThreads, 1)
             // own copies have landed.
             const int gt = (warp == 1 ? 0 : 32) + lane;
             bool ok = true;
-            // rows of the first tiles go to L2 at once; later tiles are
-            // prefetched kPrefetchAhead tiles ahead of their copy, so the copy
-            // into the (single) raw slot costs an L2 round trip, not HBM's
-            auto prefetch_tile = [&](int jt) {  // every 128-byte line a row touches (4 probes cover 352 bytes)
-                const int32_t *pids = idx_s + kTileRows * jt;
-                const int n = tile_rows(jt) * 4;
-                for (int it = gt; it < n; it += 64) {
-                    const int r = it >> 2, q = it & 3;
-                    prefetch_l2(a.src + (int64_t)pids[r] * kRowBytes + (q < 3 ? 128 * q : kRowBytes - 1));
-                }
-            };
-            for (int jt = 0; jt < kPrefetchAhead && jt < ntiles; ++jt) prefetch_tile(jt);
             for (int j = 0; j < ntiles; ++j) {
-                if (kPrefetchAhead > 0 && j + kPrefetchAhead < ntiles) prefetch_tile(j + kPrefetchAhead);
                 const int slot = j % kRawSlots;
                 if (j >= kRawSlots && !warp_wait(&bars[BAR_RAW_FREE + slot], ((j / kRawSlots) - 1) & 1, a.wait_cycles)) {
                     ok = false;

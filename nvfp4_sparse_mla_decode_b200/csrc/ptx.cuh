@@ -106,19 +106,6 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const void *tmap, int32_t
         : "memory");
 }
 
-// Tiled 2-D tensor copy from this CTA's shared memory to global memory
-// (bulk-group completion; see bulk_commit_wait_all / bulk_commit_wait_read).
-__device__ __forceinline__ void tma_store_2d(const void *tmap, const void *src, int32_t x, int32_t y) {
-    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
-                     reinterpret_cast<uint64_t>(tmap)),
-                 "r"(smem_u32(src)), "r"(x), "r"(y)
-                 : "memory");
-}
-// Commit the bulk copies issued so far and wait until they have completed
-// (their global writes done, not only their shared-memory reads).
-__device__ __forceinline__ void bulk_commit_wait_all() {
-    asm volatile("cp.async.bulk.commit_group;\n\tcp.async.bulk.wait_group 0;" ::: "memory");
-}
 // Order this thread's async-proxy accesses to global memory with its generic
 // ones (both directions), e.g. between tensor copies and a release/acquire.
 __device__ __forceinline__ void fence_proxy_async_global() {
@@ -138,13 +125,6 @@ __device__ __forceinline__ void cp_async_mbar_arrive(uint64_t *bar) {
 }
 __device__ __forceinline__ void cp_async_wait_all() {
     asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
-}
-// Bulk prefetch of `bytes` (multiple of 16, 16-byte aligned) into L2.
-__device__ __forceinline__ void bulk_prefetch_l2(const void *src, uint32_t bytes) {
-    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
-}
-__device__ __forceinline__ void prefetch_l2(const void *p) {
-    asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
 }
 
 // Bulk copy shared -> global (bulk-group completion); wait_read returns once
