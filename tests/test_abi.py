@@ -60,6 +60,18 @@ def _decode(L, **kw):
                                      a["sc"], a["out"], a["lse"], a["ws"], a["wsb"], a["st"], a["stream"])
 
 
+def test_last_cuda_error_query(L):
+    # the CUDA error behind the last NVFP4MLA_ERR_CUDA of this thread (0 and
+    # "no error" until one happens); its text is what NVFP4MLAError shows
+    code = L.nvfp4mla_last_cuda_error()
+    text = L.nvfp4mla_last_cuda_error_string()
+    assert code >= 0 and isinstance(text, bytes) and text
+    if code == 0:
+        assert text == b"no error"
+    err = nv.NVFP4MLAError(4, "call", "an illegal memory access was encountered")
+    assert "CUDA runtime error" in str(err) and "illegal memory access" in str(err) and err.status == 4
+
+
 def test_decode_argument_errors(L):
     INVALID, UNSUP, WS = 1, 2, 3
     assert _decode(L, T=0) == 0                      # nothing to do, nothing launched
