@@ -780,6 +780,7 @@ __global__ void __launch_bounds__(kTopkThreads, 1) indexer_topk_kernel(const Top
     // that starts below r1 lies in the row, which holds ctx rounded up to 4
     // floats (r0 and span are multiples of 4).
     {
+        const float tau_f = key_score(tau);  // score >= tau_f  <=>  key >= tau (scores are never NaN)
         constexpr int J = 4;
         float4 nx[J];  // the next batch's loads, in flight while this one is scanned
         auto load_batch = [&](int b0, float4 (&d)[J]) {
@@ -799,14 +800,28 @@ __global__ void __launch_bounds__(kTopkThreads, 1) indexer_topk_kernel(const Top
 #pragma unroll
             for (int j = 0; j < J; ++j) v4[j] = nx[j];
             if (b0 + kTopkThreads * 4 * J < r1) load_batch(b0 + kTopkThreads * 4 * J, nx);
-            uint32_t sel = 0;  // bit 4j+e: position wb + 128j + 4*lane + e is a candidate
+            // bit 4j+e: position wb + 128j + 4*lane + e is a candidate (its
+            // score >= tau's score, the same test as key >= tau for every
+            // score but NaN); positions past r1 are tested only in the last,
+            // partial batch
+            uint32_t sel = 0;
+            if (b0 + kTopkThreads * 4 * J <= r1) {  // block-uniform
 #pragma unroll
-            for (int j = 0; j < J; ++j) {
-                const int p = wb + 128 * j + 4 * lane;
-                sel |= (p + 0 < r1 && score_key(v4[j].x) >= tau ? 1u : 0u) << (4 * j + 0);
-                sel |= (p + 1 < r1 && score_key(v4[j].y) >= tau ? 1u : 0u) << (4 * j + 1);
-                sel |= (p + 2 < r1 && score_key(v4[j].z) >= tau ? 1u : 0u) << (4 * j + 2);
-                sel |= (p + 3 < r1 && score_key(v4[j].w) >= tau ? 1u : 0u) << (4 * j + 3);
+                for (int j = 0; j < J; ++j) {
+                    sel |= (v4[j].x >= tau_f ? 1u : 0u) << (4 * j + 0);
+                    sel |= (v4[j].y >= tau_f ? 1u : 0u) << (4 * j + 1);
+                    sel |= (v4[j].z >= tau_f ? 1u : 0u) << (4 * j + 2);
+                    sel |= (v4[j].w >= tau_f ? 1u : 0u) << (4 * j + 3);
+                }
+            } else {
+#pragma unroll
+                for (int j = 0; j < J; ++j) {
+                    const int p = wb + 128 * j + 4 * lane;
+                    sel |= (p + 0 < r1 && v4[j].x >= tau_f ? 1u : 0u) << (4 * j + 0);
+                    sel |= (p + 1 < r1 && v4[j].y >= tau_f ? 1u : 0u) << (4 * j + 1);
+                    sel |= (p + 2 < r1 && v4[j].z >= tau_f ? 1u : 0u) << (4 * j + 2);
+                    sel |= (p + 3 < r1 && v4[j].w >= tau_f ? 1u : 0u) << (4 * j + 3);
+                }
             }
             uint32_t pc = 0;  // count of load j in byte j (<= 4 per lane, <= 128 per warp)
 #pragma unroll
@@ -825,16 +840,16 @@ __global__ void __launch_bounds__(kTopkThreads, 1) indexer_topk_kernel(const Top
             for (int j = 0; j < J; ++j) {
                 uint32_t at = at_j + ((exc >> (8 * j)) & 0xFFu);
                 const int p = wb + 128 * j + 4 * lane;
-                const float v[4] = {v4[j].x, v4[j].y, v4[j].z, v4[j].w};
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    if ((sel >> (4 * j + e)) & 1u) {
-                        if (at < (uint32_t)kCandCap) {
-                            cand_key[at] = score_key(v[e]);
-                            cand_pos[at] = p + e;
-                        }
-                        ++at;
+                uint32_t bits = (sel >> (4 * j)) & 0xFu;  // few lanes hold any: visit set bits only
+                while (bits) {
+                    const int e = __ffs(bits) - 1;
+                    bits &= bits - 1u;
+                    if (at < (uint32_t)kCandCap) {
+                        const float x = e == 0 ? v4[j].x : e == 1 ? v4[j].y : e == 2 ? v4[j].z : v4[j].w;
+                        cand_key[at] = score_key(x);
+                        cand_pos[at] = p + e;
                     }
+                    ++at;
                 }
                 at_j += (tot >> (8 * j)) & 0xFFu;
             }
