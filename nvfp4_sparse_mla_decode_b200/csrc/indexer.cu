@@ -35,6 +35,7 @@
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cmath>
 
 #include "common.cuh"
@@ -318,9 +319,15 @@ static_assert(kTopkWarps == 32, "one warp reduces the per-warp minima and maxima
 constexpr int kBins = 2048;
 constexpr int kChunk = 8192;  // floats per streamed chunk
 constexpr int kRing = 3;
-constexpr int kCandCap = 12288;
+constexpr int kCandCap = 8192;    // 4 x the largest topk
 constexpr int kMaxParts = 8;
-constexpr int kTopkDynSmem = kRing * kChunk * 4 + kCandCap * 8;  // 192 KB
+// A CTA's part of the row, when it holds at most kSliceCap positions, is
+// bulk-copied into shared memory at launch (the area the general path later
+// uses as its ring), so the collect pass reads it there.
+constexpr int kSliceCap = 36 * kTopkThreads;  // 36 positions per thread
+constexpr int kAreaBytes = kSliceCap * 4 > kRing * kChunk * 4 ? kSliceCap * 4 : kRing * kChunk * 4;
+constexpr int kSlicePiece = 4096;  // positions per bulk copy of the part
+constexpr int kTopkDynSmem = kAreaBytes + kCandCap * 8;  // 216 KB
 static_assert(kCandCap >= 8192, "the sampled keys (at most 8192) share the candidate area");
 static_assert(kChunk == kTopkWarps * 256, "pass D gives each warp 256 positions of a chunk");
 
@@ -459,86 +466,111 @@ __device__ uint32_t select_in_smem(const uint32_t *keys, uint32_t n, uint32_t wa
 // by (key - min) >> shift, a monotone map onto at most 2048 bins, so every
 // bin above the one holding the want-th largest key, b*, is taken whole; the
 // few keys of b* (at most 32) are then ranked by one warp.  When b* holds
-// more than 32 keys it falls back to the radix select.  Every thread calls
-// it; `sub` is 32 words of scratch, `mm` 2.
+// more than 32 keys, they are copied to `spill` (room for n keys) and binned
+// once more over their own, narrower range; only if that fails too does the
+// radix select run, on b*'s keys.  A range below 2048 gives one key per bin,
+// so b* itself is the answer.  Keys equal to the result all fall in b*,
+// so the ties counted there are the ties overall.  Every thread calls it;
+// `sub` is 32 words of scratch, `mm` 2.
 __device__ uint32_t select_fast(const uint32_t *keys, uint32_t n, uint32_t want, uint32_t *hist, uint32_t *scratch,
-                                uint32_t *found, uint32_t *ties, uint32_t *sub, uint32_t *mm) {
+                                uint32_t *found, uint32_t *ties, uint32_t *sub, uint32_t *mm, uint32_t *spill) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    uint32_t lo = 0xFFFFFFFFu, hi = 0u;
-    for (uint32_t i = tid; i < n; i += kTopkThreads) {
-        const uint32_t k = keys[i];
-        lo = min(lo, k);
-        hi = max(hi, k);
-    }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-        lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, off));
-        hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, off));
-    }
-    if (lane == 0) {  // per-warp minima and maxima (kTopkWarps == 32)
-        scratch[warp] = lo;
-        sub[warp] = hi;
-    }
-    if (tid == 0) found[0] = 0;  // keys of b* collected so far (below)
-    for (int i = tid; i < kBins; i += kTopkThreads) hist[i] = 0;
-    __syncthreads();
-    if (warp == 0) {
-        lo = scratch[lane];
-        hi = sub[lane];
+#pragma unroll 1
+    for (int level = 0; level < 2; ++level) {
+        uint32_t lo = 0xFFFFFFFFu, hi = 0u;
+        for (uint32_t i = tid; i < n; i += kTopkThreads) {
+            const uint32_t k = keys[i];
+            lo = min(lo, k);
+            hi = max(hi, k);
+        }
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) {
             lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, off));
             hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, off));
         }
-        if (lane == 0) {
-            mm[0] = lo;
-            mm[1] = hi;
+        if (lane == 0) {  // per-warp minima and maxima (kTopkWarps == 32)
+            scratch[warp] = lo;
+            sub[warp] = hi;
         }
-    }
-    __syncthreads();
-    lo = mm[0];
-    hi = mm[1];
-    if (lo == hi) {  // all keys equal: the threshold is that key, want of them taken
-        *ties = want;
-        return lo;
-    }
-    const uint32_t range = hi - lo;
-    const int shift = max(0, 32 - __clz(range) - 11);  // range >> shift < 2048
-    for (uint32_t i = tid; i < n; i += kTopkThreads) atomicAdd(&hist[(keys[i] - lo) >> shift], 1u);
-    __syncthreads();
-    find_bin(hist, kBins, want, scratch, found + 1);  // found[1] = b*, found[2] = taken from b*
-    const uint32_t bstar = found[1], within = found[2], cnt = hist[bstar];
-    if (cnt > 32u) {  // too many keys share b*: the radix select
+        if (tid == 0) found[0] = 0;  // keys of b* collected so far (below)
+        for (int i = tid; i < kBins; i += kTopkThreads) hist[i] = 0;
         __syncthreads();
-        return select_in_smem(keys, n, want, hist, scratch, found, ties);
-    }
-    for (uint32_t i = tid; i < n; i += kTopkThreads) {
-        const uint32_t k = keys[i];
-        if (((k - lo) >> shift) == bstar) sub[atomicAdd(&found[0], 1u)] = k;
-    }
-    __syncthreads();
-    if (warp == 0) {
-        // lane i holds key i of b* (if any); the want-th largest overall is
-        // the within-th largest of b*: the key v with #(> v) < within <= #(>= v)
-        const uint32_t v = lane < (int)cnt ? sub[lane] : 0u;
-        uint32_t gt = 0, ge = 0;
-        for (uint32_t j = 0; j < cnt; ++j) {
-            const uint32_t u = __shfl_sync(0xffffffffu, v, j);
-            gt += u > v;
-            ge += u >= v;
+        if (warp == 0) {
+            lo = scratch[lane];
+            hi = sub[lane];
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) {
+                lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, off));
+                hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, off));
+            }
+            if (lane == 0) {
+                mm[0] = lo;
+                mm[1] = hi;
+            }
         }
-        const bool hit = lane < (int)cnt && gt < within && within <= ge;
-        const uint32_t who = __ballot_sync(0xffffffffu, hit);
-        if (lane == __ffs(who) - 1) {
-            mm[0] = v;
-            mm[1] = within - gt;
+        __syncthreads();
+        lo = mm[0];
+        hi = mm[1];
+        if (lo == hi) {  // all keys equal: the threshold is that key, want of them taken
+            *ties = want;
+            __syncthreads();  // mm may be reused right after
+            return lo;
         }
+        const uint32_t range = hi - lo;
+        const int shift = max(0, 32 - __clz(range) - 11);  // range >> shift < 2048
+        for (uint32_t i = tid; i < n; i += kTopkThreads) atomicAdd(&hist[(keys[i] - lo) >> shift], 1u);
+        __syncthreads();
+        find_bin(hist, kBins, want, scratch, found + 1);  // found[1] = b*, found[2] = taken from b*
+        const uint32_t bstar = found[1], within = found[2], cnt = hist[bstar];
+        if (shift == 0) {  // one key per bin: b* is the threshold, within of its keys taken
+            *ties = within;
+            __syncthreads();  // found and hist may be reused right after
+            return lo + bstar;
+        }
+        if (cnt <= 32u) {
+            for (uint32_t i = tid; i < n; i += kTopkThreads) {
+                const uint32_t k = keys[i];
+                if (((k - lo) >> shift) == bstar) sub[atomicAdd(&found[0], 1u)] = k;
+            }
+            __syncthreads();
+            if (warp == 0) {
+                // lane i holds key i of b* (if any); the want-th largest overall is
+                // the within-th largest of b*: the key v with #(> v) < within <= #(>= v)
+                const uint32_t v = lane < (int)cnt ? sub[lane] : 0u;
+                uint32_t gt = 0, ge = 0;
+                for (uint32_t j = 0; j < cnt; ++j) {
+                    const uint32_t u = __shfl_sync(0xffffffffu, v, j);
+                    gt += u > v;
+                    ge += u >= v;
+                }
+                const bool hit = lane < (int)cnt && gt < within && within <= ge;
+                const uint32_t who = __ballot_sync(0xffffffffu, hit);
+                if (lane == __ffs(who) - 1) {
+                    mm[0] = v;
+                    mm[1] = within - gt;
+                }
+            }
+            __syncthreads();
+            *ties = mm[1];
+            const uint32_t thr = mm[0];
+            __syncthreads();  // mm, sub and found may be reused right after
+            return thr;
+        }
+        if (level == 1) {  // the radix select below, over the keys spilled at level 0
+            __syncthreads();  // every thread has read hist[b*]
+            break;
+        }
+        // b*'s keys, on their own: the within-th largest of them
+        for (uint32_t i = tid; i < n; i += kTopkThreads) {
+            const uint32_t k = keys[i];
+            if (((k - lo) >> shift) == bstar) spill[atomicAdd(&found[0], 1u)] = k;
+        }
+        __syncthreads();
+        keys = spill;
+        n = cnt;
+        want = within;
     }
-    __syncthreads();
-    *ties = mm[1];
-    const uint32_t thr = mm[0];
-    __syncthreads();  // mm, sub and found may be reused right after
-    return thr;
+    return select_in_smem(keys, n, want, hist, scratch, found, ties);
 }
 
 // Score of a key (inverse of score_key).
@@ -662,9 +694,10 @@ __device__ void write_from_candidates(const uint32_t *ck, const int32_t *cp, uin
 __global__ void __launch_bounds__(kTopkThreads, 1) indexer_topk_kernel(const TopkArgs a) {
     extern __shared__ __align__(128) uint8_t dyn[];
     float *ring = reinterpret_cast<float *>(dyn);
-    uint32_t *cand_key = reinterpret_cast<uint32_t *>(dyn + kRing * kChunk * 4);
+    const float *slice = ring;  // this CTA's part of the row, until the general path
+    uint32_t *cand_key = reinterpret_cast<uint32_t *>(dyn + kAreaBytes);
     int32_t *cand_pos = reinterpret_cast<int32_t *>(cand_key + kCandCap);
-    __shared__ uint64_t full[kRing];
+    __shared__ uint64_t full[kRing + 1];  // the ring's buffers, then the part's copies
     __shared__ uint32_t hist[kBins];
     __shared__ uint32_t scratch[32], slots_a[32], slots_b[32];
     __shared__ uint32_t found[4], totals[2], sub32[32], mm2[2];
@@ -686,8 +719,12 @@ __global__ void __launch_bounds__(kTopkThreads, 1) indexer_topk_kernel(const Top
         return;
     }
     const float *s = a.scores + (int64_t)t * a.score_stride;
+    // this CTA's part of the row: P nearly equal ranges, multiples of 128
+    const int span = ((ctx + P - 1) / P + 127) / 128 * 128;
+    const int r0 = min(ctx, part * span), r1 = min(ctx, r0 + span);
+    const bool in_smem = r1 - r0 <= kSliceCap;  // block-uniform
     if (tid == 0) {
-        for (int b = 0; b < kRing; ++b) mbar_init(&full[b], 1);
+        for (int b = 0; b <= kRing; ++b) mbar_init(&full[b], 1);
         fence_mbar_init();
         ncand = 0;
     }
@@ -738,6 +775,16 @@ __global__ void __launch_bounds__(kTopkThreads, 1) indexer_topk_kernel(const Top
     };
 
     // ------------------------------------------- 1. sampled threshold tau
+    // Every CTA of the request draws the same sample of whole 32-position
+    // lines (at most 256 lines, line i of warp i % 32).  Usually the sample
+    // is cut into groups of G (a lane's 8 samples, then G / 8 lanes) and tau
+    // is a median of the groups' largest keys: each warp takes the lower
+    // median of its groups, tau is the 16th smallest of the 32 warps'.  For
+    // a short row or a large topk (no G >= 8) or a warp with fewer than 7
+    // lines, tau is taken from a binning of the whole sample instead
+    // (sample_threshold, aiming at 1.25 x topk).  Either way, a tau that
+    // catches fewer than topk positions or more than fit sends the request
+    // to the general path.
     uint32_t tau;
     {
         const int64_t lines = ((int64_t)ctx + 31) / 32;
@@ -745,7 +792,6 @@ __global__ void __launch_bounds__(kTopkThreads, 1) indexer_topk_kernel(const Top
         const int nsl = (int)((lines + lstride - 1) / lstride);  // sampled lines, <= 256
         const int last_base = (nsl - 1) * lstride * 32;
         const uint32_t S = (uint32_t)((nsl - 1) * 32 + min(32, ctx - last_base));
-        uint32_t *samp = cand_key;  // free until step 2
         uint32_t sk[(8192 / 32 + kTopkWarps - 1) / kTopkWarps];
 #pragma unroll
         for (int j = 0; j < 8; ++j) {  // all of a warp's line loads in flight at once
@@ -753,24 +799,115 @@ __global__ void __launch_bounds__(kTopkThreads, 1) indexer_topk_kernel(const Top
             const int p = i * lstride * 32 + lane;
             sk[j] = (i < nsl && p < ctx) ? score_key(__ldcg(s + p)) : 0u;  // 0 is below every score's key
         }
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const int i = warp + kTopkWarps * j;
-            if (i < nsl) samp[i * 32 + lane] = sk[j];
+        if (tid == 0 && in_smem && r1 > r0) {
+            // the part's copy, behind the sample loads; whole 16-byte units:
+            // r0 is a multiple of 128 floats and the row holds ctx rounded
+            // up to 4 floats
+            const uint32_t total = ((uint32_t)(r1 - r0) * 4u + 15u) & ~15u;
+            mbar_arrive_expect_tx(&full[kRing], total);
+            for (uint32_t off = 0; off < total; off += kSlicePiece * 4u)
+                bulk_g2s(ring + off / 4, s + r0 + off / 4, min((uint32_t)kSlicePiece * 4u, total - off),
+                         &full[kRing]);
         }
-        const uint32_t r = (uint32_t)min((int64_t)S, (int64_t)topk * S * 5 / (4 * (int64_t)ctx) + 9);
-        __syncthreads();
-        uint32_t unused;
-        (void)unused;
-        tau = sample_threshold(samp, (uint32_t)nsl * 32, r, hist, scratch, found, sub32, mm2);
+        // G = samples per group: the largest power of two in [8, 256] with
+        // ctx * ln 2 / G >= 1.4 * topk (0 if none).  The median over groups
+        // of a group's largest sample is exceeded by a share ln 2 / G of the
+        // row, so about ctx * ln 2 / G >= 1.4 * topk positions score at or
+        // above it.
+        int G = 0;
+        for (int g = 8; g <= 256; g *= 2)
+            if ((int64_t)ctx * 693 >= (int64_t)1400 * topk * g) G = g;
+        if (G > 0 && nsl >= 7 * kTopkWarps) {  // block-uniform
+            const int lg = G / 8, ng = 256 / G;  // lanes per group, groups per warp
+            uint32_t mx = sk[0];
+#pragma unroll
+            for (int j = 1; j < 8; ++j) mx = max(mx, sk[j]);
+            for (int off = 1; off < lg; off <<= 1) mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+            // lower median of the warp's ng group maxima (group k led by lane k * lg)
+            uint32_t below = 0;
+            for (int k = 0; k < ng; ++k) {
+                const uint32_t u = __shfl_sync(0xffffffffu, mx, k * lg);
+                below += u < mx || (u == mx && k * lg < lane);
+            }
+            const uint32_t who = __ballot_sync(0xffffffffu, lane % lg == 0 && below == (uint32_t)(ng - 1) / 2);
+            const uint32_t med = __shfl_sync(0xffffffffu, mx, __ffs(who) - 1);
+            if (lane == 0) sub32[warp] = med;
+            __syncthreads();
+            if (warp == 0) {  // the 16th smallest of the 32 warps' medians
+                const uint32_t e = sub32[lane];
+                uint32_t rank = 0;
+#pragma unroll
+                for (int k = 0; k < 32; ++k) {
+                    const uint32_t u = __shfl_sync(0xffffffffu, e, k);
+                    rank += u < e || (u == e && k < lane);
+                }
+                if (rank == 15u) mm2[0] = e;
+            }
+            __syncthreads();
+            tau = mm2[0];
+            __syncthreads();  // sub32 and mm2 may be reused right after
+        } else {
+            uint32_t *samp = cand_key;  // free until step 2
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const int i = warp + kTopkWarps * j;
+                if (i < nsl) samp[i * 32 + lane] = sk[j];
+            }
+            const uint32_t r = (uint32_t)min((int64_t)S, (int64_t)topk * S * 5 / (4 * (int64_t)ctx) + 9);
+            __syncthreads();
+            tau = sample_threshold(samp, (uint32_t)nsl * 32, r, hist, scratch, found, sub32, mm2);
+        }
     }
 
     // ------------------------------- 2. collect this CTA's candidates
-    const int span = ((ctx + P - 1) / P + kChunk - 1) / kChunk * kChunk;
-    const int r0 = min(ctx, part * span), r1 = min(ctx, r0 + span);
+    if (in_smem && r1 > r0 && !__syncthreads_and(mbar_wait(&full[kRing], 0))) {
+        if (tid == 0) {  // leave no copy in flight, report, leave
+            (void)mbar_wait(&full[kRing], 0);
+            flag(a.dev_status, NVFP4MLA_DEV_TIMEOUT);
+        }
+        return;
+    }
     uint32_t m = 0;  // candidates found in the range (block-uniform; may pass the cap)
-    // Straight from global memory (the row was just written and sits in L2),
-    // in batches of 16K positions: warp w takes the 512 positions
+    const float tau_f = key_score(tau);  // score >= tau_f  <=>  key >= tau (scores are never NaN)
+    if (in_smem) {
+        // From the part's copy in shared memory.  Thread i owns the run
+        // [i * L, (i + 1) * L) of the part (L / 4 odd, at most 9 float4:
+        // the eight lanes of a quarter warp then read 16-byte words in
+        // distinct banks), so position order is thread order: one pass marks
+        // the run's candidates in a 36-bit mask, one block scan of the
+        // counts places the threads, and each thread writes its few
+        // candidates.  Reads stay below 1024 * L <= kSliceCap; positions at
+        // or past the part's end n are masked.
+        const int n = r1 - r0;
+        const int l4 = ((n + kTopkThreads - 1) / kTopkThreads + 3) / 4 | 1;  // float4 per thread
+        const int base = tid * 4 * l4;
+        const float4 *v4 = reinterpret_cast<const float4 *>(slice + base);
+        uint64_t hits = 0;
+#pragma unroll
+        for (int i = 0; i < kSliceCap / kTopkThreads / 4; ++i)
+            if (i < l4) {
+                const float4 v = v4[i];
+                const int q = base + 4 * i;
+                hits |= (uint64_t)((q < n && v.x >= tau_f) | (q + 1 < n && v.y >= tau_f) << 1 |
+                                   (q + 2 < n && v.z >= tau_f) << 2 | (q + 3 < n && v.w >= tau_f) << 3)
+                        << (4 * i);
+            }
+        const uint32_t c = (uint32_t)__popcll(hits);
+        uint32_t at = block_incl_scan(c, scratch) - c;
+        m = scratch[kTopkWarps - 1];  // the block total: warp 0's scan of the warp sums
+        while (hits) {
+            const int b = __ffsll((long long)hits) - 1;
+            hits &= hits - 1;
+            if (at < (uint32_t)kCandCap) {
+                cand_key[at] = score_key(slice[base + b]);
+                cand_pos[at] = r0 + base + b;
+            }
+            ++at;
+        }
+        __syncthreads();  // every thread's candidates are written before anyone reads them
+    } else {
+    // Straight from global memory (the row was just written and sits in
+    // L2), in batches of 16K positions: warp w takes the 512 positions
     // [b0 + 512w, b0 + 512w + 512) as J = 4 float4 per lane, load j of lane
     // l covering positions 128j + 4l .. +3 (each load instruction reads 512
     // contiguous bytes; all of a lane's loads are in flight at once).
@@ -780,7 +917,6 @@ __global__ void __launch_bounds__(kTopkThreads, 1) indexer_topk_kernel(const Top
     // that starts below r1 lies in the row, which holds ctx rounded up to 4
     // floats (r0 and span are multiples of 4).
     {
-        const float tau_f = key_score(tau);  // score >= tau_f  <=>  key >= tau (scores are never NaN)
         constexpr int J = 4;
         float4 nx[J];  // the next batch's loads, in flight while this one is scanned
         auto load_batch = [&](int b0, float4 (&d)[J]) {
@@ -857,6 +993,7 @@ __global__ void __launch_bounds__(kTopkThreads, 1) indexer_topk_kernel(const Top
         }
         __syncthreads();  // every thread's candidates are written before anyone reads them
     }
+    }
 
     // ----------------------------- 3. the last CTA of the request selects
     uint32_t mtot = m;
@@ -914,7 +1051,9 @@ __global__ void __launch_bounds__(kTopkThreads, 1) indexer_topk_kernel(const Top
     }
     if (mtot >= (uint32_t)topk && mtot <= (uint32_t)kCandCap) {
         uint32_t need_eq;
-        const uint32_t thr = select_fast(cand_key, mtot, (uint32_t)topk, hist, scratch, found, &need_eq, sub32, mm2);
+        // the ring area is free in the last CTA: room for the second binning level
+        const uint32_t thr = select_fast(cand_key, mtot, (uint32_t)topk, hist, scratch, found, &need_eq, sub32, mm2,
+                                         reinterpret_cast<uint32_t *>(ring));
         write_from_candidates(cand_key, cand_pos, mtot, thr, need_eq, o, scratch);
         return;
     }
@@ -1125,7 +1264,7 @@ cudaError_t launch_indexer_scores(const uint8_t *q, const float *w, const uint8_
     if (T == 0 || max_ctx == 0) return cudaSuccess;
     using namespace idx;
     auto kern = indexer_score_kernel;
-    static bool attr_set[64] = {};
+    static std::atomic<bool> attr_set[64] = {};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
@@ -1179,7 +1318,7 @@ cudaError_t launch_indexer_topk(const float *scores, int64_t score_stride, const
                                 int32_t T, int32_t topk, int32_t *positions, void *workspace, int32_t *dev_status,
                                 cudaStream_t stream) {
     if (T == 0) return cudaSuccess;
-    static bool attr_set[64] = {};
+    static std::atomic<bool> attr_set[64] = {};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;

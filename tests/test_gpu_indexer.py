@@ -79,6 +79,36 @@ def test_topk_matches_oracle(case, topk):
     assert not bad, "tokens %s differ" % bad
 
 
+@pytest.mark.parametrize("case", ["normal", "ties", "neg_inf"])
+def test_topk_rows_longer_than_eight_ctas_hold(case):
+    # more than 8 x 53,248 positions: the row is streamed, not held on chip
+    ctx = [450000, 430001]
+    T, max_ctx = len(ctx), max(ctx)
+    stride = nv.indexer_score_stride(max_ctx)
+    s = _scores(case, T, stride, 77 + CASES.index(case))
+    pos = nv.indexer_topk(s.cuda(), torch.tensor(ctx, dtype=torch.int32, device="cuda"), max_ctx, 2048)
+    ref = indexer.topk_positions([s[t, :ctx[t]].double().numpy() for t in range(T)], 2048)
+    got = pos.cpu().numpy()
+    assert all(np.array_equal(got[t], ref[t]) for t in range(T))
+
+
+@pytest.mark.parametrize("T,top_ctx", [(160, 50000), (60, 100000), (200, 140000)])
+def test_topk_many_requests(T, top_ctx):
+    # one CTA or two per request, and more requests than the device holds
+    # at once: clusters run in waves
+    ctx = [top_ctx - (977 * t) % (top_ctx // 2) for t in range(T)]
+    max_ctx = max(ctx)
+    stride = nv.indexer_score_stride(max_ctx)
+    s = _scores("normal", T, stride, 9000 + T)
+    g = torch.Generator().manual_seed(T)
+    s[T // 3, :] = torch.randint(-3, 4, (stride,), generator=g).float()  # one request on the radix path
+    pos = nv.indexer_topk(s.cuda(), torch.tensor(ctx, dtype=torch.int32, device="cuda"), max_ctx, 2048)
+    ref = indexer.topk_positions([s[t, :ctx[t]].double().numpy() for t in range(T)], 2048)
+    got = pos.cpu().numpy()
+    bad = [t for t in range(T) if not np.array_equal(got[t], ref[t])]
+    assert not bad, "tokens %s differ" % bad
+
+
 @pytest.mark.parametrize("T", [1, 3, 35])
 def test_topk_workspace_reused_across_calls(T):
     # rows split over several CTAs meet on counters in the workspace; every
