@@ -340,7 +340,7 @@ struct TopkArgs {
     int32_t *out;
     int parts;           // P: CTAs per request
     uint32_t *arrivals;  // [T] arrival counters (zero between launches)
-    uint32_t *counts;    // [T][P] candidates found by each CTA
+    uint2 *counts;       // [T][P] per CTA: candidates found, its threshold key
     uint2 *cand;         // [T][P][kCandCap] (key, position) in position order
     int32_t *dev_status;
 };
@@ -668,6 +668,45 @@ __device__ uint32_t sample_threshold(const uint32_t *keys, uint32_t n, uint32_t 
     return tau;
 }
 
+// A median of group maxima over 8192 sampled keys (8 per thread, key 0 for
+// no sample): groups of G = 8 * lg keys (a lane's 8, then lg lanes); each
+// warp takes the lower median of its 256 / G group maxima and the result is
+// the 16th smallest of the 32 warps' medians.  For keys drawn from one
+// distribution, a share of about ln 2 / G of it lies at or above the median
+// of the groups' maxima.  Every thread calls it; `sub` is 32 words, `mm` 1.
+__device__ uint32_t group_median_key(const uint32_t (&sk)[8], int G, uint32_t *sub, uint32_t *mm) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int lg = G / 8, ng = 256 / G;  // lanes per group, groups per warp
+    uint32_t mx = sk[0];
+#pragma unroll
+    for (int j = 1; j < 8; ++j) mx = max(mx, sk[j]);
+    for (int off = 1; off < lg; off <<= 1) mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+    // lower median of the warp's ng group maxima (group k led by lane k * lg)
+    uint32_t below = 0;
+    for (int k = 0; k < ng; ++k) {
+        const uint32_t u = __shfl_sync(0xffffffffu, mx, k * lg);
+        below += u < mx || (u == mx && k * lg < lane);
+    }
+    const uint32_t who = __ballot_sync(0xffffffffu, lane % lg == 0 && below == (uint32_t)(ng - 1) / 2);
+    const uint32_t med = __shfl_sync(0xffffffffu, mx, __ffs(who) - 1);
+    if (lane == 0) sub[warp] = med;
+    __syncthreads();
+    if (warp == 0) {  // the 16th smallest of the 32 warps' medians
+        const uint32_t e = sub[lane];
+        uint32_t rank = 0;
+#pragma unroll
+        for (int k = 0; k < 32; ++k) {
+            const uint32_t u = __shfl_sync(0xffffffffu, e, k);
+            rank += u < e || (u == e && k < lane);
+        }
+        if (rank == 15u) mm[0] = e;
+    }
+    __syncthreads();
+    const uint32_t tau = mm[0];
+    __syncthreads();  // sub and mm may be reused right after
+    return tau;
+}
+
 // Write the list from m candidates held in position order: keys above thr,
 // and the first need_eq keys equal to it.
 __device__ void write_from_candidates(const uint32_t *ck, const int32_t *cp, uint32_t m, uint32_t thr,
@@ -727,8 +766,28 @@ __global__ void __launch_bounds__(kTopkThreads, 1) indexer_topk_kernel(const Top
         for (int b = 0; b <= kRing; ++b) mbar_init(&full[b], 1);
         fence_mbar_init();
         ncand = 0;
+        if (in_smem && r1 > r0) {
+            // the part's copy; whole 16-byte units: r0 is a multiple of 128
+            // floats and the row holds ctx rounded up to 4 floats
+            const uint32_t total = ((uint32_t)(r1 - r0) * 4u + 15u) & ~15u;
+            mbar_arrive_expect_tx(&full[kRing], total);
+            for (uint32_t off = 0; off < total; off += kSlicePiece * 4u)
+                bulk_g2s(ring + off / 4, s + r0 + off / 4, min((uint32_t)kSlicePiece * 4u, total - off),
+                         &full[kRing]);
+        }
     }
     __syncthreads();
+    // false (block-uniform) once the part's copy is in shared memory; true
+    // if it never landed within the bounded wait (reported: leave)
+    auto slice_lost = [&]() -> bool {
+        if (!in_smem || r1 <= r0) return false;
+        if (__syncthreads_and(mbar_wait(&full[kRing], 0))) return false;
+        if (tid == 0) {  // leave no copy in flight, report
+            (void)mbar_wait(&full[kRing], 0);
+            flag(a.dev_status, NVFP4MLA_DEV_TIMEOUT);
+        }
+        return true;
+    };
 
     // ------------------------------------------------------- streaming
     uint32_t seq = 0;     // chunks streamed through the ring so far
@@ -775,98 +834,64 @@ __global__ void __launch_bounds__(kTopkThreads, 1) indexer_topk_kernel(const Top
     };
 
     // ------------------------------------------- 1. sampled threshold tau
-    // Every CTA of the request draws the same sample of whole 32-position
-    // lines (at most 256 lines, line i of warp i % 32).  Usually the sample
-    // is cut into groups of G (a lane's 8 samples, then G / 8 lanes) and tau
-    // is a median of the groups' largest keys: each warp takes the lower
-    // median of its groups, tau is the 16th smallest of the 32 warps'.  For
-    // a short row or a large topk (no G >= 8) or a warp with fewer than 7
-    // lines, tau is taken from a binning of the whole sample instead
-    // (sample_threshold, aiming at 1.25 x topk).  Either way, a tau that
-    // catches fewer than topk positions or more than fit sends the request
-    // to the general path.
+    // tau is estimated from 8192 sampled keys (at most), 8 per thread, as a
+    // median of group maxima (group_median_key) where a group of G samples
+    // fits: G = the largest power of two in [8, 256] with
+    // ctx * ln 2 / G >= 1.4 * topk, so about 1.4 x topk or more of the
+    // sampled stretch scores at or above tau.  A CTA whose part sits in
+    // shared memory and holds at least 8192 positions samples its own part
+    // (every (n / 8192)-th position) and keeps its own tau; otherwise every
+    // CTA of the request draws the same sample of whole 32-position lines of
+    // the row (line i of warp i % 32), and when no G fits or a warp holds
+    // fewer than 7 lines, tau comes from a binning of that sample instead
+    // (sample_threshold, aiming at 1.25 x topk).  The selecting CTA checks
+    // that the exact threshold is at or above every part's tau, so every
+    // position at or above it was collected; if not, or if the candidates
+    // are fewer than topk or more than fit, the request takes the general
+    // path.
     uint32_t tau;
     {
-        const int64_t lines = ((int64_t)ctx + 31) / 32;
-        const int lstride = (int)max((int64_t)1, (lines * 32 + 8191) / 8192);
-        const int nsl = (int)((lines + lstride - 1) / lstride);  // sampled lines, <= 256
-        const int last_base = (nsl - 1) * lstride * 32;
-        const uint32_t S = (uint32_t)((nsl - 1) * 32 + min(32, ctx - last_base));
-        uint32_t sk[(8192 / 32 + kTopkWarps - 1) / kTopkWarps];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {  // all of a warp's line loads in flight at once
-            const int i = warp + kTopkWarps * j;
-            const int p = i * lstride * 32 + lane;
-            sk[j] = (i < nsl && p < ctx) ? score_key(__ldcg(s + p)) : 0u;  // 0 is below every score's key
-        }
-        if (tid == 0 && in_smem && r1 > r0) {
-            // the part's copy, behind the sample loads; whole 16-byte units:
-            // r0 is a multiple of 128 floats and the row holds ctx rounded
-            // up to 4 floats
-            const uint32_t total = ((uint32_t)(r1 - r0) * 4u + 15u) & ~15u;
-            mbar_arrive_expect_tx(&full[kRing], total);
-            for (uint32_t off = 0; off < total; off += kSlicePiece * 4u)
-                bulk_g2s(ring + off / 4, s + r0 + off / 4, min((uint32_t)kSlicePiece * 4u, total - off),
-                         &full[kRing]);
-        }
-        // G = samples per group: the largest power of two in [8, 256] with
-        // ctx * ln 2 / G >= 1.4 * topk (0 if none).  The median over groups
-        // of a group's largest sample is exceeded by a share ln 2 / G of the
-        // row, so about ctx * ln 2 / G >= 1.4 * topk positions score at or
-        // above it.
         int G = 0;
         for (int g = 8; g <= 256; g *= 2)
             if ((int64_t)ctx * 693 >= (int64_t)1400 * topk * g) G = g;
-        if (G > 0 && nsl >= 7 * kTopkWarps) {  // block-uniform
-            const int lg = G / 8, ng = 256 / G;  // lanes per group, groups per warp
-            uint32_t mx = sk[0];
+        const int n = r1 - r0;
+        uint32_t sk[(8192 / 32 + kTopkWarps - 1) / kTopkWarps];
+        if (in_smem && n >= 8192 && G > 0) {  // block-uniform
+            if (slice_lost()) return;
+            const int st = n / 8192;  // 8191 * st < n
 #pragma unroll
-            for (int j = 1; j < 8; ++j) mx = max(mx, sk[j]);
-            for (int off = 1; off < lg; off <<= 1) mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-            // lower median of the warp's ng group maxima (group k led by lane k * lg)
-            uint32_t below = 0;
-            for (int k = 0; k < ng; ++k) {
-                const uint32_t u = __shfl_sync(0xffffffffu, mx, k * lg);
-                below += u < mx || (u == mx && k * lg < lane);
-            }
-            const uint32_t who = __ballot_sync(0xffffffffu, lane % lg == 0 && below == (uint32_t)(ng - 1) / 2);
-            const uint32_t med = __shfl_sync(0xffffffffu, mx, __ffs(who) - 1);
-            if (lane == 0) sub32[warp] = med;
-            __syncthreads();
-            if (warp == 0) {  // the 16th smallest of the 32 warps' medians
-                const uint32_t e = sub32[lane];
-                uint32_t rank = 0;
-#pragma unroll
-                for (int k = 0; k < 32; ++k) {
-                    const uint32_t u = __shfl_sync(0xffffffffu, e, k);
-                    rank += u < e || (u == e && k < lane);
-                }
-                if (rank == 15u) mm2[0] = e;
-            }
-            __syncthreads();
-            tau = mm2[0];
-            __syncthreads();  // sub32 and mm2 may be reused right after
+            for (int j = 0; j < 8; ++j) sk[j] = score_key(slice[(warp * 256 + j * 32 + lane) * st]);
+            tau = group_median_key(sk, G, sub32, mm2);
         } else {
-            uint32_t *samp = cand_key;  // free until step 2
+            const int64_t lines = ((int64_t)ctx + 31) / 32;
+            const int lstride = (int)max((int64_t)1, (lines * 32 + 8191) / 8192);
+            const int nsl = (int)((lines + lstride - 1) / lstride);  // sampled lines, <= 256
+            const int last_base = (nsl - 1) * lstride * 32;
+            const uint32_t S = (uint32_t)((nsl - 1) * 32 + min(32, ctx - last_base));
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
+            for (int j = 0; j < 8; ++j) {  // all of a warp's line loads in flight at once
                 const int i = warp + kTopkWarps * j;
-                if (i < nsl) samp[i * 32 + lane] = sk[j];
+                const int p = i * lstride * 32 + lane;
+                sk[j] = (i < nsl && p < ctx) ? score_key(__ldcg(s + p)) : 0u;  // 0 is below every score's key
             }
-            const uint32_t r = (uint32_t)min((int64_t)S, (int64_t)topk * S * 5 / (4 * (int64_t)ctx) + 9);
-            __syncthreads();
-            tau = sample_threshold(samp, (uint32_t)nsl * 32, r, hist, scratch, found, sub32, mm2);
+            if (G > 0 && nsl >= 7 * kTopkWarps) {  // block-uniform
+                tau = group_median_key(sk, G, sub32, mm2);
+            } else {
+                uint32_t *samp = cand_key;  // free until step 2
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const int i = warp + kTopkWarps * j;
+                    if (i < nsl) samp[i * 32 + lane] = sk[j];
+                }
+                const uint32_t r = (uint32_t)min((int64_t)S, (int64_t)topk * S * 5 / (4 * (int64_t)ctx) + 9);
+                __syncthreads();
+                tau = sample_threshold(samp, (uint32_t)nsl * 32, r, hist, scratch, found, sub32, mm2);
+            }
         }
     }
 
     // ------------------------------- 2. collect this CTA's candidates
-    if (in_smem && r1 > r0 && !__syncthreads_and(mbar_wait(&full[kRing], 0))) {
-        if (tid == 0) {  // leave no copy in flight, report, leave
-            (void)mbar_wait(&full[kRing], 0);
-            flag(a.dev_status, NVFP4MLA_DEV_TIMEOUT);
-        }
-        return;
-    }
+    if (slice_lost()) return;
     uint32_t m = 0;  // candidates found in the range (block-uniform; may pass the cap)
     const float tau_f = key_score(tau);  // score >= tau_f  <=>  key >= tau (scores are never NaN)
     if (in_smem) {
@@ -997,12 +1022,13 @@ __global__ void __launch_bounds__(kTopkThreads, 1) indexer_topk_kernel(const Top
 
     // ----------------------------- 3. the last CTA of the request selects
     uint32_t mtot = m;
+    uint32_t tau_max = tau;  // the highest threshold among the request's parts
     if (P > 1) {
         const int64_t slot = (int64_t)t * P + part;
         const uint32_t keep = min(m, (uint32_t)kCandCap);
         uint2 *dst = a.cand + slot * kCandCap;
         for (uint32_t i = tid; i < keep; i += kTopkThreads) dst[i] = make_uint2(cand_key[i], (uint32_t)cand_pos[i]);
-        if (tid == 0) a.counts[slot] = m;
+        if (tid == 0) a.counts[slot] = make_uint2(m, tau);
         __threadfence();
         __syncthreads();
         if (tid == 0) last = atomicAdd(a.arrivals + t, 1u) == (uint32_t)(P - 1);
@@ -1011,18 +1037,21 @@ __global__ void __launch_bounds__(kTopkThreads, 1) indexer_topk_kernel(const Top
         __threadfence();
         if (tid == 0) {
             a.arrivals[t] = 0;  // ready for the next launch
-            uint32_t acc = 0;
+            uint32_t acc = 0, tmax = 0;
             bool fits = true;
             for (int q = 0; q < P; ++q) {
-                const uint32_t mq = __ldcg(a.counts + (int64_t)t * P + q);
+                const uint2 cq = __ldcg(a.counts + (int64_t)t * P + q);
                 seg_off[q] = acc;
-                acc += mq;
-                fits &= mq <= (uint32_t)kCandCap;
+                acc += cq.x;
+                fits &= cq.x <= (uint32_t)kCandCap;
+                tmax = max(tmax, cq.y);
             }
             seg_off[P] = fits ? acc : 0xFFFFFFFFu;
+            mm2[1] = tmax;
         }
         __syncthreads();
         mtot = seg_off[P];
+        tau_max = mm2[1];
         if (mtot >= (uint32_t)topk && mtot <= (uint32_t)kCandCap) {
             // concatenate in part order = position order; slot i of the
             // joined list belongs to the part q with seg_off[q] <= i <
@@ -1054,8 +1083,12 @@ __global__ void __launch_bounds__(kTopkThreads, 1) indexer_topk_kernel(const Top
         // the ring area is free in the last CTA: room for the second binning level
         const uint32_t thr = select_fast(cand_key, mtot, (uint32_t)topk, hist, scratch, found, &need_eq, sub32, mm2,
                                          reinterpret_cast<uint32_t *>(ring));
-        write_from_candidates(cand_key, cand_pos, mtot, thr, need_eq, o, scratch);
-        return;
+        // every position at or above thr was collected when thr is at or
+        // above each part's tau (block-uniform)
+        if (thr >= tau_max) {
+            write_from_candidates(cand_key, cand_pos, mtot, thr, need_eq, o, scratch);
+            return;
+        }
     }
 
     // ---------------------- tau missed: the general path over the whole row
@@ -1305,13 +1338,14 @@ int indexer_topk_parts(int32_t T, int sm_count) {
     return p < 1 ? 1 : (p > idx::kMaxParts ? idx::kMaxParts : p);
 }
 
-// Workspace of a split selection: [T] arrival counters, then [T][P] counts,
-// then [T][P][kCandCap] candidates (8 bytes each); sections 256-byte aligned.
+// Workspace of a split selection: [T] arrival counters, then [T][P] (count,
+// threshold key) pairs, then [T][P][kCandCap] candidates (8 bytes each);
+// sections 256-byte aligned.
 size_t indexer_topk_workspace_bytes(int32_t T, int sm_count) {
     const int P = indexer_topk_parts(T, sm_count);
     if (P == 1 || T <= 0) return 0;
     auto up = [](size_t x) { return (x + 255) / 256 * 256; };
-    return up((size_t)T * 4) + up((size_t)T * P * 4) + (size_t)T * P * idx::kCandCap * 8;
+    return up((size_t)T * 4) + up((size_t)T * P * 8) + (size_t)T * P * idx::kCandCap * 8;
 }
 
 cudaError_t launch_indexer_topk(const float *scores, int64_t score_stride, const int32_t *ctx_lens, int32_t max_ctx,
@@ -1345,8 +1379,8 @@ cudaError_t launch_indexer_topk(const float *scores, int64_t score_stride, const
         auto up = [](size_t x) { return (x + 255) / 256 * 256; };
         uint8_t *w = static_cast<uint8_t *>(workspace);
         a.arrivals = reinterpret_cast<uint32_t *>(w);
-        a.counts = reinterpret_cast<uint32_t *>(w + up((size_t)T * 4));
-        a.cand = reinterpret_cast<uint2 *>(w + up((size_t)T * 4) + up((size_t)T * a.parts * 4));
+        a.counts = reinterpret_cast<uint2 *>(w + up((size_t)T * 4));
+        a.cand = reinterpret_cast<uint2 *>(w + up((size_t)T * 4) + up((size_t)T * a.parts * 8));
     }
     idx::indexer_topk_kernel<<<dim3((unsigned)a.parts, (unsigned)T), idx::kTopkThreads, idx::kTopkDynSmem, stream>>>(
         a);

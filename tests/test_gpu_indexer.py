@@ -43,7 +43,7 @@ def _table(ctx, page, seed, spare_pages=3):
     return table, num_pages * page
 
 
-CASES = ["normal", "ties", "signed_zeros", "neg_inf", "alternating_lines", "rising"]
+CASES = ["normal", "ties", "signed_zeros", "neg_inf", "alternating_lines", "rising", "first_part_high"]
 
 
 def _scores(case, T, stride, seed):
@@ -62,6 +62,8 @@ def _scores(case, T, stride, seed):
         s = torch.where((line % 2 == 1)[None, :], torch.ones_like(s), s)
     elif case == "rising":               # scores grow with position
         s = s * 0.01 + torch.arange(stride, dtype=torch.float32)[None, :] / 1000
+    elif case == "first_part_high":      # one part's own threshold lies above the row's
+        s[:, :stride // 8] += 100.0
     return s
 
 
