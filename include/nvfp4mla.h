@@ -346,8 +346,8 @@ nvfp4mla_status nvfp4mla_fp8_sparse_mla_decode(const void *q_nope_f16, const voi
 
 /* Workspace of nvfp4mla_indexer_topk for T requests on the current device:
  * 0 when each request's row is handled by one CTA (T >= SMs / 2), else
- * arrival counters, per-CTA candidate counts and thresholds, and candidate
- * lists.  It must
+ * arrival counters, per-CTA candidate counts, thresholds and largest keys,
+ * and candidate lists.  It must
  * be zero-filled before its first use; every completed call leaves the
  * counters at zero again. */
 size_t nvfp4mla_indexer_topk_workspace_size(int32_t T);

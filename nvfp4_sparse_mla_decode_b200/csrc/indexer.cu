@@ -340,7 +340,7 @@ struct TopkArgs {
     int32_t *out;
     int parts;           // P: CTAs per request
     uint32_t *arrivals;  // [T] arrival counters (zero between launches)
-    uint2 *counts;       // [T][P] per CTA: candidates found, its threshold key
+    uint4 *counts;       // [T][P] per CTA: candidates found, its threshold key, its largest candidate key
     uint2 *cand;         // [T][P][kCandCap] (key, position) in position order
     int32_t *dev_status;
 };
@@ -461,6 +461,42 @@ __device__ uint32_t select_in_smem(const uint32_t *keys, uint32_t n, uint32_t wa
     return prefix;
 }
 
+// mm[0], mm[1] = the smallest and largest of n keys in shared memory (n >= 1).
+// Every thread calls it; `scratch` and `sub` are 32 words each.
+__device__ void block_min_max(const uint32_t *keys, uint32_t n, uint32_t *scratch, uint32_t *sub, uint32_t *mm) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    uint32_t lo = 0xFFFFFFFFu, hi = 0u;
+    for (uint32_t i = tid; i < n; i += kTopkThreads) {
+        const uint32_t k = keys[i];
+        lo = min(lo, k);
+        hi = max(hi, k);
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+        lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, off));
+        hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, off));
+    }
+    if (lane == 0) {  // per-warp minima and maxima (kTopkWarps == 32)
+        scratch[warp] = lo;
+        sub[warp] = hi;
+    }
+    __syncthreads();
+    if (warp == 0) {
+        lo = scratch[lane];
+        hi = sub[lane];
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, off));
+            hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, off));
+        }
+        if (lane == 0) {
+            mm[0] = lo;
+            mm[1] = hi;
+        }
+    }
+    __syncthreads();
+}
+
 // The want-th largest of n keys in shared memory (1 <= want <= n), exactly
 // as select_in_smem gives it, usually in one histogram pass: keys are binned
 // by (key - min) >> shift, a monotone map onto at most 2048 bins, so every
@@ -470,47 +506,27 @@ __device__ uint32_t select_in_smem(const uint32_t *keys, uint32_t n, uint32_t wa
 // once more over their own, narrower range; only if that fails too does the
 // radix select run, on b*'s keys.  A range below 2048 gives one key per bin,
 // so b* itself is the answer.  Keys equal to the result all fall in b*,
-// so the ties counted there are the ties overall.  Every thread calls it;
-// `sub` is 32 words of scratch, `mm` 2.
+// so the ties counted there are the ties overall.  A caller that knows a
+// range [lo0, hi0] (lo0 < hi0) holding every key skips the first min/max
+// pass.  Every thread calls it; `sub` is 32 words of scratch, `mm` 2.
 __device__ uint32_t select_fast(const uint32_t *keys, uint32_t n, uint32_t want, uint32_t *hist, uint32_t *scratch,
-                                uint32_t *found, uint32_t *ties, uint32_t *sub, uint32_t *mm, uint32_t *spill) {
+                                uint32_t *found, uint32_t *ties, uint32_t *sub, uint32_t *mm, uint32_t *spill,
+                                uint32_t lo0 = 1u, uint32_t hi0 = 0u) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 #pragma unroll 1
     for (int level = 0; level < 2; ++level) {
-        uint32_t lo = 0xFFFFFFFFu, hi = 0u;
-        for (uint32_t i = tid; i < n; i += kTopkThreads) {
-            const uint32_t k = keys[i];
-            lo = min(lo, k);
-            hi = max(hi, k);
-        }
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) {
-            lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, off));
-            hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, off));
-        }
-        if (lane == 0) {  // per-warp minima and maxima (kTopkWarps == 32)
-            scratch[warp] = lo;
-            sub[warp] = hi;
-        }
         if (tid == 0) found[0] = 0;  // keys of b* collected so far (below)
         for (int i = tid; i < kBins; i += kTopkThreads) hist[i] = 0;
-        __syncthreads();
-        if (warp == 0) {
-            lo = scratch[lane];
-            hi = sub[lane];
-#pragma unroll
-            for (int off = 16; off > 0; off >>= 1) {
-                lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, off));
-                hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, off));
+        if (level == 0 && lo0 < hi0) {  // a range holding every key is known: no min/max pass
+            if (tid == 0) {
+                mm[0] = lo0;
+                mm[1] = hi0;
             }
-            if (lane == 0) {
-                mm[0] = lo;
-                mm[1] = hi;
-            }
+            __syncthreads();
+        } else {
+            block_min_max(keys, n, scratch, sub, mm);
         }
-        __syncthreads();
-        lo = mm[0];
-        hi = mm[1];
+        const uint32_t lo = mm[0], hi = mm[1];
         if (lo == hi) {  // all keys equal: the threshold is that key, want of them taken
             *ties = want;
             __syncthreads();  // mm may be reused right after
@@ -709,21 +725,25 @@ __device__ uint32_t group_median_key(const uint32_t (&sk)[8], int G, uint32_t *s
 
 // Write the list from m candidates held in position order: keys above thr,
 // and the first need_eq keys equal to it.
+static_assert(kCandCap < 65536, "write_from_candidates packs two counts of at most kCandCap in one word");
 __device__ void write_from_candidates(const uint32_t *ck, const int32_t *cp, uint32_t m, uint32_t thr,
                                       uint32_t need_eq, int32_t *o, uint32_t *scratch) {
     const uint32_t tid = threadIdx.x;
     const uint32_t per = (m + kTopkThreads - 1) / kTopkThreads;  // each thread owns a contiguous run
     const uint32_t i0 = min(m, tid * per), i1 = min(m, i0 + per);
-    uint32_t ties = 0;
-    for (uint32_t i = i0; i < i1; ++i) ties += ck[i] == thr;
-    uint32_t tie_rank = block_incl_scan(ties, scratch) - ties;
-    uint32_t sel = 0;
+    uint32_t above = 0, ties = 0;
     for (uint32_t i = i0; i < i1; ++i) {
         const uint32_t k = ck[i];
-        sel += k > thr || (k == thr && tie_rank++ < need_eq);
+        above += k > thr;
+        ties += k == thr;
     }
-    uint32_t at = block_incl_scan(sel, scratch) - sel;
-    tie_rank -= ties;
+    // one scan of both counts, packed 16 bits each (m <= kCandCap < 65536):
+    // the run's first slot is the keys above thr before it plus the ties
+    // taken before it
+    const uint32_t packed = above | ties << 16;
+    const uint32_t ex = block_incl_scan(packed, scratch) - packed;
+    uint32_t tie_rank = ex >> 16;
+    uint32_t at = (ex & 0xFFFFu) + min(tie_rank, need_eq);
     for (uint32_t i = i0; i < i1; ++i) {
         const uint32_t k = ck[i];
         if (k > thr || (k == thr && tie_rank++ < need_eq)) o[at++] = cp[i];
@@ -741,7 +761,7 @@ __global__ void __launch_bounds__(kTopkThreads, 1) indexer_topk_kernel(const Top
     __shared__ uint32_t scratch[32], slots_a[32], slots_b[32];
     __shared__ uint32_t found[4], totals[2], sub32[32], mm2[2];
     __shared__ float red_lo[kTopkWarps], red_hi[kTopkWarps];
-    __shared__ uint32_t ncand, seg_off[kMaxParts + 1];
+    __shared__ uint32_t ncand, cmax, seg_off[kMaxParts + 1];
     __shared__ int last;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int t = blockIdx.y, part = blockIdx.x, P = a.parts;
@@ -766,17 +786,19 @@ __global__ void __launch_bounds__(kTopkThreads, 1) indexer_topk_kernel(const Top
         for (int b = 0; b <= kRing; ++b) mbar_init(&full[b], 1);
         fence_mbar_init();
         ncand = 0;
-        if (in_smem && r1 > r0) {
-            // the part's copy; whole 16-byte units: r0 is a multiple of 128
-            // floats and the row holds ctx rounded up to 4 floats
-            const uint32_t total = ((uint32_t)(r1 - r0) * 4u + 15u) & ~15u;
-            mbar_arrive_expect_tx(&full[kRing], total);
-            for (uint32_t off = 0; off < total; off += kSlicePiece * 4u)
-                bulk_g2s(ring + off / 4, s + r0 + off / 4, min((uint32_t)kSlicePiece * 4u, total - off),
-                         &full[kRing]);
-        }
+        cmax = 0;
+        if (in_smem && r1 > r0) mbar_arrive_expect_tx(&full[kRing], ((uint32_t)(r1 - r0) * 4u + 15u) & ~15u);
     }
     __syncthreads();
+    if (in_smem && r1 > r0) {
+        // the part's copy, one 16 KB piece per thread of the first warp;
+        // whole 16-byte units: r0 is a multiple of 128 floats and the row
+        // holds ctx rounded up to 4 floats
+        const uint32_t total = ((uint32_t)(r1 - r0) * 4u + 15u) & ~15u;
+        const uint32_t off = (uint32_t)tid * kSlicePiece * 4u;
+        if (tid < kSliceCap / kSlicePiece && off < total)
+            bulk_g2s(ring + off / 4, s + r0 + off / 4, min((uint32_t)kSlicePiece * 4u, total - off), &full[kRing]);
+    }
     // false (block-uniform) once the part's copy is in shared memory; true
     // if it never landed within the bounded wait (reported: leave)
     auto slice_lost = [&]() -> bool {
@@ -908,27 +930,43 @@ __global__ void __launch_bounds__(kTopkThreads, 1) indexer_topk_kernel(const Top
         const int base = tid * 4 * l4;
         const float4 *v4 = reinterpret_cast<const float4 *>(slice + base);
         uint64_t hits = 0;
+        if (base + 4 * l4 <= n) {  // the whole run lies in the part
 #pragma unroll
-        for (int i = 0; i < kSliceCap / kTopkThreads / 4; ++i)
-            if (i < l4) {
-                const float4 v = v4[i];
-                const int q = base + 4 * i;
-                hits |= (uint64_t)((q < n && v.x >= tau_f) | (q + 1 < n && v.y >= tau_f) << 1 |
-                                   (q + 2 < n && v.z >= tau_f) << 2 | (q + 3 < n && v.w >= tau_f) << 3)
-                        << (4 * i);
-            }
+            for (int i = 0; i < kSliceCap / kTopkThreads / 4; ++i)
+                if (i < l4) {
+                    const float4 v = v4[i];
+                    hits |= (uint64_t)((v.x >= tau_f) | (v.y >= tau_f) << 1 | (v.z >= tau_f) << 2 |
+                                       (v.w >= tau_f) << 3)
+                            << (4 * i);
+                }
+        } else {
+#pragma unroll
+            for (int i = 0; i < kSliceCap / kTopkThreads / 4; ++i)
+                if (i < l4) {
+                    const float4 v = v4[i];
+                    const int q = base + 4 * i;
+                    hits |= (uint64_t)((q < n && v.x >= tau_f) | (q + 1 < n && v.y >= tau_f) << 1 |
+                                       (q + 2 < n && v.z >= tau_f) << 2 | (q + 3 < n && v.w >= tau_f) << 3)
+                            << (4 * i);
+                }
+        }
         const uint32_t c = (uint32_t)__popcll(hits);
         uint32_t at = block_incl_scan(c, scratch) - c;
         m = scratch[kTopkWarps - 1];  // the block total: warp 0's scan of the warp sums
+        uint32_t kmax = 0;
         while (hits) {
             const int b = __ffsll((long long)hits) - 1;
             hits &= hits - 1;
+            const uint32_t k = score_key(slice[base + b]);
             if (at < (uint32_t)kCandCap) {
-                cand_key[at] = score_key(slice[base + b]);
+                cand_key[at] = k;
                 cand_pos[at] = r0 + base + b;
             }
+            kmax = max(kmax, k);
             ++at;
         }
+        kmax = __reduce_max_sync(0xffffffffu, kmax);
+        if (lane == 0 && kmax) atomicMax(&cmax, kmax);
         __syncthreads();  // every thread's candidates are written before anyone reads them
     } else {
     // Straight from global memory (the row was just written and sits in
@@ -943,6 +981,7 @@ __global__ void __launch_bounds__(kTopkThreads, 1) indexer_topk_kernel(const Top
     // floats (r0 and span are multiples of 4).
     {
         constexpr int J = 4;
+        uint32_t kmax = 0;  // the largest candidate key seen by this thread
         float4 nx[J];  // the next batch's loads, in flight while this one is scanned
         auto load_batch = [&](int b0, float4 (&d)[J]) {
             const int wb = b0 + warp * (32 * 4 * J);
@@ -1005,17 +1044,21 @@ __global__ void __launch_bounds__(kTopkThreads, 1) indexer_topk_kernel(const Top
                 while (bits) {
                     const int e = __ffs(bits) - 1;
                     bits &= bits - 1u;
+                    const float x = e == 0 ? v4[j].x : e == 1 ? v4[j].y : e == 2 ? v4[j].z : v4[j].w;
+                    const uint32_t k = score_key(x);
                     if (at < (uint32_t)kCandCap) {
-                        const float x = e == 0 ? v4[j].x : e == 1 ? v4[j].y : e == 2 ? v4[j].z : v4[j].w;
-                        cand_key[at] = score_key(x);
+                        cand_key[at] = k;
                         cand_pos[at] = p + e;
                     }
+                    kmax = max(kmax, k);
                     ++at;
                 }
                 at_j += (tot >> (8 * j)) & 0xFFu;
             }
             m += totals[0];
         }
+        kmax = __reduce_max_sync(0xffffffffu, kmax);
+        if (lane == 0 && kmax) atomicMax(&cmax, kmax);
         __syncthreads();  // every thread's candidates are written before anyone reads them
     }
     }
@@ -1023,12 +1066,13 @@ __global__ void __launch_bounds__(kTopkThreads, 1) indexer_topk_kernel(const Top
     // ----------------------------- 3. the last CTA of the request selects
     uint32_t mtot = m;
     uint32_t tau_max = tau;  // the highest threshold among the request's parts
+    uint32_t key_lo = tau, key_hi = cmax;  // a range holding every candidate key
     if (P > 1) {
         const int64_t slot = (int64_t)t * P + part;
         const uint32_t keep = min(m, (uint32_t)kCandCap);
         uint2 *dst = a.cand + slot * kCandCap;
         for (uint32_t i = tid; i < keep; i += kTopkThreads) dst[i] = make_uint2(cand_key[i], (uint32_t)cand_pos[i]);
-        if (tid == 0) a.counts[slot] = make_uint2(m, tau);
+        if (tid == 0) a.counts[slot] = make_uint4(m, tau, cmax, 0u);
         __threadfence();
         __syncthreads();
         if (tid == 0) last = atomicAdd(a.arrivals + t, 1u) == (uint32_t)(P - 1);
@@ -1037,21 +1081,27 @@ __global__ void __launch_bounds__(kTopkThreads, 1) indexer_topk_kernel(const Top
         __threadfence();
         if (tid == 0) {
             a.arrivals[t] = 0;  // ready for the next launch
-            uint32_t acc = 0, tmax = 0;
+            uint32_t acc = 0, tmax = 0, tmin = 0xFFFFFFFFu, kmax = 0;
             bool fits = true;
             for (int q = 0; q < P; ++q) {
-                const uint2 cq = __ldcg(a.counts + (int64_t)t * P + q);
+                const uint4 cq = __ldcg(a.counts + (int64_t)t * P + q);
                 seg_off[q] = acc;
                 acc += cq.x;
                 fits &= cq.x <= (uint32_t)kCandCap;
                 tmax = max(tmax, cq.y);
+                tmin = min(tmin, cq.y);
+                kmax = max(kmax, cq.z);
             }
             seg_off[P] = fits ? acc : 0xFFFFFFFFu;
-            mm2[1] = tmax;
+            sub32[0] = tmax;
+            sub32[1] = tmin;
+            sub32[2] = kmax;
         }
         __syncthreads();
         mtot = seg_off[P];
-        tau_max = mm2[1];
+        tau_max = sub32[0];
+        key_lo = sub32[1];
+        key_hi = sub32[2];
         if (mtot >= (uint32_t)topk && mtot <= (uint32_t)kCandCap) {
             // concatenate in part order = position order; slot i of the
             // joined list belongs to the part q with seg_off[q] <= i <
@@ -1081,8 +1131,10 @@ __global__ void __launch_bounds__(kTopkThreads, 1) indexer_topk_kernel(const Top
     if (mtot >= (uint32_t)topk && mtot <= (uint32_t)kCandCap) {
         uint32_t need_eq;
         // the ring area is free in the last CTA: room for the second binning level
+        // every candidate key lies in [key_lo, key_hi]: each is at or above
+        // its part's tau and at most its part's largest
         const uint32_t thr = select_fast(cand_key, mtot, (uint32_t)topk, hist, scratch, found, &need_eq, sub32, mm2,
-                                         reinterpret_cast<uint32_t *>(ring));
+                                         reinterpret_cast<uint32_t *>(ring), key_lo, key_hi);
         // every position at or above thr was collected when thr is at or
         // above each part's tau (block-uniform)
         if (thr >= tau_max) {
@@ -1339,13 +1391,13 @@ int indexer_topk_parts(int32_t T, int sm_count) {
 }
 
 // Workspace of a split selection: [T] arrival counters, then [T][P] (count,
-// threshold key) pairs, then [T][P][kCandCap] candidates (8 bytes each);
-// sections 256-byte aligned.
+// threshold key, largest candidate key, unused), then [T][P][kCandCap]
+// candidates (8 bytes each); sections 256-byte aligned.
 size_t indexer_topk_workspace_bytes(int32_t T, int sm_count) {
     const int P = indexer_topk_parts(T, sm_count);
     if (P == 1 || T <= 0) return 0;
     auto up = [](size_t x) { return (x + 255) / 256 * 256; };
-    return up((size_t)T * 4) + up((size_t)T * P * 8) + (size_t)T * P * idx::kCandCap * 8;
+    return up((size_t)T * 4) + up((size_t)T * P * 16) + (size_t)T * P * idx::kCandCap * 8;
 }
 
 cudaError_t launch_indexer_topk(const float *scores, int64_t score_stride, const int32_t *ctx_lens, int32_t max_ctx,
@@ -1379,8 +1431,8 @@ cudaError_t launch_indexer_topk(const float *scores, int64_t score_stride, const
         auto up = [](size_t x) { return (x + 255) / 256 * 256; };
         uint8_t *w = static_cast<uint8_t *>(workspace);
         a.arrivals = reinterpret_cast<uint32_t *>(w);
-        a.counts = reinterpret_cast<uint2 *>(w + up((size_t)T * 4));
-        a.cand = reinterpret_cast<uint2 *>(w + up((size_t)T * 4) + up((size_t)T * a.parts * 8));
+        a.counts = reinterpret_cast<uint4 *>(w + up((size_t)T * 4));
+        a.cand = reinterpret_cast<uint2 *>(w + up((size_t)T * 4) + up((size_t)T * a.parts * 16));
     }
     idx::indexer_topk_kernel<<<dim3((unsigned)a.parts, (unsigned)T), idx::kTopkThreads, idx::kTopkDynSmem, stream>>>(
         a);

@@ -219,7 +219,7 @@ def test_indexer_argument_errors(L):
     assert t(1 << 20, 4096, 1 << 20, 4096, 0, 2048, 1 << 20, None, 0, None, None) == 0
     # with 148 SMs, 2 requests split their rows over 8 CTAs each: workspace needed
     need = L.nvfp4mla_indexer_topk_workspace_size(2)
-    assert need == 256 + 256 + 2 * 8 * 8192 * 8  # (count, threshold) pairs; 8192 8-byte candidates per CTA
+    assert need == 256 + 256 + 2 * 8 * 8192 * 8  # 16 bytes of counts per CTA; 8192 8-byte candidates per CTA
     assert t(*args, 2048, 1 << 20, None, 0, None, None) == WS
     assert t(*args, 2048, 1 << 20, 1 << 20, need - 1, None, None) == WS
     assert t(*args, 2048, 1 << 20, (1 << 20) + 16, need, None, None) == INVALID  # not 256-byte aligned
@@ -230,8 +230,8 @@ def test_indexer_argument_errors(L):
     assert s(*base, 1 << 20, 1000, None, None) == WS
     assert L.nvfp4mla_indexer_workspace_size(35, 140000) == (35 * 140032 * 4 + 255) // 256 * 256 + \
         L.nvfp4mla_indexer_topk_workspace_size(35)
-    # 35 requests x 4 CTAs: counters (140 B -> 256), (count, threshold) pairs (1120 B -> 1280), candidates
-    assert L.nvfp4mla_indexer_topk_workspace_size(35) == 256 + 1280 + 35 * 4 * 8192 * 8
+    # 35 requests x 4 CTAs: counters (140 B -> 256), 16 bytes of counts per CTA (2240 B -> 2304), candidates
+    assert L.nvfp4mla_indexer_topk_workspace_size(35) == 256 + 2304 + 35 * 4 * 8192 * 8
     assert L.nvfp4mla_indexer_score_stride(140000) == 140032
 
 
