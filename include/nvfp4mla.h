@@ -165,6 +165,60 @@ nvfp4mla_status nvfp4_sparse_mla_decode(const void *q_nope_f16, const void *q_ro
                                         size_t workspace_bytes, int32_t *dev_status, void *stream);
 
 /*
+ * nvfp4mla_tuning -- launch settings a caller may fix instead of the
+ * automatic plan (sweeps, or forcing one path), for
+ * nvfp4_sparse_mla_decode_tuned.  A zero field keeps the automatic choice.
+ *   splits         CTAs sharing one token's list (S): a power of two no
+ *                  larger than 16 nor than topk's 128-row tiles; with
+ *                  S > 1, T * (H / heads_per_cta) * S must not exceed the
+ *                  device's SMs (the merge needs every CTA resident) and
+ *                  T * (H / heads_per_cta) must not exceed 512
+ *   heads_per_cta  heads of one CTA (HG, the N of its MMAs): 16, 32 or 64,
+ *                  at most H (automatic: min(H, 64))
+ *   force_staged   nonzero: decode through the staged comparison path
+ *                  (rows unpacked to 576-byte E4M3 in a staging buffer,
+ *                  then attention over them) instead of the native kernel
+ *   reserved       must be 0
+ * The pages size the decode's SM clusters from the token batch (page
+ * "Prime Intellect Launches Prime Inference, Serving 600B Tokens Daily",
+ * section "Four-bit caches make room"); these fields let a caller set that
+ * sizing by hand.
+ */
+typedef struct nvfp4mla_tuning {
+    int32_t splits;
+    int32_t heads_per_cta;
+    int32_t force_staged;
+    int32_t reserved;
+} nvfp4mla_tuning;
+
+/*
+ * nvfp4_sparse_mla_workspace_size_tuned -- nvfp4_sparse_mla_workspace_size
+ * for the plan `tuning` fixes (NULL: the automatic plan).  The staged path
+ * needs its staging buffer besides (nvfp4_staged_fp8_staging_size).  Returns
+ * 0 for a shape or setting the decode does not take.
+ */
+size_t nvfp4_sparse_mla_workspace_size_tuned(int32_t T, int32_t H, int32_t topk, const nvfp4mla_tuning *tuning);
+
+/*
+ * nvfp4_sparse_mla_decode_tuned -- nvfp4_sparse_mla_decode with the plan
+ * `tuning` fixes (NULL: exactly nvfp4_sparse_mla_decode).
+ *   workspace  as nvfp4_sparse_mla_decode, of at least
+ *              nvfp4_sparse_mla_workspace_size_tuned bytes
+ *   staging    with force_staged: [T, topk, 576] bytes, 16-byte aligned, at
+ *              least nvfp4_staged_fp8_staging_size(T, topk); else unused
+ *              (may be NULL)
+ * Results are those of nvfp4_sparse_mla_decode (of the staged path with
+ * force_staged); they differ only by FP32 rounding order between split
+ * counts.  Errors: a setting the shape cannot take returns
+ * NVFP4MLA_ERR_INVALID_ARG; the rest as nvfp4_sparse_mla_decode.
+ */
+nvfp4mla_status nvfp4_sparse_mla_decode_tuned(const void *q_nope_f16, const void *q_rope_f16, const uint8_t *cache,
+                                              int64_t num_slots, const int32_t *indices, int32_t topk, int32_t T,
+                                              int32_t H, float sm_scale, void *out_f16, float *lse, void *workspace,
+                                              size_t workspace_bytes, uint8_t *staging, size_t staging_bytes,
+                                              const nvfp4mla_tuning *tuning, int32_t *dev_status, void *stream);
+
+/*
  * nvfp4_sparse_mla_decode_host -- nvfp4_sparse_mla_decode for inputs and
  * outputs in host memory: on `stream` it copies q_nope, q_rope and indices
  * from the host into the caller's device buffers (one cudaMemcpyAsync each),

@@ -43,6 +43,12 @@ _lib = None
 _vp, _i32, _i64, _f32, _sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
 
 
+class Tuning(ctypes.Structure):
+    """nvfp4mla_tuning: fixed split count, heads per CTA, forced staged path
+    (0 = the automatic choice; `reserved` must stay 0)."""
+    _fields_ = [("splits", _i32), ("heads_per_cta", _i32), ("force_staged", _i32), ("reserved", _i32)]
+
+
 class NVFP4MLAError(RuntimeError):
     def __init__(self, status: int, what: str, detail: str | None = None):
         msg = "%s: %s (status %d)" % (what, status_string(status), status)
@@ -67,6 +73,11 @@ def lib() -> ctypes.CDLL:
         L.nvfp4_sparse_mla_decode.restype = _i32
         L.nvfp4_sparse_mla_decode.argtypes = [_vp, _vp, _vp, _i64, _vp, _i32, _i32, _i32, _f32, _vp, _vp, _vp,
                                               _sz, _vp, _vp]
+        L.nvfp4_sparse_mla_workspace_size_tuned.restype = _sz
+        L.nvfp4_sparse_mla_workspace_size_tuned.argtypes = [_i32, _i32, _i32, ctypes.POINTER(Tuning)]
+        L.nvfp4_sparse_mla_decode_tuned.restype = _i32
+        L.nvfp4_sparse_mla_decode_tuned.argtypes = [_vp, _vp, _vp, _i64, _vp, _i32, _i32, _i32, _f32, _vp, _vp, _vp,
+                                                    _sz, _vp, _sz, ctypes.POINTER(Tuning), _vp, _vp]
         L.nvfp4_sparse_mla_decode_paged.restype = _i32
         L.nvfp4_sparse_mla_decode_paged.argtypes = [_vp, _vp, _vp, _i64, _vp, _i32, _vp, _i32, _i32, _i32, _i32,
                                                     _f32, _vp, _vp, _vp, _sz, _vp, _vp]
@@ -160,7 +171,9 @@ def num_splits(T: int, H: int, topk: int = MAX_TOPK) -> int:
     return int(lib().nvfp4_sparse_mla_num_splits(T, H, topk))
 
 
-def workspace_size(T: int, H: int, topk: int = MAX_TOPK) -> int:
+def workspace_size(T: int, H: int, topk: int = MAX_TOPK, tuning: Optional[Tuning] = None) -> int:
+    if tuning is not None:
+        return int(lib().nvfp4_sparse_mla_workspace_size_tuned(T, H, topk, ctypes.byref(tuning)))
     return int(lib().nvfp4_sparse_mla_workspace_size(T, H, topk))
 
 
@@ -215,15 +228,30 @@ def _decode_args(q_nope, q_rope, cache, indices, out, lse):
 def decode(q_nope: torch.Tensor, q_rope: torch.Tensor, cache: torch.Tensor, indices: torch.Tensor,
            sm_scale: float, out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
            workspace: Optional[torch.Tensor] = None, dev_status: Optional[torch.Tensor] = None,
-           num_slots: Optional[int] = None):
+           num_slots: Optional[int] = None, tuning: Optional[Tuning] = None,
+           staging: Optional[torch.Tensor] = None):
     """Sparse MLA decode over the NVFP4 cache; returns (out [T,H,512] f16, lse [T,H] f32).
 
     A caller-supplied `workspace` must start zero-filled (its first 4096
-    bytes hold split counters that every completed call leaves at zero)."""
+    bytes hold split counters that every completed call leaves at zero).
+    `tuning` fixes the plan (nvfp4_sparse_mla_decode_tuned); with
+    force_staged the staged path runs through `staging` (allocated here when
+    not given)."""
     dev, T, H, topk, out, lse = _decode_args(q_nope, q_rope, cache, indices, out, lse)
-    ws_need = workspace_size(T, H, topk)
+    ws_need = workspace_size(T, H, topk, tuning)
     if workspace is None and ws_need:
         workspace = torch.zeros(ws_need, dtype=torch.uint8, device=dev)
+    if tuning is not None:
+        if tuning.force_staged and staging is None:
+            staging = torch.empty(max(1, staging_size(T, topk)), dtype=torch.uint8, device=dev)
+        st = lib().nvfp4_sparse_mla_decode_tuned(
+            _ptr(q_nope), _ptr(q_rope), _ptr(cache), num_slots if num_slots is not None else cache.shape[0],
+            _ptr(indices), topk, T, H, float(sm_scale), _ptr(out), _ptr(lse), _ptr(workspace),
+            workspace.numel() * workspace.element_size() if workspace is not None else 0, _ptr(staging),
+            staging.numel() * staging.element_size() if staging is not None else 0, ctypes.byref(tuning),
+            _ptr(dev_status), _stream(dev))
+        _check(st, "nvfp4_sparse_mla_decode_tuned")
+        return out, lse
     st = lib().nvfp4_sparse_mla_decode(_ptr(q_nope), _ptr(q_rope), _ptr(cache),
                                        num_slots if num_slots is not None else cache.shape[0], _ptr(indices),
                                        topk, T, H, float(sm_scale), _ptr(out), _ptr(lse), _ptr(workspace),

@@ -55,14 +55,29 @@ nvfp4mla_status from_cuda(cudaError_t e) {
     return NVFP4MLA_ERR_CUDA;
 }
 
+// The plan for (T, H, topk) with a caller's settings (tuning may be NULL):
+// UNSUPPORTED for a shape the decode does not take, INVALID_ARG for settings
+// the shape cannot take.
+nvfp4mla_status decode_plan(int32_t T, int32_t H, int32_t topk, const nvfp4mla_tuning *tuning, DecodePlan *plan) {
+    const int sms = current_device_sm_count();
+    if (!make_decode_plan(T, H, topk, sms, plan)) return NVFP4MLA_ERR_UNSUPPORTED;
+    if (!tuning) return NVFP4MLA_OK;
+    if (tuning->reserved != 0 || tuning->splits < 0 || tuning->heads_per_cta < 0) return NVFP4MLA_ERR_INVALID_ARG;
+    if (!make_decode_plan(T, H, topk, sms, plan, tuning->splits, tuning->heads_per_cta))
+        return NVFP4MLA_ERR_INVALID_ARG;
+    return NVFP4MLA_OK;
+}
+
 // Checks shared by the native and staged decode entry points.
 nvfp4mla_status check_decode(const void *q_nope, const void *q_rope, const uint8_t *cache, int64_t num_slots,
                              const int32_t *indices, int32_t topk, int32_t T, int32_t H, float sm_scale,
-                             const void *out, const float *lse, DecodePlan *plan) {
+                             const void *out, const float *lse, DecodePlan *plan,
+                             const nvfp4mla_tuning *tuning = nullptr) {
     if (T < 0 || topk < 1 || topk > NVFP4MLA_MAX_TOPK || num_slots < 1 || num_slots > INT32_MAX)
         return NVFP4MLA_ERR_INVALID_ARG;
     if (!(sm_scale == sm_scale) || sm_scale > 3.0e38f || sm_scale < -3.0e38f) return NVFP4MLA_ERR_INVALID_ARG;
-    if (!make_decode_plan(T, H, topk, current_device_sm_count(), plan)) return NVFP4MLA_ERR_UNSUPPORTED;
+    const nvfp4mla_status pst = decode_plan(T, H, topk, tuning, plan);
+    if (pst != NVFP4MLA_OK) return pst;
     if (T == 0) return NVFP4MLA_OK;
     if (!q_nope || !q_rope || !cache || !indices || !out || !lse) return NVFP4MLA_ERR_INVALID_ARG;
     if (!aligned(q_nope, 16) || !aligned(q_rope, 16) || !aligned(cache, 16) || !aligned(indices, 16) ||
@@ -126,6 +141,37 @@ nvfp4mla_status nvfp4_sparse_mla_decode(const void *q_nope_f16, const void *q_ro
     return from_cuda(launch_sparse_mla_decode(RowSource::kNvfp4Cache, q_nope_f16, q_rope_f16, cache, num_slots, indices, topk, T, H,
                                               sm_scale, out_f16, lse, workspace, plan, dev_status,
                                               static_cast<cudaStream_t>(stream)));
+}
+
+size_t nvfp4_sparse_mla_workspace_size_tuned(int32_t T, int32_t H, int32_t topk, const nvfp4mla_tuning *tuning) {
+    DecodePlan p;
+    if (T < 0 || topk < 1 || topk > NVFP4MLA_MAX_TOPK) return 0;
+    return decode_plan(T, H, topk, tuning, &p) == NVFP4MLA_OK ? p.workspace_bytes : 0;
+}
+
+nvfp4mla_status nvfp4_sparse_mla_decode_tuned(const void *q_nope_f16, const void *q_rope_f16, const uint8_t *cache,
+                                              int64_t num_slots, const int32_t *indices, int32_t topk, int32_t T,
+                                              int32_t H, float sm_scale, void *out_f16, float *lse, void *workspace,
+                                              size_t workspace_bytes, uint8_t *staging, size_t staging_bytes,
+                                              const nvfp4mla_tuning *tuning, int32_t *dev_status, void *stream) {
+    DecodePlan plan;
+    nvfp4mla_status st = check_decode(q_nope_f16, q_rope_f16, cache, num_slots, indices, topk, T, H, sm_scale,
+                                      out_f16, lse, &plan, tuning);
+    if (st != NVFP4MLA_OK || T == 0) return st;
+    if (plan.workspace_bytes > 0 && (!workspace || workspace_bytes < plan.workspace_bytes)) return NVFP4MLA_ERR_WORKSPACE;
+    if (workspace && !aligned(workspace, 256)) return NVFP4MLA_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (tuning && tuning->force_staged) {
+        if (!staging || staging_bytes < nvfp4_staged_fp8_staging_size(T, topk)) return NVFP4MLA_ERR_WORKSPACE;
+        if (!aligned(staging, 16)) return NVFP4MLA_ERR_INVALID_ARG;
+        cudaError_t e = launch_stage_fp8(cache, num_slots, indices, topk, T, staging, s);
+        if (e != cudaSuccess) return from_cuda(e);
+        return from_cuda(launch_sparse_mla_decode(RowSource::kFp8Staging, q_nope_f16, q_rope_f16, staging, num_slots,
+                                                  indices, topk, T, H, sm_scale, out_f16, lse, workspace, plan,
+                                                  dev_status, s));
+    }
+    return from_cuda(launch_sparse_mla_decode(RowSource::kNvfp4Cache, q_nope_f16, q_rope_f16, cache, num_slots, indices,
+                                              topk, T, H, sm_scale, out_f16, lse, workspace, plan, dev_status, s));
 }
 
 // Test-only (not in the public header): the NVFP4 decode with a chosen wait

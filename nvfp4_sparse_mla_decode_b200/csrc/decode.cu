@@ -889,25 +889,35 @@ int current_device_sm_count() {
     return cached[dev];
 }
 
-bool make_decode_plan(int32_t T, int32_t H, int32_t topk, int sm_count, DecodePlan *plan) {
+bool make_decode_plan(int32_t T, int32_t H, int32_t topk, int sm_count, DecodePlan *plan, int splits,
+                      int heads_per_cta) {
     DecodePlan p{};
-    if (H == 16 || H == 32 || H == 64) {
-        p.heads_per_cta = H;
-        p.head_groups = 1;
-    } else if (H == 128) {
-        p.heads_per_cta = 64;
-        p.head_groups = 2;
+    if (H != 16 && H != 32 && H != 64 && H != 128) return false;
+    if (topk < 1 || topk > kMaxTopk || T < 0 || sm_count < 1) return false;
+    if (heads_per_cta == 0) {
+        p.heads_per_cta = H < 64 ? H : 64;
+    } else if ((heads_per_cta == 16 || heads_per_cta == 32 || heads_per_cta == 64) && heads_per_cta <= H) {
+        p.heads_per_cta = heads_per_cta;  // H is a power of two: it divides H
     } else {
         return false;
     }
-    if (topk < 1 || topk > kMaxTopk || T < 0 || sm_count < 1) return false;
-    // Split a token's list over S CTAs only while the whole grid still fits
-    // in one wave of one CTA per SM (the merge needs every CTA resident).
+    p.head_groups = H / p.heads_per_cta;
     const int64_t units = (int64_t)T * p.head_groups;
     const int max_s = std::min(dec::kMaxSplits, (topk + dec::kTileRows - 1) / dec::kTileRows);
     int S = 1;
-    while (S * 2 <= max_s && units * S * 2 <= sm_count) S *= 2;
-    if (S > 1 && units > (int64_t)(kSplitCounterBytes / 8)) S = 1;
+    if (splits == 0) {
+        // Split a token's list over S CTAs only while the whole grid still
+        // fits in one wave of one CTA per SM (the merge needs every CTA
+        // resident).
+        while (S * 2 <= max_s && units * S * 2 <= sm_count) S *= 2;
+        if (S > 1 && units > (int64_t)(kSplitCounterBytes / 8)) S = 1;
+    } else {
+        // a caller's split count: a power of two the list has tiles for,
+        // with every CTA of a split grid resident and its counters in place
+        if (splits < 1 || splits > max_s || (splits & (splits - 1))) return false;
+        if (splits > 1 && (units * splits > sm_count || units > (int64_t)(kSplitCounterBytes / 8))) return false;
+        S = splits;
+    }
     p.splits = S;
     p.workspace_bytes = S > 1 ? kSplitCounterBytes + (size_t)T * S * H * (kLatent + 2) * sizeof(float) : 0;
     *plan = p;

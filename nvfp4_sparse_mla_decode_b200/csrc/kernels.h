@@ -24,7 +24,10 @@ struct DecodePlan {
 // sits at the same place for every shape.
 constexpr size_t kSplitCounterBytes = 4096;
 // sm_count: SMs of the device the launch will run on (one CTA per SM).
-bool make_decode_plan(int32_t T, int32_t H, int32_t topk, int sm_count, DecodePlan *plan);
+// splits / heads_per_cta: 0 picks them automatically; other values fix them
+// (false when the shape cannot take them).
+bool make_decode_plan(int32_t T, int32_t H, int32_t topk, int sm_count, DecodePlan *plan, int splits = 0,
+                      int heads_per_cta = 0);
 // SM count of the current device, or 148 when no device can be queried
 // (pure host use, e.g. sizing a workspace on a machine without a GPU).
 int current_device_sm_count();

@@ -52,6 +52,36 @@ def test_plan_splits_fill_the_gpu(L):
     assert nv.staging_size(35) == 35 * 2048 * 576
 
 
+def test_tuned_plan_workspace(L):
+    # nvfp4mla_tuning fixes S and HG; 0 keeps the automatic choice; settings
+    # a shape cannot take give 0 bytes (and INVALID_ARG from the decode)
+    ws = lambda T, H, topk=2048, **kw: nv.workspace_size(T, H, topk, nv.Tuning(**kw))
+    per = lambda T, S, H: 4096 + T * S * H * 514 * 4
+    assert ws(35, 64) == nv.workspace_size(35, 64) == per(35, 4, 64)
+    assert ws(35, 64, splits=1) == 0                       # one CTA per list: no merge
+    assert ws(35, 64, splits=2) == per(35, 2, 64)
+    assert ws(1, 64, splits=16) == per(1, 16, 64)
+    assert ws(1, 64, splits=16, heads_per_cta=16) == per(1, 16, 64)  # 4 groups x 16 splits = 64 CTAs
+    assert ws(35, 64, heads_per_cta=32) == per(35, 2, 64)  # automatic S for 70 units: 2
+    assert ws(35, 64, splits=8) == 0                       # 280 CTAs cannot all be resident
+    assert ws(1, 64, splits=3) == 0                        # not a power of two
+    assert ws(1, 64, 100, splits=2) == 0                   # a 100-entry list is one tile
+    assert ws(1, 64, heads_per_cta=48) == 0
+    assert ws(1, 32, heads_per_cta=64) == 0                # more heads per CTA than H
+    assert ws(1, 64, reserved=1) == 0
+    assert ws(1, 48) == 0                                  # unsupported head count
+    t = nv.Tuning(splits=3)
+    args = [1 << 20, 1 << 20, 1 << 20, 100, 1 << 20, 2048, 1, 64, 0.1, 1 << 20, 1 << 20, 1 << 20, 1 << 30,
+            None, 0]
+    assert L.nvfp4_sparse_mla_decode_tuned(*args, ctypes.byref(t), None, None) == 1        # INVALID_ARG
+    t = nv.Tuning(force_staged=1)
+    assert L.nvfp4_sparse_mla_decode_tuned(*args, ctypes.byref(t), None, None) == 3        # no staging: WS
+    args[7] = 48
+    assert L.nvfp4_sparse_mla_decode_tuned(*args, None, None, None) == 2                    # UNSUPPORTED
+    args[7], args[6] = 64, 0
+    assert L.nvfp4_sparse_mla_decode_tuned(*args, None, None, None) == 0                    # T = 0: no-op
+
+
 def _decode(L, **kw):
     a = dict(q=1 << 20, qr=1 << 20, cache=1 << 20, ns=100, idx=1 << 20, topk=2048, T=1, H=64, sc=0.1,
              out=1 << 20, lse=1 << 20, ws=1 << 20, wsb=1 << 30, st=None, stream=None)

@@ -51,6 +51,25 @@ def test_decode35x64_full():
     run(w, build_cache(w))
 
 
+@pytest.mark.parametrize("H,splits,hg,staged", [
+    (64, 1, 64, 0), (64, 2, 64, 0), (64, 16, 64, 0), (64, 0, 32, 0), (64, 4, 32, 0), (64, 0, 16, 0),
+    (64, 4, 16, 0), (64, 1, 16, 0), (64, 2, 32, 1), (128, 16, 32, 0), (128, 0, 16, 0), (32, 8, 16, 0),
+])
+def test_tuned_plans_match_oracle(H, splits, hg, staged):
+    # a caller's split count, heads per CTA and forced staged path: every
+    # token against the oracle (the staged one for the staged path)
+    T = 6 if H <= 64 else 2
+    w = synth.per_request("cuda", [20000] * T, H, seed=29 + H + splits, name="tuned")
+    cache = build_cache(w)
+    tuning = nv.Tuning(splits=splits, heads_per_cta=hg, force_staged=staged)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out, lse = nv.decode(w.q_nope, w.q_rope, cache, w.indices, w.sm_scale, dev_status=status, tuning=tuning)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    ref_o, ref_l = oracle_decode(w, range(T), staged=bool(staged))
+    check_close(out, lse, ref_o, ref_l)
+
+
 def test_staged_path_matches_staged_oracle():
     w = synth.decode35("cuda", T=6, ctx=20000)
     run(w, build_cache(w), staged=True)
