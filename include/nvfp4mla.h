@@ -111,10 +111,12 @@ nvfp4mla_status nvfp4mla_fp8_kv_append(const void *latent_bf16, int64_t latent_s
 /*
  * nvfp4_sparse_mla_num_splits -- how many CTAs the decode splits each
  * token's index list across: the largest power of two S <= 16 (and <= the
- * number of 128-row tiles of topk) with T * (H / min(H, 64)) * S no larger
- * than the SM count of the current device (148 when no device can be
- * queried).  The pages size their SM clusters from the token batch in the
- * same spirit (same section).  Host-only; returns 0 for unsupported shapes.
+ * number of 128-row tiles of topk) with T * G * S no larger than the SM
+ * count of the current device (148 when no device can be queried), where
+ * G = H / HG head groups of HG heads each: HG = min(H, 64), or 32 when H >= 64
+ * and T * (H / 32) * (the largest S the list takes) fits in the SMs.  The
+ * pages size their SM clusters from the token batch in the same spirit (same
+ * section).  Host-only; returns 0 for unsupported shapes.
  */
 int32_t nvfp4_sparse_mla_num_splits(int32_t T, int32_t H, int32_t topk);
 
