@@ -26,11 +26,12 @@
 // epilogue warps and double-buffered accumulators (2 x 64 TMEM columns).
 //
 // Selection (indexer_topk_kernel): up to 8 CTAs share a request's score row.
-// Each takes a threshold from a sample of the row, streams its part once and
-// publishes the positions at or above it in position order; the last CTA to
-// arrive (an atomic counter, nobody waits) selects exactly among them and
-// writes the list in increasing position order.  If the threshold missed,
-// that CTA falls back to binned or radix passes over the whole row.
+// Each copies its part into shared memory, takes a threshold from a sample
+// of it, marks the positions at or above it in one pass and publishes them
+// in position order; the last CTA to arrive (an atomic counter, nobody
+// waits) selects exactly among them and writes the list in increasing
+// position order.  If a threshold missed, that CTA falls back to binned or
+// radix passes over the whole row.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
@@ -283,24 +284,30 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 
 // ------------------------------------------------------------------ top-k
 // Each request's score row is shared by P CTAs of 1024 threads (P chosen so
-// the grid fills the SMs, at most 8); CTA p owns a contiguous range of the
-// row.  Every pass streams the CTA's range through a ring of three 32 KB
-// shared-memory buffers filled by bulk copies (one thread issues them, an
-// mbarrier per buffer counts the bytes).
+// the grid fills the SMs, at most 8); CTA p owns a contiguous part of the
+// row (P nearly equal parts, multiples of 128 positions).
 //
 // Usual path:
-//   1. each CTA draws the same sample of whole 32-position lines (at most
-//      8192 keys) and takes tau = the r-th largest, r chosen so that about
-//      1.25 x topk positions of the row should have a key >= tau;
-//   2. one streamed pass over the CTA's range collects the positions with
-//      key >= tau in position order and publishes them (and their count) in
-//      the workspace;
+//   0. at launch, a part of at most kSliceCap positions is bulk-copied into
+//      shared memory (nine 16 KB copies, one mbarrier counting the bytes);
+//   1. a threshold tau: a median of group maxima over 8192 sampled keys
+//      (group_median_key) chosen so that about 1.4 x topk positions or more
+//      score at or above it -- sampled from the CTA's own part when it sits
+//      in shared memory, else from whole 32-position lines of the row (the
+//      same sample in every CTA; sample_threshold when no group size fits);
+//   2. one pass marks the part's positions with score >= tau, each thread
+//      owning a run of consecutive positions, and one block scan orders
+//      them; the CTA publishes them, their count, its tau and its largest
+//      candidate key in the workspace;
 //   3. the last CTA of the request to arrive on its counter (an atomic add;
 //      nobody waits) concatenates the P lists -- again in position order --
-//      and, if topk <= m <= kCandCap candidates were found, picks the topk
-//      largest with an exact radix select and writes them in order.
-// If tau missed (too few or too many candidates) that last CTA runs the
-// general path over the whole row alone:
+//      and, if topk <= m <= kCandCap candidates were found, finds the
+//      topk-th largest key exactly (select_fast over the published key
+//      range); if that key is at or above every part's tau, every position
+//      at or above it was collected, and the CTA writes the list.
+// Otherwise (too few or too many candidates, or a key below some part's
+// tau) that last CTA runs the general path over the whole row alone,
+// streaming it through a ring of three 32 KB buffers (the area of step 0):
 //   A  min and max of the finite scores;
 //   B  histogram of a linear binning of [min, max] into 2048 bins (monotone
 //      in the score: bins above the one holding the topk-th largest score,
