@@ -43,7 +43,8 @@ def _table(ctx, page, seed, spare_pages=3):
     return table, num_pages * page
 
 
-CASES = ["normal", "ties", "signed_zeros", "neg_inf", "alternating_lines", "rising", "first_part_high"]
+CASES = ["normal", "ties", "signed_zeros", "neg_inf", "alternating_lines", "rising", "first_part_high",
+         "all_neg_inf", "constant", "pos_inf_spikes"]
 
 
 def _scores(case, T, stride, seed):
@@ -64,6 +65,12 @@ def _scores(case, T, stride, seed):
         s = s * 0.01 + torch.arange(stride, dtype=torch.float32)[None, :] / 1000
     elif case == "first_part_high":      # one part's own threshold lies above the row's
         s[:, :stride // 8] += 100.0
+    elif case == "all_neg_inf":          # every position a candidate: the general path's radix select
+        s = torch.full((T, stride), -math.inf)
+    elif case == "constant":             # one key everywhere: ties decide by position
+        s = torch.full((T, stride), 0.5)
+    elif case == "pos_inf_spikes":       # +inf above every finite score
+        s[:, 7::997] = math.inf
     return s
 
 
