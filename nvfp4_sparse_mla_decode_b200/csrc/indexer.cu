@@ -1090,15 +1090,20 @@ __global__ void __launch_bounds__(kTopkThreads, 1) indexer_topk_kernel(const Top
             a.arrivals[t] = 0;  // ready for the next launch
             uint32_t acc = 0, tmax = 0, tmin = 0xFFFFFFFFu, kmax = 0;
             bool fits = true;
-            for (int q = 0; q < P; ++q) {
-                const uint4 cq = __ldcg(a.counts + (int64_t)t * P + q);
-                seg_off[q] = acc;
-                acc += cq.x;
-                fits &= cq.x <= (uint32_t)kCandCap;
-                tmax = max(tmax, cq.y);
-                tmin = min(tmin, cq.y);
-                kmax = max(kmax, cq.z);
-            }
+            uint4 cq[kMaxParts];
+#pragma unroll
+            for (int q = 0; q < kMaxParts; ++q)  // every part's load in flight at once
+                if (q < P) cq[q] = __ldcg(a.counts + (int64_t)t * P + q);
+#pragma unroll
+            for (int q = 0; q < kMaxParts; ++q)
+                if (q < P) {
+                    seg_off[q] = acc;
+                    acc += cq[q].x;
+                    fits &= cq[q].x <= (uint32_t)kCandCap;
+                    tmax = max(tmax, cq[q].y);
+                    tmin = min(tmin, cq[q].y);
+                    kmax = max(kmax, cq[q].z);
+                }
             seg_off[P] = fits ? acc : 0xFFFFFFFFu;
             sub32[0] = tmax;
             sub32[1] = tmin;
