@@ -117,6 +117,15 @@ def test_staged_tiny():
     run(w, build_cache(w), staged=True)
 
 
+@pytest.mark.parametrize("T,H", [(1, 128), (2, 64)])
+def test_small_batches_32_heads_per_cta(T, H):
+    # the automatic plan takes 32 heads per CTA here; native and staged paths
+    w = synth.per_request("cuda", [9000] * T, H, seed=71 + T, name="small")
+    cache = build_cache(w)
+    run(w, cache)
+    run(w, cache, staged=True)
+
+
 @pytest.mark.parametrize("T", [1, 8, 32, 64, 128, 256])
 def test_sweep_h128(T):
     # every token and both head groups of every token are compared

@@ -96,6 +96,13 @@ def test_fp8_decode_ragged_tiles_all_head_counts(H):
     run(w, build_fp8_cache(w))
 
 
+@pytest.mark.parametrize("T,H", [(1, 64), (2, 128), (4, 64)])
+def test_fp8_decode_small_batches(T, H):
+    # small batches take 32 heads per CTA and 16 splits: every token
+    w = synth.per_request("cuda", [9000] * T, H, seed=37 + T, name="small")
+    run(w, build_fp8_cache(w))
+
+
 def test_fp8_decode35x64_full():
     w = synth.decode35("cuda")
     assert nv.num_splits(w.T, w.H) == 4

@@ -13,9 +13,13 @@ from harness import build_cache, check_close, oracle_decode
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("shape", ["decode35x64", "tiny", "sweep8x128", "no_split"])
+@pytest.mark.parametrize("shape", ["decode35x64", "tiny", "sweep8x128", "no_split", "t1x128", "t2x64"])
 def test_noalloc_matches_workspace_entry_point_twice(shape):
-    if shape == "decode35x64":
+    if shape == "t1x128":
+        w = synth.per_request("cuda", [6000], 128, seed=65, name="na1")        # 32 heads per CTA, S = 16
+    elif shape == "t2x64":
+        w = synth.per_request("cuda", [6000] * 2, 64, seed=66, name="na2")     # 32 heads per CTA, S = 16
+    elif shape == "decode35x64":
         w = synth.per_request("cuda", [6000] * 35, 64, seed=61, name="na35")   # S = 4
     elif shape == "tiny":
         w = synth.tiny("cuda", seed=62)                                        # S = 16
