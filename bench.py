@@ -44,7 +44,7 @@ def parse():
     ap.add_argument("--no-extras", action="store_true", help="skip staged/append/e2e/cpu legs")
     ap.add_argument("--workload", default="decode35x64",
                     choices=["decode35x64", "sweep", "padded", "prefill", "tiny", "paged", "fp8", "indexer",
-                             "blhnc", "all-others"],
+                             "blhnc", "plans", "all-others"],
                     help="decode35x64 (default) prints the one result line; the others time the remaining "
                          "workloads and print one line per shape")
     ap.add_argument("--ctx", type=int, default=140_000,
@@ -547,15 +547,55 @@ def time_blhnc(nv, synth, args):
     torch.cuda.empty_cache()
 
 
+def time_plans(nv, synth, args):
+    """Small batches under each head-group width (nvfp4mla_tuning with
+    heads_per_cta fixed, the split count left automatic): one line per
+    shape, cold single launches (L2 flushed before each, median of 20),
+    preallocated outputs and workspaces, 140,000-row contexts."""
+    import torch
+    from nvfp4_sparse_mla_decode_b200.cache import build_cache
+    flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device="cuda")
+    for H in (64, 128):
+        for T in (1, 2, 4, 8):
+            w = synth.per_request("cuda", [140_000] * T, H, seed=5 + T, name="plans")
+            cache = build_cache(w)
+            out = torch.empty(T, H, 512, dtype=torch.float16, device="cuda")
+            lse = torch.empty(T, H, dtype=torch.float32, device="cuda")
+            res = {}
+            for hg in (64, 32, 16):
+                tuning = nv.Tuning(splits=0, heads_per_cta=hg)
+                wsz = nv.workspace_size(T, H, 2048, tuning)
+                ws = torch.zeros(max(1, wsz), dtype=torch.uint8, device="cuda")
+                S = 1 if wsz == 0 else (wsz - 4096) // (T * H * 514 * 4)
+
+                def fn():
+                    nv.decode(w.q_nope, w.q_rope, cache, w.indices, w.sm_scale, out=out, lse=lse, workspace=ws,
+                              tuning=tuning)
+                res["hg%d" % hg] = {"splits": S, "ctas": T * (H // hg) * S, "us_per_launch": cold_median_us(fn, flush)}
+            ws = torch.zeros(max(1, nv.workspace_size(T, H)), dtype=torch.uint8, device="cuda")
+
+            def fn_auto():
+                nv.decode(w.q_nope, w.q_rope, cache, w.indices, w.sm_scale, out=out, lse=lse, workspace=ws)
+            auto = {"splits": nv.num_splits(T, H), "us_per_launch": cold_median_us(fn_auto, flush)}
+            print(json.dumps({"metric": METRIC, "workload": "plans T=%d H=%d" % (T, H), "T": T, "H": H,
+                              "by_heads_per_cta": res, "automatic": auto,
+                              "timing": "single launch, L2 flushed before it, median of 20", "data": "synthetic"}),
+                  flush=True)
+            del cache
+            torch.cuda.empty_cache()
+
+
 def other_workloads(args):
     import torch
     import nvfp4_sparse_mla_decode_b200 as nv
     from nvfp4_sparse_mla_decode_b200 import synth
     assert torch.cuda.is_available(), "bench.py needs a CUDA GPU"
     nv.lib()
-    names = (["tiny", "sweep", "padded", "prefill", "paged", "fp8", "indexer", "blhnc"]
+    names = (["tiny", "sweep", "padded", "prefill", "paged", "fp8", "indexer", "blhnc", "plans"]
              if args.workload == "all-others" else [args.workload])
     for name in names:
+        if name == "plans":
+            time_plans(nv, synth, args)
         if name == "blhnc":
             time_blhnc(nv, synth, args)
         if name == "indexer":
