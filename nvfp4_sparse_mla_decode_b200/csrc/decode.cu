@@ -872,21 +872,21 @@ __global__ void __launch_bounds__(dec::kThreads, 1)
 }
 
 int current_device_sm_count() {
-    static int cached[64] = {};
+    static std::atomic<int> cached[64] = {};  // 0: not asked yet
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
         (void)cudaGetLastError();  // no device: leave no error behind for later launches
         return 148;
     }
-    if (!cached[dev]) {
-        int n = 0;
+    int n = cached[dev].load();
+    if (!n) {
         if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1) {
             (void)cudaGetLastError();
             return 148;
         }
-        cached[dev] = n;
+        cached[dev].store(n);
     }
-    return cached[dev];
+    return n;
 }
 
 bool make_decode_plan(int32_t T, int32_t H, int32_t topk, int sm_count, DecodePlan *plan, int splits,
@@ -932,8 +932,9 @@ bool make_decode_plan(int32_t T, int32_t H, int32_t topk, int sm_count, DecodePl
 // Tensor maps for Q: a 2-D FP16 view [rows = T*H, cols] of q_nope (cols 512)
 // or q_rope (cols 64), box 64 cols x HG rows, 128-byte swizzle.
 static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    if (!fn) {
+    static std::atomic<PFN_cuTensorMapEncodeTiled_v12000> fn{nullptr};  // looked up once, by any thread
+    PFN_cuTensorMapEncodeTiled_v12000 f = fn.load();
+    if (!f) {
         void *p = nullptr;
         cudaDriverEntryPointQueryResult q;
         if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
@@ -941,9 +942,10 @@ static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
             (void)cudaGetLastError();
             return nullptr;
         }
-        fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+        f = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+        fn.store(f);
     }
-    return fn;
+    return f;
 }
 
 // Encoded maps are kept in a small per-thread cache keyed by (address, rows,

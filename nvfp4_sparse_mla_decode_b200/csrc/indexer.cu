@@ -1325,8 +1325,9 @@ __global__ void __launch_bounds__(kTopkThreads, 1) indexer_topk_kernel(const Top
 
 // ---------------------------------------------------------------- launch
 static PFN_cuTensorMapEncodeTiled_v12000 index_map_encoder() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    if (!fn) {
+    static std::atomic<PFN_cuTensorMapEncodeTiled_v12000> fn{nullptr};  // looked up once, by any thread
+    PFN_cuTensorMapEncodeTiled_v12000 f = fn.load();
+    if (!f) {
         void *p = nullptr;
         cudaDriverEntryPointQueryResult q;
         if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
@@ -1334,9 +1335,10 @@ static PFN_cuTensorMapEncodeTiled_v12000 index_map_encoder() {
             (void)cudaGetLastError();
             return nullptr;
         }
-        fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+        f = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+        fn.store(f);
     }
-    return fn;
+    return f;
 }
 
 // 2-D byte matrix [rows, 128] with a box of box_rows x 128 bytes, 128-byte swizzle.
