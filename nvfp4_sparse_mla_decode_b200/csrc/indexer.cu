@@ -920,6 +920,9 @@ __global__ void __launch_bounds__(kTopkThreads, 1) indexer_topk_kernel(const Top
     }
 
     // ------------------------------- 2. collect this CTA's candidates
+    // With P > 1 each candidate also goes straight to this CTA's workspace
+    // list as it is found, for the selecting CTA.
+    uint2 *const pub_dst = P > 1 ? a.cand + ((int64_t)t * P + part) * kCandCap : nullptr;
     if (slice_lost()) return;
     uint32_t m = 0;  // candidates found in the range (block-uniform; may pass the cap)
     const float tau_f = key_score(tau);  // score >= tau_f  <=>  key >= tau (scores are never NaN)
@@ -968,6 +971,7 @@ __global__ void __launch_bounds__(kTopkThreads, 1) indexer_topk_kernel(const Top
             if (at < (uint32_t)kCandCap) {
                 cand_key[at] = k;
                 cand_pos[at] = r0 + base + b;
+                if (pub_dst) pub_dst[at] = make_uint2(k, (uint32_t)(r0 + base + b));
             }
             kmax = max(kmax, k);
             ++at;
@@ -1056,6 +1060,7 @@ __global__ void __launch_bounds__(kTopkThreads, 1) indexer_topk_kernel(const Top
                     if (at < (uint32_t)kCandCap) {
                         cand_key[at] = k;
                         cand_pos[at] = p + e;
+                        if (pub_dst) pub_dst[at] = make_uint2(k, (uint32_t)(p + e));
                     }
                     kmax = max(kmax, k);
                     ++at;
@@ -1075,10 +1080,7 @@ __global__ void __launch_bounds__(kTopkThreads, 1) indexer_topk_kernel(const Top
     uint32_t tau_max = tau;  // the highest threshold among the request's parts
     uint32_t key_lo = tau, key_hi = cmax;  // a range holding every candidate key
     if (P > 1) {
-        const int64_t slot = (int64_t)t * P + part;
-        const uint32_t keep = min(m, (uint32_t)kCandCap);
-        uint2 *dst = a.cand + slot * kCandCap;
-        for (uint32_t i = tid; i < keep; i += kTopkThreads) dst[i] = make_uint2(cand_key[i], (uint32_t)cand_pos[i]);
+        const int64_t slot = (int64_t)t * P + part;  // its candidates are in the workspace already
         if (tid == 0) a.counts[slot] = make_uint4(m, tau, cmax, 0u);
         __threadfence();
         __syncthreads();
